@@ -1,0 +1,208 @@
+/*
+ * cce.h — C ABI of the flash-CCE ORPO language-model head for NVIDIA B200
+ * (sm_100a).
+ *
+ * The head takes final hidden states H[M,D], a frozen output projection
+ * W[V,D] and per-row labels y[M].  It computes per-row logp and lse without
+ * ever storing the [M,V] logits, the ORPO loss, its cotangent dL/dlogp, and
+ * dL/dH.  The operations are those of the mlx-bun design pages:
+ *
+ *   "Training — design (ORPO, flash-CCE head, prefix sharing, segmented
+ *    backward)", mlx-bun 1.0.0: §1 "The objective", §5.1 "The head: from
+ *    token-chunking to the flash-CCE kernel", §5.6 "Quantized base";
+ *   "ORPO training — design", mlx-bun 0.0.6: "Memory & speed optimization",
+ *    ranked lever 1 and its "Implementation spec — fused linear-CE log-prob
+ *    head" (forward online softmax, backward recompute from the saved lse);
+ *   "flash-CCE host-buffer pin leak — post-mortem", mlx-bun 0.0.6 (why no host
+ *    pointer outlives a call).
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Pointers are DEVICE pointers on the current CUDA device unless a comment
+ *   says "host".  Host structs (cce_head, cce_layout) are read during the call
+ *   only; their fields go to the kernels by value.  The library keeps no
+ *   pointer after a call returns.
+ * - Ownership: the caller allocates and frees everything, the workspace
+ *   included.  The library never calls cudaMalloc or cudaFree.
+ * - Asynchrony: every call enqueues work on `stream` and returns; outputs are
+ *   valid once the stream reaches them.  Nothing synchronises except
+ *   cce_device_status().
+ * - Errors: argument problems are detected before anything is enqueued and
+ *   returned synchronously (CCE_ERR_INVALID_ARGUMENT, CCE_ERR_UNSUPPORTED,
+ *   CCE_ERR_WORKSPACE_TOO_SMALL).  A failed launch returns CCE_ERR_CUDA.
+ *   Problems only the device can see (a label >= V, an empty response
+ *   segment, a mean log-prob outside the domain of log1mexp, a bounded wait
+ *   that ran out) set a bit in the status word at the start of the workspace;
+ *   the kernels then finish without trapping, and cce_device_status() reports
+ *   and clears the bits.  No C++ exception crosses this interface.
+ * - Labels: y < 0 marks an ignored row (logp = 0, no loss term, dH row
+ *   exactly 0; lse is still computed).  y >= V is an error.
+ * - Tensor-core path requirements: D % 64 == 0; 16-byte aligned pointers.
+ */
+#ifndef CCE_H_
+#define CCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* cce_stream_t;
+
+typedef enum {
+  CCE_OK = 0,
+  CCE_ERR_INVALID_ARGUMENT = 1,
+  CCE_ERR_UNSUPPORTED = 2,
+  CCE_ERR_CUDA = 3,
+  CCE_ERR_WORKSPACE_TOO_SMALL = 4,
+  CCE_ERR_LABEL_OUT_OF_RANGE = 5,  /* device: some y >= V                    */
+  CCE_ERR_DEVICE_TIMEOUT = 6,      /* device: a bounded wait ran out          */
+  CCE_ERR_EMPTY_SEGMENT = 7,       /* device: no labelled chosen/rejected row */
+  CCE_ERR_DOMAIN = 8               /* device: mean logp >= 0 (log1mexp)       */
+} cce_status;
+
+typedef enum { CCE_F32 = 0, CCE_BF16 = 1 } cce_dtype;
+
+typedef enum {
+  CCE_W_DENSE = 0,        /* w: [V, D] row-major, dtype f32 or bf16           */
+  CCE_W_AFFINE_Q4_G64 = 1 /* w: uint32 [V, D/8]; element 8k+j of a row is bits
+                             4j..4j+3 of word k (low nibble first);
+                             scales, biases: bf16 [V, D/64]; the weight is
+                             q*scale + bias (Training design §5.6).           */
+} cce_wformat;
+
+/* The frozen head (host struct; device pointers inside). */
+typedef struct {
+  cce_wformat format;
+  cce_dtype dtype;       /* dense: dtype of w; Q4: must be CCE_BF16 (scales) */
+  int64_t V, D;
+  const void* w;
+  const void* scales;    /* Q4 only, else NULL */
+  const void* biases;    /* Q4 only, else NULL */
+} cce_head;
+
+/* Disjoint head-row ranges [begin, end) of one ORPO pair (host struct).
+ * prompt rows feed the NLL term in "full" scope; chosen rows give the
+ * length-normalised mean lw, rejected rows lr (Training design §1). */
+typedef struct {
+  int64_t prompt_begin, prompt_end;
+  int64_t chosen_begin, chosen_end;
+  int64_t rejected_begin, rejected_end;
+} cce_layout;
+
+/* NLL scope of the ORPO objective (Training design §1, `sft_scope`). */
+enum { CCE_SCOPE_FULL = 0, CCE_SCOPE_RESPONSE = 1 };
+
+/* Width of one vocab block of the per-block statistics (and of one vocab
+ * tile of the kernels). */
+#define CCE_VOCAB_BLOCK 256
+
+/* Number of vocab blocks: ceil(V / CCE_VOCAB_BLOCK). */
+int64_t cce_blockmax_cols(int64_t V);
+
+/* Bytes of workspace that cce_forward and cce_backward_dh need for this
+ * problem with the default backward chunk.  A larger workspace lets the
+ * backward use wider vocab chunks (fewer passes); a smaller one (down to
+ * cce_workspace_min_bytes) narrower ones.  Returns 0 for invalid input. */
+size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W);
+size_t cce_workspace_min_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W);
+
+/*
+ * Forward of the head (Training design §5.1; ORPO design 0.0.6, fused-head
+ * spec "Forward (online-softmax over vocab tiles)"):
+ *   lse[m]  = logsumexp_v (H[m] . W[v])
+ *   logp[m] = H[m] . W[y_m] - lse[m]      (0 when y_m < 0)
+ * H: [M, D] row-major, f32 or bf16.  labels: int32 [M].
+ * logp, lse: fp32 [M] outputs.
+ * tgt_logit: optional fp32 [M] output of H[m] . W[y_m] (untouched when y < 0).
+ * blockmax: optional fp32 [cce_blockmax_cols(V), M] output, block-major:
+ *   blockmax[b*M + m] = max over v in block b of H[m] . W[v]; the backward's
+ *   block skip reads it.
+ * ws: workspace of ws_bytes (see cce_workspace_bytes); its first 256 bytes
+ *   hold the device status word and must be zeroed once before first use.
+ */
+cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M,
+                       const cce_head* W, const int32_t* labels, float* logp,
+                       float* lse, float* tgt_logit, float* blockmax, void* ws,
+                       size_t ws_bytes, cce_stream_t stream);
+
+/*
+ * ORPO loss from per-row log-probs (Training design §1, orpoLossFromLogps):
+ *   lw, lr, pm = means of logp over the labelled chosen, rejected, prompt rows
+ *   NLL  = -(sum_prompt + sum_chosen)/(n_prompt + n_chosen)   (full scope;
+ *          equal to combineFullNll) or -lw (response scope)
+ *   z    = (lw - lr) - (log1mexp(lw) - log1mexp(lr))
+ *   L_OR = -log sigmoid(z);  L = NLL + lambda * L_OR
+ * out8 (device, fp64 [8]): L, NLL, L_OR, lw, lr, pm, z, sigmoid(z).
+ * Only the first 256 bytes of ws are used (status word).
+ */
+cce_status orpo_loss_from_logps(const float* logp, const int32_t* labels,
+                                int64_t M, const cce_layout* layout,
+                                double lambda, int sft_scope, double* out8,
+                                void* ws, size_t ws_bytes,
+                                cce_stream_t stream);
+
+/*
+ * Cotangent of the ORPO loss with respect to logp (the "1/(1-P)"-scaled OR
+ * gradient plus the NLL term; ORPO design 0.0.6, regularization notes):
+ *   chosen:   lambda (sigmoid(z) - 1) / (1 - e^lw) / n_chosen + s_C
+ *   rejected: -lambda (sigmoid(z) - 1) / (1 - e^lr) / n_rejected
+ *   prompt:   s_P;   ignored rows and rows outside the layout: 0
+ * with s_C = s_P = -1/(n_prompt + n_chosen) (full) or s_C = -1/n_chosen,
+ * s_P = 0 (response).  coeff: fp32 [M] output.
+ */
+cce_status orpo_grad_coeffs(const float* logp, const int32_t* labels,
+                            int64_t M, const cce_layout* layout, double lambda,
+                            int sft_scope, float* coeff, void* ws,
+                            size_t ws_bytes, cce_stream_t stream);
+
+/*
+ * Backward of the head (ORPO design 0.0.6, fused-head spec "Backward
+ * (recompute vocab tiles from the saved LSE)"; Training design §5.1):
+ *   dH[m] = coeff[m] * sum_v (onehot(y_m)_v - p_mv) W[v],
+ *   p_mv  = exp(H[m].W[v] - lse[m]) recomputed tile by tile.
+ * coeff: fp32 [M], the cotangent dL/dlogp (e.g. from orpo_grad_coeffs).
+ * lse: fp32 [M] from cce_forward on the same H and W.
+ * filter_eps > 0 drops p_mv < filter_eps on non-target columns (the coeff
+ *   filter, Training design §5.1); 0 disables it.
+ * blockmax: optional; when given (with filter_eps > 0) a 128-row x 256-vocab
+ *   tile is skipped when every row's block probability exp(blockmax - lse) is
+ *   below filter_eps and no label of a row with coeff != 0 falls in the
+ *   block, which is exact relative to the filter.
+ * dH: fp32 [M, D] output, overwritten.
+ * skip_stats: optional device uint64 [2] incremented by (skipped tiles,
+ *   total tiles).
+ */
+cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M,
+                           const cce_head* W, const int32_t* labels,
+                           const float* lse, const float* coeff,
+                           float filter_eps, const float* blockmax, float* dH,
+                           unsigned long long* skip_stats, void* ws,
+                           size_t ws_bytes, cce_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the status word in ws, and
+ * returns the first error it holds (CCE_OK when none). */
+cce_status cce_device_status(void* ws, cce_stream_t stream);
+
+/* Human-readable name of a status. */
+const char* cce_status_string(cce_status s);
+
+/* Upper bound, in nanoseconds, of every bounded wait inside the kernels
+ * (default 2e9).  0 restores the default.  Process-wide; meant for tests of
+ * the timeout path. */
+void cce_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the timeout path: launches one CTA that waits, with the
+ * current wait limit, on an mbarrier nothing arrives on.  The wait runs out,
+ * the kernel sets CCE_ERR_DEVICE_TIMEOUT in the status word and returns;
+ * the caller reads it with cce_device_status(). */
+cce_status cce_selftest_wait_timeout(void* ws, size_t ws_bytes,
+                                     cce_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CCE_H_ */

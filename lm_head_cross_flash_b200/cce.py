@@ -1,0 +1,252 @@
+"""ctypes binding of ``libcce.so`` (declared in ``include/cce.h``).
+
+Argument marshalling only: every step of the head runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (used for device memory and
+streams); the functions keep the C names and raise ``CCEError`` for a
+synchronous error status.  The library is loaded on first use; if it is
+missing the call raises instead of falling back to anything else.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcce.so")
+
+CCE_F32, CCE_BF16 = 0, 1
+CCE_W_DENSE, CCE_W_AFFINE_Q4_G64 = 0, 1
+SCOPE = {"full": 0, "response": 1}
+VOCAB_BLOCK = 256
+
+STATUS_NAMES = {
+    0: "CCE_OK", 1: "CCE_ERR_INVALID_ARGUMENT", 2: "CCE_ERR_UNSUPPORTED",
+    3: "CCE_ERR_CUDA", 4: "CCE_ERR_WORKSPACE_TOO_SMALL",
+    5: "CCE_ERR_LABEL_OUT_OF_RANGE", 6: "CCE_ERR_DEVICE_TIMEOUT",
+    7: "CCE_ERR_EMPTY_SEGMENT", 8: "CCE_ERR_DOMAIN",
+}
+
+
+class CCEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class _Head(ctypes.Structure):
+    _fields_ = [("format", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("V", ctypes.c_int64), ("D", ctypes.c_int64),
+                ("w", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("biases", ctypes.c_void_p)]
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "prompt_begin", "prompt_end", "chosen_begin", "chosen_end",
+        "rejected_begin", "rejected_end")]
+
+
+_lib = None
+
+_SIGS = {
+    "cce_blockmax_cols": (ctypes.c_int64, [ctypes.c_int64]),
+    "cce_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_Head)]),
+    "cce_workspace_min_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_Head)]),
+    "cce_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.POINTER(_Head),
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "orpo_loss_from_logps": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                            ctypes.POINTER(_Layout), ctypes.c_double, ctypes.c_int,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                            ctypes.c_void_p]),
+    "orpo_grad_coeffs": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.POINTER(_Layout), ctypes.c_double, ctypes.c_int,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]),
+    "cce_backward_dh": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.POINTER(_Head),
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_size_t, ctypes.c_void_p]),
+    "cce_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "cce_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "cce_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+}
+
+
+def lib():
+    """Load ``libcce.so`` once; raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m lm_head_cross_flash_b200.build` (no fallback exists)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise CCEError(st, where)
+
+
+@dataclass
+class Head:
+    """The frozen head: dense ``w`` [V, D] (f32 or bf16), or a 4-bit affine
+    head (``w`` uint32 [V, D/8] stored as int32, ``scales``/``biases`` bf16
+    [V, D/64])."""
+
+    w: torch.Tensor
+    V: int
+    D: int
+    fmt: int = CCE_W_DENSE
+    scales: torch.Tensor | None = None
+    biases: torch.Tensor | None = None
+
+    @property
+    def dtype(self) -> int:
+        if self.fmt == CCE_W_AFFINE_Q4_G64:
+            return CCE_BF16
+        return CCE_F32 if self.w.dtype == torch.float32 else CCE_BF16
+
+    def c(self) -> _Head:
+        return _Head(self.fmt, self.dtype, self.V, self.D, self.w.data_ptr(),
+                     None if self.scales is None else self.scales.data_ptr(),
+                     None if self.biases is None else self.biases.data_ptr())
+
+
+def h_dtype(H: torch.Tensor) -> int:
+    return CCE_F32 if H.dtype == torch.float32 else CCE_BF16
+
+
+def blockmax_cols(V: int) -> int:
+    return int(lib().cce_blockmax_cols(V))
+
+
+def workspace_bytes(M: int, H_dtype: int, head: Head) -> int:
+    return int(lib().cce_workspace_bytes(M, H_dtype, ctypes.byref(head.c())))
+
+
+def workspace_min_bytes(M: int, H_dtype: int, head: Head) -> int:
+    return int(lib().cce_workspace_min_bytes(M, H_dtype, ctypes.byref(head.c())))
+
+
+def alloc_workspace(M: int, H_dtype: int, head: Head, device="cuda", nbytes=None):
+    """Caller-side workspace (torch allocation) with a zeroed status word."""
+    n = workspace_bytes(M, H_dtype, head) if nbytes is None else nbytes
+    if n == 0:
+        raise CCEError(1, "cce_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def cce_forward(H, head: Head, labels, logp, lse, tgt_logit=None, blockmax=None,
+                ws=None, stream=None):
+    st = lib().cce_forward(_p(H), h_dtype(H), H.shape[0], ctypes.byref(head.c()),
+                           _p(labels), _p(logp), _p(lse), _p(tgt_logit), _p(blockmax),
+                           _p(ws), ws.numel(), _stream(stream))
+    _check(st, "cce_forward")
+
+
+def _layout(layout):
+    return _Layout(*[int(x) for x in layout])
+
+
+def orpo_loss_from_logps(logp, labels, layout, lam, sft_scope, out8, ws, stream=None):
+    st = lib().orpo_loss_from_logps(_p(logp), _p(labels), logp.shape[0],
+                                    ctypes.byref(_layout(layout)), float(lam),
+                                    SCOPE.get(sft_scope, sft_scope), _p(out8), _p(ws),
+                                    ws.numel(), _stream(stream))
+    _check(st, "orpo_loss_from_logps")
+
+
+def orpo_grad_coeffs(logp, labels, layout, lam, sft_scope, coeff, ws, stream=None):
+    st = lib().orpo_grad_coeffs(_p(logp), _p(labels), logp.shape[0],
+                                ctypes.byref(_layout(layout)), float(lam),
+                                SCOPE.get(sft_scope, sft_scope), _p(coeff), _p(ws),
+                                ws.numel(), _stream(stream))
+    _check(st, "orpo_grad_coeffs")
+
+
+def cce_backward_dh(H, head: Head, labels, lse, coeff, filter_eps, blockmax, dH,
+                    skip_stats=None, ws=None, stream=None):
+    st = lib().cce_backward_dh(_p(H), h_dtype(H), H.shape[0], ctypes.byref(head.c()),
+                               _p(labels), _p(lse), _p(coeff), float(filter_eps),
+                               _p(blockmax), _p(dH), _p(skip_stats), _p(ws), ws.numel(),
+                               _stream(stream))
+    _check(st, "cce_backward_dh")
+
+
+def cce_device_status(ws, stream=None) -> int:
+    return int(lib().cce_device_status(_p(ws), _stream(stream)))
+
+
+def cce_set_wait_limit_ns(ns: int):
+    lib().cce_set_wait_limit_ns(int(ns))
+
+
+def cce_selftest_wait_timeout(ws, stream=None):
+    _check(lib().cce_selftest_wait_timeout(_p(ws), ws.numel(), _stream(stream)),
+           "cce_selftest_wait_timeout")
+
+
+# ----------------------------------------------------------------------------
+# one pass of the whole head
+# ----------------------------------------------------------------------------
+
+@dataclass
+class HeadBuffers:
+    """Device buffers of one head pass (outputs and the workspace)."""
+
+    logp: torch.Tensor
+    lse: torch.Tensor
+    tgt: torch.Tensor
+    blockmax: torch.Tensor
+    out8: torch.Tensor
+    coeff: torch.Tensor
+    dH: torch.Tensor
+    skip: torch.Tensor
+    ws: torch.Tensor
+
+    @staticmethod
+    def alloc(M: int, D: int, V: int, H_dtype: int, head: Head, device="cuda",
+              ws_bytes=None):
+        f = dict(device=device, dtype=torch.float32)
+        return HeadBuffers(
+            logp=torch.empty(M, **f), lse=torch.empty(M, **f), tgt=torch.zeros(M, **f),
+            blockmax=torch.empty(blockmax_cols(V), M, **f),
+            out8=torch.empty(8, device=device, dtype=torch.float64),
+            coeff=torch.empty(M, **f), dH=torch.empty(M, D, **f),
+            skip=torch.zeros(2, device=device, dtype=torch.int64),
+            ws=alloc_workspace(M, H_dtype, head, device, ws_bytes))
+
+
+def orpo_head_pass(H, head: Head, labels, layout, lam, sft_scope, filter_eps,
+                   block_skip: bool, buf: HeadBuffers, stream=None):
+    """Forward, ORPO loss, cotangent and dH, all enqueued on one stream."""
+    cce_forward(H, head, labels, buf.logp, buf.lse, buf.tgt, buf.blockmax, buf.ws, stream)
+    orpo_loss_from_logps(buf.logp, labels, layout, lam, sft_scope, buf.out8, buf.ws, stream)
+    orpo_grad_coeffs(buf.logp, labels, layout, lam, sft_scope, buf.coeff, buf.ws, stream)
+    cce_backward_dh(H, head, labels, buf.lse, buf.coeff, filter_eps,
+                    buf.blockmax if block_skip else None, buf.dH, buf.skip, buf.ws, stream)

@@ -1,0 +1,249 @@
+// aux_kernels.cuh — the small, bandwidth- or latency-bound steps of the head:
+// the cross-block LSE merge, the ORPO epilogue (loss and cotangent), the
+// block-skip planner, operand preparation, and the timeout self-test.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "gemm_tc.cuh"
+
+namespace cce {
+
+// ------------------------------------------------------------ LSE merge --
+// lse[m] = max_b part_m[b,m] + log(sum_b part_s[b,m] exp(part_m[b,m] - max));
+// logp[m] = tgt[m] - lse[m] for 0 <= y < V, else 0.  (Cross-block merge of
+// the per-block partials; Training design §5.1, "Vocab-parallel grid":
+// the merge is a cheap reduction of (blockMax, block sum-exp) partials.)
+// One warp per row: lanes stride over the blocks, then a shuffle reduction.
+__global__ void __launch_bounds__(256) merge_lse_kernel(
+    const float* __restrict__ part_m, const float* __restrict__ part_s,
+    int cols, int M, const int32_t* __restrict__ labels, int V,
+    const float* __restrict__ tgt, float* __restrict__ logp,
+    float* __restrict__ lse, uint32_t* status) {
+  const int warps = blockDim.x >> 5;
+  const int row = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  float m = -INFINITY, s = 0.f;
+  for (int b = lane; b < cols; b += 32) {
+    const float mb = part_m[static_cast<size_t>(b) * M + row];
+    const float sb = part_s[static_cast<size_t>(b) * M + row];
+    const float mn = fmaxf(m, mb);
+    s = s * expf(m - mn) + sb * expf(mb - mn);
+    m = mn;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+    const float so = __shfl_xor_sync(0xffffffffu, s, off);
+    const float mn = fmaxf(m, mo);
+    const float a = (m == -INFINITY) ? 0.f : s * expf(m - mn);
+    const float bb = (mo == -INFINITY) ? 0.f : so * expf(mo - mn);
+    s = a + bb;
+    m = mn;
+  }
+  if (lane == 0) {
+    const float l = m + logf(s);
+    lse[row] = l;
+    const int y = labels[row];
+    if (y >= V) set_status(status, ST_LABEL);
+    logp[row] = (y >= 0 && y < V) ? tgt[row] - l : 0.f;
+  }
+}
+
+// ------------------------------------------------------- ORPO epilogue --
+struct OrpoArgs {
+  int64_t pb, pe, cb, ce, rb, re;  // layout
+  double lambda;
+  int scope;                       // 0 full, 1 response
+  int want_coeff;
+};
+
+// log(1 - e^x), x < 0: two-branch form (Maechler 2012), fp64.
+__device__ __forceinline__ double log1mexp_d(double x) {
+  return x > -0.6931471805599453 ? log(-expm1(x)) : log1p(-exp(x));
+}
+
+__device__ __forceinline__ double softplus_d(double x) {
+  return fmax(x, 0.0) + log1p(exp(-fabs(x)));
+}
+
+// One block: fp64 segment sums (warp shuffles + shared memory), then thread 0
+// forms lw, lr, pm, NLL, z, L_OR, L (Training design §1) and, in coefficient
+// mode, every thread writes dL/dlogp for its rows.
+__global__ void __launch_bounds__(1024) orpo_kernel(
+    const float* __restrict__ logp, const int32_t* __restrict__ labels,
+    int64_t M, OrpoArgs o, double* __restrict__ out8,
+    float* __restrict__ coeff, uint32_t* status) {
+  double s[3] = {0.0, 0.0, 0.0};
+  double n[3] = {0.0, 0.0, 0.0};
+  for (int64_t m = threadIdx.x; m < M; m += blockDim.x) {
+    if (labels[m] < 0) continue;
+    const double v = static_cast<double>(logp[m]);
+    if (m >= o.pb && m < o.pe) { s[0] += v; n[0] += 1.0; }
+    if (m >= o.cb && m < o.ce) { s[1] += v; n[1] += 1.0; }
+    if (m >= o.rb && m < o.re) { s[2] += v; n[2] += 1.0; }
+  }
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      s[i] += __shfl_xor_sync(0xffffffffu, s[i], off);
+      n[i] += __shfl_xor_sync(0xffffffffu, n[i], off);
+    }
+  }
+  __shared__ double red[32][6];
+  __shared__ double sc[8];  // c_prompt, c_chosen, c_rejected, ok
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0)
+    for (int i = 0; i < 3; ++i) { red[warp][i] = s[i]; red[warp][3 + i] = n[i]; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t[6] = {0, 0, 0, 0, 0, 0};
+    const int nw = (blockDim.x + 31) >> 5;
+    for (int w = 0; w < nw; ++w)
+      for (int i = 0; i < 6; ++i) t[i] += red[w][i];
+    const double sP = t[0], sC = t[1], sR = t[2];
+    const double nP = t[3], nC = t[4], nR = t[5];
+    double res[8];
+    const double qnan = __longlong_as_double(0x7ff8000000000000ll);
+    double cP = 0.0, cC = 0.0, cR = 0.0;
+    bool ok = true;
+    if (nC == 0.0 || nR == 0.0) {
+      set_status(status, ST_EMPTY);
+      ok = false;
+    }
+    const double lw = ok ? sC / nC : qnan;
+    const double lr = ok ? sR / nR : qnan;
+    if (ok && !(lw < 0.0 && lr < 0.0)) {
+      set_status(status, ST_DOMAIN);
+      ok = false;
+    }
+    if (ok) {
+      const double pm = nP > 0.0 ? sP / nP : 0.0;
+      const double nll = o.scope == 0 ? -(sP + sC) / (nP + nC) : -lw;
+      const double z = (lw - lr) - (log1mexp_d(lw) - log1mexp_d(lr));
+      const double lor = softplus_d(-z);
+      const double sig = z >= 0.0 ? 1.0 / (1.0 + exp(-z)) : exp(z) / (1.0 + exp(z));
+      res[0] = nll + o.lambda * lor;
+      res[1] = nll;
+      res[2] = lor;
+      res[3] = lw;
+      res[4] = lr;
+      res[5] = pm;
+      res[6] = z;
+      res[7] = sig;
+      const double aw = 1.0 / (-expm1(lw));
+      const double ar = 1.0 / (-expm1(lr));
+      const double dz = sig - 1.0;
+      const double sNll = o.scope == 0 ? -1.0 / (nP + nC) : -1.0 / nC;
+      cP = o.scope == 0 ? sNll : 0.0;
+      cC = o.lambda * dz * aw / nC + sNll;
+      cR = -o.lambda * dz * ar / nR;
+    } else {
+      for (int i = 0; i < 8; ++i) res[i] = qnan;
+    }
+    if (out8 != nullptr)
+      for (int i = 0; i < 8; ++i) out8[i] = res[i];
+    sc[0] = cP;
+    sc[1] = cC;
+    sc[2] = cR;
+  }
+  if (!o.want_coeff) return;
+  __syncthreads();
+  const float cP = static_cast<float>(sc[0]);
+  const float cC = static_cast<float>(sc[1]);
+  const float cR = static_cast<float>(sc[2]);
+  for (int64_t m = threadIdx.x; m < M; m += blockDim.x) {
+    float c = 0.f;
+    if (labels[m] >= 0) {
+      if (m >= o.pb && m < o.pe) c = cP;
+      else if (m >= o.cb && m < o.ce) c = cC;
+      else if (m >= o.rb && m < o.re) c = cR;
+    }
+    coeff[m] = c;
+  }
+}
+
+// ----------------------------------------------------- block-skip planner --
+// tile_skip[rt, b] = 1 when, for every row m of row tile rt with coeff != 0,
+// the block's largest softmax probability exp(blockmax[b,m] - lse[m]) is
+// below eps and y_m is not in block b: every term of that tile would be
+// dropped by the coefficient filter.  row_skip[rt] = 1 when every row of the
+// tile has coeff == 0.  One warp per (rt, b).
+__global__ void __launch_bounds__(256) skip_plan_kernel(
+    const float* __restrict__ blockmax, const float* __restrict__ lse,
+    const int32_t* __restrict__ labels, const float* __restrict__ coeff,
+    int M, int cols, int n_rt, float eps, uint8_t* __restrict__ tile_skip,
+    uint8_t* __restrict__ row_skip, unsigned long long* stats) {
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (unit >= static_cast<int64_t>(n_rt) * cols) return;
+  const int rt = static_cast<int>(unit / cols);
+  const int b = static_cast<int>(unit - static_cast<int64_t>(rt) * cols);
+  bool all_zero = true, skip = true;
+  for (int i = lane; i < BM; i += 32) {
+    const int m = rt * BM + i;
+    if (m >= M) continue;
+    const float c = coeff[m];
+    if (c == 0.f) continue;
+    all_zero = false;
+    const int y = labels[m];
+    if (y >= b * BN && y < (b + 1) * BN) skip = false;
+    if (blockmax == nullptr) { skip = false; continue; }
+    const float p = softmax_p(blockmax[static_cast<size_t>(b) * M + m], -lse[m] * LOG2E);
+    if (!(p < eps)) skip = false;
+  }
+  all_zero = __all_sync(0xffffffffu, all_zero);
+  skip = __all_sync(0xffffffffu, skip) && !all_zero;
+  if (lane == 0) {
+    tile_skip[unit] = skip ? 1 : 0;
+    if (b == 0) row_skip[rt] = all_zero ? 1 : 0;
+    if (stats != nullptr) {
+      if (skip || all_zero) atomicAdd(&stats[0], 1ull);
+      atomicAdd(&stats[1], 1ull);
+    }
+  }
+}
+
+// ------------------------------------------------------ operand preparation --
+// Split an fp32 matrix [rows, D] into bf16 parts so that three bf16 products
+// reproduce an fp32 product to ~2^-16: x = hi + lo, hi = bf16(x),
+// lo = bf16(x - hi).  dst is [rows, 3*D]; `order` selects the part written to
+// each third: 0 -> (hi, hi, lo) for the left operand, 1 -> (hi, lo, hi) for
+// the right operand, so that the K-concatenated product is
+// hi*hi + hi*lo + lo*hi.
+__global__ void split_f32_kernel(const float* __restrict__ src, int64_t rows,
+                                 int D, int order,
+                                 __nv_bfloat16* __restrict__ dst) {
+  const int64_t n = rows * D;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / D;
+    const int d = static_cast<int>(i - r * D);
+    const float x = src[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    __nv_bfloat16* o = dst + r * (3 * static_cast<int64_t>(D));
+    o[d] = hi;
+    o[D + d] = order == 0 ? hi : lo;
+    o[2 * D + d] = order == 0 ? lo : hi;
+  }
+}
+
+// ------------------------------------------------------ timeout self-test --
+__global__ void selftest_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: the wait must run out.
+    if (!wait_bounded(&bar, 0, limit_ns, nullptr)) set_status(status, ST_TIMEOUT);
+  }
+}
+
+}  // namespace cce

@@ -1,0 +1,501 @@
+// cce.cu — host side of the C ABI declared in include/cce.h: argument
+// validation, workspace layout, TMA tensor maps and kernel launches on the
+// caller's stream.  Nothing here allocates device memory; the caller's
+// workspace holds every intermediate.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/cce.h"
+#include "aux_kernels.cuh"
+#include "gemm_tc.cuh"
+
+using namespace cce;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+constexpr int64_t kDefaultChunkBytes = 256ll << 20;  // G' chunk, default
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------ driver API --
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                   void*, const cuuint64_t*, const cuuint64_t*,
+                                   const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D tensor map over a row-major [rows, cols] 16-bit matrix with row
+// stride `ld` elements, box {box_c, box_r}, 128-byte swizzle, zero OOB fill.
+bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
+              uint64_t rows, uint64_t ld, uint32_t box_c, uint32_t box_r) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_c, box_r};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------- device facts --
+struct DevInfo {
+  int sms = 0;
+  bool attrs = false;
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+cce_status device_info(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.attrs) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return CCE_ERR_CUDA;
+    if (cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+      return CCE_ERR_CUDA;
+    d.attrs = true;
+  }
+  *sms = d.sms;
+  return CCE_OK;
+}
+
+// ------------------------------------------------------------ validation --
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cce_status check_head(const cce_head* W, cce_dtype h_dtype) {
+  if (W == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  if (W->V <= 0 || W->D <= 0 || W->w == nullptr || !aligned16(W->w))
+    return CCE_ERR_INVALID_ARGUMENT;
+  if (W->V > (int64_t(1) << 30) || W->D > (int64_t(1) << 16)) return CCE_ERR_UNSUPPORTED;
+  if (W->D % 64 != 0) return CCE_ERR_UNSUPPORTED;
+  if (W->format == CCE_W_DENSE) {
+    if (W->dtype != CCE_F32 && W->dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
+    if (W->dtype != h_dtype) return CCE_ERR_UNSUPPORTED;
+    return CCE_OK;
+  }
+  if (W->format == CCE_W_AFFINE_Q4_G64) return CCE_ERR_UNSUPPORTED;
+  return CCE_ERR_INVALID_ARGUMENT;
+}
+
+// ------------------------------------------------------ workspace layout --
+struct Layout {
+  size_t status = 0;
+  size_t part_s = 0, part_m = 0, tgt = 0;  // forward
+  size_t hs = 0, ws = 0;                   // f32 split operands
+  size_t g = 0, tile_skip = 0, row_skip = 0;
+  int64_t vc = 0;                          // backward vocab chunk
+  size_t total = 0;
+};
+
+Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc) {
+  Layout L;
+  const int64_t cols = ceil_div(W->V, BN);
+  const int64_t n_rt = ceil_div(M, BM);
+  size_t o = kStatusBytes;
+  // forward region
+  size_t f = o;
+  L.part_s = f; f += align_up(size_t(cols) * M * 4);
+  L.part_m = f; f += align_up(size_t(cols) * M * 4);
+  L.tgt = f; f += align_up(size_t(M) * 4);
+  // backward region (shares the space after the status word)
+  size_t b = o;
+  L.g = b; b += align_up(size_t(M) * vc * 2);
+  L.tile_skip = b; b += align_up(size_t(n_rt) * cols);
+  L.row_skip = b; b += align_up(size_t(n_rt));
+  // split operands live after both regions
+  size_t s = std::max(f, b);
+  if (h == CCE_F32) {
+    L.hs = s; s += align_up(size_t(M) * 3 * W->D * 2);
+    L.ws = s; s += align_up(size_t(W->V) * 3 * W->D * 2);
+  }
+  L.vc = vc;
+  L.total = s;
+  return L;
+}
+
+int64_t default_vc(int64_t M, const cce_head* W) {
+  const int64_t vmax = ceil_div(W->V, BN) * BN;
+  int64_t vc = (kDefaultChunkBytes / (2 * M)) / BN * BN;
+  return std::max<int64_t>(BN, std::min(vc, vmax));
+}
+
+// Widest chunk whose layout fits in ws_bytes (0 if even the narrowest
+// does not fit).
+int64_t fit_vc(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes) {
+  const int64_t vmax = ceil_div(W->V, BN) * BN;
+  if (make_layout(M, h, W, BN).total > ws_bytes) return 0;
+  int64_t lo = 1, hi = vmax / BN;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) / 2;
+    if (make_layout(M, h, W, mid * BN).total <= ws_bytes) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo * BN;
+}
+
+uint32_t* status_word(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
+
+cce_status launch_ok() {
+  return cudaGetLastError() == cudaSuccess ? CCE_OK : CCE_ERR_CUDA;
+}
+
+int grid_for(int64_t tiles, int sms) {
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, sms)));
+}
+
+// Operands of the tensor-core GEMMs for one problem: 16-bit A (head rows)
+// and B (head) with their K extents.
+struct Operands {
+  const void* a;   // [M, ka] 16-bit
+  const void* b;   // [V, kb] 16-bit
+  int64_t k;       // contraction length used by the S GEMM
+  int64_t ld_a, ld_b;
+  bool bf16;
+  int64_t d_pass_off;  // kDh: offset (elements) of the lo half of a split head
+  int npass_dh;
+};
+
+cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_head* W,
+                            const Layout& L, void* ws, cudaStream_t st, Operands* op) {
+  const int64_t D = W->D;
+  if (h == CCE_BF16) {
+    op->a = H;
+    op->b = W->w;
+    op->k = D;
+    op->ld_a = D;
+    op->ld_b = D;
+    op->bf16 = true;
+    op->d_pass_off = 0;
+    op->npass_dh = 1;
+    return CCE_OK;
+  }
+  // fp32: three-part bf16 split, K = 3D.
+  auto* hs = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + L.hs);
+  auto* wsb = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + L.ws);
+  split_f32_kernel<<<1184, 256, 0, st>>>(static_cast<const float*>(H), M, int(D), 0, hs);
+  split_f32_kernel<<<1184, 256, 0, st>>>(static_cast<const float*>(W->w), W->V, int(D), 1, wsb);
+  if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  op->a = hs;
+  op->b = wsb;
+  op->k = 3 * D;
+  op->ld_a = 3 * D;
+  op->ld_b = 3 * D;
+  op->bf16 = true;
+  op->d_pass_off = D;  // columns [D, 2D) of the right split hold lo
+  op->npass_dh = 2;
+  return CCE_OK;
+}
+
+}  // namespace
+
+// ========================================================================
+extern "C" {
+
+const char* cce_status_string(cce_status s) {
+  switch (s) {
+    case CCE_OK: return "CCE_OK";
+    case CCE_ERR_INVALID_ARGUMENT: return "CCE_ERR_INVALID_ARGUMENT";
+    case CCE_ERR_UNSUPPORTED: return "CCE_ERR_UNSUPPORTED";
+    case CCE_ERR_CUDA: return "CCE_ERR_CUDA";
+    case CCE_ERR_WORKSPACE_TOO_SMALL: return "CCE_ERR_WORKSPACE_TOO_SMALL";
+    case CCE_ERR_LABEL_OUT_OF_RANGE: return "CCE_ERR_LABEL_OUT_OF_RANGE";
+    case CCE_ERR_DEVICE_TIMEOUT: return "CCE_ERR_DEVICE_TIMEOUT";
+    case CCE_ERR_EMPTY_SEGMENT: return "CCE_ERR_EMPTY_SEGMENT";
+    case CCE_ERR_DOMAIN: return "CCE_ERR_DOMAIN";
+  }
+  return "CCE_UNKNOWN_STATUS";
+}
+
+void cce_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns); }
+
+int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
+
+size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
+  if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
+  return make_layout(M, h_dtype, W, default_vc(M, W)).total;
+}
+
+size_t cce_workspace_min_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
+  if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
+  return make_layout(M, h_dtype, W, BN).total;
+}
+
+cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
+                       const int32_t* labels, float* logp, float* lse, float* tgt_logit,
+                       float* blockmax, void* ws, size_t ws_bytes, cce_stream_t stream) {
+  if (H == nullptr || labels == nullptr || logp == nullptr || lse == nullptr || ws == nullptr)
+    return CCE_ERR_INVALID_ARGUMENT;
+  if (M <= 0 || M > (int64_t(1) << 30)) return CCE_ERR_INVALID_ARGUMENT;
+  if (h_dtype != CCE_F32 && h_dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(H) || !aligned16(ws)) return CCE_ERR_INVALID_ARGUMENT;
+  cce_status s = check_head(W, h_dtype);
+  if (s != CCE_OK) return s;
+  const Layout L = make_layout(M, h_dtype, W, BN);
+  if (L.total > ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = device_info(&sms)) != CCE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* wsc = static_cast<char*>(ws);
+
+  Operands op;
+  if ((s = prepare_operands(H, h_dtype, M, W, L, ws, st, &op)) != CCE_OK) return s;
+  const int64_t V = W->V;
+  const int64_t cols = ceil_div(V, BN);
+  const int64_t n_rt = ceil_div(M, BM);
+  float* part_s = reinterpret_cast<float*>(wsc + L.part_s);
+  float* part_m = blockmax != nullptr ? blockmax : reinterpret_cast<float*>(wsc + L.part_m);
+  float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
+
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM) ||
+      !make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN))
+    return CCE_ERR_CUDA;
+
+  TileArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = int(M);
+  a.n_rt = int(n_rt);
+  a.n_ct = int(cols);
+  a.nk = int(op.k / BK);
+  a.npass = 1;
+  a.b_row0 = 0;
+  a.V = int(V);
+  a.D = int(W->D);
+  a.fmt = op.bf16 ? 1 : 0;
+  a.wait_ns = g_wait_ns.load();
+  a.status = status_word(ws);
+  a.labels = labels;
+  a.part_m = part_m;
+  a.part_s = part_s;
+  a.tgt = tgt;
+  a.ct_off = 0;
+  cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a);
+  if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+
+  const int rows_per_block = 8;
+  merge_lse_kernel<<<int(ceil_div(M, rows_per_block)), rows_per_block * 32, 0, st>>>(
+      part_m, part_s, int(cols), int(M), labels, int(V), tgt, logp, lse, status_word(ws));
+  return launch_ok();
+}
+
+static cce_status check_layout(const cce_layout* L, int64_t M) {
+  if (L == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  const int64_t r[3][2] = {{L->prompt_begin, L->prompt_end},
+                           {L->chosen_begin, L->chosen_end},
+                           {L->rejected_begin, L->rejected_end}};
+  for (int i = 0; i < 3; ++i) {
+    if (r[i][0] < 0 || r[i][1] < r[i][0] || r[i][1] > M) return CCE_ERR_INVALID_ARGUMENT;
+    for (int j = 0; j < i; ++j)
+      if (r[i][0] < r[j][1] && r[j][0] < r[i][1]) return CCE_ERR_INVALID_ARGUMENT;
+  }
+  if (r[1][1] == r[1][0] || r[2][1] == r[2][0]) return CCE_ERR_INVALID_ARGUMENT;
+  return CCE_OK;
+}
+
+static cce_status orpo_common(const float* logp, const int32_t* labels, int64_t M,
+                              const cce_layout* layout, double lambda, int scope,
+                              double* out8, float* coeff, void* ws, size_t ws_bytes,
+                              cce_stream_t stream) {
+  if (logp == nullptr || labels == nullptr || ws == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  if (M <= 0 || M > (int64_t(1) << 31)) return CCE_ERR_INVALID_ARGUMENT;
+  if (!(lambda >= 0.0) || lambda > 1e30) return CCE_ERR_INVALID_ARGUMENT;
+  if (scope != CCE_SCOPE_FULL && scope != CCE_SCOPE_RESPONSE) return CCE_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < kStatusBytes || !aligned16(ws)) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  cce_status s = check_layout(layout, M);
+  if (s != CCE_OK) return s;
+  OrpoArgs o;
+  o.pb = layout->prompt_begin;
+  o.pe = layout->prompt_end;
+  o.cb = layout->chosen_begin;
+  o.ce = layout->chosen_end;
+  o.rb = layout->rejected_begin;
+  o.re = layout->rejected_end;
+  o.lambda = lambda;
+  o.scope = scope;
+  o.want_coeff = coeff != nullptr;
+  orpo_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      logp, labels, M, o, out8, coeff, status_word(ws));
+  return launch_ok();
+}
+
+cce_status orpo_loss_from_logps(const float* logp, const int32_t* labels, int64_t M,
+                                const cce_layout* layout, double lambda, int sft_scope,
+                                double* out8, void* ws, size_t ws_bytes,
+                                cce_stream_t stream) {
+  if (out8 == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  return orpo_common(logp, labels, M, layout, lambda, sft_scope, out8, nullptr, ws,
+                     ws_bytes, stream);
+}
+
+cce_status orpo_grad_coeffs(const float* logp, const int32_t* labels, int64_t M,
+                            const cce_layout* layout, double lambda, int sft_scope,
+                            float* coeff, void* ws, size_t ws_bytes, cce_stream_t stream) {
+  if (coeff == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  return orpo_common(logp, labels, M, layout, lambda, sft_scope, nullptr, coeff, ws,
+                     ws_bytes, stream);
+}
+
+cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
+                           const int32_t* labels, const float* lse, const float* coeff,
+                           float filter_eps, const float* blockmax, float* dH,
+                           unsigned long long* skip_stats, void* ws, size_t ws_bytes,
+                           cce_stream_t stream) {
+  if (H == nullptr || labels == nullptr || lse == nullptr || coeff == nullptr ||
+      dH == nullptr || ws == nullptr)
+    return CCE_ERR_INVALID_ARGUMENT;
+  if (M <= 0 || M > (int64_t(1) << 30)) return CCE_ERR_INVALID_ARGUMENT;
+  if (h_dtype != CCE_F32 && h_dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
+  if (!(filter_eps >= 0.f) || filter_eps > 1.f) return CCE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(H) || !aligned16(ws) || !aligned16(dH)) return CCE_ERR_INVALID_ARGUMENT;
+  cce_status s = check_head(W, h_dtype);
+  if (s != CCE_OK) return s;
+  const int64_t vc = fit_vc(M, h_dtype, W, ws_bytes);
+  if (vc == 0) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  const Layout L = make_layout(M, h_dtype, W, vc);
+  int sms = 0;
+  if ((s = device_info(&sms)) != CCE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* wsc = static_cast<char*>(ws);
+
+  Operands op;
+  if ((s = prepare_operands(H, h_dtype, M, W, L, ws, st, &op)) != CCE_OK) return s;
+  const int64_t V = W->V, D = W->D;
+  const int64_t cols = ceil_div(V, BN);
+  const int64_t n_rt = ceil_div(M, BM);
+  const int64_t n_dt = ceil_div(D, BN);
+  uint16_t* g = reinterpret_cast<uint16_t*>(wsc + L.g);
+  uint8_t* tile_skip = reinterpret_cast<uint8_t*>(wsc + L.tile_skip);
+  uint8_t* row_skip = reinterpret_cast<uint8_t*>(wsc + L.row_skip);
+
+  // Plan: rows whose coefficient is 0 everywhere in a tile, and (with the
+  // filter and blockmax) vocab blocks the filter would empty.
+  {
+    const int64_t units = n_rt * cols;
+    const int wpb = 8;
+    skip_plan_kernel<<<int(ceil_div(units, wpb)), wpb * 32, 0, st>>>(
+        filter_eps > 0.f ? blockmax : nullptr, lse, labels, coeff, int(M), int(cols),
+        int(n_rt), filter_eps, tile_skip, row_skip, skip_stats);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+
+  CUtensorMap ma, mb, mg, mw;
+  if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM) ||
+      !make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN) ||
+      !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK))
+    return CCE_ERR_CUDA;
+
+  TileArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = int(M);
+  a.n_rt = int(n_rt);
+  a.V = int(V);
+  a.D = int(D);
+  a.fmt = op.bf16 ? 1 : 0;
+  a.wait_ns = g_wait_ns.load();
+  a.status = status_word(ws);
+  a.labels = labels;
+  a.lse = lse;
+  a.filter_eps = filter_eps;
+  a.g_out = g;
+  a.g_ld = int(vc);
+  a.tile_skip = tile_skip;
+  a.skip_ld = int(cols);
+  a.row_skip = row_skip;
+  a.coeff = coeff;
+  a.dh = dH;
+
+  for (int64_t v0 = 0; v0 < V; v0 += vc) {
+    const int64_t w = std::min<int64_t>(vc, V - v0);
+    const int64_t ct_n = ceil_div(w, BN);
+    // G' = onehot - softmax for this chunk
+    TileArgs ag = a;
+    ag.n_ct = int(ct_n);
+    ag.nk = int(op.k / BK);
+    ag.npass = 1;
+    ag.b_row0 = int(v0);
+    ag.ct_off = int(v0 / BN);
+    cce_tc_kernel<Mode::kGrad><<<grid_for(n_rt * ct_n, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+        ma, mb, ag);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    // dH (+)= coeff * G' . W[chunk]
+    if (!make_map(&mg, g, op.bf16, ct_n * BN, M, vc, BK, BM)) return CCE_ERR_CUDA;
+    TileArgs ad = a;
+    ad.n_ct = int(n_dt);
+    ad.nk = int(ct_n * BN / BK);
+    ad.npass = op.npass_dh;
+    ad.b_pass_off = int(op.d_pass_off);
+    ad.b_row0 = int(v0);
+    ad.first_chunk = v0 == 0 ? 1 : 0;
+    cce_tc_kernel<Mode::kDh><<<grid_for(n_rt * n_dt, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+        mg, mw, ad);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+  return CCE_OK;
+}
+
+cce_status cce_device_status(void* ws, cce_stream_t stream) {
+  if (ws == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return CCE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return CCE_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return CCE_ERR_CUDA;
+  }
+  if (word & ST_LABEL) return CCE_ERR_LABEL_OUT_OF_RANGE;
+  if (word & ST_TIMEOUT) return CCE_ERR_DEVICE_TIMEOUT;
+  if (word & ST_EMPTY) return CCE_ERR_EMPTY_SEGMENT;
+  if (word & ST_DOMAIN) return CCE_ERR_DOMAIN;
+  return CCE_OK;
+}
+
+cce_status cce_selftest_wait_timeout(void* ws, size_t ws_bytes, cce_stream_t stream) {
+  if (ws == nullptr || ws_bytes < kStatusBytes || !aligned16(ws)) return CCE_ERR_INVALID_ARGUMENT;
+  selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      status_word(ws), g_wait_ns.load());
+  return launch_ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,218 @@
+"""GPU parity of the C-ABI library against the float64 oracle on small,
+ragged shapes (several tiles plus tails), the integer-exact indexing design,
+the ORPO epilogue, device-side error reporting and the timeout path."""
+
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_cross_flash_b200 import cce
+from lm_head_cross_flash_b200 import synthetic as S
+from oracle import flash_cce as O
+
+from helpers import TOL_DH, TOL_LOGP, TOL_LOSS, oracle_W, rel_fro, run_pass, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _forward(wl):
+    H, head, labels = upload(wl)
+    hd = cce.h_dtype(H)
+    ws = cce.alloc_workspace(wl.M, hd, head)
+    f = dict(device="cuda", dtype=torch.float32)
+    logp, lse, tgt = torch.empty(wl.M, **f), torch.empty(wl.M, **f), torch.zeros(wl.M, **f)
+    bm = torch.empty(cce.blockmax_cols(wl.V), wl.M, **f)
+    cce.cce_forward(H, head, labels, logp, lse, tgt, bm, ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0
+    return (H, head, labels, ws), logp.cpu().numpy(), lse.cpu().numpy(), tgt.cpu().numpy(), bm.cpu().numpy()
+
+
+SMALL = [
+    # (cfg recipe, (P, Rc, Rr), D, V)
+    (1, (1, 1, 1), 64, 31),
+    (1, (3, 2, 2), 64, 1),
+    (1, (40, 44, 44), 128, 256),
+    (1, (40, 45, 44), 64, 257),
+    (2, (100, 150, 131), 256, 4097),
+    (1, (64, 200, 300), 192, 1000),
+    (0, (8, 60, 60), 64, 300),
+    (0, (32, 96, 128), 256, 4096),
+]
+
+
+@pytest.mark.parametrize("cfg,split,D,V", SMALL)
+def test_forward_matches_oracle(cfg, split, D, V):
+    wl = S.make_custom(cfg, M_split=split, D=D, V=V)
+    _, logp, lse, tgt, bm = _forward(wl)
+    ologp, olse, otgt = O.head_forward(wl.H, oracle_W(wl), wl.labels)
+    assert np.max(np.abs(lse - olse)) <= TOL_LOGP
+    assert np.max(np.abs(logp - ologp)) <= TOL_LOGP
+    ok = wl.labels >= 0
+    assert np.all(logp[~ok] == 0.0)
+    assert np.max(np.abs(tgt[ok] - otgt[ok])) <= TOL_LOGP
+    # blockmax: max logit per 256-wide vocab block
+    Z = wl.H.astype(np.float64) @ oracle_W(wl).T
+    nb = cce.blockmax_cols(V)
+    want = np.stack([Z[:, b * 256:(b + 1) * 256].max(axis=1) for b in range(nb)])
+    assert np.max(np.abs(bm - want)) <= TOL_LOGP
+
+
+def test_integer_design_is_bit_exact():
+    """Small-integer H and W are exact in bf16 and their dot products exact in
+    fp32, so the gathered target logit must equal the integer exactly, for
+    labels in every tile including the tail and the tile edges."""
+    P, Rc, Rr, D, V = 50, 60, 70, 128, 1100
+    M = P + Rc + Rr
+    g = np.random.default_rng(5)
+    H = g.integers(-3, 4, size=(M, D)).astype(np.float32)
+    W = g.integers(-2, 3, size=(V, D)).astype(np.float32)
+    labels = g.integers(0, V, size=M).astype(np.int32)
+    edge = [0, 255, 256, 511, 512, 1023, 1024, 1099]
+    labels[1:1 + len(edge)] = edge
+    labels[0] = -1
+    labels[17] = -5
+    wl = S.make_custom(1, M_split=(P, Rc, Rr), D=D, V=V)
+    wl.H, wl.W, wl.labels = H, W, labels
+    wl.H_bits, wl.W_bits = S.f32_to_bf16_bits(H), S.f32_to_bf16_bits(W)
+    _, logp, lse, tgt, _ = _forward(wl)
+    exact = (H.astype(np.int64) @ W.astype(np.int64).T)
+    ok = labels >= 0
+    want = exact[np.nonzero(ok)[0], labels[ok]].astype(np.float32)
+    assert np.array_equal(tgt[ok], want)
+    assert np.all(logp[~ok] == 0.0)
+
+
+@pytest.mark.parametrize("cfg,split,D,V", [(1, (40, 45, 44), 64, 257),
+                                           (2, (100, 150, 131), 256, 4097),
+                                           (0, (8, 60, 60), 64, 300)])
+def test_backward_random_cotangent(cfg, split, D, V):
+    """dH with a non-uniform cotangent (rows with zero cotangent stay 0)."""
+    wl = S.make_custom(cfg, M_split=split, D=D, V=V)
+    (H, head, labels, ws), logp, lse, _, bm = _forward(wl)
+    g = S.random_cotangent(wl)
+    g[5:9] = 0.0
+    coeff = torch.from_numpy(g).cuda()
+    dH = torch.full((wl.M, wl.D), float("nan"), device="cuda")
+    lse_t = torch.from_numpy(lse).cuda()
+    cce.cce_backward_dh(H, head, labels, lse_t, coeff, 0.0, None, dH, None, ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0
+    dH = dH.cpu().numpy()
+    want = O.head_dh(wl.H, oracle_W(wl), wl.labels, g, O.head_forward(wl.H, oracle_W(wl), wl.labels)[1])
+    assert rel_fro(dH, want) <= TOL_DH, rel_fro(dH, want)
+    assert np.all(dH[wl.labels < 0] == 0.0)
+    assert np.all(dH[5:9] == 0.0)
+
+
+def test_backward_narrow_workspace_chunks():
+    """A workspace that only fits a 256-wide vocab chunk gives the same dH."""
+    wl = S.make_custom(2, M_split=(60, 70, 80), D=128, V=1500)
+    (H, head, labels, ws), logp, lse, _, _ = _forward(wl)
+    g = torch.from_numpy(S.random_cotangent(wl)).cuda()
+    lse_t = torch.from_numpy(lse).cuda()
+    d1 = torch.empty(wl.M, wl.D, device="cuda")
+    cce.cce_backward_dh(H, head, labels, lse_t, g, 0.0, None, d1, None, ws)
+    small = cce.alloc_workspace(wl.M, cce.h_dtype(H), head,
+                                nbytes=cce.workspace_min_bytes(wl.M, cce.h_dtype(H), head))
+    d2 = torch.empty(wl.M, wl.D, device="cuda")
+    cce.cce_backward_dh(H, head, labels, lse_t, g, 0.0, None, d2, None, small)
+    torch.cuda.synchronize()
+    assert rel_fro(d2.cpu().numpy(), d1.cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("scope", ["full", "response"])
+def test_full_pass_small(scope):
+    wl = S.make_custom(0, M_split=(32, 96, 128), D=256, V=4096)
+    wl.scope = scope
+    _, _, _, buf, st = run_pass(wl)
+    assert st == 0
+    W = oracle_W(wl)
+    L = O.Layout(*wl.layout_tuple)
+    ologp, olse, _ = O.head_forward(wl.H, W, wl.labels)
+    o = O.orpo_loss_from_logps(ologp, wl.labels, L, wl.lam, scope)
+    g = O.orpo_grad_coeffs(ologp, wl.labels, L, wl.lam, scope)
+    odh = O.head_dh(wl.H, W, wl.labels, g, olse)
+    assert np.max(np.abs(buf.logp.cpu().numpy() - ologp)) <= TOL_LOGP
+    assert np.max(np.abs(buf.lse.cpu().numpy() - olse)) <= TOL_LOGP
+    out8 = buf.out8.cpu().numpy()
+    assert abs(out8[0] - o.loss) <= TOL_LOSS * abs(o.loss)
+    assert rel_fro(buf.coeff.cpu().numpy(), g) <= 1e-5
+    assert rel_fro(buf.dH.cpu().numpy(), odh) <= TOL_DH
+
+
+def test_orpo_epilogue_matches_oracle_at_full_size():
+    """The ORPO epilogue on seeded log-probs of the long-pair shape."""
+    P, Rc, Rr = 1024, 3584, 3584
+    M = P + Rc + Rr
+    lp = S.random_logps(M, seed=3)
+    y = np.random.default_rng(4).integers(-1, 1000, size=M).astype(np.int32)
+    y[0] = -1
+    L = O.Layout.contiguous(P, Rc, Rr)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    out8 = torch.empty(8, dtype=torch.float64, device="cuda")
+    coeff = torch.empty(M, device="cuda")
+    lpt, yt = torch.from_numpy(lp).cuda(), torch.from_numpy(y).cuda()
+    for scope in ("full", "response"):
+        for lam in (0.0, 0.1, 1.0):
+            cce.orpo_loss_from_logps(lpt, yt, dataclasses.astuple(L), lam, scope, out8, ws)
+            cce.orpo_grad_coeffs(lpt, yt, dataclasses.astuple(L), lam, scope, coeff, ws)
+            torch.cuda.synchronize()
+            assert cce.cce_device_status(ws) == 0
+            o = O.orpo_loss_from_logps(lp, y, L, lam, scope)
+            got = out8.cpu().numpy()
+            want = np.array(o.as8())
+            assert np.allclose(got, want, rtol=1e-12, atol=1e-14), (got, want)
+            g = O.orpo_grad_coeffs(lp, y, L, lam, scope)
+            assert np.allclose(coeff.cpu().numpy(), g, rtol=1e-6, atol=1e-12)
+
+
+def test_device_errors_are_reported_not_trapped():
+    wl = S.make_custom(1, M_split=(4, 4, 4), D=64, V=100)
+    wl.labels[3] = 100  # == V
+    H, head, labels = upload(wl)
+    ws = cce.alloc_workspace(wl.M, cce.h_dtype(H), head)
+    f = dict(device="cuda", dtype=torch.float32)
+    logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+    cce.cce_forward(H, head, labels, logp, lse, None, None, ws)
+    assert cce.cce_device_status(ws) == 5          # label out of range
+    assert cce.cce_device_status(ws) == 0          # cleared
+    # empty rejected segment: every rejected row ignored
+    y = labels.clone()
+    y[8:] = -1
+    out8 = torch.empty(8, dtype=torch.float64, device="cuda")
+    cce.orpo_loss_from_logps(logp, y, wl.layout_tuple, 0.1, "full", out8, ws)
+    assert cce.cce_device_status(ws) == 7
+    assert torch.isnan(out8).all()
+    # the context is still usable
+    cce.cce_forward(H, head, labels.clamp(max=99), logp, lse, None, None, ws)
+    assert cce.cce_device_status(ws) == 0
+
+
+def test_timeout_path_reports_and_recovers():
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    cce.cce_set_wait_limit_ns(2_000_000)  # 2 ms
+    try:
+        cce.cce_selftest_wait_timeout(ws)
+        assert cce.cce_device_status(ws) == 6
+    finally:
+        cce.cce_set_wait_limit_ns(0)
+    assert cce.cce_device_status(ws) == 0
+
+
+def test_synchronous_argument_errors():
+    wl = S.make_custom(1, M_split=(4, 4, 4), D=64, V=100)
+    H, head, labels = upload(wl)
+    ws = cce.alloc_workspace(wl.M, cce.h_dtype(H), head)
+    f = dict(device="cuda", dtype=torch.float32)
+    logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+    with pytest.raises(cce.CCEError) as e:
+        cce.cce_forward(H, head, labels, logp, lse, None, None, ws[:1024])
+    assert e.value.status == 4
+    bad = cce.Head(w=head.w, V=wl.V, D=96)
+    with pytest.raises(cce.CCEError) as e:
+        cce.cce_forward(H, bad, labels, logp, lse, None, None, ws)
+    assert e.value.status == 2
