@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the flash-CCE ORPO head on B200.
+
+One step = one pass of the whole head on one ORPO pair of the long-pair
+workload (M = 8,192 head rows, D = 2,048, V = 262,144, bf16): forward GEMM
+with the online-LSE epilogue, LSE merge, ORPO loss, cotangent, and the
+backward (recompute, G', dH contraction).  Inputs are seeded synthetic
+arrays with that shape and a random-initialised head.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 the script runs under torchrun: every rank processes its own pair
+on its own GPU (independent problems, no data-path collective; weak
+scaling); timing is the max over ranks.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the float64 CPU oracle (the only reference this
+head has) on a bounded sample of rows per step, on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "flash-CCE fwd+bwd tokens/sec and % of bf16 tensor peak at M=8192,V=262144"
+WORKLOAD_ID = 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", type=int, default=WORKLOAD_ID)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers --
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "lm_head_cross_flash_b200", "csrc")
+    for n in sorted(os.listdir(src)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(src, n), "rb") as f:
+                h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kind: str, workload: str):
+    """Per-launch DRAM bytes of `kind` from the committed ncu summary, if it
+    was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kind)
+    if not e or e.get("src_hash") != source_hash() or e.get("workload") != workload:
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples of one GPU while it runs."""
+
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.5)
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                c, m, pw = float(f[1]), float(f[2]), float(f[3])
+            except ValueError:
+                continue
+            mx = max(mx, m)
+            if pw < 250.0:  # idle samples before the GPU ramps up
+                continue
+            sm.append(c)
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(dev) -> str:
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # pragma: no cover
+        return str(dev)
+
+
+def aggregate(dist, local_ms: float, local_tokens: float, device=None):
+    """Max step time and summed tokens over ranks (identity when not
+    distributed)."""
+    if dist is None or not dist.is_initialized():
+        return local_ms, local_tokens
+    import torch
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    n = torch.tensor([local_tokens], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_rows(wl, W64, rows, g):
+    """The oracle's per-row work of one head pass (forward and dH) on `rows`."""
+    from oracle import flash_cce as O
+    logp, lse, _ = O.head_forward(wl.H[rows], W64, wl.labels[rows], block=len(rows))
+    O.head_dh(wl.H[rows], W64, wl.labels[rows], g[rows], lse, block=len(rows))
+    return logp
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, seconds: float, rows_per_block: int = 8):
+    """Oracle throughput (rows/s) on a time-bounded sample of rows."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from lm_head_cross_flash_b200 import synthetic as S
+    cores = cpu_threads()
+    W64 = wl.W.astype(np.float64)
+    g = S.random_cotangent(wl).astype(np.float64)
+    order = np.random.default_rng(0).permutation(wl.M)
+    done, t0 = 0, time.perf_counter()
+    with threadpool_limits(limits=cores):
+        while time.perf_counter() - t0 < seconds and done < wl.M:
+            rows = np.sort(order[done:done + rows_per_block])
+            oracle_rows(wl, W64, rows, g)
+            done += len(rows)
+    dt = time.perf_counter() - t0
+    return done / dt, cores, done, dt
+
+
+# -------------------------------------------------------------- our arm --
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from lm_head_cross_flash_b200 import cce
+    from lm_head_cross_flash_b200 import synthetic as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    wl = S.make_workload(args.workload)
+    if wl.dtype == "bf16":
+        H = torch.from_numpy(wl.H_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        head = cce.Head(w=torch.from_numpy(wl.W_bits.view(np.int16)).to(dev).view(torch.bfloat16),
+                        V=wl.V, D=wl.D)
+    else:
+        H = torch.from_numpy(wl.H).to(dev)
+        head = cce.Head(w=torch.from_numpy(wl.W).to(dev), V=wl.V, D=wl.D)
+    labels = torch.from_numpy(wl.labels).to(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_alloc = torch.cuda.memory_allocated(dev)
+    free0, _ = torch.cuda.mem_get_info(dev)
+    buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cce.orpo_head_pass(H, head, labels, wl.layout_tuple, wl.lam, wl.scope, wl.filter_eps,
+                           wl.block_skip, buf, stream)
+
+    sampler = ClockSampler(gpu_uuid(dev))
+    sampler.start()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    st = cce.cce_device_status(buf.ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    cce.cce_profile_enable(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    prof = cce.cce_profile_read()
+    cce.cce_profile_enable(False)
+    sampler.stop()
+    peak_mem = torch.cuda.max_memory_allocated(dev) - base_alloc
+    free1, _ = torch.cuda.mem_get_info(dev)
+    st = cce.cce_device_status(buf.ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+
+    ms_max, tokens = aggregate(dist if world > 1 else None, ms_total, float(wl.M * args.steps), dev)
+    ms_step = ms_max / args.steps
+
+    # end to end through the public API: host H and labels in, dH and loss out
+    e2e = None
+    if not args.no_e2e:
+        hH = (torch.from_numpy(wl.H_bits.view(np.int16)).view(torch.bfloat16)
+              if wl.dtype == "bf16" else torch.from_numpy(wl.H)).pin_memory()
+        hy = torch.from_numpy(wl.labels).pin_memory()
+        hdH = torch.empty(wl.M, wl.D, dtype=torch.float32).pin_memory()
+        hout = torch.empty(8, dtype=torch.float64).pin_memory()
+        Hd = torch.empty_like(H)
+        yd = torch.empty_like(labels)
+
+        def e2e_step():
+            Hd.copy_(hH, non_blocking=True)
+            yd.copy_(hy, non_blocking=True)
+            cce.orpo_head_pass(Hd, head, yd, wl.layout_tuple, wl.lam, wl.scope, wl.filter_eps,
+                               wl.block_skip, buf, stream)
+            hdH.copy_(buf.dH, non_blocking=True)
+            hout.copy_(buf.out8, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e_ms, e_tok = aggregate(dist if world > 1 else None, e0.elapsed_time(e1),
+                                float(wl.M * args.steps), dev)
+        if not np.isfinite(hout.numpy()[0]):
+            raise RuntimeError("non-finite loss in the end-to-end pass")
+        e2e = {"value": e_tok / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(hH.numel() * hH.element_size() + hy.numel() * 4),
+               "d2h_bytes_per_step": int(hdH.numel() * 4 + hout.numel() * 8)}
+
+    clk = sampler.summary()
+    if world > 1:
+        allc = [None] * world
+        dist.all_gather_object(allc, clk)
+        meds = [c["sm_mhz"] for c in allc if c["sm_mhz"]]
+        clk = {"sm_mhz": min(meds) if meds else None,
+               "sm_max_mhz": max((c["sm_max_mhz"] or 0) for c in allc) or None,
+               "reasons": sorted(set(r for c in allc for r in c["reasons"])),
+               "samples": sum(c["samples"] for c in allc)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rps, cores, rows, dt = time_oracle(wl, args.cpu_seconds)
+        cpu = {"value": rps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} rows of the {wl.name} workload (forward logp/lse and dH per "
+                         f"row, float64, logits materialised per row block) in {dt:.1f} s"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peaks_src = load_peaks()
+    flop_step = 6.0 * wl.M * wl.V * wl.D
+    tflops = flop_step / (ms_step / 1e3) / 1e12
+    # roofline of the dominant kernel kind (largest summed time)
+    per_kind_flops = {"fwd_lse_gemm": 2.0 * wl.M * wl.V * wl.D,
+                      "bwd_grad_gemm": 2.0 * wl.M * wl.V * wl.D,
+                      "bwd_dh_gemm": 2.0 * wl.M * wl.V * wl.D}
+    kinds = {k: v for k, v in prof.items() if v[1] > 0}
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    dom_ms, dom_n = kinds[dom]
+    launches_per_step = dom_n / args.steps
+    peak_s = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if dom in per_kind_flops:
+        achieved = per_kind_flops[dom] * args.steps / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_s,
+                "unit": "TFLOP/s", "frac": achieved / peak_s,
+                "traffic": load_traffic(dom, wl.name),
+                "launches_per_step": launches_per_step,
+                "avg_launch_ms": dom_ms / dom_n,
+                "flops_per_launch": per_kind_flops[dom] / launches_per_step,
+                "peak_source": f"{peaks_src} bf16 sustained (MEASURED_PEAKS.json)"}
+    else:  # pragma: no cover
+        roof = {"bound": "hbm", "kernel": dom, "achieved": None, "peak": peaks.get("hbm_gbs"),
+                "unit": "GB/s", "frac": None, "traffic": None}
+    gpu_launches = int(sum(v[1] for v in kinds.values()))
+    out = {
+        "metric": METRIC,
+        "value": tokens / (ms_max / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic: seeded inputs of the workload recipe, random-init head",
+        "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "V": wl.V, "P": wl.P,
+                   "Rc": wl.Rc, "Rr": wl.Rr, "sft_scope": wl.scope, "lambda": wl.lam,
+                   "filter_eps": wl.filter_eps, "block_skip": wl.block_skip,
+                   "parallelism": f"dp{world} (independent pairs, no collective)",
+                   "l2": "inputs larger than L2 (W is 1.07 GB, L2 126 MB); no flush"},
+        "tflops": tflops,
+        "pct_bf16_peak": {"sustained": 100.0 * tflops / peak_s,
+                          "burst": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+                          "source": peaks_src},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": gpu_launches,
+        "clocks": clk,
+        "kernels_ms_per_step": {k: v[0] / args.steps for k, v in kinds.items()},
+        "kernel_launches_per_step": {k: v[1] / args.steps for k, v in kinds.items()},
+        "peak_mem_bytes": int(peak_mem),
+        "mem_get_info_delta_bytes": int(free0 - free1),
+        "logits_bytes_avoided": int(wl.M) * int(wl.V) * 4,
+        "skip_tiles": buf.skip.cpu().tolist(),
+    }
+    return out
+
+
+# -------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from lm_head_cross_flash_b200 import synthetic as S
+    wl = S.make_workload(args.workload)
+    W64 = wl.W.astype(np.float64)
+    g = S.random_cotangent(wl).astype(np.float64)
+    cores = cpu_threads()
+    rows_per_step = 4
+    order = np.random.default_rng(1).permutation(wl.M)
+    with threadpool_limits(limits=cores):
+        for i in range(max(3, args.warmup)):
+            oracle_rows(wl, W64, np.sort(order[:rows_per_step]), g)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            r = np.sort(order[(i * rows_per_step) % wl.M:][:rows_per_step])
+            oracle_rows(wl, W64, r, g)
+        dt = time.perf_counter() - t0
+    value = rows_per_step * args.steps / dt
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: seeded inputs of the workload recipe, random-init head",
+        "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "V": wl.V,
+                   "sample_rows_per_step": rows_per_step},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows_per_step} rows per step of the {wl.name} workload "
+                                   "(forward logp/lse and dH per row, float64)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

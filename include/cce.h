@@ -202,6 +202,20 @@ void cce_set_wait_limit_ns(uint64_t ns);
 cce_status cce_selftest_wait_timeout(void* ws, size_t ws_bytes,
                                      cce_stream_t stream);
 
+
+/* Optional per-kernel timing for benchmarks.  While enabled, every kernel the
+ * library launches is bracketed by a pair of CUDA events recorded on its own
+ * launch stream.  cce_profile_enable(1) starts (and clears) a recording,
+ * cce_profile_enable(0) stops it.  cce_profile_read() waits for the recorded
+ * events, writes per kernel kind the summed milliseconds and the number of
+ * launches into ms[0..n) and launches[0..n) (host arrays, either may be
+ * NULL), clears the records and returns the number of kinds.
+ * cce_profile_kind_name() names a kind.  Process-wide; not for concurrent
+ * use from several host threads. */
+void cce_profile_enable(int on);
+int cce_profile_read(double* ms, long long* launches, int n);
+const char* cce_profile_kind_name(int kind);
+
 #ifdef __cplusplus
 }
 #endif

@@ -75,7 +75,26 @@ _SIGS = {
     "cce_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "cce_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "cce_profile_enable": (None, [ctypes.c_int]),
+    "cce_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
+                                        ctypes.POINTER(ctypes.c_longlong), ctypes.c_int]),
+    "cce_profile_kind_name": (ctypes.c_char_p, [ctypes.c_int]),
 }
+
+PROFILE_KINDS = 8
+
+
+def cce_profile_enable(on: bool):
+    lib().cce_profile_enable(1 if on else 0)
+
+
+def cce_profile_read() -> dict:
+    """{kind name: (total ms, launches)} of the kernels recorded since
+    ``cce_profile_enable(True)``; clears the records."""
+    ms = (ctypes.c_double * PROFILE_KINDS)()
+    n = (ctypes.c_longlong * PROFILE_KINDS)()
+    k = lib().cce_profile_read(ms, n, PROFILE_KINDS)
+    return {lib().cce_profile_kind_name(i).decode(): (ms[i], n[i]) for i in range(k)}
 
 
 def lib():

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/cce.h"
 #include "aux_kernels.cuh"
@@ -68,6 +69,58 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+
+// -------------------------------------------------------------- profiler --
+// Optional per-kernel timing: while enabled, every kernel launch is
+// bracketed by a CUDA event pair recorded on its own stream.
+enum ProfKind {
+  PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_N
+};
+const char* const kProfNames[PK_N] = {"split_f32",     "fwd_lse_gemm", "lse_merge",
+                                      "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
+                                      "bwd_dh_gemm",   "selftest"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_ev_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_ev_pool.empty()) {
+    cudaEvent_t e = g_ev_pool.back();
+    g_ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+class ProfScope {
+ public:
+  ProfScope(int kind, cudaStream_t st) : kind_(kind), st_(st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_on) return;
+    a_ = pool_event();
+    b_ = pool_event();
+    if (a_ != nullptr && b_ != nullptr) cudaEventRecord(a_, st_);
+  }
+  ~ProfScope() {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (a_ == nullptr || b_ == nullptr) return;
+    cudaEventRecord(b_, st_);
+    g_prof.push_back({kind_, a_, b_});
+  }
+
+ private:
+  int kind_;
+  cudaStream_t st_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
 
 // --------------------------------------------------------- device facts --
 struct DevInfo {
@@ -211,8 +264,11 @@ cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_hea
   // fp32: three-part bf16 split, K = 3D.
   auto* hs = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + L.hs);
   auto* wsb = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + L.ws);
-  split_f32_kernel<<<1184, 256, 0, st>>>(static_cast<const float*>(H), M, int(D), 0, hs);
-  split_f32_kernel<<<1184, 256, 0, st>>>(static_cast<const float*>(W->w), W->V, int(D), 1, wsb);
+  {
+    ProfScope ps(PK_SPLIT, st);
+    split_f32_kernel<<<1184, 256, 0, st>>>(static_cast<const float*>(H), M, int(D), 0, hs);
+    split_f32_kernel<<<1184, 256, 0, st>>>(static_cast<const float*>(W->w), W->V, int(D), 1, wsb);
+  }
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   op->a = hs;
   op->b = wsb;
@@ -308,12 +364,18 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.part_s = part_s;
   a.tgt = tgt;
   a.ct_off = 0;
-  cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a);
+  {
+    ProfScope ps(PK_LSE, st);
+    cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a);
+  }
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
 
   const int rows_per_block = 8;
-  merge_lse_kernel<<<int(ceil_div(M, rows_per_block)), rows_per_block * 32, 0, st>>>(
-      part_m, part_s, int(cols), int(M), labels, int(V), tgt, logp, lse, status_word(ws));
+  {
+    ProfScope ps(PK_MERGE, st);
+    merge_lse_kernel<<<int(ceil_div(M, rows_per_block)), rows_per_block * 32, 0, st>>>(
+        part_m, part_s, int(cols), int(M), labels, int(V), tgt, logp, lse, status_word(ws));
+  }
   return launch_ok();
 }
 
@@ -352,8 +414,11 @@ static cce_status orpo_common(const float* logp, const int32_t* labels, int64_t 
   o.lambda = lambda;
   o.scope = scope;
   o.want_coeff = coeff != nullptr;
-  orpo_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      logp, labels, M, o, out8, coeff, status_word(ws));
+  {
+    ProfScope ps(PK_ORPO, reinterpret_cast<cudaStream_t>(stream));
+    orpo_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        logp, labels, M, o, out8, coeff, status_word(ws));
+  }
   return launch_ok();
 }
 
@@ -411,6 +476,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   {
     const int64_t units = n_rt * cols;
     const int wpb = 8;
+    ProfScope ps(PK_SKIP, st);
     skip_plan_kernel<<<int(ceil_div(units, wpb)), wpb * 32, 0, st>>>(
         filter_eps > 0.f ? blockmax : nullptr, lse, labels, coeff, int(M), int(cols),
         int(n_rt), filter_eps, tile_skip, row_skip, skip_stats);
@@ -453,8 +519,11 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ag.npass = 1;
     ag.b_row0 = int(v0);
     ag.ct_off = int(v0 / BN);
-    cce_tc_kernel<Mode::kGrad><<<grid_for(n_rt * ct_n, sms), NUM_THREADS, SMEM_BYTES, st>>>(
-        ma, mb, ag);
+    {
+      ProfScope ps(PK_GRAD, st);
+      cce_tc_kernel<Mode::kGrad><<<grid_for(n_rt * ct_n, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+          ma, mb, ag);
+    }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     // dH (+)= coeff * G' . W[chunk]
     if (!make_map(&mg, g, op.bf16, ct_n * BN, M, vc, BK, BM)) return CCE_ERR_CUDA;
@@ -465,11 +534,49 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ad.b_pass_off = int(op.d_pass_off);
     ad.b_row0 = int(v0);
     ad.first_chunk = v0 == 0 ? 1 : 0;
-    cce_tc_kernel<Mode::kDh><<<grid_for(n_rt * n_dt, sms), NUM_THREADS, SMEM_BYTES, st>>>(
-        mg, mw, ad);
+    {
+      ProfScope ps(PK_DH, st);
+      cce_tc_kernel<Mode::kDh><<<grid_for(n_rt * n_dt, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+          mg, mw, ad);
+    }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
   return CCE_OK;
+}
+
+
+void cce_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    g_ev_pool.push_back(r.a);
+    g_ev_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  g_prof_on = on != 0;
+}
+
+int cce_profile_read(double* ms, long long* launches, int n) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int k = 0; k < n && k < PK_N; ++k) {
+    if (ms != nullptr) ms[k] = 0.0;
+    if (launches != nullptr) launches[k] = 0;
+  }
+  for (auto& r : g_prof) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess &&
+        cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess && r.kind < n) {
+      if (ms != nullptr) ms[r.kind] += t;
+      if (launches != nullptr) launches[r.kind] += (r.kind == PK_SPLIT) ? 2 : 1;
+    }
+    g_ev_pool.push_back(r.a);
+    g_ev_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  return PK_N;
+}
+
+const char* cce_profile_kind_name(int kind) {
+  return (kind >= 0 && kind < PK_N) ? kProfNames[kind] : "unknown";
 }
 
 cce_status cce_device_status(void* ws, cce_stream_t stream) {
@@ -493,6 +600,7 @@ cce_status cce_device_status(void* ws, cce_stream_t stream) {
 
 cce_status cce_selftest_wait_timeout(void* ws, size_t ws_bytes, cce_stream_t stream) {
   if (ws == nullptr || ws_bytes < kStatusBytes || !aligned16(ws)) return CCE_ERR_INVALID_ARGUMENT;
+  ProfScope ps(PK_SELFTEST, reinterpret_cast<cudaStream_t>(stream));
   selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       status_word(ws), g_wait_ns.load());
   return launch_ok();

@@ -1,0 +1,82 @@
+"""GPU parity at the full workload sizes.
+
+* tiny fp32 pair and small bf16 pair: the whole pass (logp, lse, loss,
+  cotangent, dH) against the oracle on every row;
+* long bf16 pairs: logp / lse on stratified sampled rows, and dH on sampled
+  rows for a seeded non-uniform cotangent (the oracle cannot afford every
+  row); the filtered + block-skipped backward is compared with the
+  unfiltered oracle, and block skipping must not change a single bit of dH.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_cross_flash_b200 import cce
+from lm_head_cross_flash_b200 import synthetic as S
+from oracle import flash_cce as O
+
+from helpers import TOL_DH, TOL_LOGP, TOL_LOSS, oracle_W, oracle_layout, rel_fro, run_pass, upload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_full_pass_every_row(cfg):
+    wl = S.make_workload(cfg)
+    _, _, _, buf, st = run_pass(wl)
+    assert st == 0
+    W = oracle_W(wl)
+    L = oracle_layout(wl)
+    logp, lse, _ = O.head_forward(wl.H, W, wl.labels)
+    o = O.orpo_loss_from_logps(logp, wl.labels, L, wl.lam, wl.scope)
+    g = O.orpo_grad_coeffs(logp, wl.labels, L, wl.lam, wl.scope)
+    dH = O.head_dh(wl.H, W, wl.labels, g, lse)
+    assert np.max(np.abs(buf.logp.cpu().numpy() - logp)) <= TOL_LOGP
+    assert np.max(np.abs(buf.lse.cpu().numpy() - lse)) <= TOL_LOGP
+    out8 = buf.out8.cpu().numpy()
+    assert abs(out8[0] - o.loss) <= TOL_LOSS * abs(o.loss)
+    assert rel_fro(buf.dH.cpu().numpy(), dH) <= TOL_DH
+    d = buf.dH.cpu().numpy()
+    assert np.all(d[wl.labels < 0] == 0.0)
+    if wl.scope == "response":
+        assert np.all(d[:wl.P] == 0.0)
+
+
+def _sampled(wl, filter_eps, block_skip):
+    H, head, labels = upload(wl)
+    hd = cce.h_dtype(H)
+    buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+    cce.cce_forward(H, head, labels, buf.logp, buf.lse, buf.tgt, buf.blockmax, buf.ws)
+    g = S.random_cotangent(wl)
+    coeff = torch.from_numpy(g).cuda()
+    cce.cce_backward_dh(H, head, labels, buf.lse, coeff, filter_eps,
+                        buf.blockmax if block_skip else None, buf.dH, buf.skip, buf.ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(buf.ws) == 0
+    return (H, head, labels, coeff), buf, g
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_long_pair_sampled_rows(cfg):
+    wl = S.make_workload(cfg)
+    (H, head, labels, coeff), buf, g = _sampled(wl, wl.filter_eps, wl.block_skip)
+    rows = S.sample_rows(wl, n_uniform=40)
+    W = oracle_W(wl)
+    logp, lse, _ = O.head_forward(wl.H, W, wl.labels, rows=rows)
+    assert np.max(np.abs(buf.logp.cpu().numpy()[rows] - logp)) <= TOL_LOGP
+    assert np.max(np.abs(buf.lse.cpu().numpy()[rows] - lse)) <= TOL_LOGP
+    # dH against the UNFILTERED oracle
+    want = O.head_dh(wl.H, W, wl.labels, g, lse, rows=rows)
+    got = buf.dH.cpu().numpy()[rows]
+    err = rel_fro(got, want)
+    print(f"workload {cfg}: sampled dH rel err {err:.3e}; skip tiles {buf.skip.cpu().tolist()}")
+    assert err <= TOL_DH
+    assert np.all(got[wl.labels[rows] < 0] == 0.0)
+    if wl.block_skip:
+        # the block skip is exact relative to the filter: bit-identical dH
+        d2 = torch.empty_like(buf.dH)
+        cce.cce_backward_dh(H, head, labels, buf.lse, coeff, wl.filter_eps, None, d2, None,
+                            buf.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(d2, buf.dH)

@@ -1,0 +1,134 @@
+"""Host-only checks of the C-ABI library: it loads, exports every entry point
+that include/cce.h declares, and rejects bad arguments synchronously before
+touching the GPU (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from lm_head_cross_flash_b200 import build, cce
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return cce.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", txt, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "defined")))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "cce_forward" in names and "cce_backward_dh" in names
+    assert "orpo_loss_from_logps" in names and "orpo_grad_coeffs" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in cce.STATUS_NAMES.items():
+        assert lib.cce_status_string(code).decode() == name
+
+
+def test_blockmax_cols(lib):
+    assert lib.cce_blockmax_cols(1) == 1
+    assert lib.cce_blockmax_cols(256) == 1
+    assert lib.cce_blockmax_cols(257) == 2
+    assert lib.cce_blockmax_cols(262144) == 1024
+    assert lib.cce_blockmax_cols(73440) == 287
+    assert lib.cce_blockmax_cols(0) == 0
+
+
+def _head(V=1000, D=128, dtype=cce.CCE_BF16, w=4096, fmt=cce.CCE_W_DENSE):
+    return cce._Head(fmt, dtype, V, D, w, None, None)
+
+
+def test_workspace_sizes_monotonic(lib):
+    h = _head()
+    sz = [lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h)) for M in (1, 100, 1000, 5000)]
+    assert all(a <= b for a, b in zip(sz, sz[1:])) and sz[0] > 0
+    lo = lib.cce_workspace_min_bytes(1000, cce.CCE_BF16, ctypes.byref(h))
+    assert 0 < lo <= sz[2]
+    big = _head(V=262144, D=2048)
+    assert lib.cce_workspace_bytes(8192, cce.CCE_BF16, ctypes.byref(big)) < 400 << 20
+    assert lib.cce_workspace_bytes(0, cce.CCE_BF16, ctypes.byref(h)) == 0
+    bad = _head(D=96)
+    assert lib.cce_workspace_bytes(10, cce.CCE_BF16, ctypes.byref(bad)) == 0
+
+
+def test_forward_rejects_bad_arguments_before_launch(lib):
+    h = _head()
+    hp = ctypes.byref(h)
+    P = ctypes.c_void_p
+    a = P(4096)
+    # null pointers
+    assert lib.cce_forward(None, 1, 10, hp, a, a, a, None, None, a, 1 << 20, None) == 1
+    assert lib.cce_forward(a, 1, 10, hp, None, a, a, None, None, a, 1 << 20, None) == 1
+    # M <= 0, bad dtype, misaligned
+    assert lib.cce_forward(a, 1, 0, hp, a, a, a, None, None, a, 1 << 20, None) == 1
+    assert lib.cce_forward(a, 7, 10, hp, a, a, a, None, None, a, 1 << 20, None) == 1
+    assert lib.cce_forward(P(4097), 1, 10, hp, a, a, a, None, None, a, 1 << 20, None) == 1
+    # D not a multiple of 64, mixed dtypes, Q4 with f32 rows
+    assert lib.cce_forward(a, 1, 10, ctypes.byref(_head(D=96)), a, a, a, None, None, a, 1 << 20, None) == 2
+    assert lib.cce_forward(a, 0, 10, hp, a, a, a, None, None, a, 1 << 20, None) == 2
+    # workspace too small
+    assert lib.cce_forward(a, 1, 10, hp, a, a, a, None, None, a, 1024, None) == 4
+
+
+def test_backward_rejects_bad_arguments_before_launch(lib):
+    h = _head()
+    hp = ctypes.byref(h)
+    P = ctypes.c_void_p
+    a = P(4096)
+    f = ctypes.c_float
+    assert lib.cce_backward_dh(a, 1, 10, hp, a, a, None, f(0), None, a, None, a, 1 << 24, None) == 1
+    assert lib.cce_backward_dh(a, 1, 10, hp, a, a, a, f(-1.0), None, a, None, a, 1 << 24, None) == 1
+    assert lib.cce_backward_dh(a, 1, 10, hp, a, a, a, f(float("nan")), None, a, None, a, 1 << 24, None) == 1
+    assert lib.cce_backward_dh(a, 1, 10, hp, a, a, a, f(0), None, P(4100), None, a, 1 << 24, None) == 1
+    assert lib.cce_backward_dh(a, 1, 10, hp, a, a, a, f(0), None, a, None, a, 4096, None) == 4
+
+
+def test_orpo_rejects_bad_layouts(lib):
+    P = ctypes.c_void_p
+    a = P(4096)
+    ws_ok = 1 << 12
+
+    def L(*v):
+        return ctypes.byref(cce._Layout(*v))
+
+    bad = [
+        (0, 10, 5, 15, 15, 20),    # overlap prompt / chosen
+        (0, 5, 5, 5, 5, 20),       # empty chosen
+        (0, 5, 5, 10, 10, 10),     # empty rejected
+        (0, 5, 5, 10, 10, 21),     # beyond M
+        (-1, 5, 5, 10, 10, 20),    # negative
+        (0, 5, 10, 5, 10, 20),     # end < begin
+    ]
+    for lay in bad:
+        assert lib.orpo_loss_from_logps(a, a, 20, L(*lay), 0.1, 0, a, a, ws_ok, None) == 1
+        assert lib.orpo_grad_coeffs(a, a, 20, L(*lay), 0.1, 0, a, a, ws_ok, None) == 1
+    good = L(0, 5, 5, 10, 10, 20)
+    assert lib.orpo_loss_from_logps(a, a, 20, good, -0.1, 0, a, a, ws_ok, None) == 1
+    assert lib.orpo_loss_from_logps(a, a, 20, good, float("nan"), 0, a, a, ws_ok, None) == 1
+    assert lib.orpo_loss_from_logps(a, a, 20, good, 0.1, 2, a, a, ws_ok, None) == 1
+    assert lib.orpo_loss_from_logps(a, a, 20, good, 0.1, 0, None, a, ws_ok, None) == 1
+    assert lib.orpo_loss_from_logps(a, a, 20, good, 0.1, 0, a, a, 16, None) == 4
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(cce, "_lib", None)
+    monkeypatch.setattr(cce, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        cce.lib()
