@@ -216,6 +216,41 @@ void cce_profile_enable(int on);
 int cce_profile_read(double* ms, long long* launches, int n);
 const char* cce_profile_kind_name(int kind);
 
+/*
+ * Forward without a caller workspace (no counterpart on the pages; it is a
+ * convenience of this library).
+ *
+ * For callers that cannot allocate device memory: plugins and plain-C hosts
+ * that receive only input and output pointers from a framework owning every
+ * device allocation, and runtimes whose device-memory budget is fixed at
+ * start-up.  Computes exactly what cce_forward computes, for bf16 H and a
+ * dense bf16 head, with the forward's scratch (per-block partials, gathered
+ * target logits, status word) in a fixed device array of
+ * CCE_NOALLOC_SCRATCH_BYTES inside the library.  Every GPU that loads the
+ * library holds that array until the process exits.
+ *
+ * - Needs 256 + 8*ceil(V/256)*M + 4*M bytes of scratch (each term rounded up
+ *   to 256) when tgt_logit and blockmax are NULL; a non-NULL blockmax or
+ *   tgt_logit is written directly and its share is unused.  Larger problems
+ *   return CCE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls share the one array and it keeps the last call's contents.
+ *   Calls whose work overlaps on the GPU (several streams, several host
+ *   threads) race on it; serialise them.
+ * - status: optional device uint32 output; it is zeroed, then receives the
+ *   device error bits (bit 0: a label >= V, bit 1: a bounded wait ran out).
+ *   With NULL the bits go to the array and are not reported.
+ * - Other arguments as for cce_forward; H is bf16 [M, D], W dense bf16.
+ */
+#define CCE_NOALLOC_SCRATCH_BYTES (32u << 20)
+cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_head* W,
+                               const int32_t* labels, float* logp, float* lse,
+                               float* tgt_logit, float* blockmax,
+                               uint32_t* status, cce_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -79,7 +79,24 @@ _SIGS = {
     "cce_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_longlong), ctypes.c_int]),
     "cce_profile_kind_name": (ctypes.c_char_p, [ctypes.c_int]),
+    "cce_forward_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(_Head),
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p]),
 }
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def cce_forward_noalloc(H, head: "Head", labels, logp, lse, tgt_logit=None, blockmax=None,
+                        status=None, stream=None):
+    """Forward for callers that cannot allocate device memory: the library's
+    fixed scratch array (NOALLOC_SCRATCH_BYTES) replaces the workspace.
+    Calls share that array, so calls that overlap on the GPU race."""
+    st = lib().cce_forward_noalloc(_p(H), H.shape[0], ctypes.byref(head.c()), _p(labels),
+                                   _p(logp), _p(lse), _p(tgt_logit), _p(blockmax), _p(status),
+                                   _stream(stream))
+    _check(st, "cce_forward_noalloc")
 
 PROFILE_KINDS = 8
 

@@ -607,3 +607,97 @@ cce_status cce_selftest_wait_timeout(void* ws, size_t ws_bytes, cce_stream_t str
 }
 
 }  // extern "C"
+
+// ========================================================================
+// Forward without a caller workspace.
+//
+// Some callers cannot allocate device memory: plugins and plain-C hosts that
+// receive only input and output pointers from a framework owning every
+// device allocation, and runtimes whose memory budget is fixed at start-up
+// and may not grow afterwards.  For them cce_forward_noalloc runs the same
+// forward kernels with their scratch (per-block partials, the gathered target
+// logits and the status word) in the fixed-size device array below.  The
+// array is a module global: every GPU that loads this library holds it until
+// the process exits.
+namespace {
+
+constexpr size_t kNoallocBytes = size_t(CCE_NOALLOC_SCRATCH_BYTES);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code only sees a host-side stand-in for the symbol).
+cce_status noalloc_scratch(char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CCE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return CCE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<char*>(g_noalloc_ptr[dev]);
+  return CCE_OK;
+}
+
+}  // namespace
+
+extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_head* W,
+                                          const int32_t* labels, float* logp, float* lse,
+                                          float* tgt_logit, float* blockmax,
+                                          uint32_t* status, cce_stream_t stream) {
+  if (H == nullptr || labels == nullptr || logp == nullptr || lse == nullptr)
+    return CCE_ERR_INVALID_ARGUMENT;
+  if (M <= 0 || M > (int64_t(1) << 30) || !aligned16(H)) return CCE_ERR_INVALID_ARGUMENT;
+  cce_status s = check_head(W, CCE_BF16);
+  if (s != CCE_OK) return s;
+  const int64_t V = W->V, D = W->D;
+  const int64_t cols = ceil_div(V, BN);
+  const int64_t n_rt = ceil_div(M, BM);
+  // scratch: status word | part_s [cols, M] | part_m [cols, M] | tgt [M]
+  const size_t o_s = kStatusBytes;
+  const size_t o_m = o_s + align_up(size_t(cols) * M * 4);
+  const size_t o_t = o_m + align_up(size_t(cols) * M * 4);
+  const size_t need = o_t + align_up(size_t(M) * 4);
+  if (need > kNoallocBytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = device_info(&sms)) != CCE_OK) return s;
+  char* scr = nullptr;
+  if ((s = noalloc_scratch(&scr)) != CCE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  uint32_t* st_word = status != nullptr ? status : reinterpret_cast<uint32_t*>(scr);
+  if (cudaMemsetAsync(st_word, 0, sizeof(uint32_t), st) != cudaSuccess) return CCE_ERR_CUDA;
+  float* part_s = reinterpret_cast<float*>(scr + o_s);
+  float* part_m = blockmax != nullptr ? blockmax : reinterpret_cast<float*>(scr + o_m);
+  float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(scr + o_t);
+
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, H, true, D, M, D, BK, BM) || !make_map(&mb, W->w, true, D, V, D, BK, BN))
+    return CCE_ERR_CUDA;
+  TileArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = int(M);
+  a.n_rt = int(n_rt);
+  a.n_ct = int(cols);
+  a.nk = int(D / BK);
+  a.npass = 1;
+  a.V = int(V);
+  a.D = int(D);
+  a.fmt = 1;
+  a.wait_ns = g_wait_ns.load();
+  a.status = st_word;
+  a.labels = labels;
+  a.part_m = part_m;
+  a.part_s = part_s;
+  a.tgt = tgt;
+  cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a);
+  if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  const int rows_per_block = 8;
+  merge_lse_kernel<<<int(ceil_div(M, rows_per_block)), rows_per_block * 32, 0, st>>>(
+      part_m, part_s, int(cols), int(M), labels, int(V), tgt, logp, lse, st_word);
+  return launch_ok();
+}
