@@ -98,7 +98,7 @@ def cce_forward_noalloc(H, head: "Head", labels, logp, lse, tgt_logit=None, bloc
                                    _stream(stream))
     _check(st, "cce_forward_noalloc")
 
-PROFILE_KINDS = 8
+PROFILE_KINDS = 16
 
 
 def cce_profile_enable(on: bool):

@@ -232,6 +232,25 @@ __global__ void split_f32_kernel(const float* __restrict__ src, int64_t rows,
   }
 }
 
+// ------------------------------------------------- K-split partial sums --
+// dH += parts[0] + parts[1] + ... (fixed order, so the result is
+// deterministic); n4 = M*D/4 float4 elements per buffer.
+__global__ void add_parts_kernel(float4* __restrict__ dh, const float4* __restrict__ parts,
+                                 int nparts, int64_t n4) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 v = dh[i];
+    for (int p = 0; p < nparts; ++p) {
+      const float4 q = parts[p * n4 + i];
+      v.x += q.x;
+      v.y += q.y;
+      v.z += q.z;
+      v.w += q.w;
+    }
+    dh[i] = v;
+  }
+}
+
 // ------------------------------------------------------ timeout self-test --
 __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
   __shared__ uint64_t bar;

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -75,11 +76,11 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // Optional per-kernel timing: while enabled, every kernel launch is
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
-  PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_N
+  PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM, PK_N
 };
 const char* const kProfNames[PK_N] = {"split_f32",     "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
-                                      "bwd_dh_gemm",   "selftest"};
+                                      "bwd_dh_gemm",   "selftest",     "dh_split_sum"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -122,6 +123,24 @@ class ProfScope {
   cudaEvent_t a_ = nullptr, b_ = nullptr;
 };
 
+// General tiled tensor map (rank 2 or 3, row-major, strides in bytes for
+// dimensions 1..rank-1), zero OOB fill.
+bool make_map_ex(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int rank,
+                 const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                 CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t d[3], st[2];
+  cuuint32_t b[3], e[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+  return fn(m, dt, rank, const_cast<void*>(ptr), d, st, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // --------------------------------------------------------- device facts --
 struct DevInfo {
   int sms = 0;
@@ -138,12 +157,12 @@ cce_status device_info(int* sms) {
   if (!d.attrs) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return CCE_ERR_CUDA;
-    if (cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes<Mode::kLse>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes<Mode::kGrad>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes<Mode::kDh>()) != cudaSuccess)
       return CCE_ERR_CUDA;
     d.attrs = true;
   }
@@ -175,11 +194,46 @@ struct Layout {
   size_t part_s = 0, part_m = 0, tgt = 0;  // forward
   size_t hs = 0, ws = 0;                   // f32 split operands
   size_t g = 0, tile_skip = 0, row_skip = 0;
+  size_t dh_part = 0;                      // K-split partial dH buffers
   int64_t vc = 0;                          // backward vocab chunk
+  int ksplit = 1;
   size_t total = 0;
 };
 
-Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc) {
+// SM count of the current device (148 on B200 when no device is visible).
+int sm_count_guess() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    return n;
+  cudaGetLastError();
+  return 148;
+}
+
+// K split of the dH GEMM: the smallest S in 1..4 whose tile count fills the
+// persistent grid's last wave best (each split needs its own fp32 partial
+// buffer, summed once at the end).  Every chunk has at least 4 K steps, so
+// every split gets at least one.
+int choose_ksplit(int64_t tiles, int sms) {
+  auto eff = [&](int S) {
+    const double w = double(tiles) * S / sms;
+    return w / std::ceil(w);
+  };
+  int best = 1;
+  double be = eff(1);
+  for (int S = 2; S <= 4; ++S)
+    if (eff(S) > be + 0.03) {
+      best = S;
+      be = eff(S);
+    }
+  return best;
+}
+
+int ksplit_for(int64_t M, const cce_head* W, int sms) {
+  return choose_ksplit(ceil_div(M, BM) * ceil_div(W->D, BN), sms);
+}
+
+Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ksplit = 1) {
   Layout L;
   const int64_t cols = ceil_div(W->V, BN);
   const int64_t n_rt = ceil_div(M, BM);
@@ -194,6 +248,8 @@ Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc) {
   L.g = b; b += align_up(size_t(M) * vc * 2);
   L.tile_skip = b; b += align_up(size_t(n_rt) * cols);
   L.row_skip = b; b += align_up(size_t(n_rt));
+  L.dh_part = b; b += align_up(size_t(ksplit - 1) * M * W->D * 4);
+  L.ksplit = ksplit;
   // split operands live after both regions
   size_t s = std::max(f, b);
   if (h == CCE_F32) {
@@ -213,13 +269,13 @@ int64_t default_vc(int64_t M, const cce_head* W) {
 
 // Widest chunk whose layout fits in ws_bytes (0 if even the narrowest
 // does not fit).
-int64_t fit_vc(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes) {
+int64_t fit_vc(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes, int ksplit) {
   const int64_t vmax = ceil_div(W->V, BN) * BN;
-  if (make_layout(M, h, W, BN).total > ws_bytes) return 0;
+  if (make_layout(M, h, W, BN, ksplit).total > ws_bytes) return 0;
   int64_t lo = 1, hi = vmax / BN;
   while (lo < hi) {
     const int64_t mid = (lo + hi + 1) / 2;
-    if (make_layout(M, h, W, mid * BN).total <= ws_bytes) lo = mid;
+    if (make_layout(M, h, W, mid * BN, ksplit).total <= ws_bytes) lo = mid;
     else hi = mid - 1;
   }
   return lo * BN;
@@ -307,12 +363,12 @@ int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
 
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
-  return make_layout(M, h_dtype, W, default_vc(M, W)).total;
+  return make_layout(M, h_dtype, W, default_vc(M, W), ksplit_for(M, W, sm_count_guess())).total;
 }
 
 size_t cce_workspace_min_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
-  return make_layout(M, h_dtype, W, BN).total;
+  return make_layout(M, h_dtype, W, BN, ksplit_for(M, W, sm_count_guess())).total;
 }
 
 cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
@@ -366,7 +422,8 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.ct_off = 0;
   {
     ProfScope ps(PK_LSE, st);
-    cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a);
+    cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+        ma, mb, ma, ma, a);
   }
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
 
@@ -453,9 +510,13 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   if (!aligned16(H) || !aligned16(ws) || !aligned16(dH)) return CCE_ERR_INVALID_ARGUMENT;
   cce_status s = check_head(W, h_dtype);
   if (s != CCE_OK) return s;
-  const int64_t vc = fit_vc(M, h_dtype, W, ws_bytes);
+  // K split of the dH GEMM; fall back to fewer splits if the workspace
+  // cannot hold their partial buffers.
+  int ksplit = ksplit_for(M, W, sm_count_guess());
+  int64_t vc = 0;
+  while ((vc = fit_vc(M, h_dtype, W, ws_bytes, ksplit)) == 0 && ksplit > 1) --ksplit;
   if (vc == 0) return CCE_ERR_WORKSPACE_TOO_SMALL;
-  const Layout L = make_layout(M, h_dtype, W, vc);
+  const Layout L = make_layout(M, h_dtype, W, vc, ksplit);
   int sms = 0;
   if ((s = device_info(&sms)) != CCE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -483,11 +544,27 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
 
-  CUtensorMap ma, mb, mg, mw;
+  CUtensorMap ma, mb, mg, mw, mgs, md0, md1;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM) ||
       !make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN) ||
       !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK))
     return CCE_ERR_CUDA;
+  {
+    // dH and the K-split partial buffers as [nbuf, M, D] fp32, 32x32 boxes
+    const uint64_t dd[3] = {uint64_t(D), uint64_t(M), 1};
+    const uint64_t ds[2] = {uint64_t(D) * 4, uint64_t(M) * D * 4};
+    const uint32_t db[3] = {32, 32, 1};
+    if (!make_map_ex(&md0, dH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dd, ds, db,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return CCE_ERR_CUDA;
+    md1 = md0;
+    if (ksplit > 1) {
+      const uint64_t pd[3] = {uint64_t(D), uint64_t(M), uint64_t(ksplit - 1)};
+      if (!make_map_ex(&md1, wsc + L.dh_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, pd, ds, db,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+        return CCE_ERR_CUDA;
+    }
+  }
 
   TileArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -508,6 +585,8 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   a.row_skip = row_skip;
   a.coeff = coeff;
   a.dh = dH;
+  a.dh_part = reinterpret_cast<float*>(wsc + L.dh_part);
+  a.ksplit = ksplit;
 
   for (int64_t v0 = 0; v0 < V; v0 += vc) {
     const int64_t w = std::min<int64_t>(vc, V - v0);
@@ -520,9 +599,19 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ag.b_row0 = int(v0);
     ag.ct_off = int(v0 / BN);
     {
+      // G'' store map: [M, chunk columns] 16-bit, 32x32 boxes, 64-byte swizzle
+      const uint64_t gd[2] = {uint64_t(ct_n * BN), uint64_t(M)};
+      const uint64_t gs[1] = {uint64_t(vc) * 2};
+      const uint32_t gb[2] = {32, 32};
+      if (!make_map_ex(&mgs, g, op.bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                       2, gd, gs, gb, CU_TENSOR_MAP_SWIZZLE_64B))
+        return CCE_ERR_CUDA;
+    }
+    {
       ProfScope ps(PK_GRAD, st);
-      cce_tc_kernel<Mode::kGrad><<<grid_for(n_rt * ct_n, sms), NUM_THREADS, SMEM_BYTES, st>>>(
-          ma, mb, ag);
+      cce_tc_kernel<Mode::kGrad><<<grid_for(n_rt * ct_n, sms), NUM_THREADS,
+                                   smem_bytes<Mode::kGrad>(), st>>>(ma, mb, mgs, mgs, ag);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     // dH (+)= coeff * G' . W[chunk]
@@ -536,9 +625,17 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ad.first_chunk = v0 == 0 ? 1 : 0;
     {
       ProfScope ps(PK_DH, st);
-      cce_tc_kernel<Mode::kDh><<<grid_for(n_rt * n_dt, sms), NUM_THREADS, SMEM_BYTES, st>>>(
-          mg, mw, ad);
+      cce_tc_kernel<Mode::kDh><<<grid_for(n_rt * n_dt * ksplit, sms), NUM_THREADS,
+                                 smem_bytes<Mode::kDh>(), st>>>(mg, mw, md0, md1, ad);
     }
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+  if (ksplit > 1) {
+    ProfScope ps(PK_DHSUM, st);
+    const int64_t n4 = M * D / 4;
+    add_parts_kernel<<<std::max<int>(1, std::min<int64_t>(ceil_div(n4, 256), 4 * sms)), 256, 0,
+                       st>>>(reinterpret_cast<float4*>(dH),
+                             reinterpret_cast<const float4*>(wsc + L.dh_part), ksplit - 1, n4);
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
   return CCE_OK;
@@ -694,7 +791,8 @@ extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_he
   a.part_m = part_m;
   a.part_s = part_s;
   a.tgt = tgt;
-  cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a);
+  cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+      ma, mb, ma, ma, a);
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   const int rows_per_block = 8;
   merge_lse_kernel<<<int(ceil_div(M, rows_per_block)), rows_per_block * 32, 0, st>>>(

@@ -38,11 +38,23 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2 };
+
+// Epilogue staging for TMA stores: per epilogue warp two buffers of
+// 32 rows x 32 columns (kGrad: 16-bit G'', 64-byte rows; kDh: fp32 dH,
+// 128-byte rows).
+template <Mode MODE>
+__host__ __device__ constexpr int staging_buf_bytes() {
+  return MODE == Mode::kGrad ? 32 * 64 : MODE == Mode::kDh ? 32 * 128 : 0;
+}
+template <Mode MODE>
+__host__ __device__ constexpr int smem_bytes() {
+  return STAGES * STAGE_BYTES + 4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
+}
+constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr uint64_t DRAIN_LIMIT_NS = 1000000000ull;
 
-enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2 };
 
 struct TileArgs {
   int M;         // rows of A (head rows)
@@ -73,9 +85,34 @@ struct TileArgs {
   const uint8_t* row_skip;   // [n_rt] or null
   // kDh
   const float* coeff;
-  float* dh;  // [M, D]
+  float* dh;       // [M, D]; K-split 0 accumulates here
+  float* dh_part;  // K-split s >= 1 accumulates in dh_part + (s-1)*M*D
+  int ksplit;      // kDh: the chunk's K range is split in `ksplit` parts
   int first_chunk;
 };
+
+// Tile t of a launch.  kLse/kGrad: row tile fastest, so the CTAs in flight
+// share one vocab tile of W (L2) and H stays resident.  kDh: d-tile fastest,
+// then K split, then row tile, so the CTAs in flight share a G' row tile.
+struct TileCoord {
+  int rt, ct, s;
+};
+
+template <Mode MODE>
+__device__ __forceinline__ TileCoord tile_coord(const TileArgs& a, int t) {
+  TileCoord c;
+  if (MODE == Mode::kDh) {
+    c.ct = t % a.n_ct;
+    const int r = t / a.n_ct;
+    c.s = r % a.ksplit;
+    c.rt = r / a.ksplit;
+  } else {
+    c.rt = t % a.n_rt;
+    c.ct = t / a.n_rt;
+    c.s = 0;
+  }
+  return c;
+}
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
@@ -108,14 +145,53 @@ __device__ __forceinline__ float softmax_p(float s, float nl) {
   return ex2_approx(fmaf(s, LOG2E, nl));
 }
 
+// Drains `nchunks` 32-column chunks of this warp's accumulator lanes through
+// two register buffers, so the TMEM load of chunk c+1 overlaps the work on
+// chunk c.  f(c, r) receives the 32 fp32 values (as bits) of chunk c.
+template <class F>
+__device__ __forceinline__ void drain_chunks(uint32_t taddr, int nchunks, F&& f) {
+  uint32_t ra[32], rb[32];
+  if (nchunks <= 0) return;
+  __syncwarp();
+  tmem_ld32(taddr, ra);
+  tmem_ld_wait(ra);
+#pragma unroll 1
+  for (int c = 0; c < nchunks; c += 2) {
+    const bool more = c + 1 < nchunks;
+    if (more) {
+      __syncwarp();
+      tmem_ld32(taddr + (c + 1) * 32, rb);
+    }
+    f(c, ra);
+    if (more) {
+      __syncwarp();
+      tmem_ld_wait(rb);
+      const bool more2 = c + 2 < nchunks;
+      if (more2) tmem_ld32(taddr + (c + 2) * 32, ra);
+      f(c + 1, rb);
+      if (more2) {
+        __syncwarp();
+        tmem_ld_wait(ra);
+      }
+    }
+  }
+}
+
 template <Mode MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     cce_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                  const __grid_constant__ CUtensorMap tmB, const TileArgs a) {
+                  const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmC,
+                  const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
+  // tmA/tmB: operand loads.  tmC: kGrad G'' store map [M, chunk] (box 32x32,
+  // 64-byte swizzle); kDh dH [1, M, D] (box 1x32x32, 128-byte swizzle).
+  // tmC2: kDh partial buffers [ksplit-1, M, D].
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * STAGE_BYTES);
+  uint8_t* staging = base + STAGES * STAGE_BYTES;
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -125,8 +201,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = a.n_rt * a.n_ct;
-  const int ksteps = a.nk * a.npass;
+  const int nsplit = MODE == Mode::kDh ? a.ksplit : 1;
+  const int ntiles = a.n_rt * a.n_ct * nsplit;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -160,9 +236,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
+      // H (kLse/kGrad) and the W chunk (kDh) are re-read by many tiles:
+      // keep them in L2 ahead of streaming data.
+      const uint64_t keep = l2_policy_evict_last();
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int rt = t % a.n_rt, ct = t / a.n_rt;
-        if (tile_kind<MODE>(a, rt, ct) != 0) continue;
+        const TileCoord tc = tile_coord<MODE>(a, t);
+        if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
+        const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
+        const int ksteps = nks * a.npass;
         for (int kk = 0; kk < ksteps; ++kk) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
             ok = false;
@@ -171,16 +252,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sA = base + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          const int pass = kk / a.nk, k = kk - pass * a.nk;
-          tma_load_2d(sA, &tmA, &full[stage], k * BK, rt * BM);
+          const int pass = kk / nks, k = kb + (kk - pass * nks);
           if (MODE == Mode::kDh) {
+            tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sB + j * (64 * BK * 2), &tmB, &full[stage],
-                          ct * BN + j * 64 + pass * a.b_pass_off,
-                          a.b_row0 + k * BK);
+              tma_load_2d_hint(sB + j * (64 * BK * 2), &tmB, &full[stage],
+                               tc.ct * BN + j * 64 + pass * a.b_pass_off,
+                               a.b_row0 + k * BK, keep);
           } else {
-            tma_load_2d(sB, &tmB, &full[stage], k * BK, a.b_row0 + ct * BN);
+            tma_load_2d_hint(sA, &tmA, &full[stage], k * BK, tc.rt * BM, keep);
+            tma_load_2d(sB, &tmB, &full[stage], k * BK, a.b_row0 + tc.ct * BN);
           }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -210,8 +292,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int acc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int rt = t % a.n_rt, ct = t / a.n_rt;
-        if (tile_kind<MODE>(a, rt, ct) != 0) continue;
+        const TileCoord tc = tile_coord<MODE>(a, t);
+        if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
+        const int ksteps =
+            ((tc.s + 1) * a.nk / nsplit - tc.s * a.nk / nsplit) * a.npass;
         const int b = acc & 1;
         if (!wait_bounded(&acc_empty[b], ((acc >> 1) & 1) ^ 1u, a.wait_ns,
                           abort_flag)) {
@@ -261,8 +345,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int rin = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     int acc = 0;
+    uint8_t* const stage_base = staging + quad * 2 * staging_buf_bytes<MODE>();
+    uint32_t nstore = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const int rt = t % a.n_rt, ct = t / a.n_rt;
+      const TileCoord tc = tile_coord<MODE>(a, t);
+      const int rt = tc.rt, ct = tc.ct;
+      float* const dh_buf =
+          tc.s == 0 ? a.dh : a.dh_part + static_cast<size_t>(tc.s - 1) * a.M * a.D;
       const int kind = tile_kind<MODE>(a, rt, ct);
       const int row = rt * BM + rin;
       const bool live = row < a.M;
@@ -277,7 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else if (MODE == Mode::kDh) {
           if (live) {
             for (int d0 = ct * BN; d0 < min(a.D, ct * BN + BN); d0 += 4)
-              *reinterpret_cast<float4*>(a.dh + static_cast<size_t>(row) * a.D + d0) =
+              *reinterpret_cast<float4*>(dh_buf + static_cast<size_t>(row) * a.D + d0) =
                   make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
@@ -295,42 +384,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (MODE == Mode::kLse) {
         const int y = live ? a.labels[row] : -1;
         const int vbase = a.b_row0 + ct * BN;
+        const int nchunks = min(BN / 32, (a.V - vbase + 31) / 32);
         float m_run = -INFINITY, s_run = 0.f, tval = 0.f;
         bool found = false;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        drain_chunks(taddr, nchunks, [&](int c, const uint32_t (&r)[32]) {
           const int v0 = vbase + c * 32;
           const int nvalid = min(32, a.V - v0);
-          if (nvalid <= 0) break;
-          __syncwarp();
-          uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
           float cm = -INFINITY;
+          float s0 = 0.f, s1 = 0.f;
           if (nvalid == 32) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) cm = fmaxf(cm, u2f(r[j]));
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) cm = fmaxf(cm, u2f(r[j]));
-          }
-          const float mn = fmaxf(m_run, cm);
-          const float nb = -mn * LOG2E;
-          float s0 = 0.f, s1 = 0.f;
-          if (nvalid == 32) {
+            const float mn = fmaxf(m_run, cm);
+            const float nb = -mn * LOG2E;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               s0 += ex2_approx(fmaf(u2f(r[j]), LOG2E, nb));
               s1 += ex2_approx(fmaf(u2f(r[j + 1]), LOG2E, nb));
             }
+            s_run = s_run * ex2_approx((m_run - mn) * LOG2E) + (s0 + s1);
+            m_run = mn;
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
+              if (j < nvalid) cm = fmaxf(cm, u2f(r[j]));
+            const float mn = fmaxf(m_run, cm);
+            const float nb = -mn * LOG2E;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
               if (j < nvalid) s0 += ex2_approx(fmaf(u2f(r[j]), LOG2E, nb));
+            s_run = s_run * ex2_approx((m_run - mn) * LOG2E) + s0;
+            m_run = mn;
           }
-          s_run = s_run * ex2_approx((m_run - mn) * LOG2E) + (s0 + s1);
-          m_run = mn;
           const int tt = y - v0;
           const bool hit = static_cast<unsigned>(tt) < static_cast<unsigned>(nvalid);
           if (__any_sync(0xffffffffu, hit)) {
@@ -340,8 +425,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (j == tt) tval = u2f(r[j]);
               found = true;
             }
+            __syncwarp();
           }
-        }
+        });
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
         if (live) {
@@ -351,78 +437,109 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (found) a.tgt[row] = tval;
         }
       } else if (MODE == Mode::kGrad) {
+        // G'' = softmax - onehot (the dH step applies -coeff), 16-bit.
         const int y = live ? a.labels[row] : -1;
         const float nl = live ? -a.lse[row] * LOG2E : 0.f;
         const float eps = a.filter_eps;
         const int vbase = a.b_row0 + ct * BN;
-        uint16_t* gdst = a.g_out + static_cast<size_t>(live ? row : 0) * a.g_ld + ct * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        drain_chunks(taddr, BN / 32, [&](int c, const uint32_t (&r)[32]) {
           const int v0 = vbase + c * 32;
-          __syncwarp();
-          uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
+          const int tt = y - v0;
+          // Warp-uniform: a chunk inside the vocab with no label of this warp
+          // takes the short path (one FFMA + one ex2 per logit).
+          const bool slow = (v0 + 32 > a.V) ||
+                            __any_sync(0xffffffffu, static_cast<unsigned>(tt) < 32u);
           uint32_t pk[16];
+          if (!slow) {
+            if (eps > 0.f) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float g2[2];
+              for (int j = 0; j < 32; j += 2) {
+                float p0 = softmax_p(u2f(r[j]), nl), p1 = softmax_p(u2f(r[j + 1]), nl);
+                p0 = p0 < eps ? 0.f : p0;
+                p1 = p1 < eps ? 0.f : p1;
+                pk[j >> 1] = pack2(p0, p1, a.fmt);
+              }
+            } else {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int v = v0 + j + h;
-              float p = softmax_p(u2f(r[j + h]), nl);
-              const bool tgt = (v == y);
-              if (p < eps && !tgt) p = 0.f;
-              g2[h] = v < a.V ? (tgt ? 1.f - p : -p) : 0.f;
+              for (int j = 0; j < 32; j += 2)
+                pk[j >> 1] = pack2(softmax_p(u2f(r[j]), nl), softmax_p(u2f(r[j + 1]), nl), a.fmt);
             }
-            pk[j >> 1] = pack2(g2[0], g2[1], a.fmt);
-          }
-          if (live) {
-            uint4* dst = reinterpret_cast<uint4*>(gdst + c * 32);
+          } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int j = 0; j < 32; j += 2) {
+              float g2[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int v = v0 + j + h;
+                float p = softmax_p(u2f(r[j + h]), nl);
+                const bool tgt = (v == y);
+                if (p < eps && !tgt) p = 0.f;
+                g2[h] = v < a.V ? (tgt ? p - 1.f : p) : 0.f;
+              }
+              pk[j >> 1] = pack2(g2[0], g2[1], a.fmt);
+            }
           }
-        }
+          // Stage the 32x32 block in shared memory (64-byte swizzle: 16-byte
+          // chunk i of row r sits at chunk i ^ ((r >> 1) & 3)) and let TMA
+          // write it; rows past M are clipped by the tensor map.
+          uint8_t* sb = stage_base + (nstore & 1) * staging_buf_bytes<MODE>();
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(sb + lane * 64 + ((i ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, sb, ct * BN + c * 32, rt * BM + quad * 32);
+            bulk_commit();
+          }
+          ++nstore;
+        });
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
-      } else {  // kDh
-        const float g = live ? a.coeff[row] : 0.f;
+      } else {  // kDh: dH (+)= -coeff * (G'' . W)
+        const float g = live ? -a.coeff[row] : 0.f;
         const int dbase = ct * BN;
-        float* drow = a.dh + static_cast<size_t>(live ? row : 0) * a.D;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int d0 = dbase + c * 32;
-          if (d0 >= a.D) break;
+        const int nchunks = min(BN / 32, (a.D - dbase) / 32);
+        const CUtensorMap* dmap = tc.s == 0 ? &tmC : &tmC2;
+        const int dz = tc.s == 0 ? 0 : tc.s - 1;
+        drain_chunks(taddr, nchunks, [&](int c, const uint32_t (&r)[32]) {
+          // Stage g * acc as a 32x32 fp32 block (128-byte swizzle: chunk i of
+          // row r at chunk i ^ (r & 7)); the first vocab chunk stores it, the
+          // later ones add it in L2 (one add per element per launch, so the
+          // result does not depend on timing).
+          uint8_t* sb = stage_base + (nstore & 1) * staging_buf_bytes<MODE>();
+          if (lane == 0) bulk_wait_read<1>();
           __syncwarp();
-          uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
-          if (live) {
-            float4* dst = reinterpret_cast<float4*>(drow + d0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 o;
-              o.x = g == 0.f ? 0.f : g * u2f(r[4 * i + 0]);
-              o.y = g == 0.f ? 0.f : g * u2f(r[4 * i + 1]);
-              o.z = g == 0.f ? 0.f : g * u2f(r[4 * i + 2]);
-              o.w = g == 0.f ? 0.f : g * u2f(r[4 * i + 3]);
-              if (!a.first_chunk) {
-                const float4 p = dst[i];
-                o.x += p.x;
-                o.y += p.y;
-                o.z += p.z;
-                o.w += p.w;
-              }
-              dst[i] = o;
-            }
+          for (int i = 0; i < 8; ++i) {
+            const float4 o =
+                g == 0.f ? make_float4(0.f, 0.f, 0.f, 0.f)
+                         : make_float4(g * u2f(r[4 * i]), g * u2f(r[4 * i + 1]),
+                                       g * u2f(r[4 * i + 2]), g * u2f(r[4 * i + 3]));
+            *reinterpret_cast<float4*>(sb + lane * 128 + ((i ^ (lane & 7)) << 4)) = o;
           }
-        }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (a.first_chunk)
+              tma_store_3d(dmap, sb, dbase + c * 32, rt * BM + quad * 32, dz);
+            else
+              tma_reduce_add_3d(dmap, sb, dbase + c * 32, rt * BM + quad * 32, dz);
+            bulk_commit();
+          }
+          ++nstore;
+        });
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
       }
       ++acc;
     }
+    // Every TMA store / reduction of this warp has completed before exit.
+    if (MODE != Mode::kLse && lane == 0) bulk_wait<0>();
+    __syncwarp();
   }
 
   tc_fence_before();
