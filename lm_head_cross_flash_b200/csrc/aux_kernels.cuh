@@ -232,6 +232,25 @@ __global__ void split_f32_kernel(const float* __restrict__ src, int64_t rows,
   }
 }
 
+// fp16 copy of bf16 rows [rows, D] for a 4-bit head, with element e of every
+// group of 8 columns stored at position q4_pos(e) (the order in which the
+// dequantiser lays out the weights along K).  n8 = rows*D/8.
+__global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
+                                     uint4* __restrict__ dst) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    __half h[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t bits = (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+      h[q4_pos(e)] = __float2half_rn(__uint_as_float(bits << 16));
+    }
+    dst[i] = *reinterpret_cast<const uint4*>(h);
+  }
+}
+
 // ------------------------------------------------- K-split partial sums --
 // dH += parts[0] + parts[1] + ... (fixed order, so the result is
 // deterministic); n4 = M*D/4 float4 elements per buffer.

@@ -157,12 +157,13 @@ cce_status device_info(int* sms) {
   if (!d.attrs) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return CCE_ERR_CUDA;
-    if (cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes<Mode::kLse>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes<Mode::kGrad>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes<Mode::kDh>()) != cudaSuccess)
+    const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    if (cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse, false>, attr, smem_bytes<Mode::kLse>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad, false>, attr, smem_bytes<Mode::kGrad>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh, false>, attr, smem_bytes<Mode::kDh>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse, true>, attr, smem_bytes<Mode::kLse>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad, true>, attr, smem_bytes<Mode::kGrad>()) != cudaSuccess ||
+        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh, true>, attr, smem_bytes<Mode::kDh>()) != cudaSuccess)
       return CCE_ERR_CUDA;
     d.attrs = true;
   }
@@ -184,7 +185,13 @@ cce_status check_head(const cce_head* W, cce_dtype h_dtype) {
     if (W->dtype != h_dtype) return CCE_ERR_UNSUPPORTED;
     return CCE_OK;
   }
-  if (W->format == CCE_W_AFFINE_Q4_G64) return CCE_ERR_UNSUPPORTED;
+  if (W->format == CCE_W_AFFINE_Q4_G64) {
+    if (W->dtype != CCE_BF16 || W->scales == nullptr || W->biases == nullptr ||
+        (reinterpret_cast<uintptr_t>(W->scales) & 1u) || (reinterpret_cast<uintptr_t>(W->biases) & 1u))
+      return CCE_ERR_INVALID_ARGUMENT;
+    if (h_dtype != CCE_BF16) return CCE_ERR_UNSUPPORTED;
+    return CCE_OK;
+  }
   return CCE_ERR_INVALID_ARGUMENT;
 }
 
@@ -255,6 +262,8 @@ Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ks
   if (h == CCE_F32) {
     L.hs = s; s += align_up(size_t(M) * 3 * W->D * 2);
     L.ws = s; s += align_up(size_t(W->V) * 3 * W->D * 2);
+  } else if (W->format == CCE_W_AFFINE_Q4_G64) {
+    L.hs = s; s += align_up(size_t(M) * W->D * 2);  // fp16, K-permuted rows
   }
   L.vc = vc;
   L.total = s;
@@ -291,11 +300,25 @@ int grid_for(int64_t tiles, int sms) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, sms)));
 }
 
+// Launch one tensor-core step; a 4-bit head adds the dequantisation warps.
+template <Mode MODE>
+void launch_tc(bool q4, int64_t tiles, int sms, cudaStream_t st, const CUtensorMap& ma,
+               const CUtensorMap& mb, const CUtensorMap& mc, const CUtensorMap& mc2,
+               const TileArgs& args) {
+  if (q4)
+    cce_tc_kernel<MODE, true><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
+        ma, mb, mc, mc2, args);
+  else
+    cce_tc_kernel<MODE, false><<<grid_for(tiles, sms), NUM_THREADS, smem_bytes<MODE>(), st>>>(
+        ma, mb, mc, mc2, args);
+}
+
 // Operands of the tensor-core GEMMs for one problem: 16-bit A (head rows)
 // and B (head) with their K extents.
 struct Operands {
+  bool q4;         // 4-bit head: B is dequantised in-kernel, A is fp16
   const void* a;   // [M, ka] 16-bit
-  const void* b;   // [V, kb] 16-bit
+  const void* b;   // [V, kb] 16-bit (dense heads)
   int64_t k;       // contraction length used by the S GEMM
   int64_t ld_a, ld_b;
   bool bf16;
@@ -306,6 +329,24 @@ struct Operands {
 cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_head* W,
                             const Layout& L, void* ws, cudaStream_t st, Operands* op) {
   const int64_t D = W->D;
+  op->q4 = W->format == CCE_W_AFFINE_Q4_G64;
+  if (op->q4) {
+    uint4* h16 = reinterpret_cast<uint4*>(static_cast<char*>(ws) + L.hs);
+    {
+      ProfScope ps(PK_SPLIT, st);
+      h_to_f16_perm_kernel<<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+    }
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    op->a = h16;
+    op->b = nullptr;
+    op->k = D;
+    op->ld_a = D;
+    op->ld_b = D;
+    op->bf16 = false;
+    op->d_pass_off = 0;
+    op->npass_dh = 1;
+    return CCE_OK;
+  }
   if (h == CCE_BF16) {
     op->a = H;
     op->b = W->w;
@@ -398,9 +439,9 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
 
   CUtensorMap ma, mb;
-  if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM) ||
-      !make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN))
-    return CCE_ERR_CUDA;
+  if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
+  if (op.q4) mb = ma;  // unused: B is dequantised in-kernel
+  else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN)) return CCE_ERR_CUDA;
 
   TileArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -420,10 +461,12 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.part_s = part_s;
   a.tgt = tgt;
   a.ct_off = 0;
+  a.q_w = static_cast<const uint32_t*>(W->w);
+  a.q_scale = static_cast<const uint16_t*>(W->scales);
+  a.q_bias = static_cast<const uint16_t*>(W->biases);
   {
     ProfScope ps(PK_LSE, st);
-    cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
-        ma, mb, ma, ma, a);
+    launch_tc<Mode::kLse>(op.q4, n_rt * cols, sms, st, ma, mb, ma, ma, a);
   }
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
 
@@ -545,10 +588,14 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   }
 
   CUtensorMap ma, mb, mg, mw, mgs, md0, md1;
-  if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM) ||
-      !make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN) ||
-      !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK))
+  if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
+  if (op.q4) {
+    mb = ma;  // unused: B is dequantised in-kernel
+    mw = ma;
+  } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN) ||
+             !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK)) {
     return CCE_ERR_CUDA;
+  }
   {
     // dH and the K-split partial buffers as [nbuf, M, D] fp32, 32x32 boxes
     const uint64_t dd[3] = {uint64_t(D), uint64_t(M), 1};
@@ -587,6 +634,9 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   a.dh = dH;
   a.dh_part = reinterpret_cast<float*>(wsc + L.dh_part);
   a.ksplit = ksplit;
+  a.q_w = static_cast<const uint32_t*>(W->w);
+  a.q_scale = static_cast<const uint16_t*>(W->scales);
+  a.q_bias = static_cast<const uint16_t*>(W->biases);
 
   for (int64_t v0 = 0; v0 < V; v0 += vc) {
     const int64_t w = std::min<int64_t>(vc, V - v0);
@@ -610,8 +660,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     }
     {
       ProfScope ps(PK_GRAD, st);
-      cce_tc_kernel<Mode::kGrad><<<grid_for(n_rt * ct_n, sms), NUM_THREADS,
-                                   smem_bytes<Mode::kGrad>(), st>>>(ma, mb, mgs, mgs, ag);
+      launch_tc<Mode::kGrad>(op.q4, n_rt * ct_n, sms, st, ma, mb, mgs, mgs, ag);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     // dH (+)= coeff * G' . W[chunk]
@@ -625,8 +674,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ad.first_chunk = v0 == 0 ? 1 : 0;
     {
       ProfScope ps(PK_DH, st);
-      cce_tc_kernel<Mode::kDh><<<grid_for(n_rt * n_dt * ksplit, sms), NUM_THREADS,
-                                 smem_bytes<Mode::kDh>(), st>>>(mg, mw, md0, md1, ad);
+      launch_tc<Mode::kDh>(op.q4, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
@@ -751,6 +799,7 @@ extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_he
   if (M <= 0 || M > (int64_t(1) << 30) || !aligned16(H)) return CCE_ERR_INVALID_ARGUMENT;
   cce_status s = check_head(W, CCE_BF16);
   if (s != CCE_OK) return s;
+  if (W->format != CCE_W_DENSE) return CCE_ERR_UNSUPPORTED;
   const int64_t V = W->V, D = W->D;
   const int64_t cols = ceil_div(V, BN);
   const int64_t n_rt = ceil_div(M, BM);
@@ -791,7 +840,7 @@ extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_he
   a.part_m = part_m;
   a.part_s = part_s;
   a.tgt = tgt;
-  cce_tc_kernel<Mode::kLse><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+  cce_tc_kernel<Mode::kLse, false><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
       ma, mb, ma, ma, a);
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   const int rows_per_block = 8;

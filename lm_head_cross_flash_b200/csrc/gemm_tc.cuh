@@ -36,7 +36,9 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 192;     // TMA, MMA, 4 epilogue warps
+constexpr int NUM_THREADS_Q4 = 320;  // + 4 dequantisation warps (4-bit head)
+constexpr int DQ_WARP0 = 6;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2 };
 
@@ -89,7 +91,42 @@ struct TileArgs {
   float* dh_part;  // K-split s >= 1 accumulates in dh_part + (s-1)*M*D
   int ksplit;      // kDh: the chunk's K range is split in `ksplit` parts
   int first_chunk;
+  // 4-bit affine head (group 64): words [V, D/8], scales/biases bf16 [V, D/64]
+  const uint32_t* q_w;
+  const uint16_t* q_scale;
+  const uint16_t* q_bias;
 };
+
+// Position, inside its group of 8, at which the 4-bit dequantiser stores
+// element e of the group: the int4 -> fp16 conversion yields the pairs
+// (e0,e4), (e1,e5), (e2,e6), (e3,e7).  The hidden rows are stored with the
+// same order along K, so every dot product is unchanged.
+__host__ __device__ constexpr int q4_pos(int e) { return e < 4 ? 2 * e : 2 * e - 7; }
+
+// Dequantise the 64 weights of one (row, group): w = q * scale + bias, with
+// q read from 8 packed words (element 8c+j = bits 4j..4j+3 of word c) and
+// the result rounded once to fp16 (fma.rn.f16x2 on q, scale, bias, all exact
+// in fp16).  q comes from the bit pattern 0x6400 | q = 1024 + q in fp16.
+// out[c] holds the 8 fp16 values of word c in q4_pos order.
+__device__ __forceinline__ void dequant_group64(const uint4& wa, const uint4& wb, uint16_t sbits,
+                                                uint16_t bbits, uint4 (&out)[8]) {
+  const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
+  const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bbits) << 16));
+  const __half2 k1024 = __float2half2_rn(1024.f);
+  const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t x = ((words[c] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
+      __half2 h = *reinterpret_cast<const __half2*>(&x);
+      h = __hfma2(__hsub2(h, k1024), s2, b2);
+      t[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    out[c] = make_uint4(t[0], t[1], t[2], t[3]);
+  }
+}
 
 // Tile t of a launch.  kLse/kGrad: row tile fastest, so the CTAs in flight
 // share one vocab tile of W (L2) and H stays resident.  kDh: d-tile fastest,
@@ -177,8 +214,8 @@ __device__ __forceinline__ void drain_chunks(uint32_t taddr, int nchunks, F&& f)
   }
 }
 
-template <Mode MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <Mode MODE, bool Q4 = false>
+__global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     cce_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                   const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC,
@@ -206,7 +243,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], Q4 ? 1 + 4 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -251,9 +288,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint8_t* sA = base + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
           const int pass = kk / nks, k = kb + (kk - pass * nks);
-          if (MODE == Mode::kDh) {
+          if (Q4) {
+            // B comes from the dequantisation warps.
+            mbar_arrive_expect_tx(&full[stage], A_BYTES);
+            if (MODE == Mode::kDh)
+              tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
+            else
+              tma_load_2d_hint(sA, &tmA, &full[stage], k * BK, tc.rt * BM, keep);
+          } else if (MODE == Mode::kDh) {
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
             tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
@@ -261,6 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                tc.ct * BN + j * 64 + pass * a.b_pass_off,
                                a.b_row0 + k * BK, keep);
           } else {
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
             tma_load_2d_hint(sA, &tmA, &full[stage], k * BK, tc.rt * BM, keep);
             tma_load_2d(sB, &tmB, &full[stage], k * BK, a.b_row0 + tc.ct * BN);
           }
@@ -338,6 +383,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // All MMAs issued by this thread complete before TMEM is released.
       umma_commit(drain);
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
+    }
+  } else if (Q4 && warp >= DQ_WARP0) {
+    // --------------------------------------------- 4-bit dequantisation --
+    // 128 threads fill the B half of every stage: 256 (row, group) units of
+    // 64 weights per K step, 2 per thread, read from global memory (words,
+    // scale, bias), dequantised to fp16 and written in the 128-byte-swizzled
+    // layout the TMA would produce (16-byte chunk c of row r at c ^ (r & 7)).
+    const int dq = threadIdx.x - DQ_WARP0 * 32;
+    const int gpr = a.D / 64;  // groups per head row
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    struct Unit {
+      uint4 wa, wb;
+      uint16_t sc, bi;
+      bool valid;
+    };
+    // unit u of K step k of tile tc: source row, group and smem offset
+    auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& off) {
+      if (MODE == Mode::kDh) {
+        const int r = u & 63, j = u >> 6;
+        v = a.b_row0 + k * BK + r;
+        g = tc.ct * (BN / 64) + j;
+        off = j * (64 * BK * 2) + r * 128;
+      } else {
+        v = a.b_row0 + tc.ct * BN + u;
+        g = k;
+        off = u * 128;
+      }
+    };
+    auto load = [&](const TileCoord& tc, int k, int u) {
+      Unit x;
+      int v, g, off;
+      locate(tc, k, u, v, g, off);
+      x.valid = v < a.V && g < gpr;
+      if (x.valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.q_w + static_cast<size_t>(v) * (a.D / 8) + g * 8);
+        x.wa = __ldg(src);
+        x.wb = __ldg(src + 1);
+        x.sc = __ldg(a.q_scale + static_cast<size_t>(v) * gpr + g);
+        x.bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
+      } else {
+        x.wa = x.wb = make_uint4(0, 0, 0, 0);
+        x.sc = x.bi = 0;
+      }
+      return x;
+    };
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      const TileCoord tc = tile_coord<MODE>(a, t);
+      if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
+      const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
+      Unit c0 = load(tc, kb, dq), c1 = load(tc, kb, dq + 128);
+      for (int kk = 0; kk < nks; ++kk) {
+        Unit n0, n1;
+        if (kk + 1 < nks) {
+          n0 = load(tc, kb + kk + 1, dq);
+          n1 = load(tc, kb + kk + 1, dq + 128);
+        }
+        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sB = base + stage * STAGE_BYTES + A_BYTES;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const Unit& x = h == 0 ? c0 : c1;
+          const int u = dq + h * 128;
+          int v, g, off;
+          locate(tc, kb + kk, u, v, g, off);
+          const int r = MODE == Mode::kDh ? (u & 63) : u;
+          uint4 out[8];
+          if (x.valid) {
+            dequant_group64(x.wa, x.wb, x.sc, x.bi, out);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(sB + off + ((c ^ (r & 7)) << 4)) = out[c];
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        c0 = n0;
+        c1 = n1;
+      }
+    }
+    if (!ok) {
+      set_status(a.status, ST_TIMEOUT);
+      *abort_flag = 1;
     }
   } else {
     // ---------------------------------------------------------- epilogue --
@@ -515,10 +655,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
+            // accumulator column of output column j (4-bit heads permute K
+            // inside groups of 8, so the dH columns come out permuted too)
+            constexpr auto src = [](int j) { return Q4 ? (j & ~7) + q4_pos(j & 7) : j; };
             const float4 o =
                 g == 0.f ? make_float4(0.f, 0.f, 0.f, 0.f)
-                         : make_float4(g * u2f(r[4 * i]), g * u2f(r[4 * i + 1]),
-                                       g * u2f(r[4 * i + 2]), g * u2f(r[4 * i + 3]));
+                         : make_float4(g * u2f(r[src(4 * i)]), g * u2f(r[src(4 * i + 1)]),
+                                       g * u2f(r[src(4 * i + 2)]), g * u2f(r[src(4 * i + 3)]));
             *reinterpret_cast<float4*>(sb + lane * 128 + ((i ^ (lane & 7)) << 4)) = o;
           }
           fence_proxy_async_smem();

@@ -2,7 +2,8 @@
 
 * tiny fp32 pair and small bf16 pair: the whole pass (logp, lse, loss,
   cotangent, dH) against the oracle on every row;
-* long bf16 pairs: logp / lse on stratified sampled rows, and dH on sampled
+* long bf16 pairs and the long-context 4-bit pair: logp / lse on stratified
+  sampled rows, and dH on sampled
   rows for a seeded non-uniform cotangent (the oracle cannot afford every
   row); the filtered + block-skipped backward is compared with the
   unfiltered oracle, and block skipping must not change a single bit of dH.
@@ -57,7 +58,7 @@ def _sampled(wl, filter_eps, block_skip):
     return (H, head, labels, coeff), buf, g
 
 
-@pytest.mark.parametrize("cfg", [2, 3])
+@pytest.mark.parametrize("cfg", [2, 3, 4])
 def test_long_pair_sampled_rows(cfg):
     wl = S.make_workload(cfg)
     (H, head, labels, coeff), buf, g = _sampled(wl, wl.filter_eps, wl.block_skip)

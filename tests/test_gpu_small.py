@@ -41,6 +41,9 @@ SMALL = [
     (1, (64, 200, 300), 192, 1000),
     (0, (8, 60, 60), 64, 300),
     (0, (32, 96, 128), 256, 4096),
+    (4, (40, 45, 44), 128, 257),
+    (4, (100, 150, 131), 256, 4097),
+    (4, (64, 200, 300), 320, 1000),
 ]
 
 
@@ -88,7 +91,9 @@ def test_integer_design_is_bit_exact():
 
 @pytest.mark.parametrize("cfg,split,D,V", [(1, (40, 45, 44), 64, 257),
                                            (2, (100, 150, 131), 256, 4097),
-                                           (0, (8, 60, 60), 64, 300)])
+                                           (0, (8, 60, 60), 64, 300),
+                                           (4, (100, 150, 131), 256, 4097),
+                                           (4, (64, 200, 300), 320, 1000)])
 def test_backward_random_cotangent(cfg, split, D, V):
     """dH with a non-uniform cotangent (rows with zero cotangent stay 0)."""
     wl = S.make_custom(cfg, M_split=split, D=D, V=V)
@@ -124,9 +129,9 @@ def test_backward_narrow_workspace_chunks():
     assert rel_fro(d2.cpu().numpy(), d1.cpu().numpy()) < 1e-5
 
 
-@pytest.mark.parametrize("scope", ["full", "response"])
-def test_full_pass_small(scope):
-    wl = S.make_custom(0, M_split=(32, 96, 128), D=256, V=4096)
+@pytest.mark.parametrize("cfg,scope", [(0, "full"), (0, "response"), (4, "full")])
+def test_full_pass_small(cfg, scope):
+    wl = S.make_custom(cfg, M_split=(32, 96, 128), D=256, V=4096)
     wl.scope = scope
     _, _, _, buf, st = run_pass(wl)
     assert st == 0
