@@ -164,6 +164,15 @@ def aggregate(dist, local_ms: float, local_tokens: float, device=None):
 
 # ------------------------------------------------------------ CPU oracle --
 
+def oracle_head(wl):
+    """The head's weights as the method defines them, float64."""
+    import numpy as np
+    from oracle import flash_cce as O
+    if wl.wformat == "q4g64":
+        return O.dequant_affine_q4(wl.q_packed, wl.q_scales, wl.q_biases)
+    return wl.W.astype(np.float64)
+
+
 def oracle_rows(wl, W64, rows, g):
     """The oracle's per-row work of one head pass (forward and dH) on `rows`."""
     from oracle import flash_cce as O
@@ -186,7 +195,7 @@ def time_oracle(wl, seconds: float, rows_per_block: int = 8):
 
     from lm_head_cross_flash_b200 import synthetic as S
     cores = cpu_threads()
-    W64 = wl.W.astype(np.float64)
+    W64 = oracle_head(wl)
     g = S.random_cotangent(wl).astype(np.float64)
     order = np.random.default_rng(0).permutation(wl.M)
     done, t0 = 0, time.perf_counter()
@@ -221,14 +230,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     wl = S.make_workload(args.workload)
-    if wl.dtype == "bf16":
-        H = torch.from_numpy(wl.H_bits.view(np.int16)).to(dev).view(torch.bfloat16)
-        head = cce.Head(w=torch.from_numpy(wl.W_bits.view(np.int16)).to(dev).view(torch.bfloat16),
-                        V=wl.V, D=wl.D)
-    else:
-        H = torch.from_numpy(wl.H).to(dev)
-        head = cce.Head(w=torch.from_numpy(wl.W).to(dev), V=wl.V, D=wl.D)
-    labels = torch.from_numpy(wl.labels).to(dev)
+    H, head, labels = cce.upload_workload(wl, dev)
     torch.cuda.reset_peak_memory_stats(dev)
     base_alloc = torch.cuda.memory_allocated(dev)
     free0, _ = torch.cuda.mem_get_info(dev)
@@ -339,7 +341,7 @@ def run_ours(args):
     flop_step = 6.0 * wl.M * wl.V * wl.D
     tflops = flop_step / (ms_step / 1e3) / 1e12
     # roofline of the dominant kernel kind (largest summed time)
-    per_kind_flops = {"fwd_lse_gemm": 2.0 * wl.M * wl.V * wl.D,
+    per_kind_flops = {"fwd_lse_gemm": 2.0 * wl.M * wl.V * wl.D,  # per step
                       "bwd_grad_gemm": 2.0 * wl.M * wl.V * wl.D,
                       "bwd_dh_gemm": 2.0 * wl.M * wl.V * wl.D}
     kinds = {k: v for k, v in prof.items() if v[1] > 0}
@@ -371,7 +373,8 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "dtype": ("f16 (4-bit head dequantised in-kernel)" if wl.wformat == "q4g64"
+                  else "bf16" if wl.dtype == "bf16" else "f32"),
         "data": "synthetic: seeded inputs of the workload recipe, random-init head",
         "config": {"workload": wl.name, "M": wl.M, "D": wl.D, "V": wl.V, "P": wl.P,
                    "Rc": wl.Rc, "Rr": wl.Rr, "sft_scope": wl.scope, "lambda": wl.lam,
@@ -408,7 +411,7 @@ def run_reference(args):
 
     from lm_head_cross_flash_b200 import synthetic as S
     wl = S.make_workload(args.workload)
-    W64 = wl.W.astype(np.float64)
+    W64 = oracle_head(wl)
     g = S.random_cotangent(wl).astype(np.float64)
     cores = cpu_threads()
     rows_per_step = 4

@@ -286,3 +286,24 @@ def orpo_head_pass(H, head: Head, labels, layout, lam, sft_scope, filter_eps,
     orpo_grad_coeffs(buf.logp, labels, layout, lam, sft_scope, buf.coeff, buf.ws, stream)
     cce_backward_dh(H, head, labels, buf.lse, buf.coeff, filter_eps,
                     buf.blockmax if block_skip else None, buf.dH, buf.skip, buf.ws, stream)
+
+
+def upload_workload(wl, device="cuda"):
+    """Device tensors (H, Head, labels) of a ``synthetic.Workload``."""
+    import numpy as np
+    if wl.dtype == "bf16":
+        H = torch.from_numpy(wl.H_bits.view(np.int16)).to(device).view(torch.bfloat16)
+    else:
+        H = torch.from_numpy(wl.H).to(device)
+    if wl.wformat == "q4g64":
+        head = Head(w=torch.from_numpy(wl.q_packed.view(np.int32)).to(device), V=wl.V, D=wl.D,
+                    fmt=CCE_W_AFFINE_Q4_G64,
+                    scales=torch.from_numpy(wl.q_scales.view(np.int16)).to(device).view(torch.bfloat16),
+                    biases=torch.from_numpy(wl.q_biases.view(np.int16)).to(device).view(torch.bfloat16))
+    elif wl.dtype == "bf16":
+        head = Head(w=torch.from_numpy(wl.W_bits.view(np.int16)).to(device).view(torch.bfloat16),
+                    V=wl.V, D=wl.D)
+    else:
+        head = Head(w=torch.from_numpy(wl.W).to(device), V=wl.V, D=wl.D)
+    labels = torch.from_numpy(wl.labels).to(device)
+    return H, head, labels

@@ -270,9 +270,19 @@ Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ks
   return L;
 }
 
+// Row tiles per raster group of the S GEMMs: as many as keep about 48 MB of
+// the hidden rows (the re-used operand) in L2.
+int group_rows(int64_t n_rt, int64_t k_elems) {
+  const int64_t per = int64_t(BM) * k_elems * 2;
+  return int(std::max<int64_t>(1, std::min<int64_t>(n_rt, (int64_t(48) << 20) / per)));
+}
+
+// Default G'' chunk: 256 MB, or four times dH when that is larger (every
+// chunk adds into dH once, so wider chunks save dH traffic when M*D is big).
 int64_t default_vc(int64_t M, const cce_head* W) {
   const int64_t vmax = ceil_div(W->V, BN) * BN;
-  int64_t vc = (kDefaultChunkBytes / (2 * M)) / BN * BN;
+  const int64_t budget = std::max<int64_t>(kDefaultChunkBytes, 4 * M * W->D * 4);
+  int64_t vc = (budget / (2 * M)) / BN * BN;
   return std::max<int64_t>(BN, std::min(vc, vmax));
 }
 
@@ -464,6 +474,7 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.q_w = static_cast<const uint32_t*>(W->w);
   a.q_scale = static_cast<const uint16_t*>(W->scales);
   a.q_bias = static_cast<const uint16_t*>(W->biases);
+  a.group_rt = group_rows(n_rt, op.k);
   {
     ProfScope ps(PK_LSE, st);
     launch_tc<Mode::kLse>(op.q4, n_rt * cols, sms, st, ma, mb, ma, ma, a);
@@ -637,6 +648,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   a.q_w = static_cast<const uint32_t*>(W->w);
   a.q_scale = static_cast<const uint16_t*>(W->scales);
   a.q_bias = static_cast<const uint16_t*>(W->biases);
+  a.group_rt = group_rows(n_rt, op.k);
 
   for (int64_t v0 = 0; v0 < V; v0 += vc) {
     const int64_t w = std::min<int64_t>(vc, V - v0);
@@ -836,6 +848,7 @@ extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_he
   a.fmt = 1;
   a.wait_ns = g_wait_ns.load();
   a.status = st_word;
+  a.group_rt = int(n_rt);
   a.labels = labels;
   a.part_m = part_m;
   a.part_s = part_s;

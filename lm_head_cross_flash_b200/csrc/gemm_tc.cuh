@@ -37,7 +37,8 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;     // TMA, MMA, 4 epilogue warps
-constexpr int NUM_THREADS_Q4 = 320;  // + 4 dequantisation warps (4-bit head)
+constexpr int DQ_WARPS = 8;          // dequantisation warps (4-bit head), 2 per SMSP
+constexpr int NUM_THREADS_Q4 = NUM_THREADS + 32 * DQ_WARPS;
 constexpr int DQ_WARP0 = 6;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2 };
@@ -91,6 +92,7 @@ struct TileArgs {
   float* dh_part;  // K-split s >= 1 accumulates in dh_part + (s-1)*M*D
   int ksplit;      // kDh: the chunk's K range is split in `ksplit` parts
   int first_chunk;
+  int group_rt;    // kLse/kGrad: row tiles per raster group
   // 4-bit affine head (group 64): words [V, D/8], scales/biases bf16 [V, D/64]
   const uint32_t* q_w;
   const uint16_t* q_scale;
@@ -128,9 +130,12 @@ __device__ __forceinline__ void dequant_group64(const uint4& wa, const uint4& wb
   }
 }
 
-// Tile t of a launch.  kLse/kGrad: row tile fastest, so the CTAs in flight
-// share one vocab tile of W (L2) and H stays resident.  kDh: d-tile fastest,
-// then K split, then row tile, so the CTAs in flight share a G' row tile.
+// Tile t of a launch.  kLse/kGrad: row tiles are taken in groups of
+// `group_rt` (sized so a group of H rows stays in L2); inside a group the row
+// tile is fastest, so the CTAs in flight share one vocab tile of W, and the
+// group sweeps the whole vocabulary before the next group starts.  kDh:
+// d-tile fastest, then K split, then row tile, so the CTAs in flight share a
+// G' row tile.
 struct TileCoord {
   int rt, ct, s;
 };
@@ -144,8 +149,13 @@ __device__ __forceinline__ TileCoord tile_coord(const TileArgs& a, int t) {
     c.s = r % a.ksplit;
     c.rt = r / a.ksplit;
   } else {
-    c.rt = t % a.n_rt;
-    c.ct = t / a.n_rt;
+    const int per_group = a.group_rt * a.n_ct;
+    const int grp = t / per_group;
+    const int r = t - grp * per_group;
+    const int g0 = grp * a.group_rt;
+    const int gn = min(a.group_rt, a.n_rt - g0);
+    c.rt = g0 + r % gn;
+    c.ct = r / gn;
     c.s = 0;
   }
   return c;
@@ -243,7 +253,7 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], Q4 ? 1 + 4 : 1);
+      mbar_init(&full[s], Q4 ? 1 + DQ_WARPS : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -386,8 +396,8 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     }
   } else if (Q4 && warp >= DQ_WARP0) {
     // --------------------------------------------- 4-bit dequantisation --
-    // 128 threads fill the B half of every stage: 256 (row, group) units of
-    // 64 weights per K step, 2 per thread, read from global memory (words,
+    // 256 threads fill the B half of every stage: 256 (row, group) units of
+    // 64 weights per K step, one per thread, read from global memory (words,
     // scale, bias), dequantised to fp16 and written in the 128-byte-swizzled
     // layout the TMA would produce (16-byte chunk c of row r at c ^ (r & 7)).
     const int dq = threadIdx.x - DQ_WARP0 * 32;
@@ -434,22 +444,18 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       const TileCoord tc = tile_coord<MODE>(a, t);
       if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
       const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
-      Unit c0 = load(tc, kb, dq), c1 = load(tc, kb, dq + 128);
+      Unit c0 = load(tc, kb, dq);
       for (int kk = 0; kk < nks; ++kk) {
-        Unit n0, n1;
-        if (kk + 1 < nks) {
-          n0 = load(tc, kb + kk + 1, dq);
-          n1 = load(tc, kb + kk + 1, dq + 128);
-        }
+        Unit n0;
+        if (kk + 1 < nks) n0 = load(tc, kb + kk + 1, dq);
         if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
           ok = false;
           break;
         }
         uint8_t* sB = base + stage * STAGE_BYTES + A_BYTES;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const Unit& x = h == 0 ? c0 : c1;
-          const int u = dq + h * 128;
+        {
+          const Unit& x = c0;
+          const int u = dq;
           int v, g, off;
           locate(tc, kb + kk, u, v, g, off);
           const int r = MODE == Mode::kDh ? (u & 63) : u;
@@ -472,7 +478,6 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           phase ^= 1u;
         }
         c0 = n0;
-        c1 = n1;
       }
     }
     if (!ok) {

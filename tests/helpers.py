@@ -19,23 +19,7 @@ TOL_DH = 1e-2
 
 def upload(wl: S.Workload, device="cuda"):
     """Device tensors (H, head, labels) of a workload."""
-    if wl.dtype == "bf16":
-        H = torch.from_numpy(wl.H_bits.view(np.int16)).to(device).view(torch.bfloat16)
-    else:
-        H = torch.from_numpy(wl.H).to(device)
-    if wl.wformat == "q4g64":
-        head = cce.Head(
-            w=torch.from_numpy(wl.q_packed.view(np.int32)).to(device), V=wl.V, D=wl.D,
-            fmt=cce.CCE_W_AFFINE_Q4_G64,
-            scales=torch.from_numpy(wl.q_scales.view(np.int16)).to(device).view(torch.bfloat16),
-            biases=torch.from_numpy(wl.q_biases.view(np.int16)).to(device).view(torch.bfloat16))
-    elif wl.dtype == "bf16":
-        head = cce.Head(w=torch.from_numpy(wl.W_bits.view(np.int16)).to(device).view(torch.bfloat16),
-                        V=wl.V, D=wl.D)
-    else:
-        head = cce.Head(w=torch.from_numpy(wl.W).to(device), V=wl.V, D=wl.D)
-    labels = torch.from_numpy(wl.labels).to(device)
-    return H, head, labels
+    return cce.upload_workload(wl, device)
 
 
 def oracle_W(wl: S.Workload) -> np.ndarray:
