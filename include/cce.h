@@ -160,6 +160,36 @@ cce_status orpo_grad_coeffs(const float* logp, const int32_t* labels,
                             size_t ws_bytes, cce_stream_t stream);
 
 /*
+ * Objective siblings on the same log-prob engine (Training design §8.3
+ * "Objective variants"; the UltraFeedback research notes §6.1-6.3):
+ *   CCE_OBJ_ORPO        the ORPO loss above (lambda, sft_scope; beta, gamma
+ *                       unused)
+ *   CCE_OBJ_SIMPO       L = -log sigmoid(beta (lw - lr) - gamma), no NLL term
+ *   CCE_OBJ_ORPO_MARGIN L = NLL + lambda * [-log sigmoid(beta (lw - lr) - gamma)]
+ *                       (ORPO's NLL anchor with SimPO's target margin)
+ * For the SimPO kinds out8 holds L, NLL, the SimPO term, lw, lr, pm,
+ * u = beta (lw - lr) - gamma, sigmoid(u); the cotangent follows by the chain
+ * rule (d/du softplus(-u) = sigmoid(u) - 1).  Host struct, read during the
+ * call.  lambda >= 0, beta >= 0, gamma finite.
+ */
+typedef enum { CCE_OBJ_ORPO = 0, CCE_OBJ_SIMPO = 1, CCE_OBJ_ORPO_MARGIN = 2 } cce_objective_kind;
+typedef struct {
+  cce_objective_kind kind;
+  double lambda, beta, gamma;
+  int sft_scope;
+} cce_objective;
+
+cce_status pref_loss_from_logps(const float* logp, const int32_t* labels,
+                                int64_t M, const cce_layout* layout,
+                                const cce_objective* obj, double* out8,
+                                void* ws, size_t ws_bytes,
+                                cce_stream_t stream);
+cce_status pref_grad_coeffs(const float* logp, const int32_t* labels,
+                            int64_t M, const cce_layout* layout,
+                            const cce_objective* obj, float* coeff, void* ws,
+                            size_t ws_bytes, cce_stream_t stream);
+
+/*
  * Backward of the head (ORPO design 0.0.6, fused-head spec "Backward
  * (recompute vocab tiles from the saved LSE)"; Training design §5.1):
  *   dH[m] = coeff[m] * sum_v (onehot(y_m)_v - p_mv) W[v],

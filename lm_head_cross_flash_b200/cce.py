@@ -44,6 +44,14 @@ class _Head(ctypes.Structure):
                 ("biases", ctypes.c_void_p)]
 
 
+class _Objective(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("lam", ctypes.c_double), ("beta", ctypes.c_double),
+                ("gamma", ctypes.c_double), ("sft_scope", ctypes.c_int)]
+
+
+OBJECTIVES = {"orpo": 0, "simpo": 1, "orpo_margin": 2}
+
+
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "prompt_begin", "prompt_end", "chosen_begin", "chosen_end",
@@ -75,6 +83,14 @@ _SIGS = {
     "cce_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "cce_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "pref_loss_from_logps": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                            ctypes.POINTER(_Layout), ctypes.POINTER(_Objective),
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                            ctypes.c_void_p]),
+    "pref_grad_coeffs": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.POINTER(_Layout), ctypes.POINTER(_Objective),
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]),
     "cce_profile_enable": (None, [ctypes.c_int]),
     "cce_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_longlong), ctypes.c_int]),
@@ -307,3 +323,26 @@ def upload_workload(wl, device="cuda"):
         head = Head(w=torch.from_numpy(wl.W).to(device), V=wl.V, D=wl.D)
     labels = torch.from_numpy(wl.labels).to(device)
     return H, head, labels
+
+
+def _objective(kind, lam, beta, gamma, sft_scope):
+    return _Objective(OBJECTIVES.get(kind, kind), float(lam), float(beta), float(gamma),
+                      SCOPE.get(sft_scope, sft_scope))
+
+
+def pref_loss_from_logps(logp, labels, layout, kind, lam, beta, gamma, sft_scope, out8, ws,
+                         stream=None):
+    st = lib().pref_loss_from_logps(_p(logp), _p(labels), logp.shape[0],
+                                    ctypes.byref(_layout(layout)),
+                                    ctypes.byref(_objective(kind, lam, beta, gamma, sft_scope)),
+                                    _p(out8), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "pref_loss_from_logps")
+
+
+def pref_grad_coeffs(logp, labels, layout, kind, lam, beta, gamma, sft_scope, coeff, ws,
+                     stream=None):
+    st = lib().pref_grad_coeffs(_p(logp), _p(labels), logp.shape[0],
+                                ctypes.byref(_layout(layout)),
+                                ctypes.byref(_objective(kind, lam, beta, gamma, sft_scope)),
+                                _p(coeff), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "pref_grad_coeffs")

@@ -58,6 +58,8 @@ struct OrpoArgs {
   double lambda;
   int scope;                       // 0 full, 1 response
   int want_coeff;
+  int kind;                        // 0 ORPO, 1 SimPO, 2 ORPO + SimPO margin
+  double beta, gamma;              // SimPO scale and target margin
 };
 
 // log(1 - e^x), x < 0: two-branch form (Maechler 2012), fp64.
@@ -116,11 +118,33 @@ __global__ void __launch_bounds__(1024) orpo_kernel(
     }
     const double lw = ok ? sC / nC : qnan;
     const double lr = ok ? sR / nR : qnan;
-    if (ok && !(lw < 0.0 && lr < 0.0)) {
+    if (ok && o.kind == 0 && !(lw < 0.0 && lr < 0.0)) {
       set_status(status, ST_DOMAIN);
       ok = false;
     }
-    if (ok) {
+    if (ok && o.kind != 0) {
+      // SimPO term softplus(-u), u = beta (lw - lr) - gamma; ORPO + margin
+      // adds it, weighted by lambda, to the NLL term.
+      const double pm = nP > 0.0 ? sP / nP : 0.0;
+      const double nll = o.scope == 0 ? -(sP + sC) / (nP + nC) : -lw;
+      const double u = o.beta * (lw - lr) - o.gamma;
+      const double term = softplus_d(-u);
+      const double sig = u >= 0.0 ? 1.0 / (1.0 + exp(-u)) : exp(u) / (1.0 + exp(u));
+      const double w = o.kind == 1 ? 1.0 : o.lambda;
+      res[0] = o.kind == 1 ? term : nll + o.lambda * term;
+      res[1] = nll;
+      res[2] = term;
+      res[3] = lw;
+      res[4] = lr;
+      res[5] = pm;
+      res[6] = u;
+      res[7] = sig;
+      const double d = w * (sig - 1.0) * o.beta;
+      const double sNll = o.kind == 1 ? 0.0 : (o.scope == 0 ? -1.0 / (nP + nC) : -1.0 / nC);
+      cP = (o.kind == 1 || o.scope == 1) ? 0.0 : sNll;
+      cC = d / nC + sNll;
+      cR = -d / nR;
+    } else if (ok) {
       const double pm = nP > 0.0 ? sP / nP : 0.0;
       const double nll = o.scope == 0 ? -(sP + sC) / (nP + nC) : -lw;
       const double z = (lw - lr) - (log1mexp_d(lw) - log1mexp_d(lr));

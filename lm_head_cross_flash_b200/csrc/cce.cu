@@ -507,10 +507,13 @@ static cce_status check_layout(const cce_layout* L, int64_t M) {
 static cce_status orpo_common(const float* logp, const int32_t* labels, int64_t M,
                               const cce_layout* layout, double lambda, int scope,
                               double* out8, float* coeff, void* ws, size_t ws_bytes,
-                              cce_stream_t stream) {
+                              cce_stream_t stream, int kind = 0, double beta = 1.0,
+                              double gamma = 0.0) {
   if (logp == nullptr || labels == nullptr || ws == nullptr) return CCE_ERR_INVALID_ARGUMENT;
   if (M <= 0 || M > (int64_t(1) << 31)) return CCE_ERR_INVALID_ARGUMENT;
   if (!(lambda >= 0.0) || lambda > 1e30) return CCE_ERR_INVALID_ARGUMENT;
+  if (kind < 0 || kind > 2 || !(beta >= 0.0) || beta > 1e30 || !(std::fabs(gamma) <= 1e30))
+    return CCE_ERR_INVALID_ARGUMENT;
   if (scope != CCE_SCOPE_FULL && scope != CCE_SCOPE_RESPONSE) return CCE_ERR_INVALID_ARGUMENT;
   if (ws_bytes < kStatusBytes || !aligned16(ws)) return CCE_ERR_WORKSPACE_TOO_SMALL;
   cce_status s = check_layout(layout, M);
@@ -525,6 +528,9 @@ static cce_status orpo_common(const float* logp, const int32_t* labels, int64_t 
   o.lambda = lambda;
   o.scope = scope;
   o.want_coeff = coeff != nullptr;
+  o.kind = kind;
+  o.beta = beta;
+  o.gamma = gamma;
   {
     ProfScope ps(PK_ORPO, reinterpret_cast<cudaStream_t>(stream));
     orpo_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
@@ -548,6 +554,33 @@ cce_status orpo_grad_coeffs(const float* logp, const int32_t* labels, int64_t M,
   if (coeff == nullptr) return CCE_ERR_INVALID_ARGUMENT;
   return orpo_common(logp, labels, M, layout, lambda, sft_scope, nullptr, coeff, ws,
                      ws_bytes, stream);
+}
+
+static cce_status objective_args(const cce_objective* obj) {
+  if (obj == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  if (obj->kind != CCE_OBJ_ORPO && obj->kind != CCE_OBJ_SIMPO && obj->kind != CCE_OBJ_ORPO_MARGIN)
+    return CCE_ERR_INVALID_ARGUMENT;
+  return CCE_OK;
+}
+
+cce_status pref_loss_from_logps(const float* logp, const int32_t* labels, int64_t M,
+                                const cce_layout* layout, const cce_objective* obj,
+                                double* out8, void* ws, size_t ws_bytes, cce_stream_t stream) {
+  cce_status s = objective_args(obj);
+  if (s != CCE_OK) return s;
+  if (out8 == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  return orpo_common(logp, labels, M, layout, obj->lambda, obj->sft_scope, out8, nullptr, ws,
+                     ws_bytes, stream, int(obj->kind), obj->beta, obj->gamma);
+}
+
+cce_status pref_grad_coeffs(const float* logp, const int32_t* labels, int64_t M,
+                            const cce_layout* layout, const cce_objective* obj, float* coeff,
+                            void* ws, size_t ws_bytes, cce_stream_t stream) {
+  cce_status s = objective_args(obj);
+  if (s != CCE_OK) return s;
+  if (coeff == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  return orpo_common(logp, labels, M, layout, obj->lambda, obj->sft_scope, nullptr, coeff, ws,
+                     ws_bytes, stream, int(obj->kind), obj->beta, obj->gamma);
 }
 
 cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,

@@ -346,3 +346,83 @@ def dequant_affine_q4(packed, scales, biases, group: int = 64) -> np.ndarray:
     s = np.repeat(bf16_bits_to_f64(scales), group, axis=1)
     b = np.repeat(bf16_bits_to_f64(biases), group, axis=1)
     return q * s + b
+
+
+# ----------------------------------------------------------------------------
+# objective siblings on the same log-prob engine
+# ----------------------------------------------------------------------------
+#
+# Training design §8.3 ("Objective variants and data") lists SimPO as a cheap
+# sibling once the shared logp engine exists, and the UltraFeedback research
+# notes (§6.1-6.3) define:
+#   SimPO:            L = -log sigmoid(beta * (lw - lr) - gamma)   (no NLL term)
+#   ORPO + margin:    L = NLL(chosen) + lambda * [-log sigmoid(beta*(lw-lr) - gamma)]
+# (§6.2, the "gamma-hybrid", equal to the "SFT + SimPO single-stage" of §6.3).
+# The design record writes the SimPO term as softplus(-beta((lw-lr) - gamma)),
+# with gamma inside the beta product; the notes and the published SimPO loss
+# (Meng et al. 2024) subtract gamma after scaling.  The latter is used here.
+
+OBJECTIVES = ("orpo", "simpo", "orpo_margin")
+
+
+def simpo_margin(lw: float, lr: float, beta: float, gamma: float) -> float:
+    """u = beta * (lw - lr) - gamma; the SimPO term is softplus(-u)."""
+    return beta * (lw - lr) - gamma
+
+
+def pref_loss_from_logps(logp, labels, layout: Layout, kind: str, lam: float,
+                         beta: float = 1.0, gamma: float = 0.0,
+                         sft_scope: str = "full") -> OrpoOut:
+    """Loss of one objective from per-row log-probs.
+
+    ``orpo`` is ``orpo_loss_from_logps``.  For ``simpo`` and ``orpo_margin``
+    the returned fields are: loss, nll (reported, added only by
+    ``orpo_margin``), l_or = the SimPO term softplus(-u), lw, lr, pm, z = u,
+    sig = sigmoid(u).
+    """
+    if kind == "orpo":
+        return orpo_loss_from_logps(logp, labels, layout, lam, sft_scope)
+    if kind not in OBJECTIVES:
+        raise ValueError(kind)
+    logp = _as64(logp)
+    labels = np.asarray(labels)
+    L = layout
+    nP, sP = _segment_stats(logp, labels, L.prompt_begin, L.prompt_end)
+    nC, sC = _segment_stats(logp, labels, L.chosen_begin, L.chosen_end)
+    nR, sR = _segment_stats(logp, labels, L.rejected_begin, L.rejected_end)
+    if nC == 0 or nR == 0:
+        raise ValueError("chosen and rejected need at least one labelled row")
+    lw, lr = sC / nC, sR / nR
+    pm = sP / nP if nP > 0 else 0.0
+    nll = -(sP + sC) / (nP + nC) if sft_scope == "full" else -lw
+    u = simpo_margin(lw, lr, beta, gamma)
+    term = softplus(-u)
+    loss = term if kind == "simpo" else nll + lam * term
+    return OrpoOut(loss=loss, nll=nll, l_or=term, lw=lw, lr=lr, pm=pm, z=u,
+                   sig=sigmoid(u), n_prompt=nP, n_chosen=nC, n_rejected=nR)
+
+
+def pref_grad_coeffs(logp, labels, layout: Layout, kind: str, lam: float,
+                     beta: float = 1.0, gamma: float = 0.0,
+                     sft_scope: str = "full") -> np.ndarray:
+    """dL/dlogp of one objective (chain rule: d softplus(-u)/du = sigmoid(u) - 1,
+    du/dlw = beta, du/dlr = -beta, dlw/dlogp = 1/n_chosen on chosen rows)."""
+    if kind == "orpo":
+        return orpo_grad_coeffs(logp, labels, layout, lam, sft_scope)
+    labels = np.asarray(labels)
+    o = pref_loss_from_logps(logp, labels, layout, kind, lam, beta, gamma, sft_scope)
+    L = layout
+    g = np.zeros(labels.shape[0])
+    w = 1.0 if kind == "simpo" else lam
+    d = w * (o.sig - 1.0) * beta
+    if kind == "simpo":
+        s_c = s_p = 0.0
+    elif sft_scope == "full":
+        s_c = s_p = -1.0 / (o.n_prompt + o.n_chosen)
+    else:
+        s_c, s_p = -1.0 / o.n_chosen, 0.0
+    g[L.prompt_begin:L.prompt_end] = s_p
+    g[L.chosen_begin:L.chosen_end] = d / o.n_chosen + s_c
+    g[L.rejected_begin:L.rejected_end] = -d / o.n_rejected
+    g[labels < 0] = 0.0
+    return g

@@ -81,3 +81,28 @@ def test_long_pair_sampled_rows(cfg):
                             buf.ws)
         torch.cuda.synchronize()
         assert torch.equal(d2, buf.dH)
+
+
+def test_residency_no_logits_buffer_and_no_hidden_allocation():
+    """A whole pass at the long-pair shape allocates nothing on the device
+    (the library never calls cudaMalloc), and every buffer the caller holds
+    is far smaller than the [M, V] logits."""
+    wl = S.make_workload(2)
+    H, head, labels = upload(wl)
+    buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head)
+    args = (H, head, labels, wl.layout_tuple, wl.lam, wl.scope, 0.0, False, buf)
+    cce.orpo_head_pass(*args)          # first call: module load, attributes
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    torch.cuda.reset_peak_memory_stats()
+    before = torch.cuda.memory_allocated()
+    cce.orpo_head_pass(*args)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.max_memory_allocated() == before
+    held = sum(t.numel() * t.element_size() for t in
+               (buf.logp, buf.lse, buf.tgt, buf.blockmax, buf.out8, buf.coeff, buf.dH, buf.ws))
+    logits = wl.M * wl.V * 2           # even bf16 logits
+    assert held < logits / 8, (held, logits)
+    assert cce.cce_device_status(buf.ws) == 0

@@ -221,3 +221,29 @@ def test_synchronous_argument_errors():
     with pytest.raises(cce.CCEError) as e:
         cce.cce_forward(H, bad, labels, logp, lse, None, None, ws)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("kind", ["orpo", "simpo", "orpo_margin"])
+def test_objective_siblings_match_oracle(kind):
+    """ORPO, SimPO and ORPO + SimPO margin on seeded log-probs (full size)."""
+    P, Rc, Rr = 1024, 3584, 3584
+    M = P + Rc + Rr
+    lp = S.random_logps(M, seed=5, scale=3.0)
+    y = np.random.default_rng(6).integers(-1, 1000, size=M).astype(np.int32)
+    L = O.Layout.contiguous(P, Rc, Rr)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    out8 = torch.empty(8, dtype=torch.float64, device="cuda")
+    coeff = torch.empty(M, device="cuda")
+    lpt, yt = torch.from_numpy(lp).cuda(), torch.from_numpy(y).cuda()
+    for scope in ("full", "response"):
+        for lam, beta, gamma in ((0.1, 2.0, 0.5), (1.0, 0.5, 0.0)):
+            cce.pref_loss_from_logps(lpt, yt, dataclasses.astuple(L), kind, lam, beta, gamma,
+                                     scope, out8, ws)
+            cce.pref_grad_coeffs(lpt, yt, dataclasses.astuple(L), kind, lam, beta, gamma,
+                                 scope, coeff, ws)
+            torch.cuda.synchronize()
+            assert cce.cce_device_status(ws) == 0
+            o = O.pref_loss_from_logps(lp, y, L, kind, lam, beta, gamma, scope)
+            assert np.allclose(out8.cpu().numpy(), np.array(o.as8()), rtol=1e-12, atol=1e-14)
+            g = O.pref_grad_coeffs(lp, y, L, kind, lam, beta, gamma, scope)
+            assert np.allclose(coeff.cpu().numpy(), g, rtol=1e-6, atol=1e-12)

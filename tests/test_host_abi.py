@@ -132,3 +132,15 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(cce, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         cce.lib()
+
+
+def test_objective_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    a = P(4096)
+    lay = ctypes.byref(cce._Layout(0, 5, 5, 10, 10, 20))
+    for obj in [cce._Objective(3, 0.1, 1.0, 0.0, 0), cce._Objective(1, 0.1, -1.0, 0.0, 0),
+                cce._Objective(1, 0.1, 1.0, float("inf"), 0), cce._Objective(2, -0.1, 1.0, 0.0, 0),
+                cce._Objective(1, 0.1, 1.0, 0.0, 5)]:
+        assert lib.pref_loss_from_logps(a, a, 20, lay, ctypes.byref(obj), a, a, 4096, None) == 1
+        assert lib.pref_grad_coeffs(a, a, 20, lay, ctypes.byref(obj), a, a, 4096, None) == 1
+    assert lib.pref_loss_from_logps(a, a, 20, lay, None, a, a, 4096, None) == 1

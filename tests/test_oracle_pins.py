@@ -345,3 +345,50 @@ def test_dequant_groups_select_their_own_scale():
     bi = np.array([[0x0000, 0x3F80]] * V, dtype=np.uint16)      # 0.0 | 1.0
     w = O.dequant_affine_q4(words, sc, bi)
     assert np.all(w[:, :64] == 1.0) and np.all(w[:, 64:] == 3.0)
+
+
+# --------------------------------------------------------------------------
+# objective siblings (SimPO, ORPO + margin)
+# --------------------------------------------------------------------------
+
+def test_simpo_equal_means_closed_form():
+    _, _, y, L = tiny_case(P=4, Rc=3, Rr=5, seed=2)
+    logp = np.full(len(y), -1.7)
+    for gamma in (0.0, 0.5, 2.0):
+        o = O.pref_loss_from_logps(logp, y, L, "simpo", 0.1, beta=2.5, gamma=gamma)
+        assert o.loss == pytest.approx(math.log1p(math.exp(gamma)), rel=1e-14)
+        h = O.pref_loss_from_logps(logp, y, L, "orpo_margin", 0.3, beta=2.5, gamma=gamma)
+        assert h.loss == pytest.approx(1.7 + 0.3 * math.log1p(math.exp(gamma)), rel=1e-14)
+
+
+def test_simpo_against_published_form():
+    _, _, y, L = tiny_case(P=4, Rc=3, Rr=5, seed=3)
+    g = np.random.default_rng(4)
+    logp = -g.random(len(y)) * 3 - 0.1
+    logp[y < 0] = 0.0
+    o = O.pref_loss_from_logps(logp, y, L, "simpo", 0.0, beta=2.0, gamma=0.7)
+    lw = logp[L.chosen_begin:L.chosen_end][y[L.chosen_begin:L.chosen_end] >= 0].mean()
+    lr = logp[L.rejected_begin:L.rejected_end][y[L.rejected_begin:L.rejected_end] >= 0].mean()
+    assert o.loss == pytest.approx(-sps.log_expit(2.0 * (lw - lr) - 0.7), rel=1e-13)
+
+
+@pytest.mark.parametrize("kind", ["simpo", "orpo_margin"])
+@pytest.mark.parametrize("scope", ["full", "response"])
+def test_sibling_coeffs_are_dL_dlogp(kind, scope):
+    _, _, y, L = tiny_case(P=4, Rc=3, Rr=5, seed=1, ignore=(0, 5))
+    g = np.random.default_rng(8)
+    logp = -g.random(len(y)) * 4 - 0.05
+    logp[y < 0] = 0.0
+    args = dict(lam=0.4, beta=1.7, gamma=0.3, sft_scope=scope)
+    coef = O.pref_grad_coeffs(logp, y, L, kind, **args)
+    h = 1e-6
+    for m in range(len(y)):
+        if y[m] < 0:
+            assert coef[m] == 0.0
+            continue
+        lp, lm = logp.copy(), logp.copy()
+        lp[m] += h
+        lm[m] -= h
+        fd = (O.pref_loss_from_logps(lp, y, L, kind, **args).loss
+              - O.pref_loss_from_logps(lm, y, L, kind, **args).loss) / (2 * h)
+        assert coef[m] == pytest.approx(fd, rel=1e-6, abs=1e-9)
