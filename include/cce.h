@@ -67,11 +67,16 @@ typedef enum {
 typedef enum { CCE_F32 = 0, CCE_BF16 = 1 } cce_dtype;
 
 typedef enum {
-  CCE_W_DENSE = 0,        /* w: [V, D] row-major, dtype f32 or bf16           */
-  CCE_W_AFFINE_Q4_G64 = 1 /* w: uint32 [V, D/8]; element 8k+j of a row is bits
-                             4j..4j+3 of word k (low nibble first);
-                             scales, biases: bf16 [V, D/64]; the weight is
-                             q*scale + bias (Training design §5.6).           */
+  CCE_W_DENSE = 0,         /* w: [V, D] row-major, dtype f32 or bf16          */
+  CCE_W_AFFINE_Q4_G64 = 1, /* w: uint32 [V, D/8]; element 8k+j of a row is bits
+                              4j..4j+3 of word k (low nibble first);
+                              scales, biases: bf16 [V, D/64]; the weight is
+                              q*scale + bias (Training design §5.6).          */
+  CCE_W_AFFINE_Q8_G64 = 2  /* w: uint32 [V, D/4]; element 4k+j of a row is byte
+                              j of word k (low byte first); scales, biases as
+                              for the 4-bit head.  Quantised heads compute in
+                              fp16 (H converted once; weights dequantised
+                              in-kernel and rounded once to fp16).           */
 } cce_wformat;
 
 /* The frozen head (host struct; device pointers inside). */
@@ -82,6 +87,9 @@ typedef struct {
   const void* w;
   const void* scales;    /* Q4 only, else NULL */
   const void* biases;    /* Q4 only, else NULL */
+  float softcap;         /* > 0: logits are softcap * tanh(h.W_v / softcap)
+                            (Gemma-style final-logit capping; the backward
+                            applies 1 - tanh^2); 0 = none */
 } cce_head;
 
 /* Disjoint head-row ranges [begin, end) of one ORPO pair (host struct).

@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcce.so")
 
 CCE_F32, CCE_BF16 = 0, 1
-CCE_W_DENSE, CCE_W_AFFINE_Q4_G64 = 0, 1
+CCE_W_DENSE, CCE_W_AFFINE_Q4_G64, CCE_W_AFFINE_Q8_G64 = 0, 1, 2
 SCOPE = {"full": 0, "response": 1}
 VOCAB_BLOCK = 256
 
@@ -41,7 +41,7 @@ class _Head(ctypes.Structure):
     _fields_ = [("format", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("V", ctypes.c_int64), ("D", ctypes.c_int64),
                 ("w", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("biases", ctypes.c_void_p)]
+                ("biases", ctypes.c_void_p), ("softcap", ctypes.c_float)]
 
 
 class _Objective(ctypes.Structure):
@@ -174,17 +174,19 @@ class Head:
     fmt: int = CCE_W_DENSE
     scales: torch.Tensor | None = None
     biases: torch.Tensor | None = None
+    softcap: float = 0.0
 
     @property
     def dtype(self) -> int:
-        if self.fmt == CCE_W_AFFINE_Q4_G64:
+        if self.fmt in (CCE_W_AFFINE_Q4_G64, CCE_W_AFFINE_Q8_G64):
             return CCE_BF16
         return CCE_F32 if self.w.dtype == torch.float32 else CCE_BF16
 
     def c(self) -> _Head:
         return _Head(self.fmt, self.dtype, self.V, self.D, self.w.data_ptr(),
                      None if self.scales is None else self.scales.data_ptr(),
-                     None if self.biases is None else self.biases.data_ptr())
+                     None if self.biases is None else self.biases.data_ptr(),
+                     float(self.softcap))
 
 
 def h_dtype(H: torch.Tensor) -> int:
@@ -311,9 +313,9 @@ def upload_workload(wl, device="cuda"):
         H = torch.from_numpy(wl.H_bits.view(np.int16)).to(device).view(torch.bfloat16)
     else:
         H = torch.from_numpy(wl.H).to(device)
-    if wl.wformat == "q4g64":
+    if wl.wformat in ("q4g64", "q8g64"):
         head = Head(w=torch.from_numpy(wl.q_packed.view(np.int32)).to(device), V=wl.V, D=wl.D,
-                    fmt=CCE_W_AFFINE_Q4_G64,
+                    fmt=CCE_W_AFFINE_Q4_G64 if wl.wformat == "q4g64" else CCE_W_AFFINE_Q8_G64,
                     scales=torch.from_numpy(wl.q_scales.view(np.int16)).to(device).view(torch.bfloat16),
                     biases=torch.from_numpy(wl.q_biases.view(np.int16)).to(device).view(torch.bfloat16))
     elif wl.dtype == "bf16":

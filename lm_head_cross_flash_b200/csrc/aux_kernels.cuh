@@ -256,9 +256,10 @@ __global__ void split_f32_kernel(const float* __restrict__ src, int64_t rows,
   }
 }
 
-// fp16 copy of bf16 rows [rows, D] for a 4-bit head, with element e of every
-// group of 8 columns stored at position q4_pos(e) (the order in which the
-// dequantiser lays out the weights along K).  n8 = rows*D/8.
+// fp16 copy of bf16 rows [rows, D] for a quantised head, with element e of
+// every block of 8 columns stored at position qpos<QB>(e) (the order in which
+// the dequantiser lays out the weights along K).  n8 = rows*D/8.
+template <int QB>
 __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
                                      uint4* __restrict__ dst) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
@@ -269,7 +270,7 @@ __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint32_t bits = (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-      h[q4_pos(e)] = __float2half_rn(__uint_as_float(bits << 16));
+      h[qpos<QB>(e)] = __float2half_rn(__uint_as_float(bits << 16));
     }
     dst[i] = *reinterpret_cast<const uint4*>(h);
   }

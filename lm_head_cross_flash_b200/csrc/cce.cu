@@ -158,12 +158,14 @@ cce_status device_info(int* sms) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return CCE_ERR_CUDA;
     const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-    if (cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse, false>, attr, smem_bytes<Mode::kLse>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad, false>, attr, smem_bytes<Mode::kGrad>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh, false>, attr, smem_bytes<Mode::kDh>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kLse, true>, attr, smem_bytes<Mode::kLse>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kGrad, true>, attr, smem_bytes<Mode::kGrad>()) != cudaSuccess ||
-        cudaFuncSetAttribute(cce_tc_kernel<Mode::kDh, true>, attr, smem_bytes<Mode::kDh>()) != cudaSuccess)
+    bool ok = true;
+#define CCE_SET_SMEM(MODE, QB) \
+    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, QB>, attr, smem_bytes<MODE>()) == cudaSuccess;
+    CCE_SET_SMEM(Mode::kLse, 0) CCE_SET_SMEM(Mode::kGrad, 0) CCE_SET_SMEM(Mode::kDh, 0)
+    CCE_SET_SMEM(Mode::kLse, 4) CCE_SET_SMEM(Mode::kGrad, 4) CCE_SET_SMEM(Mode::kDh, 4)
+    CCE_SET_SMEM(Mode::kLse, 8) CCE_SET_SMEM(Mode::kGrad, 8) CCE_SET_SMEM(Mode::kDh, 8)
+#undef CCE_SET_SMEM
+    if (!ok)
       return CCE_ERR_CUDA;
     d.attrs = true;
   }
@@ -180,12 +182,13 @@ cce_status check_head(const cce_head* W, cce_dtype h_dtype) {
     return CCE_ERR_INVALID_ARGUMENT;
   if (W->V > (int64_t(1) << 30) || W->D > (int64_t(1) << 16)) return CCE_ERR_UNSUPPORTED;
   if (W->D % 64 != 0) return CCE_ERR_UNSUPPORTED;
+  if (!(W->softcap >= 0.f) || W->softcap > 1e30f) return CCE_ERR_INVALID_ARGUMENT;
   if (W->format == CCE_W_DENSE) {
     if (W->dtype != CCE_F32 && W->dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
     if (W->dtype != h_dtype) return CCE_ERR_UNSUPPORTED;
     return CCE_OK;
   }
-  if (W->format == CCE_W_AFFINE_Q4_G64) {
+  if (W->format == CCE_W_AFFINE_Q4_G64 || W->format == CCE_W_AFFINE_Q8_G64) {
     if (W->dtype != CCE_BF16 || W->scales == nullptr || W->biases == nullptr ||
         (reinterpret_cast<uintptr_t>(W->scales) & 1u) || (reinterpret_cast<uintptr_t>(W->biases) & 1u))
       return CCE_ERR_INVALID_ARGUMENT;
@@ -262,7 +265,7 @@ Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ks
   if (h == CCE_F32) {
     L.hs = s; s += align_up(size_t(M) * 3 * W->D * 2);
     L.ws = s; s += align_up(size_t(W->V) * 3 * W->D * 2);
-  } else if (W->format == CCE_W_AFFINE_Q4_G64) {
+  } else if (W->format != CCE_W_DENSE) {
     L.hs = s; s += align_up(size_t(M) * W->D * 2);  // fp16, K-permuted rows
   }
   L.vc = vc;
@@ -310,23 +313,27 @@ int grid_for(int64_t tiles, int sms) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, sms)));
 }
 
-// Launch one tensor-core step; a 4-bit head adds the dequantisation warps.
+// Launch one tensor-core step; a quantised head adds the dequantisation
+// warps.
 template <Mode MODE>
-void launch_tc(bool q4, int64_t tiles, int sms, cudaStream_t st, const CUtensorMap& ma,
+void launch_tc(int qb, int64_t tiles, int sms, cudaStream_t st, const CUtensorMap& ma,
                const CUtensorMap& mb, const CUtensorMap& mc, const CUtensorMap& mc2,
                const TileArgs& args) {
-  if (q4)
-    cce_tc_kernel<MODE, true><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
+  if (qb == 4)
+    cce_tc_kernel<MODE, 4><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
+        ma, mb, mc, mc2, args);
+  else if (qb == 8)
+    cce_tc_kernel<MODE, 8><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
         ma, mb, mc, mc2, args);
   else
-    cce_tc_kernel<MODE, false><<<grid_for(tiles, sms), NUM_THREADS, smem_bytes<MODE>(), st>>>(
+    cce_tc_kernel<MODE, 0><<<grid_for(tiles, sms), NUM_THREADS, smem_bytes<MODE>(), st>>>(
         ma, mb, mc, mc2, args);
 }
 
 // Operands of the tensor-core GEMMs for one problem: 16-bit A (head rows)
 // and B (head) with their K extents.
 struct Operands {
-  bool q4;         // 4-bit head: B is dequantised in-kernel, A is fp16
+  int qb;          // 4 / 8: quantised head, B is dequantised in-kernel, A is fp16
   const void* a;   // [M, ka] 16-bit
   const void* b;   // [V, kb] 16-bit (dense heads)
   int64_t k;       // contraction length used by the S GEMM
@@ -339,12 +346,15 @@ struct Operands {
 cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_head* W,
                             const Layout& L, void* ws, cudaStream_t st, Operands* op) {
   const int64_t D = W->D;
-  op->q4 = W->format == CCE_W_AFFINE_Q4_G64;
-  if (op->q4) {
+  op->qb = W->format == CCE_W_AFFINE_Q4_G64 ? 4 : W->format == CCE_W_AFFINE_Q8_G64 ? 8 : 0;
+  if (op->qb) {
     uint4* h16 = reinterpret_cast<uint4*>(static_cast<char*>(ws) + L.hs);
     {
       ProfScope ps(PK_SPLIT, st);
-      h_to_f16_perm_kernel<<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+      if (op->qb == 4)
+        h_to_f16_perm_kernel<4><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+      else
+        h_to_f16_perm_kernel<8><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     op->a = h16;
@@ -450,7 +460,7 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
 
   CUtensorMap ma, mb;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
-  if (op.q4) mb = ma;  // unused: B is dequantised in-kernel
+  if (op.qb) mb = ma;  // unused: B is dequantised in-kernel
   else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN)) return CCE_ERR_CUDA;
 
   TileArgs a;
@@ -475,9 +485,11 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.q_scale = static_cast<const uint16_t*>(W->scales);
   a.q_bias = static_cast<const uint16_t*>(W->biases);
   a.group_rt = group_rows(n_rt, op.k);
+  a.softcap = W->softcap;
+  a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
   {
     ProfScope ps(PK_LSE, st);
-    launch_tc<Mode::kLse>(op.q4, n_rt * cols, sms, st, ma, mb, ma, ma, a);
+    launch_tc<Mode::kLse>(op.qb, n_rt * cols, sms, st, ma, mb, ma, ma, a);
   }
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
 
@@ -633,7 +645,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
 
   CUtensorMap ma, mb, mg, mw, mgs, md0, md1;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
-  if (op.q4) {
+  if (op.qb) {
     mb = ma;  // unused: B is dequantised in-kernel
     mw = ma;
   } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN) ||
@@ -682,6 +694,8 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   a.q_scale = static_cast<const uint16_t*>(W->scales);
   a.q_bias = static_cast<const uint16_t*>(W->biases);
   a.group_rt = group_rows(n_rt, op.k);
+  a.softcap = W->softcap;
+  a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
 
   for (int64_t v0 = 0; v0 < V; v0 += vc) {
     const int64_t w = std::min<int64_t>(vc, V - v0);
@@ -705,7 +719,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     }
     {
       ProfScope ps(PK_GRAD, st);
-      launch_tc<Mode::kGrad>(op.q4, n_rt * ct_n, sms, st, ma, mb, mgs, mgs, ag);
+      launch_tc<Mode::kGrad>(op.qb, n_rt * ct_n, sms, st, ma, mb, mgs, mgs, ag);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     // dH (+)= coeff * G' . W[chunk]
@@ -719,7 +733,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ad.first_chunk = v0 == 0 ? 1 : 0;
     {
       ProfScope ps(PK_DH, st);
-      launch_tc<Mode::kDh>(op.q4, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);
+      launch_tc<Mode::kDh>(op.qb, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
@@ -882,11 +896,13 @@ extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_he
   a.wait_ns = g_wait_ns.load();
   a.status = st_word;
   a.group_rt = int(n_rt);
+  a.softcap = W->softcap;
+  a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
   a.labels = labels;
   a.part_m = part_m;
   a.part_s = part_s;
   a.tgt = tgt;
-  cce_tc_kernel<Mode::kLse, false><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
+  cce_tc_kernel<Mode::kLse, 0><<<grid_for(n_rt * cols, sms), NUM_THREADS, SMEM_BYTES, st>>>(
       ma, mb, ma, ma, a);
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   const int rows_per_block = 8;

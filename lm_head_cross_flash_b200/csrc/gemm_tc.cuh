@@ -93,17 +93,48 @@ struct TileArgs {
   int ksplit;      // kDh: the chunk's K range is split in `ksplit` parts
   int first_chunk;
   int group_rt;    // kLse/kGrad: row tiles per raster group
+  float softcap;   // > 0: logits are cap * tanh(s / cap)
+  float inv_cap;
   // 4-bit affine head (group 64): words [V, D/8], scales/biases bf16 [V, D/64]
   const uint32_t* q_w;
   const uint16_t* q_scale;
   const uint16_t* q_bias;
 };
 
-// Position, inside its group of 8, at which the 4-bit dequantiser stores
-// element e of the group: the int4 -> fp16 conversion yields the pairs
-// (e0,e4), (e1,e5), (e2,e6), (e3,e7).  The hidden rows are stored with the
-// same order along K, so every dot product is unchanged.
+// Position, inside its block of 8, at which the dequantiser stores element e
+// of the block.  4-bit: the int4 -> fp16 conversion yields the pairs
+// (e0,e4), (e1,e5), (e2,e6), (e3,e7); 8-bit: the pairs (e0,e2), (e1,e3) of
+// each word.  The hidden rows are stored with the same order along K, so
+// every dot product is unchanged.
 __host__ __device__ constexpr int q4_pos(int e) { return e < 4 ? 2 * e : 2 * e - 7; }
+__host__ __device__ constexpr int q8_pos(int e) {
+  return (e & 4) + ((e & 3) == 1 ? 2 : (e & 3) == 2 ? 1 : (e & 3));
+}
+template <int QB>
+__host__ __device__ constexpr int qpos(int e) { return QB == 8 ? q8_pos(e) : q4_pos(e); }
+
+// 8-bit variant: 16 packed words (element 4c+j = byte j of word c).
+__device__ __forceinline__ void dequant_group64_q8(const uint4 (&wv)[4], uint16_t sbits,
+                                                   uint16_t bbits, uint4 (&out)[8]) {
+  const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
+  const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bbits) << 16));
+  const __half2 k1024 = __float2half2_rn(1024.f);
+  const uint32_t words[16] = {wv[0].x, wv[0].y, wv[0].z, wv[0].w, wv[1].x, wv[1].y,
+                              wv[1].z, wv[1].w, wv[2].x, wv[2].y, wv[2].z, wv[2].w,
+                              wv[3].x, wv[3].y, wv[3].z, wv[3].w};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t x = ((words[2 * c + (i >> 1)] >> (8 * (i & 1))) & 0x00FF00FFu) | 0x64006400u;
+      __half2 h = *reinterpret_cast<const __half2*>(&x);
+      h = __hfma2(__hsub2(h, k1024), s2, b2);
+      t[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    out[c] = make_uint4(t[0], t[1], t[2], t[3]);
+  }
+}
 
 // Dequantise the 64 weights of one (row, group): w = q * scale + bias, with
 // q read from 8 packed words (element 8c+j = bits 4j..4j+3 of word c) and
@@ -186,6 +217,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, int fmt) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// tanh(x) from one ex2: t = 2^(2 x log2 e), tanh = (t - 1) / (t + 1); |x| is
+// clamped at 15, where tanh is 1 to fp32 precision.  Absolute error ~1e-7.
+__device__ __forceinline__ float tanh_ex2(float x) {
+  x = fminf(fmaxf(x, -15.f), 15.f);
+  const float t = ex2_approx(x * (2.f * LOG2E));
+  return __fdividef(t - 1.f, t + 1.f);
+}
+
 // Softmax probability of logit s given nl = -lse * log2(e).  The block-skip
 // planner uses the same expression, so its decisions agree with the filter.
 __device__ __forceinline__ float softmax_p(float s, float nl) {
@@ -224,8 +263,8 @@ __device__ __forceinline__ void drain_chunks(uint32_t taddr, int nchunks, F&& f)
   }
 }
 
-template <Mode MODE, bool Q4 = false>
-__global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
+template <Mode MODE, int QB = 0>
+__global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     cce_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                   const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC,
@@ -253,7 +292,7 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], Q4 ? 1 + DQ_WARPS : 1);
+      mbar_init(&full[s], QB ? 1 + DQ_WARPS : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -299,7 +338,7 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           uint8_t* sA = base + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
           const int pass = kk / nks, k = kb + (kk - pass * nks);
-          if (Q4) {
+          if (QB) {
             // B comes from the dequantisation warps.
             mbar_arrive_expect_tx(&full[stage], A_BYTES);
             if (MODE == Mode::kDh)
@@ -394,7 +433,7 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       umma_commit(drain);
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
     }
-  } else if (Q4 && warp >= DQ_WARP0) {
+  } else if (QB && warp >= DQ_WARP0) {
     // --------------------------------------------- 4-bit dequantisation --
     // 256 threads fill the B half of every stage: 256 (row, group) units of
     // 64 weights per K step, one per thread, read from global memory (words,
@@ -405,8 +444,9 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    constexpr int NV = QB == 8 ? 4 : 2;  // 16-byte vectors per (row, group)
     struct Unit {
-      uint4 wa, wb;
+      uint4 w[NV];
       uint16_t sc, bi;
       bool valid;
     };
@@ -429,13 +469,15 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       locate(tc, k, u, v, g, off);
       x.valid = v < a.V && g < gpr;
       if (x.valid) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.q_w + static_cast<size_t>(v) * (a.D / 8) + g * 8);
-        x.wa = __ldg(src);
-        x.wb = __ldg(src + 1);
+        const uint4* src = reinterpret_cast<const uint4*>(
+            a.q_w + static_cast<size_t>(v) * (a.D / (32 / (QB ? QB : 4))) + g * (2 * QB));
+#pragma unroll
+        for (int i = 0; i < NV; ++i) x.w[i] = __ldg(src + i);
         x.sc = __ldg(a.q_scale + static_cast<size_t>(v) * gpr + g);
         x.bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
       } else {
-        x.wa = x.wb = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) x.w[i] = make_uint4(0, 0, 0, 0);
         x.sc = x.bi = 0;
       }
       return x;
@@ -461,7 +503,10 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           const int r = MODE == Mode::kDh ? (u & 63) : u;
           uint4 out[8];
           if (x.valid) {
-            dequant_group64(x.wa, x.wb, x.sc, x.bi, out);
+            if constexpr (QB == 8)
+              dequant_group64_q8(x.w, x.sc, x.bi, out);
+            else
+              dequant_group64(x.w[0], x.w[QB == 8 ? 0 : 1], x.sc, x.bi, out);
           } else {
 #pragma unroll
             for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
@@ -535,29 +580,36 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         drain_chunks(taddr, nchunks, [&](int c, const uint32_t (&r)[32]) {
           const int v0 = vbase + c * 32;
           const int nvalid = min(32, a.V - v0);
+          float x[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] = u2f(r[j]);
+          if (a.softcap > 0.f) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = a.softcap * tanh_ex2(x[j] * a.inv_cap);
+          }
           float cm = -INFINITY;
           float s0 = 0.f, s1 = 0.f;
           if (nvalid == 32) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) cm = fmaxf(cm, u2f(r[j]));
+            for (int j = 0; j < 32; ++j) cm = fmaxf(cm, x[j]);
             const float mn = fmaxf(m_run, cm);
             const float nb = -mn * LOG2E;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              s0 += ex2_approx(fmaf(u2f(r[j]), LOG2E, nb));
-              s1 += ex2_approx(fmaf(u2f(r[j + 1]), LOG2E, nb));
+              s0 += ex2_approx(fmaf(x[j], LOG2E, nb));
+              s1 += ex2_approx(fmaf(x[j + 1], LOG2E, nb));
             }
             s_run = s_run * ex2_approx((m_run - mn) * LOG2E) + (s0 + s1);
             m_run = mn;
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < nvalid) cm = fmaxf(cm, u2f(r[j]));
+              if (j < nvalid) cm = fmaxf(cm, x[j]);
             const float mn = fmaxf(m_run, cm);
             const float nb = -mn * LOG2E;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < nvalid) s0 += ex2_approx(fmaf(u2f(r[j]), LOG2E, nb));
+              if (j < nvalid) s0 += ex2_approx(fmaf(x[j], LOG2E, nb));
             s_run = s_run * ex2_approx((m_run - mn) * LOG2E) + s0;
             m_run = mn;
           }
@@ -567,7 +619,7 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             if (hit) {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (j == tt) tval = u2f(r[j]);
+                if (j == tt) tval = x[j];
               found = true;
             }
             __syncwarp();
@@ -595,7 +647,23 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           const bool slow = (v0 + 32 > a.V) ||
                             __any_sync(0xffffffffu, static_cast<unsigned>(tt) < 32u);
           uint32_t pk[16];
-          if (!slow) {
+          if (a.softcap > 0.f) {
+            // capped logits; each term carries 1 - tanh^2(s / cap)
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float g2[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int v = v0 + j + h;
+                const float th = tanh_ex2(u2f(r[j + h]) * a.inv_cap);
+                float p = softmax_p(a.softcap * th, nl);
+                const bool tgt = (v == y);
+                if (p < eps && !tgt) p = 0.f;
+                g2[h] = v < a.V ? (tgt ? p - 1.f : p) * (1.f - th * th) : 0.f;
+              }
+              pk[j >> 1] = pack2(g2[0], g2[1], a.fmt);
+            }
+          } else if (!slow) {
             if (eps > 0.f) {
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
@@ -662,7 +730,7 @@ __global__ void __launch_bounds__(Q4 ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           for (int i = 0; i < 8; ++i) {
             // accumulator column of output column j (4-bit heads permute K
             // inside groups of 8, so the dH columns come out permuted too)
-            constexpr auto src = [](int j) { return Q4 ? (j & ~7) + q4_pos(j & 7) : j; };
+            constexpr auto src = [](int j) { return QB ? (j & ~7) + qpos<QB>(j & 7) : j; };
             const float4 o =
                 g == 0.f ? make_float4(0.f, 0.f, 0.f, 0.f)
                          : make_float4(g * u2f(r[src(4 * i)]), g * u2f(r[src(4 * i + 1)]),

@@ -110,6 +110,33 @@ def quantize_affine_q4(w: np.ndarray, group: int = 64):
     return packed, sb, bb
 
 
+def quantize_affine_q8(w: np.ndarray, group: int = 64):
+    """Store float32 rows [V, D] as 8-bit affine groups of ``group`` along D.
+
+    As ``quantize_affine_q4`` with 255 levels: bias = min, scale =
+    (max - min) / 255 (1 if constant), both bf16; q = clip(rint((w - bias) /
+    scale), 0, 255).  Packing: element ``4k + j`` of a row is byte ``j`` of
+    uint32 word ``k`` (low byte first).  Returns (packed uint32 [V, D/4],
+    scales bf16 bits [V, D/group], biases bf16 bits [V, D/group]).
+    """
+    V, D = w.shape
+    assert D % group == 0 and D % 4 == 0
+    wg = w.reshape(V, D // group, group)
+    mn = wg.min(axis=2)
+    mx = wg.max(axis=2)
+    scale = (mx - mn) / np.float32(255.0)
+    scale = np.where(scale == 0, np.float32(1.0), scale).astype(np.float32)
+    sb = f32_to_bf16_bits(scale)
+    bb = f32_to_bf16_bits(mn)
+    s = bf16_bits_to_f32(sb)[:, :, None]
+    b = bf16_bits_to_f32(bb)[:, :, None]
+    q = np.clip(np.rint((wg - b) / s), 0, 255).astype(np.uint32).reshape(V, D)
+    packed = np.zeros((V, D // 4), dtype=np.uint32)
+    for j in range(4):
+        packed |= q[:, j::4] << np.uint32(8 * j)
+    return packed, sb, bb
+
+
 # ----------------------------------------------------------------------------
 # workload
 # ----------------------------------------------------------------------------
@@ -121,8 +148,8 @@ class Workload:
     * ``H``: float32 [M, D] (bf16-representable values for bf16 workloads);
       ``H_bits`` the bf16 bit patterns (uint16) or None for fp32.
     * dense head: ``W`` float32 [V, D] (bf16-representable for bf16) and
-      ``W_bits``; 4-bit head: ``q_packed`` uint32 [V, D/8], ``q_scales`` /
-      ``q_biases`` bf16 bits [V, D/64], and ``W`` None.
+      ``W_bits``; 4-bit (8-bit) head: ``q_packed`` uint32 [V, D/8] ([V, D/4]),
+      ``q_scales`` / ``q_biases`` bf16 bits [V, D/64], and ``W`` None.
     """
 
     cfg_id: int
@@ -214,15 +241,17 @@ def _make(cfg_id, c, seed, threads) -> Workload:
                   scope=c["scope"], lam=LAMBDA, filter_eps=c["filter_eps"],
                   block_skip=c["block_skip"], labels=labels, H=H, H_bits=None)
 
-    if c["wformat"] == "q4g64":
-        packed = np.empty((V, D // 8), dtype=np.uint32)
+    if c["wformat"] in ("q4g64", "q8g64"):
+        per_word = 8 if c["wformat"] == "q4g64" else 4
+        quant = quantize_affine_q4 if per_word == 8 else quantize_affine_q8
+        packed = np.empty((V, D // per_word), dtype=np.uint32)
         sc = np.empty((V, D // 64), dtype=np.uint16)
         bi = np.empty((V, D // 64), dtype=np.uint16)
         blk = 4096
 
         def qwork(i):
             r0, r1 = i * blk, min(V, (i + 1) * blk)
-            p_, s_, b_ = quantize_affine_q4(Wf[r0:r1])
+            p_, s_, b_ = quant(Wf[r0:r1])
             packed[r0:r1], sc[r0:r1], bi[r0:r1] = p_, s_, b_
 
         with ThreadPoolExecutor(threads) as ex:

@@ -146,14 +146,22 @@ def _as64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
-def head_forward(H, W, labels, rows=None, block: int = 64):
+def softcap_logits(Z, softcap: float):
+    """Gemma-style logit soft-capping, cap * tanh(z / cap) (ORPO design
+    (0.0.6), fused-head spec: "Gemma applies final_logit_softcapping"); a cap
+    of 0 means none."""
+    return Z if not softcap else softcap * np.tanh(Z / softcap)
+
+
+def head_forward(H, W, labels, rows=None, block: int = 64, softcap: float = 0.0):
     """Per-row lse, target logit and logp of the LM head (Training design §5.1).
 
     ``H`` [M, D] and ``W`` [V, D] hold exactly the values the GPU consumes
     (bf16-rounded, or dequantised), converted to float64.  ``rows`` optionally
     restricts the computation to a subset of rows (sampled parity).  Returns
     ``(logp, lse, tgt)`` for the selected rows; ``logp`` and ``tgt`` are 0 for
-    ignored rows (label < 0).
+    ignored rows (label < 0).  With ``softcap`` the logits are capped first
+    and everything (lse, target, logp) uses the capped values.
     """
     H = _as64(H)
     W = _as64(W)
@@ -165,7 +173,7 @@ def head_forward(H, W, labels, rows=None, block: int = 64):
     tgt = np.zeros(n)
     for r0 in range(0, n, block):
         sel = idx[r0:r0 + block]
-        Z = H[sel] @ W.T                                   # [rows, V] logits
+        Z = softcap_logits(H[sel] @ W.T, softcap)           # [rows, V] logits
         mx = Z.max(axis=1)
         lse[r0:r0 + len(sel)] = mx + np.log(np.exp(Z - mx[:, None]).sum(axis=1))
         y = labels[sel]
@@ -179,7 +187,7 @@ def head_forward(H, W, labels, rows=None, block: int = 64):
 
 
 def head_dh(H, W, labels, coeff, lse, rows=None, filter_eps: float = 0.0,
-            block: int = 64):
+            block: int = 64, softcap: float = 0.0):
     """dh_t = sum_v g_t (onehot(y_t)_v - p_tv) W_v, p = exp(z - lse).
 
     ORPO design (0.0.6), fused-head spec "Backward (recompute vocab tiles from
@@ -187,7 +195,9 @@ def head_dh(H, W, labels, coeff, lse, rows=None, filter_eps: float = 0.0,
     dh = that . W.  ``coeff`` is g = dL/dlogp per row (0 for ignored rows).
     ``lse`` is the per-row lse of the selected rows.  With ``filter_eps`` > 0 a
     term whose softmax is below eps on a non-target column is dropped
-    (Training design §5.1, "coeff filter").
+    (Training design §5.1, "coeff filter").  With ``softcap`` the softmax is
+    over the capped logits and each term carries d(capped)/d(raw) =
+    1 - tanh^2(raw / cap) (the fused-head spec's "x sech^2").
     """
     H = _as64(H)
     W = _as64(W)
@@ -200,7 +210,8 @@ def head_dh(H, W, labels, coeff, lse, rows=None, filter_eps: float = 0.0,
     for r0 in range(0, idx.shape[0], block):
         sel = idx[r0:r0 + block]
         k = len(sel)
-        Z = H[sel] @ W.T
+        Zr = H[sel] @ W.T
+        Z = softcap_logits(Zr, softcap)
         P = np.exp(Z - lse[r0:r0 + k, None])
         y = labels[sel]
         onehot = np.zeros_like(P)
@@ -211,6 +222,8 @@ def head_dh(H, W, labels, coeff, lse, rows=None, filter_eps: float = 0.0,
             P = np.where(drop, 0.0, P)
         c = np.where(ok, coeff[sel], 0.0)
         G = c[:, None] * (onehot - P)
+        if softcap:
+            G = G * (1.0 - np.tanh(Zr / softcap) ** 2)
         out[r0:r0 + k] = G @ W
     return out
 
@@ -304,18 +317,19 @@ def orpo_grad_coeffs(logp, labels, layout: Layout, lam: float,
 
 
 def orpo_head_loss(H, W, labels, layout: Layout, lam: float,
-                   sft_scope: str = "full") -> float:
+                   sft_scope: str = "full", softcap: float = 0.0) -> float:
     """Scalar ORPO loss of the head as a function of H (for finite differences)."""
-    logp, _, _ = head_forward(H, W, labels)
+    logp, _, _ = head_forward(H, W, labels, softcap=softcap)
     return orpo_loss_from_logps(logp, labels, layout, lam, sft_scope).loss
 
 
 def orpo_head_grad(H, W, labels, layout: Layout, lam: float,
-                   sft_scope: str = "full", filter_eps: float = 0.0):
+                   sft_scope: str = "full", filter_eps: float = 0.0,
+                   softcap: float = 0.0):
     """dL/dH through the head: coefficients, then ``head_dh``."""
-    logp, lse, _ = head_forward(H, W, labels)
+    logp, lse, _ = head_forward(H, W, labels, softcap=softcap)
     g = orpo_grad_coeffs(logp, labels, layout, lam, sft_scope)
-    return head_dh(H, W, labels, g, lse, filter_eps=filter_eps)
+    return head_dh(H, W, labels, g, lse, filter_eps=filter_eps, softcap=softcap)
 
 
 # ----------------------------------------------------------------------------
@@ -426,3 +440,19 @@ def pref_grad_coeffs(logp, labels, layout: Layout, kind: str, lam: float,
     g[L.rejected_begin:L.rejected_end] = -d / o.n_rejected
     g[labels < 0] = 0.0
     return g
+
+
+def dequant_affine_q8(packed, scales, biases, group: int = 64) -> np.ndarray:
+    """8-bit affine groups: w[v, d] = q[v, d] * scale + bias, element
+    ``4*k + j`` of a row in byte ``j`` of word ``k`` (low byte first);
+    the 8-bit variant of the quantised head (Training design §5.1, "in-Metal
+    4/8-bit affine dequant").  ``scales``/``biases``: bf16 bits [V, D/group]."""
+    packed = np.asarray(packed, dtype=np.uint32)
+    V, W4 = packed.shape
+    D = W4 * 4
+    q = np.empty((V, D), dtype=np.float64)
+    for j in range(4):
+        q[:, j::4] = ((packed >> np.uint32(8 * j)) & np.uint32(0xFF)).astype(np.float64)
+    s = np.repeat(bf16_bits_to_f64(scales), group, axis=1)
+    b = np.repeat(bf16_bits_to_f64(biases), group, axis=1)
+    return q * s + b

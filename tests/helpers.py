@@ -26,6 +26,8 @@ def oracle_W(wl: S.Workload) -> np.ndarray:
     """The head's weights exactly as the method defines them (float64)."""
     if wl.wformat == "q4g64":
         return O.dequant_affine_q4(wl.q_packed, wl.q_scales, wl.q_biases)
+    if wl.wformat == "q8g64":
+        return O.dequant_affine_q8(wl.q_packed, wl.q_scales, wl.q_biases)
     return wl.W.astype(np.float64)
 
 

@@ -247,3 +247,53 @@ def test_objective_siblings_match_oracle(kind):
             assert np.allclose(out8.cpu().numpy(), np.array(o.as8()), rtol=1e-12, atol=1e-14)
             g = O.pref_grad_coeffs(lp, y, L, kind, lam, beta, gamma, scope)
             assert np.allclose(coeff.cpu().numpy(), g, rtol=1e-6, atol=1e-12)
+
+
+@pytest.mark.parametrize("cfg,cap", [(1, 30.0), (2, 2.0), (4, 30.0), (0, 5.0)])
+def test_softcap_forward_and_backward(cfg, cap):
+    """Gemma-style logit capping: capped logits in the forward, the
+    1 - tanh^2 factor in the backward."""
+    wl = S.make_custom(cfg, M_split=(60, 70, 80), D=128, V=1500)
+    H, head, labels = upload(wl)
+    head.softcap = cap
+    hd = cce.h_dtype(H)
+    ws = cce.alloc_workspace(wl.M, hd, head)
+    f = dict(device="cuda", dtype=torch.float32)
+    logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+    cce.cce_forward(H, head, labels, logp, lse, None, None, ws)
+    g = S.random_cotangent(wl)
+    dH = torch.empty(wl.M, wl.D, **f)
+    cce.cce_backward_dh(H, head, labels, lse, torch.from_numpy(g).cuda(), 0.0, None, dH, None, ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0
+    W = oracle_W(wl)
+    ologp, olse, _ = O.head_forward(wl.H, W, wl.labels, softcap=cap)
+    assert np.max(np.abs(logp.cpu().numpy() - ologp)) <= TOL_LOGP
+    assert np.max(np.abs(lse.cpu().numpy() - olse)) <= TOL_LOGP
+    want = O.head_dh(wl.H, W, wl.labels, g, olse, softcap=cap)
+    assert rel_fro(dH.cpu().numpy(), want) <= TOL_DH
+
+
+@pytest.mark.parametrize("split,D,V,cap", [((40, 45, 44), 128, 257, 0.0),
+                                           ((100, 150, 131), 256, 4097, 0.0),
+                                           ((64, 200, 300), 320, 1000, 30.0)])
+def test_q8_head_forward_and_backward(split, D, V, cap):
+    """8-bit affine head (group 64), dequantised in-kernel."""
+    wl = S.make_custom(4, M_split=split, D=D, V=V, wformat="q8g64")
+    H, head, labels = upload(wl)
+    head.softcap = cap
+    ws = cce.alloc_workspace(wl.M, cce.h_dtype(H), head)
+    f = dict(device="cuda", dtype=torch.float32)
+    logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+    cce.cce_forward(H, head, labels, logp, lse, None, None, ws)
+    g = S.random_cotangent(wl)
+    dH = torch.empty(wl.M, wl.D, **f)
+    cce.cce_backward_dh(H, head, labels, lse, torch.from_numpy(g).cuda(), 0.0, None, dH, None, ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0
+    W = oracle_W(wl)
+    ologp, olse, _ = O.head_forward(wl.H, W, wl.labels, softcap=cap)
+    assert np.max(np.abs(logp.cpu().numpy() - ologp)) <= TOL_LOGP
+    assert np.max(np.abs(lse.cpu().numpy() - olse)) <= TOL_LOGP
+    want = O.head_dh(wl.H, W, wl.labels, g, olse, softcap=cap)
+    assert rel_fro(dH.cpu().numpy(), want) <= TOL_DH

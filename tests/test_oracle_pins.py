@@ -392,3 +392,50 @@ def test_sibling_coeffs_are_dL_dlogp(kind, scope):
         fd = (O.pref_loss_from_logps(lp, y, L, kind, **args).loss
               - O.pref_loss_from_logps(lm, y, L, kind, **args).loss) / (2 * h)
         assert coef[m] == pytest.approx(fd, rel=1e-6, abs=1e-9)
+
+
+# --------------------------------------------------------------------------
+# logit softcap
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cap", [0.7, 3.0])
+def test_softcap_finite_differences(cap):
+    H, W, y, L = tiny_case(seed=13)
+    H = H * 2.0
+    dH = O.orpo_head_grad(H, W, y, L, 0.3, "full", softcap=cap)
+    h = 1e-6
+    fd = np.zeros_like(H)
+    for m in range(H.shape[0]):
+        for d in range(H.shape[1]):
+            Hp, Hm = H.copy(), H.copy()
+            Hp[m, d] += h
+            Hm[m, d] -= h
+            fd[m, d] = (O.orpo_head_loss(Hp, W, y, L, 0.3, "full", softcap=cap)
+                        - O.orpo_head_loss(Hm, W, y, L, 0.3, "full", softcap=cap)) / (2 * h)
+    assert np.allclose(dH, fd, rtol=1e-6, atol=1e-9)
+
+
+def test_softcap_limits():
+    H, W, y, L = tiny_case(P=5, Rc=7, Rr=6, D=24, V=97, seed=3)
+    plain = O.head_forward(H, W, y)
+    big = O.head_forward(H, W, y, softcap=1e7)
+    for a, b in zip(plain, big):
+        assert np.allclose(a, b, rtol=1e-9, atol=1e-9)
+    cap = 0.5
+    logp, lse, tgt = O.head_forward(H, W, y, softcap=cap)
+    Z = cap * np.tanh((H @ W.T) / cap)
+    assert np.all(np.abs(tgt) <= cap)
+    assert np.allclose(lse, sps.logsumexp(Z, axis=1), rtol=1e-14, atol=1e-13)
+
+
+def test_dequant_q8_byte_order_and_affine():
+    words = np.zeros((1, 16), dtype=np.uint32)
+    words[0, 0] = 0x03020100
+    words[0, 1] = 0xFF807F10
+    one = np.array([[0x3F80]], dtype=np.uint16)
+    zero = np.array([[0x0000]], dtype=np.uint16)
+    w = O.dequant_affine_q8(words, one, zero)
+    assert w.shape == (1, 64)
+    assert w[0, :8].tolist() == [0, 1, 2, 3, 16, 127, 128, 255]
+    w2 = O.dequant_affine_q8(words, np.array([[0x3E80]], np.uint16), np.array([[0xBF80]], np.uint16))
+    assert np.array_equal(w2, w * 0.25 - 1.0)

@@ -48,3 +48,13 @@ def test_sample_rows_cover_segments():
     r = S.sample_rows(wl, n_uniform=10)
     assert r[0] == 0 and 40 in r and 69 in r and 70 in r and 99 in r
     assert np.all(np.diff(r) > 0)
+
+
+def test_q8_roundtrip_error_bounded_by_half_step():
+    g = np.random.default_rng(2)
+    w = (g.standard_normal((23, 128)) / 16).astype(np.float32)
+    packed, sc, bi = S.quantize_affine_q8(w)
+    deq = O.dequant_affine_q8(packed, sc, bi)
+    step = np.repeat(O.bf16_bits_to_f64(sc), 64, axis=1)
+    assert np.all(np.abs(deq - w) <= 1.01 * step)
+    assert np.mean(np.abs(deq - w) <= 0.5 * step + 1e-7) > 0.97
