@@ -221,6 +221,29 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M,
                            unsigned long long* skip_stats, void* ws,
                            size_t ws_bytes, cce_stream_t stream);
 
+/*
+ * Prefix-shared ORPO pair (Training design §5.4, "Shared prompt-prefix
+ * forward"): one forward over [prompt(P); chosen(Rc); rejected(Rr)] gives
+ * H_cat [P+Rc+Rr, D], and the head gathers chosen[k] <- H_cat[P-1+k],
+ * rejected[0] <- H_cat[P-1], rejected[k>=1] <- H_cat[P+Rc+k-1]; prompt row m
+ * (the position predicting prompt token m) <- H_cat[m-1], and the unlabelled
+ * head row 0 <- H_cat[0].
+ * cce_prefix_gather writes those head rows, in the layout [prompt | chosen |
+ * rejected] used by every other call, into H_head [P+Rc+Rr, D] (dtype f32 or
+ * bf16, row bytes a multiple of 16).
+ * cce_prefix_scatter is its adjoint for the backward: dH_cat [P+Rc+Rr, D]
+ * fp32 (overwritten) = the sum of dH_head rows that read each row, so row
+ * P-1 receives the gradients of the first chosen and the first rejected
+ * token (the two branches' cotangents meet in the shared prefix).
+ * Deterministic, bandwidth-bound; P, Rc, Rr >= 1.
+ */
+cce_status cce_prefix_gather(const void* H_cat, cce_dtype dtype, int64_t P,
+                             int64_t Rc, int64_t Rr, int64_t D, void* H_head,
+                             cce_stream_t stream);
+cce_status cce_prefix_scatter(const float* dH_head, int64_t P, int64_t Rc,
+                              int64_t Rr, int64_t D, float* dH_cat,
+                              cce_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the status word in ws, and
  * returns the first error it holds (CCE_OK when none). */
 cce_status cce_device_status(void* ws, cce_stream_t stream);

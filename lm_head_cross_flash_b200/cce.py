@@ -91,6 +91,12 @@ _SIGS = {
                                         ctypes.POINTER(_Layout), ctypes.POINTER(_Objective),
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]),
+    "cce_prefix_gather": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                         ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "cce_prefix_scatter": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                          ctypes.c_void_p]),
     "cce_profile_enable": (None, [ctypes.c_int]),
     "cce_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_longlong), ctypes.c_int]),
@@ -348,3 +354,13 @@ def pref_grad_coeffs(logp, labels, layout, kind, lam, beta, gamma, sft_scope, co
                                 ctypes.byref(_objective(kind, lam, beta, gamma, sft_scope)),
                                 _p(coeff), _p(ws), ws.numel(), _stream(stream))
     _check(st, "pref_grad_coeffs")
+
+
+def cce_prefix_gather(H_cat, P, Rc, Rr, H_head, stream=None):
+    _check(lib().cce_prefix_gather(_p(H_cat), h_dtype(H_cat), P, Rc, Rr, H_cat.shape[1],
+                                   _p(H_head), _stream(stream)), "cce_prefix_gather")
+
+
+def cce_prefix_scatter(dH_head, P, Rc, Rr, dH_cat, stream=None):
+    _check(lib().cce_prefix_scatter(_p(dH_head), P, Rc, Rr, dH_head.shape[1], _p(dH_cat),
+                                    _stream(stream)), "cce_prefix_scatter")

@@ -276,6 +276,48 @@ __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
   }
 }
 
+// ----------------------------------------------- prefix-shared ORPO pair --
+// Source row of head row m (Training design §5.4): m - 1 for m >= 1 except
+// the first rejected row m = P + Rc, which reads P - 1; head row 0 reads 0.
+__device__ __forceinline__ int64_t prefix_src(int64_t m, int64_t P, int64_t Rc) {
+  return m == 0 ? 0 : (m == P + Rc ? P - 1 : m - 1);
+}
+
+// H_head[m] = H_cat[prefix_src(m)], rows of `row_bytes` (multiple of 16).
+__global__ void prefix_gather_kernel(const uint4* __restrict__ src, int64_t M, int64_t P,
+                                     int64_t Rc, int64_t row16, uint4* __restrict__ dst) {
+  const int64_t n = M * row16;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / row16, c = i - m * row16;
+    dst[i] = src[prefix_src(m, P, Rc) * row16 + c];
+  }
+}
+
+// Adjoint: dH_cat[r] = sum over head rows m with prefix_src(m) == r of
+// dH_head[m], added in increasing m (deterministic).  Rows P + Rc - 1 and
+// M - 1 receive nothing.
+__global__ void prefix_scatter_kernel(const float4* __restrict__ dh, int64_t M, int64_t P,
+                                      int64_t Rc, int64_t row4, float4* __restrict__ out) {
+  const int64_t n = M * row4;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / row4, c = i - r * row4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add = [&](int64_t m) {
+      const float4 v = dh[m * row4 + c];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    };
+    if (r == 0) add(0);
+    if (r + 1 < M && r + 1 != P + Rc) add(r + 1);
+    if (r == P - 1) add(P + Rc);
+    out[i] = acc;
+  }
+}
+
 // ------------------------------------------------- K-split partial sums --
 // dH += parts[0] + parts[1] + ... (fixed order, so the result is
 // deterministic); n4 = M*D/4 float4 elements per buffer.

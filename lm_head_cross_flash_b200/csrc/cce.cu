@@ -76,11 +76,13 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // Optional per-kernel timing: while enabled, every kernel launch is
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
-  PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM, PK_N
+  PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM,
+  PK_PREFIX, PK_N
 };
-const char* const kProfNames[PK_N] = {"split_f32",     "fwd_lse_gemm", "lse_merge",
+const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
-                                      "bwd_dh_gemm",   "selftest",     "dh_split_sum"};
+                                      "bwd_dh_gemm",   "selftest",     "dh_split_sum",
+                                      "prefix_gather_scatter"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -781,6 +783,42 @@ int cce_profile_read(double* ms, long long* launches, int n) {
 
 const char* cce_profile_kind_name(int kind) {
   return (kind >= 0 && kind < PK_N) ? kProfNames[kind] : "unknown";
+}
+
+static cce_status prefix_args(int64_t P, int64_t Rc, int64_t Rr, int64_t D) {
+  if (P < 1 || Rc < 1 || Rr < 1 || D <= 0) return CCE_ERR_INVALID_ARGUMENT;
+  if (P + Rc + Rr > (int64_t(1) << 31) || D > (int64_t(1) << 20)) return CCE_ERR_INVALID_ARGUMENT;
+  return CCE_OK;
+}
+
+cce_status cce_prefix_gather(const void* H_cat, cce_dtype dtype, int64_t P, int64_t Rc,
+                             int64_t Rr, int64_t D, void* H_head, cce_stream_t stream) {
+  if (H_cat == nullptr || H_head == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  if (dtype != CCE_F32 && dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
+  cce_status s = prefix_args(P, Rc, Rr, D);
+  if (s != CCE_OK) return s;
+  const int64_t row_bytes = D * (dtype == CCE_F32 ? 4 : 2);
+  if (row_bytes % 16 != 0 || !aligned16(H_cat) || !aligned16(H_head)) return CCE_ERR_INVALID_ARGUMENT;
+  const int64_t M = P + Rc + Rr, row16 = row_bytes / 16;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope ps(PK_PREFIX, st);
+  prefix_gather_kernel<<<int(std::min<int64_t>(ceil_div(M * row16, 256), 4096)), 256, 0, st>>>(
+      static_cast<const uint4*>(H_cat), M, P, Rc, row16, static_cast<uint4*>(H_head));
+  return launch_ok();
+}
+
+cce_status cce_prefix_scatter(const float* dH_head, int64_t P, int64_t Rc, int64_t Rr, int64_t D,
+                              float* dH_cat, cce_stream_t stream) {
+  if (dH_head == nullptr || dH_cat == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  cce_status s = prefix_args(P, Rc, Rr, D);
+  if (s != CCE_OK) return s;
+  if (D % 4 != 0 || !aligned16(dH_head) || !aligned16(dH_cat)) return CCE_ERR_INVALID_ARGUMENT;
+  const int64_t M = P + Rc + Rr, row4 = D / 4;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope ps(PK_PREFIX, st);
+  prefix_scatter_kernel<<<int(std::min<int64_t>(ceil_div(M * row4, 256), 4096)), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(dH_head), M, P, Rc, row4, reinterpret_cast<float4*>(dH_cat));
+  return launch_ok();
 }
 
 cce_status cce_device_status(void* ws, cce_stream_t stream) {

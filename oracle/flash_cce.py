@@ -456,3 +456,41 @@ def dequant_affine_q8(packed, scales, biases, group: int = 64) -> np.ndarray:
     s = np.repeat(bf16_bits_to_f64(scales), group, axis=1)
     b = np.repeat(bf16_bits_to_f64(biases), group, axis=1)
     return q * s + b
+
+
+# ----------------------------------------------------------------------------
+# prefix-shared pair: head rows gathered from one concatenated forward
+# ----------------------------------------------------------------------------
+
+def prefix_gather_index(P: int, Rc: int, Rr: int) -> np.ndarray:
+    """Source row of every head row for a prefix-shared pair.
+
+    Training design §5.4: one forward over [prompt(P); chosen(Rc);
+    rejected(Rr)] yields H_cat; the head gathers chosen[k] <- H_cat[P-1+k],
+    rejected[0] <- H_cat[P-1], rejected[k>=1] <- H_cat[P+Rc+k-1].  The prompt
+    rows of the ``full`` scope are the positions that predict the next prompt
+    token, prompt row m <- H_cat[m-1].  Head row 0 (unlabelled: nothing
+    predicts the first prompt token) reads H_cat[0].
+    """
+    M = P + Rc + Rr
+    idx = np.empty(M, dtype=np.int64)
+    idx[0] = 0
+    idx[1:P] = np.arange(0, P - 1)                   # prompt
+    idx[P:P + Rc] = P - 1 + np.arange(Rc)            # chosen[k] <- P-1+k
+    idx[P + Rc] = P - 1                              # rejected[0] <- P-1
+    idx[P + Rc + 1:] = P + Rc + np.arange(1, Rr) - 1  # rejected[k] <- P+Rc+k-1
+    return idx
+
+
+def prefix_gather(H_cat, P: int, Rc: int, Rr: int) -> np.ndarray:
+    return np.asarray(H_cat)[prefix_gather_index(P, Rc, Rr)]
+
+
+def prefix_scatter(dH_head, P: int, Rc: int, Rr: int) -> np.ndarray:
+    """Adjoint of ``prefix_gather``: dH_cat[r] = sum of dH_head[m] over the
+    head rows m that read row r (reverse mode sums the two branches'
+    cotangents into the shared prefix)."""
+    dH_head = _as64(dH_head)
+    out = np.zeros_like(dH_head)
+    np.add.at(out, prefix_gather_index(P, Rc, Rr), dH_head)
+    return out

@@ -297,3 +297,34 @@ def test_q8_head_forward_and_backward(split, D, V, cap):
     assert np.max(np.abs(lse.cpu().numpy() - olse)) <= TOL_LOGP
     want = O.head_dh(wl.H, W, wl.labels, g, olse, softcap=cap)
     assert rel_fro(dH.cpu().numpy(), want) <= TOL_DH
+
+
+def test_prefix_shared_pair_end_to_end():
+    """Gather the head rows of a prefix-shared pair from one concatenated
+    forward, run the head, scatter dH back; compare with the oracle."""
+    P, Rc, Rr, D, V = 40, 70, 90, 128, 1500
+    wl = S.make_custom(2, M_split=(P, Rc, Rr), D=D, V=V)
+    Hcat, head, labels = upload(wl)           # treat the drawn rows as H_cat
+    Hh = torch.empty_like(Hcat)
+    cce.cce_prefix_gather(Hcat, P, Rc, Rr, Hh)
+    torch.cuda.synchronize()
+    idx = O.prefix_gather_index(P, Rc, Rr)
+    assert torch.equal(Hh, Hcat[torch.from_numpy(idx).cuda()])
+    buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(Hh), head)
+    cce.orpo_head_pass(Hh, head, labels, wl.layout_tuple, wl.lam, wl.scope, 0.0, False, buf)
+    dcat = torch.empty_like(buf.dH)
+    cce.cce_prefix_scatter(buf.dH, P, Rc, Rr, dcat)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(buf.ws) == 0
+    W = oracle_W(wl)
+    L = O.Layout(*wl.layout_tuple)
+    Hh64 = O.prefix_gather(wl.H, P, Rc, Rr)
+    want = O.prefix_scatter(O.orpo_head_grad(Hh64, W, wl.labels, L, wl.lam, wl.scope), P, Rc, Rr)
+    assert rel_fro(dcat.cpu().numpy(), want) <= TOL_DH
+    assert np.all(dcat.cpu().numpy()[P + Rc - 1] == 0)
+    # the scatter is exact: sums of at most two fp32 values, in a fixed order
+    G = np.random.default_rng(12).standard_normal((wl.M, D)).astype(np.float32)
+    out = torch.empty(wl.M, D, device="cuda")
+    cce.cce_prefix_scatter(torch.from_numpy(G).cuda(), P, Rc, Rr, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), O.prefix_scatter(G, P, Rc, Rr).astype(np.float32))

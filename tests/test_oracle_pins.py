@@ -439,3 +439,55 @@ def test_dequant_q8_byte_order_and_affine():
     assert w[0, :8].tolist() == [0, 1, 2, 3, 16, 127, 128, 255]
     w2 = O.dequant_affine_q8(words, np.array([[0x3E80]], np.uint16), np.array([[0xBF80]], np.uint16))
     assert np.array_equal(w2, w * 0.25 - 1.0)
+
+
+# --------------------------------------------------------------------------
+# prefix-shared gather
+# --------------------------------------------------------------------------
+
+def test_prefix_gather_index_matches_the_stated_map():
+    P, Rc, Rr = 5, 3, 4
+    idx = O.prefix_gather_index(P, Rc, Rr)
+    assert idx.tolist() == [0, 0, 1, 2, 3,     # prompt rows 1..4 <- 0..3
+                            4, 5, 6,           # chosen[k] <- P-1+k
+                            4,                 # rejected[0] <- P-1
+                            8, 9, 10]          # rejected[k] <- P+Rc+k-1
+
+
+def test_prefix_scatter_is_the_adjoint():
+    g = np.random.default_rng(9)
+    P, Rc, Rr, D = 6, 5, 7, 3
+    M = P + Rc + Rr
+    Hc = g.standard_normal((M, D))
+    G = g.standard_normal((M, D))
+    lhs = np.sum(O.prefix_gather(Hc, P, Rc, Rr) * G)
+    rhs = np.sum(Hc * O.prefix_scatter(G, P, Rc, Rr))
+    assert lhs == pytest.approx(rhs, rel=1e-13)
+    d = O.prefix_scatter(G, P, Rc, Rr)
+    assert np.allclose(d[P - 1], G[P] + G[P + Rc])   # both first response tokens
+    assert np.all(d[P + Rc - 1] == 0) and np.all(d[M - 1] == 0)
+
+
+def test_prefix_shared_loss_gradient_by_finite_differences():
+    """The whole prefix-shared head: L(H_cat) and its gradient."""
+    g = np.random.default_rng(10)
+    P, Rc, Rr, D, V = 4, 3, 3, 8, 20
+    M = P + Rc + Rr
+    Hc = g.standard_normal((M, D))
+    W = g.standard_normal((V, D)) / math.sqrt(D)
+    y = g.integers(0, V, size=M).astype(np.int32)
+    y[0] = -1
+    L = O.Layout.contiguous(P, Rc, Rr)
+
+    def loss(Hc_):
+        return O.orpo_head_loss(O.prefix_gather(Hc_, P, Rc, Rr), W, y, L, 0.2)
+
+    grad = O.prefix_scatter(O.orpo_head_grad(O.prefix_gather(Hc, P, Rc, Rr), W, y, L, 0.2),
+                            P, Rc, Rr)
+    h = 1e-6
+    for r in range(M):
+        for d in range(D):
+            Hp, Hm = Hc.copy(), Hc.copy()
+            Hp[r, d] += h
+            Hm[r, d] -= h
+            assert grad[r, d] == pytest.approx((loss(Hp) - loss(Hm)) / (2 * h), rel=1e-6, abs=1e-9)
