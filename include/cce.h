@@ -244,6 +244,25 @@ cce_status cce_prefix_scatter(const float* dH_head, int64_t P, int64_t Rc,
                               int64_t Rr, int64_t D, float* dH_cat,
                               cce_stream_t stream);
 
+/*
+ * Backward of a trainable head: cce_backward_dh plus the weight gradient
+ *   dW[v] = sum_m coeff[m] (onehot(y_m)_v - p_mv) H[m]   (times 1 - tanh^2
+ *   under a softcap, with the same coefficient filter),
+ * for when the head stops being frozen (ORPO design 0.0.6, fused-head spec:
+ * the head's explicit VJP inputs and the "dC"/head-LoRA follow-on).  It reuses
+ * each vocab chunk of the backward: dW[chunk] = -(G''^T . (coeff * H)), a
+ * tensor-core GEMM over the rows.  dW: fp32 [V, D] output, overwritten.
+ * Dense heads only (quantised heads return CCE_ERR_UNSUPPORTED).  Other
+ * arguments as for cce_backward_dh.
+ */
+cce_status cce_backward_dh_dw(const void* H, cce_dtype h_dtype, int64_t M,
+                              const cce_head* W, const int32_t* labels,
+                              const float* lse, const float* coeff,
+                              float filter_eps, const float* blockmax,
+                              float* dH, float* dW,
+                              unsigned long long* skip_stats, void* ws,
+                              size_t ws_bytes, cce_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the status word in ws, and
  * returns the first error it holds (CCE_OK when none). */
 cce_status cce_device_status(void* ws, cce_stream_t stream);

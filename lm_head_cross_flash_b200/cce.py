@@ -79,6 +79,11 @@ _SIGS = {
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_void_p]),
+    "cce_backward_dh_dw": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                          ctypes.POINTER(_Head), ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "cce_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "cce_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
@@ -364,3 +369,12 @@ def cce_prefix_gather(H_cat, P, Rc, Rr, H_head, stream=None):
 def cce_prefix_scatter(dH_head, P, Rc, Rr, dH_cat, stream=None):
     _check(lib().cce_prefix_scatter(_p(dH_head), P, Rc, Rr, dH_head.shape[1], _p(dH_cat),
                                     _stream(stream)), "cce_prefix_scatter")
+
+
+def cce_backward_dh_dw(H, head: Head, labels, lse, coeff, filter_eps, blockmax, dH, dW,
+                       skip_stats=None, ws=None, stream=None):
+    st = lib().cce_backward_dh_dw(_p(H), h_dtype(H), H.shape[0], ctypes.byref(head.c()),
+                                  _p(labels), _p(lse), _p(coeff), float(filter_eps),
+                                  _p(blockmax), _p(dH), _p(dW), _p(skip_stats), _p(ws),
+                                  ws.numel(), _stream(stream))
+    _check(st, "cce_backward_dh_dw")

@@ -276,6 +276,23 @@ __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
   }
 }
 
+// ---------------------------------------------------- trainable head --
+// hg[m, d] = bf16(coeff[m] * H[m, d]): the B operand of the dW GEMM (the row
+// cotangent enters along K, so it is folded into the rows of H).
+template <typename T>
+__global__ void scale_rows_bf16_kernel(const T* __restrict__ H, const float* __restrict__ coeff,
+                                       int64_t M, int D, __nv_bfloat16* __restrict__ out) {
+  const int64_t n = M * D;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / D;
+    float h;
+    if constexpr (sizeof(T) == 4) h = H[i];
+    else h = __bfloat162float(H[i]);
+    out[i] = __float2bfloat16_rn(coeff[m] * h);
+  }
+}
+
 // ----------------------------------------------- prefix-shared ORPO pair --
 // Source row of head row m (Training design §5.4): m - 1 for m >= 1 except
 // the first rejected row m = P + Rc, which reads P - 1; head row 0 reads 0.

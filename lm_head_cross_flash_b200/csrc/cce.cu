@@ -77,12 +77,12 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
   PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM,
-  PK_PREFIX, PK_N
+  PK_PREFIX, PK_DW, PK_N
 };
 const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
                                       "bwd_dh_gemm",   "selftest",     "dh_split_sum",
-                                      "prefix_gather_scatter"};
+                                      "prefix_gather_scatter", "bwd_dw_gemm"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -166,6 +166,7 @@ cce_status device_info(int* sms) {
     CCE_SET_SMEM(Mode::kLse, 0) CCE_SET_SMEM(Mode::kGrad, 0) CCE_SET_SMEM(Mode::kDh, 0)
     CCE_SET_SMEM(Mode::kLse, 4) CCE_SET_SMEM(Mode::kGrad, 4) CCE_SET_SMEM(Mode::kDh, 4)
     CCE_SET_SMEM(Mode::kLse, 8) CCE_SET_SMEM(Mode::kGrad, 8) CCE_SET_SMEM(Mode::kDh, 8)
+    CCE_SET_SMEM(Mode::kDw, 0)
 #undef CCE_SET_SMEM
     if (!ok)
       return CCE_ERR_CUDA;
@@ -207,6 +208,7 @@ struct Layout {
   size_t hs = 0, ws = 0;                   // f32 split operands
   size_t g = 0, tile_skip = 0, row_skip = 0;
   size_t dh_part = 0;                      // K-split partial dH buffers
+  size_t hg = 0;                           // coeff * H (bf16), trainable head
   int64_t vc = 0;                          // backward vocab chunk
   int ksplit = 1;
   size_t total = 0;
@@ -262,6 +264,9 @@ Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ks
   L.row_skip = b; b += align_up(size_t(n_rt));
   L.dh_part = b; b += align_up(size_t(ksplit - 1) * M * W->D * 4);
   L.ksplit = ksplit;
+  if (W->format == CCE_W_DENSE) {
+    L.hg = b; b += align_up(size_t(M) * W->D * 2);  // coeff * H for the dW GEMM
+  }
   // split operands live after both regions
   size_t s = std::max(f, b);
   if (h == CCE_F32) {
@@ -597,11 +602,37 @@ cce_status pref_grad_coeffs(const float* logp, const int32_t* labels, int64_t M,
                      ws_bytes, stream, int(obj->kind), obj->beta, obj->gamma);
 }
 
+static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
+                                const int32_t* labels, const float* lse, const float* coeff,
+                                float filter_eps, const float* blockmax, float* dH, float* dW,
+                                unsigned long long* skip_stats, void* ws, size_t ws_bytes,
+                                cce_stream_t stream);
+
 cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
                            const int32_t* labels, const float* lse, const float* coeff,
                            float filter_eps, const float* blockmax, float* dH,
                            unsigned long long* skip_stats, void* ws, size_t ws_bytes,
                            cce_stream_t stream) {
+  return backward_impl(H, h_dtype, M, W, labels, lse, coeff, filter_eps, blockmax, dH, nullptr,
+                       skip_stats, ws, ws_bytes, stream);
+}
+
+cce_status cce_backward_dh_dw(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
+                              const int32_t* labels, const float* lse, const float* coeff,
+                              float filter_eps, const float* blockmax, float* dH, float* dW,
+                              unsigned long long* skip_stats, void* ws, size_t ws_bytes,
+                              cce_stream_t stream) {
+  if (dW == nullptr || !aligned16(dW)) return CCE_ERR_INVALID_ARGUMENT;
+  if (W != nullptr && W->format != CCE_W_DENSE) return CCE_ERR_UNSUPPORTED;
+  return backward_impl(H, h_dtype, M, W, labels, lse, coeff, filter_eps, blockmax, dH, dW,
+                       skip_stats, ws, ws_bytes, stream);
+}
+
+static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
+                                const int32_t* labels, const float* lse, const float* coeff,
+                                float filter_eps, const float* blockmax, float* dH, float* dW,
+                                unsigned long long* skip_stats, void* ws, size_t ws_bytes,
+                                cce_stream_t stream) {
   if (H == nullptr || labels == nullptr || lse == nullptr || coeff == nullptr ||
       dH == nullptr || ws == nullptr)
     return CCE_ERR_INVALID_ARGUMENT;
@@ -699,6 +730,29 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
   a.softcap = W->softcap;
   a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
 
+  // Trainable head: B operand coeff * H and the dW output map.
+  CUtensorMap mhg, mdw;
+  __nv_bfloat16* hg = reinterpret_cast<__nv_bfloat16*>(wsc + L.hg);
+  if (dW != nullptr) {
+    {
+      ProfScope ps(PK_SPLIT, st);
+      if (h_dtype == CCE_F32)
+        scale_rows_bf16_kernel<float><<<1184, 256, 0, st>>>(static_cast<const float*>(H), coeff, M,
+                                                            int(D), hg);
+      else
+        scale_rows_bf16_kernel<__nv_bfloat16><<<1184, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(H), coeff, M, int(D), hg);
+    }
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    const uint64_t wd[3] = {uint64_t(D), uint64_t(V), 1};
+    const uint64_t wsd[2] = {uint64_t(D) * 4, uint64_t(V) * D * 4};
+    const uint32_t wb[3] = {32, 32, 1};
+    if (!make_map(&mhg, hg, true, D, M, D, 64, BK) ||
+        !make_map_ex(&mdw, dW, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wd, wsd, wb,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return CCE_ERR_CUDA;
+  }
+
   for (int64_t v0 = 0; v0 < V; v0 += vc) {
     const int64_t w = std::min<int64_t>(vc, V - v0);
     const int64_t ct_n = ceil_div(w, BN);
@@ -709,6 +763,7 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
     ag.npass = 1;
     ag.b_row0 = int(v0);
     ag.ct_off = int(v0 / BN);
+    ag.zero_skip_rows = dW != nullptr ? 1 : 0;
     {
       // G'' store map: [M, chunk columns] 16-bit, 32x32 boxes, 64-byte swizzle
       const uint64_t gd[2] = {uint64_t(ct_n * BN), uint64_t(M)};
@@ -738,6 +793,25 @@ cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M, const cc
       launch_tc<Mode::kDh>(op.qb, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    if (dW != nullptr) {
+      // dW[v0 : v0 + w] = -(G''^T . coeff*H): vocab tiles of 128 rows, K = M.
+      CUtensorMap mga;
+      if (!make_map(&mga, g, true, ct_n * BN, M, vc, 64, BK)) return CCE_ERR_CUDA;
+      TileArgs aw = a;
+      aw.n_rt = int(ct_n * BN / BM);
+      aw.n_ct = int(n_dt);
+      aw.nk = int(ceil_div(M, BK));
+      aw.npass = 1;
+      aw.b_row0 = int(v0);
+      aw.ksplit = 1;
+      aw.fmt = 1;
+      {
+        ProfScope ps(PK_DW, st);
+        cce_tc_kernel<Mode::kDw, 0><<<grid_for(int64_t(aw.n_rt) * n_dt, sms), NUM_THREADS,
+                                      smem_bytes<Mode::kDw>(), st>>>(mga, mhg, mdw, mdw, aw);
+      }
+      if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    }
   }
   if (ksplit > 1) {
     ProfScope ps(PK_DHSUM, st);

@@ -41,14 +41,14 @@ constexpr int DQ_WARPS = 8;          // dequantisation warps (4-bit head), 2 per
 constexpr int NUM_THREADS_Q4 = NUM_THREADS + 32 * DQ_WARPS;
 constexpr int DQ_WARP0 = 6;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2 };
+enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2, kDw = 3 };
 
 // Epilogue staging for TMA stores: per epilogue warp two buffers of
 // 32 rows x 32 columns (kGrad: 16-bit G'', 64-byte rows; kDh: fp32 dH,
 // 128-byte rows).
 template <Mode MODE>
 __host__ __device__ constexpr int staging_buf_bytes() {
-  return MODE == Mode::kGrad ? 32 * 64 : MODE == Mode::kDh ? 32 * 128 : 0;
+  return MODE == Mode::kGrad ? 32 * 64 : (MODE == Mode::kDh || MODE == Mode::kDw) ? 32 * 128 : 0;
 }
 template <Mode MODE>
 __host__ __device__ constexpr int smem_bytes() {
@@ -93,6 +93,7 @@ struct TileArgs {
   int ksplit;      // kDh: the chunk's K range is split in `ksplit` parts
   int first_chunk;
   int group_rt;    // kLse/kGrad: row tiles per raster group
+  int zero_skip_rows;  // kGrad: write zeros (not nothing) for row-skipped tiles
   float softcap;   // > 0: logits are cap * tanh(s / cap)
   float inv_cap;
   // 4-bit affine head (group 64): words [V, D/8], scales/biases bf16 [V, D/64]
@@ -174,7 +175,7 @@ struct TileCoord {
 template <Mode MODE>
 __device__ __forceinline__ TileCoord tile_coord(const TileArgs& a, int t) {
   TileCoord c;
-  if (MODE == Mode::kDh) {
+  if (MODE == Mode::kDh || MODE == Mode::kDw) {
     c.ct = t % a.n_ct;
     const int r = t / a.n_ct;
     c.s = r % a.ksplit;
@@ -197,10 +198,10 @@ __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 // 0 = compute, 1 = write zeros only, 2 = nothing.
 template <Mode MODE>
 __device__ __forceinline__ int tile_kind(const TileArgs& a, int rt, int ct) {
-  if (MODE == Mode::kLse) return 0;
+  if (MODE == Mode::kLse || MODE == Mode::kDw) return 0;
   const bool rs = a.row_skip != nullptr && a.row_skip[rt] != 0;
   if (MODE == Mode::kGrad) {
-    if (rs) return 2;
+    if (rs) return a.zero_skip_rows ? 1 : 2;
     if (a.tile_skip != nullptr && a.tile_skip[rt * a.skip_ld + a.ct_off + ct]) return 1;
     return 0;
   }
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nsplit = MODE == Mode::kDh ? a.ksplit : 1;
+  const int nsplit = (MODE == Mode::kDh || MODE == Mode::kDw) ? a.ksplit : 1;
   const int ntiles = a.n_rt * a.n_ct * nsplit;
 
   if (threadIdx.x == 0) {
@@ -345,6 +346,17 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
               tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
             else
               tma_load_2d_hint(sA, &tmA, &full[stage], k * BK, tc.rt * BM, keep);
+          } else if (MODE == Mode::kDw) {
+            // A = G'' as an MN-major operand (vocab contiguous), two 64x64
+            // boxes; B = coeff * H, MN-major (d contiguous), four boxes.
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j)
+              tma_load_2d(sA + j * (64 * BK * 2), &tmA, &full[stage], tc.rt * BM + j * 64, k * BK);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d_hint(sB + j * (64 * BK * 2), &tmB, &full[stage], tc.ct * BN + j * 64,
+                               k * BK, keep);
           } else if (MODE == Mode::kDh) {
             mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
             tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
@@ -379,8 +391,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      const uint32_t idesc =
-          idesc_f16(BM, BN, a.fmt, false, MODE == Mode::kDh);
+      const uint32_t idesc = idesc_f16(BM, BN, a.fmt, MODE == Mode::kDw,
+                                       MODE == Mode::kDh || MODE == Mode::kDw);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -408,9 +420,11 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           const uint32_t sB = sA + A_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t ad = sdesc_sw128(sA + j * 32, 16, 1024);
+            const uint64_t ad = MODE == Mode::kDw
+                                    ? sdesc_sw128(sA + j * 16 * 128, 64 * BK * 2, 1024)
+                                    : sdesc_sw128(sA + j * 32, 16, 1024);
             const uint64_t bd =
-                MODE == Mode::kDh
+                (MODE == Mode::kDh || MODE == Mode::kDw)
                     ? sdesc_sw128(sB + j * 16 * 128, 64 * BK * 2, 1024)
                     : sdesc_sw128(sB + j * 32, 16, 1024);
             umma_f16_ss(d_tmem, ad, bd, idesc, (kk | j) != 0 ? 1u : 0u);
@@ -712,12 +726,14 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         });
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
-      } else {  // kDh: dH (+)= -coeff * (G'' . W)
-        const float g = live ? -a.coeff[row] : 0.f;
+      } else {  // kDh: dH (+)= -coeff * (G'' . W);  kDw: dW[chunk] = -(G''^T . coeff*H)
+        const float g = MODE == Mode::kDw ? -1.f : (live ? -a.coeff[row] : 0.f);
         const int dbase = ct * BN;
         const int nchunks = min(BN / 32, (a.D - dbase) / 32);
         const CUtensorMap* dmap = tc.s == 0 ? &tmC : &tmC2;
         const int dz = tc.s == 0 ? 0 : tc.s - 1;
+        const int orow0 = (MODE == Mode::kDw ? a.b_row0 : 0) + rt * BM + quad * 32;
+        const bool store = MODE == Mode::kDw || a.first_chunk;
         drain_chunks(taddr, nchunks, [&](int c, const uint32_t (&r)[32]) {
           // Stage g * acc as a 32x32 fp32 block (128-byte swizzle: chunk i of
           // row r at chunk i ^ (r & 7)); the first vocab chunk stores it, the
@@ -740,10 +756,10 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (a.first_chunk)
-              tma_store_3d(dmap, sb, dbase + c * 32, rt * BM + quad * 32, dz);
+            if (store)
+              tma_store_3d(dmap, sb, dbase + c * 32, orow0, dz);
             else
-              tma_reduce_add_3d(dmap, sb, dbase + c * 32, rt * BM + quad * 32, dz);
+              tma_reduce_add_3d(dmap, sb, dbase + c * 32, orow0, dz);
             bulk_commit();
           }
           ++nstore;

@@ -494,3 +494,42 @@ def prefix_scatter(dH_head, P: int, Rc: int, Rr: int) -> np.ndarray:
     out = np.zeros_like(dH_head)
     np.add.at(out, prefix_gather_index(P, Rc, Rr), dH_head)
     return out
+
+
+# ----------------------------------------------------------------------------
+# trainable head: gradient with respect to W
+# ----------------------------------------------------------------------------
+
+def head_dw(H, W, labels, coeff, lse, filter_eps: float = 0.0, softcap: float = 0.0,
+            block: int = 64) -> np.ndarray:
+    """dW[v] = sum_m g_m (onehot(y_m)_v - p_mv) * cap'(s_mv) * H[m].
+
+    The head's weight gradient for when the head stops being frozen (ORPO
+    design (0.0.6), fused-head spec: explicit VJP inputs (h, baseW, ...), and
+    the follow-on "head-LoRA / dC"): the same per-logit cotangent as
+    ``head_dh``, contracted with H over the rows instead of with W over the
+    vocabulary.  ``lse`` covers every row.
+    """
+    H = _as64(H)
+    W = _as64(W)
+    labels = np.asarray(labels)
+    coeff = _as64(coeff)
+    lse = _as64(lse)
+    out = np.zeros_like(W)
+    for r0 in range(0, H.shape[0], block):
+        sel = slice(r0, r0 + block)
+        Zr = H[sel] @ W.T
+        Z = softcap_logits(Zr, softcap)
+        P = np.exp(Z - lse[sel, None])
+        y = labels[sel]
+        onehot = np.zeros_like(P)
+        ok = y >= 0
+        onehot[np.nonzero(ok)[0], y[ok]] = 1.0
+        if filter_eps > 0.0:
+            P = np.where((P < filter_eps) & (onehot == 0.0), 0.0, P)
+        c = np.where(ok, coeff[sel], 0.0)
+        G = c[:, None] * (onehot - P)
+        if softcap:
+            G = G * (1.0 - np.tanh(Zr / softcap) ** 2)
+        out += G.T @ H[sel]
+    return out

@@ -328,3 +328,51 @@ def test_prefix_shared_pair_end_to_end():
     cce.cce_prefix_scatter(torch.from_numpy(G).cuda(), P, Rc, Rr, out)
     torch.cuda.synchronize()
     assert np.array_equal(out.cpu().numpy(), O.prefix_scatter(G, P, Rc, Rr).astype(np.float32))
+
+
+@pytest.mark.parametrize("cfg,split,D,V,cap,eps", [
+    (1, (40, 45, 44), 128, 257, 0.0, 0.0),
+    (2, (100, 150, 131), 256, 4097, 0.0, 0.0),
+    (0, (8, 60, 60), 64, 300, 0.0, 0.0),
+    (1, (64, 200, 300), 192, 1000, 30.0, 0.0),
+    (3, (100, 150, 131), 256, 4097, 0.0, 1e-4),
+])
+def test_trainable_head_dw(cfg, split, D, V, cap, eps):
+    """dW = sum_m coeff (onehot - p) H_m, and dH unchanged by asking for dW."""
+    wl = S.make_custom(cfg, M_split=split, D=D, V=V)
+    H, head, labels = upload(wl)
+    head.softcap = cap
+    hd = cce.h_dtype(H)
+    ws = cce.alloc_workspace(wl.M, hd, head)
+    f = dict(device="cuda", dtype=torch.float32)
+    logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+    cce.cce_forward(H, head, labels, logp, lse, None, None, ws)
+    g = S.random_cotangent(wl)
+    g[: split[0] // 2] = 0.0            # a run of zero-cotangent rows
+    coeff = torch.from_numpy(g).cuda()
+    dH1 = torch.empty(wl.M, wl.D, **f)
+    cce.cce_backward_dh(H, head, labels, lse, coeff, eps, None, dH1, None, ws)
+    dH2 = torch.empty(wl.M, wl.D, **f)
+    dW = torch.full((wl.V, wl.D), float("nan"), **f)
+    cce.cce_backward_dh_dw(H, head, labels, lse, coeff, eps, None, dH2, dW, None, ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0
+    assert torch.equal(dH1, dH2)
+    W = oracle_W(wl)
+    olse = O.head_forward(wl.H, W, wl.labels, softcap=cap)[1]
+    want = O.head_dw(wl.H, W, wl.labels, g, olse, filter_eps=eps, softcap=cap)
+    if eps > 0:  # the filter is an approximation: compare with the unfiltered dW
+        want = O.head_dw(wl.H, W, wl.labels, g, olse, softcap=cap)
+    assert rel_fro(dW.cpu().numpy(), want) <= TOL_DH, rel_fro(dW.cpu().numpy(), want)
+
+
+def test_trainable_head_rejects_quantised_heads():
+    wl = S.make_custom(4, M_split=(8, 8, 8), D=128, V=300)
+    H, head, labels = upload(wl)
+    ws = cce.alloc_workspace(wl.M, cce.h_dtype(H), head)
+    f = dict(device="cuda", dtype=torch.float32)
+    z = torch.zeros(wl.M, **f)
+    with pytest.raises(cce.CCEError) as e:
+        cce.cce_backward_dh_dw(H, head, labels, z, z, 0.0, None, torch.empty(wl.M, wl.D, **f),
+                               torch.empty(wl.V, wl.D, **f), None, ws)
+    assert e.value.status == 2

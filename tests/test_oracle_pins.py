@@ -491,3 +491,24 @@ def test_prefix_shared_loss_gradient_by_finite_differences():
             Hp[r, d] += h
             Hm[r, d] -= h
             assert grad[r, d] == pytest.approx((loss(Hp) - loss(Hm)) / (2 * h), rel=1e-6, abs=1e-9)
+
+
+# --------------------------------------------------------------------------
+# trainable head: dL/dW
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cap", [0.0, 2.0])
+def test_head_dw_finite_differences(cap):
+    H, W, y, L = tiny_case(P=3, Rc=2, Rr=3, D=6, V=10, seed=17)
+    logp, lse, _ = O.head_forward(H, W, y, softcap=cap)
+    g = O.orpo_grad_coeffs(logp, y, L, 0.4, "full")
+    dW = O.head_dw(H, W, y, g, lse, softcap=cap)
+    h = 1e-6
+    for v in range(W.shape[0]):
+        for d in range(W.shape[1]):
+            Wp, Wm = W.copy(), W.copy()
+            Wp[v, d] += h
+            Wm[v, d] -= h
+            fd = (O.orpo_head_loss(H, Wp, y, L, 0.4, "full", softcap=cap)
+                  - O.orpo_head_loss(H, Wm, y, L, 0.4, "full", softcap=cap)) / (2 * h)
+            assert dW[v, d] == pytest.approx(fd, rel=1e-6, abs=1e-9)
