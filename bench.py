@@ -46,6 +46,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--workspace-mb", type=int, default=0,
+                   help="workspace size (default: the library's default)")
     return p.parse_args(argv)
 
 
@@ -234,7 +236,8 @@ def run_ours(args):
     torch.cuda.reset_peak_memory_stats(dev)
     base_alloc = torch.cuda.memory_allocated(dev)
     free0, _ = torch.cuda.mem_get_info(dev)
-    buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head, dev)
+    buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head, dev,
+                                ws_bytes=(args.workspace_mb << 20) or None)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -380,7 +383,8 @@ def run_ours(args):
                    "Rc": wl.Rc, "Rr": wl.Rr, "sft_scope": wl.scope, "lambda": wl.lam,
                    "filter_eps": wl.filter_eps, "block_skip": wl.block_skip,
                    "parallelism": f"dp{world} (independent pairs, no collective)",
-                   "l2": "inputs larger than L2 (W is 1.07 GB, L2 126 MB); no flush"},
+                   "l2": "inputs larger than L2 (W is 1.07 GB, L2 126 MB); no flush",
+                   "workspace_bytes": int(buf.ws.numel())},
         "tflops": tflops,
         "pct_bf16_peak": {"sustained": 100.0 * tflops / peak_s,
                           "burst": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),

@@ -275,6 +275,12 @@ const char* cce_status_string(cce_status s);
  * the timeout path. */
 void cce_set_wait_limit_ns(uint64_t ns);
 
+/* Dense heads run the tensor-core GEMMs on CTA pairs (clusters of two
+ * CTAs on one TPC, tcgen05 cta_group::2, 256x256 tiles) by default; 0 selects
+ * single-CTA 128x256 tiles.  Both give the same results to rounding.
+ * Process-wide; a workspace sized under one setting fits the other. */
+void cce_set_cta_pairs(int on);
+
 /* Self-test of the timeout path: launches one CTA that waits, with the
  * current wait limit, on an mbarrier nothing arrives on.  The wait runs out,
  * the kernel sets CCE_ERR_DEVICE_TIMEOUT in the status word and returns;

@@ -87,6 +87,7 @@ _SIGS = {
     "cce_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "cce_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "cce_set_cta_pairs": (None, [ctypes.c_int]),
     "cce_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "pref_loss_from_logps": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                             ctypes.POINTER(_Layout), ctypes.POINTER(_Objective),
@@ -378,3 +379,7 @@ def cce_backward_dh_dw(H, head: Head, labels, lse, coeff, filter_eps, blockmax, 
                                   _p(blockmax), _p(dH), _p(dW), _p(skip_stats), _p(ws),
                                   ws.numel(), _stream(stream))
     _check(st, "cce_backward_dh_dw")
+
+
+def cce_set_cta_pairs(on: bool):
+    lib().cce_set_cta_pairs(1 if on else 0)

@@ -27,6 +27,7 @@ constexpr int64_t kDefaultChunkBytes = 256ll << 20;  // G' chunk, default
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_pairs{1};  // 2-CTA (cta_group::2) tiles for dense heads
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -146,8 +147,30 @@ bool make_map_ex(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int ra
 // --------------------------------------------------------- device facts --
 struct DevInfo {
   int sms = 0;
+  int pairs = 0;  // CTA pairs (clusters of 2) resident at once, 0 = none
   bool attrs = false;
 };
+
+template <Mode MODE>
+int max_pairs_of() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<MODE, true>();
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, cce_tc_kernel<MODE, 0, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
 
@@ -168,12 +191,27 @@ cce_status device_info(int* sms) {
     CCE_SET_SMEM(Mode::kLse, 8) CCE_SET_SMEM(Mode::kGrad, 8) CCE_SET_SMEM(Mode::kDh, 8)
     CCE_SET_SMEM(Mode::kDw, 0)
 #undef CCE_SET_SMEM
+#define CCE_SET_SMEM2(MODE) \
+    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, 0, true>, attr, smem_bytes<MODE, true>()) == cudaSuccess;
+    CCE_SET_SMEM2(Mode::kLse) CCE_SET_SMEM2(Mode::kGrad) CCE_SET_SMEM2(Mode::kDh)
+#undef CCE_SET_SMEM2
+    if (ok)
+      d.pairs = std::min(max_pairs_of<Mode::kLse>(),
+                         std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
     if (!ok)
       return CCE_ERR_CUDA;
     d.attrs = true;
   }
   *sms = d.sms;
   return CCE_OK;
+}
+
+// CTA pairs resident at once on the current device (0: pairs unavailable).
+int device_pairs() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  return g_dev[dev].pairs;
 }
 
 // ------------------------------------------------------------ validation --
@@ -243,7 +281,11 @@ int choose_ksplit(int64_t tiles, int sms) {
   return best;
 }
 
+// Dense heads run the S and dH GEMMs on CTA pairs unless switched off.
+bool pairs_wanted(const cce_head* W) { return g_pairs.load() != 0 && W->format == CCE_W_DENSE; }
+
 int ksplit_for(int64_t M, const cce_head* W, int sms) {
+  if (pairs_wanted(W)) return choose_ksplit(ceil_div(M, 2 * BM) * ceil_div(W->D, BN), sms / 2);
   return choose_ksplit(ceil_div(M, BM) * ceil_div(W->D, BN), sms);
 }
 
@@ -318,6 +360,27 @@ cce_status launch_ok() {
 
 int grid_for(int64_t tiles, int sms) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, sms)));
+}
+
+// Launch a tensor-core step on CTA pairs (clusters of two, cta_group::2).
+template <Mode MODE>
+cudaError_t launch_tc_pairs(int64_t pair_tiles, int max_pairs, cudaStream_t st,
+                            const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
+                            const CUtensorMap& mc2, const TileArgs& args) {
+  cudaLaunchConfig_t cfg = {};
+  const int pairs = int(std::max<int64_t>(1, std::min<int64_t>(pair_tiles, max_pairs)));
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<MODE, true>();
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, cce_tc_kernel<MODE, 0, true>, ma, mb, mc, mc2, args);
 }
 
 // Launch one tensor-core step; a quantised head adds the dequantisation
@@ -427,6 +490,8 @@ const char* cce_status_string(cce_status s) {
 
 void cce_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns); }
 
+void cce_set_cta_pairs(int on) { g_pairs.store(on != 0 ? 1 : 0); }
+
 int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
 
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
@@ -465,10 +530,13 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   float* part_m = blockmax != nullptr ? blockmax : reinterpret_cast<float*>(wsc + L.part_m);
   float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
 
+  const int max_pairs = pairs_wanted(W) ? device_pairs() : 0;
+  const bool pairs = max_pairs > 0;
   CUtensorMap ma, mb;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
   if (op.qb) mb = ma;  // unused: B is dequantised in-kernel
-  else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN)) return CCE_ERR_CUDA;
+  else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN))
+    return CCE_ERR_CUDA;
 
   TileArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -494,9 +562,19 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.group_rt = group_rows(n_rt, op.k);
   a.softcap = W->softcap;
   a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
+  a.n_rt128 = int(n_rt);
   {
     ProfScope ps(PK_LSE, st);
-    launch_tc<Mode::kLse>(op.qb, n_rt * cols, sms, st, ma, mb, ma, ma, a);
+    if (pairs) {
+      TileArgs a2 = a;
+      a2.n_rt = int(ceil_div(M, 2 * BM));
+      a2.group_rt = std::max(1, a.group_rt / 2);
+      if (launch_tc_pairs<Mode::kLse>(int64_t(a2.n_rt) * cols, max_pairs, st, ma, mb, ma, ma,
+                                      a2) != cudaSuccess)
+        return CCE_ERR_CUDA;
+    } else {
+      launch_tc<Mode::kLse>(op.qb, n_rt * cols, sms, st, ma, mb, ma, ma, a);
+    }
   }
   if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
 
@@ -677,11 +755,13 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   }
 
   CUtensorMap ma, mb, mg, mw, mgs, md0, md1;
+  const int max_pairs = pairs_wanted(W) ? device_pairs() : 0;
+  const bool pairs = max_pairs > 0 && ksplit == ksplit_for(M, W, sm_count_guess());
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
   if (op.qb) {
     mb = ma;  // unused: B is dequantised in-kernel
     mw = ma;
-  } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, BN) ||
+  } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN) ||
              !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK)) {
     return CCE_ERR_CUDA;
   }
@@ -729,6 +809,8 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   a.group_rt = group_rows(n_rt, op.k);
   a.softcap = W->softcap;
   a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
+  a.n_rt128 = int(n_rt);
+  const int64_t n_rt2 = ceil_div(M, 2 * BM);
 
   // Trainable head: B operand coeff * H and the dW output map.
   CUtensorMap mhg, mdw;
@@ -776,7 +858,16 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
     }
     {
       ProfScope ps(PK_GRAD, st);
-      launch_tc<Mode::kGrad>(op.qb, n_rt * ct_n, sms, st, ma, mb, mgs, mgs, ag);
+      if (pairs) {
+        TileArgs a2 = ag;
+        a2.n_rt = int(n_rt2);
+        a2.group_rt = std::max(1, ag.group_rt / 2);
+        if (launch_tc_pairs<Mode::kGrad>(n_rt2 * ct_n, max_pairs, st, ma, mb, mgs, mgs, a2) !=
+            cudaSuccess)
+          return CCE_ERR_CUDA;
+      } else {
+        launch_tc<Mode::kGrad>(op.qb, n_rt * ct_n, sms, st, ma, mb, mgs, mgs, ag);
+      }
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     // dH (+)= coeff * G' . W[chunk]
@@ -790,7 +881,15 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
     ad.first_chunk = v0 == 0 ? 1 : 0;
     {
       ProfScope ps(PK_DH, st);
-      launch_tc<Mode::kDh>(op.qb, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);
+      if (pairs) {
+        TileArgs a2 = ad;
+        a2.n_rt = int(n_rt2);
+        if (launch_tc_pairs<Mode::kDh>(n_rt2 * n_dt * ksplit, max_pairs, st, mg, mw, md0, md1,
+                                       a2) != cudaSuccess)
+          return CCE_ERR_CUDA;
+      } else {
+        launch_tc<Mode::kDh>(op.qb, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);
+      }
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     if (dW != nullptr) {

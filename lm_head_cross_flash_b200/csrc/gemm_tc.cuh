@@ -50,9 +50,15 @@ template <Mode MODE>
 __host__ __device__ constexpr int staging_buf_bytes() {
   return MODE == Mode::kGrad ? 32 * 64 : (MODE == Mode::kDh || MODE == Mode::kDw) ? 32 * 128 : 0;
 }
-template <Mode MODE>
+// CTA pairs (cta_group::2): a 256x256 tile per pair, each CTA loads its 128
+// rows of A and half (128 columns) of B, so a stage is 32 KB and 6 fit.
+constexpr int STAGES2 = 6;
+constexpr int B_HALF_BYTES = (BN / 2) * BK * 2;
+constexpr int STAGE2_BYTES = A_BYTES + B_HALF_BYTES;
+template <Mode MODE, bool C2 = false>
 __host__ __device__ constexpr int smem_bytes() {
-  return STAGES * STAGE_BYTES + 4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
+  return (C2 ? STAGES2 * STAGE2_BYTES : STAGES * STAGE_BYTES) +
+         4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
@@ -94,6 +100,7 @@ struct TileArgs {
   int first_chunk;
   int group_rt;    // kLse/kGrad: row tiles per raster group
   int zero_skip_rows;  // kGrad: write zeros (not nothing) for row-skipped tiles
+  int n_rt128;     // 128-row tiles of A (pairs: n_rt counts 256-row tiles)
   float softcap;   // > 0: logits are cap * tanh(s / cap)
   float inv_cap;
   // 4-bit affine head (group 64): words [V, D/8], scales/biases bf16 [V, D/64]
@@ -209,6 +216,19 @@ __device__ __forceinline__ int tile_kind(const TileArgs& a, int rt, int ct) {
   return 0;
 }
 
+// Kind of a pair tile (two 128-row halves): computed when either half is.
+template <Mode MODE>
+__device__ __forceinline__ int pair_kind(const TileArgs& a, int rt2, int ct) {
+  const int k0 = tile_kind<MODE>(a, 2 * rt2, ct);
+  const int k1 = 2 * rt2 + 1 < a.n_rt128 ? tile_kind<MODE>(a, 2 * rt2 + 1, ct) : 2;
+  return (k0 == 0 || k1 == 0) ? 0 : 1;
+}
+
+template <Mode MODE, bool C2>
+__device__ __forceinline__ int launch_kind(const TileArgs& a, int rt, int ct) {
+  return C2 ? pair_kind<MODE>(a, rt, ct) : tile_kind<MODE>(a, rt, ct);
+}
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, int fmt) {
   if (fmt == 1) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -264,23 +284,33 @@ __device__ __forceinline__ void drain_chunks(uint32_t taddr, int nchunks, F&& f)
   }
 }
 
-template <Mode MODE, int QB = 0>
+template <Mode MODE, int QB = 0, bool C2 = false>
 __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     cce_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                   const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC,
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
+  static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
+  static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
+  constexpr int NST = C2 ? STAGES2 : STAGES;
+  constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES;
+  // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
+  // rank 0 (the leader) issues the MMAs for both; each CTA loads its own
+  // 128 rows of A and its half of B and drains its own 128 TMEM lanes.
+  const uint32_t rank = C2 ? cluster_ctarank() : 0u;
+  const int tile0 = C2 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int tstride = C2 ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
   // tmA/tmB: operand loads.  tmC: kGrad G'' store map [M, chunk] (box 32x32,
   // 64-byte swizzle); kDh dH [1, M, D] (box 1x32x32, 128-byte swizzle).
   // tmC2: kDh partial buffers [ksplit-1, M, D].
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t* staging = base + STAGES * STAGE_BYTES;
+  uint8_t* staging = base + NST * SBYTES;
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
-  uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
+  uint64_t* empty = full + NST;
+  uint64_t* acc_full = empty + NST;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -292,13 +322,13 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   const int ntiles = a.n_rt * a.n_ct * nsplit;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], QB ? 1 + DQ_WARPS : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4 * 32);
+      mbar_init(&acc_empty[b], (C2 ? 2 : 1) * 4 * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -308,11 +338,17 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (C2) {
+      tmem_alloc2(tmem_slot, TMEM_COLS);
+      tmem_relinquish2();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (C2) cluster_sync_all();  // barriers of both CTAs initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -326,9 +362,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       // H (kLse/kGrad) and the W chunk (kDh) are re-read by many tiles:
       // keep them in L2 ahead of streaming data.
       const uint64_t keep = l2_policy_evict_last();
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int t = tile0; t < ntiles && ok; t += tstride) {
         const TileCoord tc = tile_coord<MODE>(a, t);
-        if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
+        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct) != 0) continue;
         const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
         const int ksteps = nks * a.npass;
         for (int kk = 0; kk < ksteps; ++kk) {
@@ -336,10 +372,29 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             ok = false;
             break;
           }
-          uint8_t* sA = base + stage * STAGE_BYTES;
+          uint8_t* sA = base + stage * SBYTES;
           uint8_t* sB = sA + A_BYTES;
           const int pass = kk / nks, k = kb + (kk - pass * nks);
-          if (QB) {
+          if constexpr (C2) {
+            // Both CTAs' copies are counted on the leader's barrier.
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * SBYTES);
+            const int arow = (tc.rt * 2 + static_cast<int>(rank)) * BM;
+            if (MODE == Mode::kDh) {
+              tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, l2_policy_evict_normal());
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j)
+                tma_load_2d_pair(sB + j * (64 * BK * 2), &tmB, bar,
+                                 tc.ct * BN + static_cast<int>(rank) * (BN / 2) + j * 64 +
+                                     pass * a.b_pass_off,
+                                 a.b_row0 + k * BK, keep);
+            } else {
+              tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, keep);
+              tma_load_2d_pair(sB, &tmB, bar, k * BK,
+                               a.b_row0 + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
+                               l2_policy_evict_normal());
+            }
+          } else if (QB) {
             // B comes from the dequantisation warps.
             mbar_arrive_expect_tx(&full[stage], A_BYTES);
             if (MODE == Mode::kDh)
@@ -372,7 +427,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
@@ -382,24 +437,27 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         set_status(a.status, ST_TIMEOUT);
         *abort_flag = 1;
       }
-      // Let every issued copy land before the CTA can exit.
-      for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s))
-          wait_bounded(&full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS,
-                       nullptr);
+      // Let every issued copy land before the CTA can exit (in a pair the
+      // leader's barriers also count the other CTA's copies; the final
+      // cluster barrier keeps both CTAs alive until then).
+      if (!C2 || rank == 0)
+        for (int s = 0; s < NST; ++s)
+          if (issued_mask & (1u << s))
+            wait_bounded(&full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS,
+                         nullptr);
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16(BM, BN, a.fmt, MODE == Mode::kDw,
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_f16(C2 ? 2 * BM : BM, BN, a.fmt, MODE == Mode::kDw,
                                        MODE == Mode::kDh || MODE == Mode::kDw);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int t = tile0; t < ntiles && ok; t += tstride) {
         const TileCoord tc = tile_coord<MODE>(a, t);
-        if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
+        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct) != 0) continue;
         const int ksteps =
             ((tc.s + 1) * a.nk / nsplit - tc.s * a.nk / nsplit) * a.npass;
         const int b = acc & 1;
@@ -416,7 +474,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_u32(base + stage * STAGE_BYTES);
+          const uint32_t sA = smem_u32(base + stage * SBYTES);
           const uint32_t sB = sA + A_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
@@ -427,16 +485,22 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                 (MODE == Mode::kDh || MODE == Mode::kDw)
                     ? sdesc_sw128(sB + j * 16 * 128, 64 * BK * 2, 1024)
                     : sdesc_sw128(sB + j * 32, 16, 1024);
-            umma_f16_ss(d_tmem, ad, bd, idesc, (kk | j) != 0 ? 1u : 0u);
+            if constexpr (C2)
+              umma_f16_ss2(d_tmem, ad, bd, idesc, (kk | j) != 0 ? 1u : 0u);
+            else
+              umma_f16_ss(d_tmem, ad, bd, idesc, (kk | j) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
-          if (++stage == STAGES) {
+          // the stage is free in both CTAs once these MMAs have read it
+          if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
+          else umma_commit(&empty[stage]);
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&acc_full[b]);
+        if constexpr (C2) umma_commit2_mc(&acc_full[b], 0x3);
+        else umma_commit(&acc_full[b]);
         ++acc;
       }
       if (!ok) {
@@ -444,7 +508,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         *abort_flag = 1;
       }
       // All MMAs issued by this thread complete before TMEM is released.
-      umma_commit(drain);
+      if constexpr (C2) umma_commit2_mc(drain, 0x1);
+      else umma_commit(drain);
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
     }
   } else if (QB && warp >= DQ_WARP0) {
@@ -496,7 +561,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       }
       return x;
     };
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+    for (int t = tile0; t < ntiles && ok; t += tstride) {
       const TileCoord tc = tile_coord<MODE>(a, t);
       if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
       const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
@@ -508,7 +573,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           ok = false;
           break;
         }
-        uint8_t* sB = base + stage * STAGE_BYTES + A_BYTES;
+        uint8_t* sB = base + stage * SBYTES + A_BYTES;
         {
           const Unit& x = c0;
           const int u = dq;
@@ -532,7 +597,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == STAGES) {
+        if (++stage == NST) {
           stage = 0;
           phase ^= 1u;
         }
@@ -551,14 +616,37 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     int acc = 0;
     uint8_t* const stage_base = staging + quad * 2 * staging_buf_bytes<MODE>();
     uint32_t nstore = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    // Leader's acc_empty barriers (a pair's MMA waits for both CTAs).
+    uint32_t acc_empty_leader[2] = {0u, 0u};
+    if constexpr (C2) {
+      acc_empty_leader[0] = mapa_shared(smem_u32(&acc_empty[0]), 0);
+      acc_empty_leader[1] = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    }
+    for (int t = tile0; t < ntiles; t += tstride) {
       const TileCoord tc = tile_coord<MODE>(a, t);
-      const int rt = tc.rt, ct = tc.ct;
+      // this CTA's 128-row tile
+      const int rt = C2 ? tc.rt * 2 + static_cast<int>(rank) : tc.rt, ct = tc.ct;
       float* const dh_buf =
           tc.s == 0 ? a.dh : a.dh_part + static_cast<size_t>(tc.s - 1) * a.M * a.D;
-      const int kind = tile_kind<MODE>(a, rt, ct);
+      const int kind_launch = launch_kind<MODE, C2>(a, tc.rt, ct);
+      const int kind = !C2 ? kind_launch
+                           : (rt < a.n_rt128 ? tile_kind<MODE>(a, rt, ct) : 2);
       const int row = rt * BM + rin;
       const bool live = row < a.M;
+      if (C2 && kind_launch == 0 && kind != 0) {
+        // The pair computed this tile for the other half: take the
+        // accumulator round trip without using it, then do this half's
+        // zeros (kind 1) or nothing (kind 2).
+        const int b = acc & 1;
+        if (!wait_bounded(&acc_full[b], (acc >> 1) & 1, a.wait_ns, abort_flag)) {
+          set_status(a.status, ST_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(acc_empty_leader[b]);
+        ++acc;
+      }
       if (kind == 2) continue;
       if (kind == 1) {
         if (MODE == Mode::kGrad) {
@@ -640,7 +728,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           }
         });
         tc_fence_before();
-        mbar_arrive(&acc_empty[b]);
+        if constexpr (C2) mbar_arrive_cluster(acc_empty_leader[b]);
+        else mbar_arrive(&acc_empty[b]);
         if (live) {
           const size_t o = static_cast<size_t>(a.ct_off + ct) * a.M + row;
           a.part_m[o] = m_run;
@@ -725,7 +814,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           ++nstore;
         });
         tc_fence_before();
-        mbar_arrive(&acc_empty[b]);
+        if constexpr (C2) mbar_arrive_cluster(acc_empty_leader[b]);
+        else mbar_arrive(&acc_empty[b]);
       } else {  // kDh: dH (+)= -coeff * (G'' . W);  kDw: dW[chunk] = -(G''^T . coeff*H)
         const float g = MODE == Mode::kDw ? -1.f : (live ? -a.coeff[row] : 0.f);
         const int dbase = ct * BN;
@@ -765,7 +855,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           ++nstore;
         });
         tc_fence_before();
-        mbar_arrive(&acc_empty[b]);
+        if constexpr (C2) mbar_arrive_cluster(acc_empty_leader[b]);
+        else mbar_arrive(&acc_empty[b]);
       }
       ++acc;
     }
@@ -776,10 +867,14 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // A pair stays resident until both CTAs are done with each other's shared
+  // memory, barriers and tensor memory.
+  if constexpr (C2) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (C2) tmem_dealloc2(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 

@@ -376,3 +376,28 @@ def test_trainable_head_rejects_quantised_heads():
         cce.cce_backward_dh_dw(H, head, labels, z, z, 0.0, None, torch.empty(wl.M, wl.D, **f),
                                torch.empty(wl.V, wl.D, **f), None, ws)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("cfg,split,D,V", [(1, (40, 45, 44), 128, 257),
+                                           (2, (100, 150, 131), 256, 4097),
+                                           (1, (300, 400, 500), 512, 3000),
+                                           (0, (8, 60, 60), 64, 300)])
+def test_cta_pairs_match_single_cta(cfg, split, D, V):
+    """The 2-CTA (cta_group::2) tiles and the single-CTA tiles agree, and both
+    match the oracle."""
+    wl = S.make_custom(cfg, M_split=split, D=D, V=V)
+    outs = []
+    for pairs in (True, False):
+        cce.cce_set_cta_pairs(pairs)
+        try:
+            _, _, _, buf, st = run_pass(wl)
+        finally:
+            cce.cce_set_cta_pairs(True)
+        assert st == 0
+        outs.append((buf.logp.cpu().numpy(), buf.lse.cpu().numpy(), buf.dH.cpu().numpy()))
+    (lp1, ls1, d1), (lp0, ls0, d0) = outs
+    assert np.max(np.abs(lp1 - lp0)) <= 1e-5 and np.max(np.abs(ls1 - ls0)) <= 1e-5
+    assert rel_fro(d1, d0) <= 1e-3
+    W = oracle_W(wl)
+    ologp, olse, _ = O.head_forward(wl.H, W, wl.labels)
+    assert np.max(np.abs(lp1 - ologp)) <= TOL_LOGP
