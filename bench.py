@@ -48,6 +48,9 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--workspace-mb", type=int, default=0,
                    help="workspace size (default: the library's default)")
+    p.add_argument("--sweep", choices=["small_m"], default=None,
+                   help="small_m: the W-stream (HBM-bound) regime, M in {64, 128, 256} at "
+                        "D=2048, V=262144; one JSON line per M")
     return p.parse_args(argv)
 
 
@@ -404,6 +407,87 @@ def run_ours(args):
     return out
 
 
+# ------------------------------------------------------ small-M sweep --
+
+def run_small_m(args):
+    """Forward and backward of the head at M = 64, 128, 256 (D = 2,048,
+    V = 262,144, bf16, flat H): the regime where streaming W from HBM bounds
+    the time.  Achieved GB/s counts the method's minimum bytes: W once per
+    pass, H in, dH out and the per-row / per-block statistics.  This
+    implementation's backward reads W twice (the G'' recompute and the dH
+    contraction are separate GEMMs) and moves G'' through HBM; those bytes are
+    reported as design_bytes."""
+    import torch
+
+    from lm_head_cross_flash_b200 import cce
+    from lm_head_cross_flash_b200 import synthetic as S
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peaks_src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    lines = []
+    for M in (64, 128, 256):
+        P = M // 8
+        Rc = (M - P) // 2
+        wl = S.make_custom(2, M_split=(P, Rc, M - P - Rc), D=2048, V=262144)
+        H, head, labels = cce.upload_workload(wl, dev)
+        buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head, dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def fwd():
+            cce.cce_forward(H, head, labels, buf.logp, buf.lse, buf.tgt, buf.blockmax, buf.ws,
+                            stream)
+
+        def bwd():
+            cce.cce_backward_dh(H, head, labels, buf.lse, buf.coeff, wl.filter_eps, None,
+                                buf.dH, buf.skip, buf.ws, stream)
+
+        fwd()
+        cce.orpo_grad_coeffs(buf.logp, labels, wl.layout_tuple, wl.lam, wl.scope, buf.coeff,
+                             buf.ws, stream)
+        for _ in range(max(3, args.warmup)):
+            fwd()
+            bwd()
+        torch.cuda.synchronize(dev)
+
+        def timed(f):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                f()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1) / args.steps
+
+        t_f, t_b = timed(fwd), timed(bwd)
+        st = cce.cce_device_status(buf.ws)
+        if st != 0:
+            raise RuntimeError(f"device status {st} in the small-M sweep (M={M})")
+        wbytes = 2.0 * wl.V * wl.D
+        cols = cce.blockmax_cols(wl.V)
+        stats = 4.0 * M * cols + 4.0 * 4 * M
+        fwd_bytes = wbytes + 2.0 * M * wl.D + stats
+        bwd_bytes = wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 3 * 4.0 * M
+        bwd_design = 2 * wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 2 * 2.0 * M * wl.V
+        line = {"sweep": "small_m", "M": M, "D": wl.D, "V": wl.V, "dtype": "bf16",
+                "steps": args.steps, "fwd_ms": t_f, "bwd_ms": t_b,
+                "fwd_gbs": fwd_bytes / (t_f / 1e3) / 1e9,
+                "bwd_gbs": bwd_bytes / (t_b / 1e3) / 1e9,
+                "fwd_frac_hbm": fwd_bytes / (t_f / 1e3) / 1e9 / hbm,
+                "bwd_frac_hbm": bwd_bytes / (t_b / 1e3) / 1e9 / hbm,
+                "fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes,
+                "bwd_design_bytes": bwd_design,
+                "bwd_design_gbs": bwd_design / (t_b / 1e3) / 1e9,
+                "tokens_per_s": M / ((t_f + t_b) / 1e3),
+                "hbm_peak_gbs": hbm, "peak_source": f"{peaks_src} hbm_gbs (MEASURED_PEAKS.json)",
+                "l2": "W (1.07 GB) larger than L2; no flush"}
+        lines.append(line)
+        del buf, H, head, labels
+        torch.cuda.empty_cache()
+    return lines
+
+
 # -------------------------------------------------------- reference arm --
 
 def run_reference(args):
@@ -455,6 +539,10 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.sweep == "small_m":
+        for line in run_small_m(args):
+            print(json.dumps(line), flush=True)
+        return
     out = run_reference(args) if args.impl == "reference" else run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)

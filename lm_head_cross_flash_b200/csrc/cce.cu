@@ -281,11 +281,17 @@ int choose_ksplit(int64_t tiles, int sms) {
   return best;
 }
 
-// Dense heads run the S and dH GEMMs on CTA pairs unless switched off.
-bool pairs_wanted(const cce_head* W) { return g_pairs.load() != 0 && W->format == CCE_W_DENSE; }
+// Dense heads run the S and dH GEMMs on CTA pairs unless switched off, or
+// unless padding the rows to 256-row pair tiles would add more than an eighth
+// to the 128-row tiles' work (M <= 128: a single row tile, HBM-bound on W).
+bool pairs_wanted(int64_t M, const cce_head* W) {
+  if (g_pairs.load() == 0 || W->format != CCE_W_DENSE) return false;
+  const int64_t n128 = ceil_div(M, BM);
+  return n128 >= 2 && 8 * (2 * ceil_div(M, 2 * BM) - n128) <= n128;
+}
 
 int ksplit_for(int64_t M, const cce_head* W, int sms) {
-  if (pairs_wanted(W)) return choose_ksplit(ceil_div(M, 2 * BM) * ceil_div(W->D, BN), sms / 2);
+  if (pairs_wanted(M, W)) return choose_ksplit(ceil_div(M, 2 * BM) * ceil_div(W->D, BN), sms / 2);
   return choose_ksplit(ceil_div(M, BM) * ceil_div(W->D, BN), sms);
 }
 
@@ -530,7 +536,7 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   float* part_m = blockmax != nullptr ? blockmax : reinterpret_cast<float*>(wsc + L.part_m);
   float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
 
-  const int max_pairs = pairs_wanted(W) ? device_pairs() : 0;
+  const int max_pairs = pairs_wanted(M, W) ? device_pairs() : 0;
   const bool pairs = max_pairs > 0;
   CUtensorMap ma, mb;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
@@ -755,7 +761,7 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   }
 
   CUtensorMap ma, mb, mg, mw, mgs, md0, md1;
-  const int max_pairs = pairs_wanted(W) ? device_pairs() : 0;
+  const int max_pairs = pairs_wanted(M, W) ? device_pairs() : 0;
   const bool pairs = max_pairs > 0 && ksplit == ksplit_for(M, W, sm_count_guess());
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
   if (op.qb) {

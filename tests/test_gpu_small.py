@@ -379,12 +379,17 @@ def test_trainable_head_rejects_quantised_heads():
 
 
 @pytest.mark.parametrize("cfg,split,D,V", [(1, (40, 45, 44), 128, 257),
-                                           (2, (100, 150, 131), 256, 4097),
+                                           (2, (100, 150, 262), 256, 4097),
                                            (1, (300, 400, 500), 512, 3000),
-                                           (0, (8, 60, 60), 64, 300)])
+                                           (1, (300, 400, 400), 448, 2000),
+                                           (0, (8, 60, 188), 64, 300),
+                                           (0, (40, 100, 116), 256, 1000)])
 def test_cta_pairs_match_single_cta(cfg, split, D, V):
     """The 2-CTA (cta_group::2) tiles and the single-CTA tiles agree, and both
-    match the oracle."""
+    match the oracle.  Row counts are ones that take pairs (at least two
+    128-row tiles, at most an eighth of padding): 129, 512, 1200, 1100 (nine
+    row tiles, the last pair half empty) and 256 rows; K depths from 2 to 12
+    steps of 64 wrap the 6-stage ring."""
     wl = S.make_custom(cfg, M_split=split, D=D, V=V)
     outs = []
     for pairs in (True, False):
