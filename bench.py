@@ -48,6 +48,10 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--workspace-mb", type=int, default=0,
                    help="workspace size (default: the library's default)")
+    p.add_argument("--quant-staging", type=int, choices=[0, 1, 2], default=0,
+                   help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
+    p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
+                   help="1: 2-CTA (cta_group::2) tiles where they apply; 0: single-CTA tiles")
     p.add_argument("--sweep", choices=["small_m"], default=None,
                    help="small_m: the W-stream (HBM-bound) regime, M in {64, 128, 256} at "
                         "D=2048, V=262144; one JSON line per M")
@@ -233,6 +237,8 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    cce.cce_set_quant_staging(args.quant_staging)
+    cce.cce_set_cta_pairs(bool(args.cta_pairs))
 
     wl = S.make_workload(args.workload)
     H, head, labels = cce.upload_workload(wl, dev)
@@ -387,7 +393,9 @@ def run_ours(args):
                    "filter_eps": wl.filter_eps, "block_skip": wl.block_skip,
                    "parallelism": f"dp{world} (independent pairs, no collective)",
                    "l2": "inputs larger than L2 (W is 1.07 GB, L2 126 MB); no flush",
-                   "workspace_bytes": int(buf.ws.numel())},
+                   "workspace_bytes": int(buf.ws.numel()),
+                   "cta_pairs": bool(args.cta_pairs),
+                   "quant_staging": ["choose", "in-kernel", "staged"][args.quant_staging]},
         "tflops": tflops,
         "pct_bf16_peak": {"sustained": 100.0 * tflops / peak_s,
                           "burst": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),

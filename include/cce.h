@@ -114,7 +114,8 @@ int64_t cce_blockmax_cols(int64_t V);
 /* Bytes of workspace that cce_forward and cce_backward_dh need for this
  * problem with the default backward chunk.  A larger workspace lets the
  * backward use wider vocab chunks (fewer passes); a smaller one (down to
- * cce_workspace_min_bytes) narrower ones.  Returns 0 for invalid input. */
+ * cce_workspace_min_bytes: one 256-column chunk, no K split of the dH GEMM)
+ * narrower ones and fewer K splits.  Returns 0 for invalid input. */
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W);
 size_t cce_workspace_min_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W);
 
@@ -280,6 +281,45 @@ void cce_set_wait_limit_ns(uint64_t ns);
  * single-CTA 128x256 tiles.  Both give the same results to rounding.
  * Process-wide; a workspace sized under one setting fits the other. */
 void cce_set_cta_pairs(int on);
+
+/* How the GEMMs read a 4- or 8-bit head (the dequantisation step of the
+ * quantised-head design, Training design, MLX affine quantisation):
+ *   0  choose (default): staged when M spans at least 8 row tiles of 128 and
+ *      the workspace holds chunks of at least 8,192 head rows, else in-kernel;
+ *   1  in-kernel: extra warps of the GEMM kernels dequantise each B tile into
+ *      shared memory (reads 4.25 or 8.25 bits per weight; the small-M choice);
+ *   2  staged: each vocabulary chunk is first dequantised once into an fp16
+ *      [chunk, D] buffer in the workspace, then the dense fp16 GEMMs (CTA
+ *      pairs) run on it, so the dequantisation is not repeated per row tile.
+ * Both produce the same fp16 weights (w = q*scale + bias rounded once), so
+ * results agree to accumulation order.  Process-wide.  Any other value is
+ * taken as 0.  A workspace of cce_workspace_bytes() under 0 fits every mode
+ * (staged falls back to in-kernel when the chunk would be too narrow). */
+void cce_set_quant_staging(int mode);
+
+/* The execution plan cce_forward and cce_backward_dh would take for this
+ * problem and workspace size under the current settings (host-only: no
+ * launch, no device memory; with no device visible the SM count is taken as
+ * 148).  No counterpart on the pages: it exposes how the workspace size
+ * shapes the chunking, for sizing workspaces and for tests.
+ *   fwd_ok / bwd_ok   1 when the workspace is large enough for the call;
+ *   fwd_chunk         vocab rows per forward launch (the padded vocabulary
+ *                     when the forward runs as one launch);
+ *   bwd_chunk         vocab rows per backward G'' chunk;
+ *   bwd_ksplit        K splits of the dH GEMM (fp32 partial buffers);
+ *   *_staged          1 when a 4/8-bit head runs as staged fp16 chunks;
+ *   *_cta_pairs       1 when the GEMMs are planned on CTA pairs (used if the
+ *                     device can co-schedule them).
+ * Returns CCE_ERR_INVALID_ARGUMENT / UNSUPPORTED as the calls would. */
+typedef struct {
+  int fwd_ok, bwd_ok;
+  int64_t fwd_chunk, bwd_chunk;
+  int bwd_ksplit;
+  int fwd_staged, bwd_staged;
+  int fwd_cta_pairs, bwd_cta_pairs;
+} cce_plan;
+cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
+                          cce_plan* out);
 
 /* Self-test of the timeout path: launches one CTA that waits, with the
  * current wait limit, on an mbarrier nothing arrives on.  The wait runs out,

@@ -58,6 +58,14 @@ class _Layout(ctypes.Structure):
         "rejected_begin", "rejected_end")]
 
 
+class _Plan(ctypes.Structure):
+    _fields_ = [("fwd_ok", ctypes.c_int), ("bwd_ok", ctypes.c_int),
+                ("fwd_chunk", ctypes.c_int64), ("bwd_chunk", ctypes.c_int64),
+                ("bwd_ksplit", ctypes.c_int),
+                ("fwd_staged", ctypes.c_int), ("bwd_staged", ctypes.c_int),
+                ("fwd_cta_pairs", ctypes.c_int), ("bwd_cta_pairs", ctypes.c_int)]
+
+
 _lib = None
 
 _SIGS = {
@@ -88,6 +96,9 @@ _SIGS = {
     "cce_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "cce_set_cta_pairs": (None, [ctypes.c_int]),
+    "cce_set_quant_staging": (None, [ctypes.c_int]),
+    "cce_query_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_Head),
+                                      ctypes.c_size_t, ctypes.POINTER(_Plan)]),
     "cce_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "pref_loss_from_logps": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                             ctypes.POINTER(_Layout), ctypes.POINTER(_Objective),
@@ -383,3 +394,18 @@ def cce_backward_dh_dw(H, head: Head, labels, lse, coeff, filter_eps, blockmax, 
 
 def cce_set_cta_pairs(on: bool):
     lib().cce_set_cta_pairs(1 if on else 0)
+
+
+def cce_set_quant_staging(mode: int):
+    """0: choose; 1: dequantise inside the GEMMs; 2: staged fp16 chunks."""
+    lib().cce_set_quant_staging(int(mode))
+
+
+def cce_query_plan(M: int, H_dtype: int, head: "Head | _Head", ws_bytes: int) -> dict:
+    """The chunking, K split, staging and CTA-pair plan the forward and
+    backward would take with a workspace of ``ws_bytes`` (host-only)."""
+    out = _Plan()
+    h = head.c() if isinstance(head, Head) else head
+    _check(lib().cce_query_plan(M, H_dtype, ctypes.byref(h), ws_bytes, ctypes.byref(out)),
+           "cce_query_plan")
+    return {n: getattr(out, n) for n, _ in _Plan._fields_}

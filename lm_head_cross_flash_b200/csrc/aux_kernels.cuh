@@ -276,6 +276,57 @@ __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
   }
 }
 
+// ---------------------------------------------- staged dequantisation --
+// fp16 rows [rows, D] of a 4- or 8-bit affine head, vocab rows v0 .. v0+rows,
+// in natural column order: w = q * scale + bias per group of 64 along D.  The
+// values are those the in-kernel dequantiser produces (same fp16 fma), only
+// the K-interleaved pairs it emits are put back in order with byte permutes.
+// One thread per (row, group): 32 (4-bit) or 64 (8-bit) bytes in, 128 out.
+template <int QB>
+__global__ void dequant_rows_f16_kernel(const uint32_t* __restrict__ qw,
+                                        const uint16_t* __restrict__ scales,
+                                        const uint16_t* __restrict__ biases, int64_t v0,
+                                        int64_t rows, int D, uint4* __restrict__ out) {
+  static_assert(QB == 4 || QB == 8, "4- or 8-bit heads");
+  const int gpr = D / 64;
+  const int64_t units = rows * gpr;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = u / gpr;
+    const int g = static_cast<int>(u - r * gpr);
+    const int64_t v = v0 + r;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        qw + static_cast<size_t>(v) * (D / (32 / QB)) + static_cast<size_t>(g) * (2 * QB));
+    const uint16_t sc = __ldg(scales + static_cast<size_t>(v) * gpr + g);
+    const uint16_t bi = __ldg(biases + static_cast<size_t>(v) * gpr + g);
+    uint4 h[8];
+    if constexpr (QB == 8) {
+      uint4 wv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wv[i] = __ldg(src + i);
+      dequant_group64_q8(wv, sc, bi, h);
+    } else {
+      dequant_group64(__ldg(src), __ldg(src + 1), sc, bi, h);
+    }
+    uint4* dst = out + (static_cast<size_t>(r) * D + static_cast<size_t>(g) * 64) / 8;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      // 4-bit: halves (e0,e4) (e1,e5) (e2,e6) (e3,e7); 8-bit: (e0,e2) (e1,e3)
+      // (e4,e6) (e5,e7).  Natural order is (e0,e1) (e2,e3) (e4,e5) (e6,e7).
+      const uint32_t t0 = h[c].x, t1 = h[c].y, t2 = h[c].z, t3 = h[c].w;
+      uint4 n;
+      if constexpr (QB == 4) {
+        n = make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t2, t3, 0x5410),
+                       __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x7632));
+      } else {
+        n = make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632),
+                       __byte_perm(t2, t3, 0x5410), __byte_perm(t2, t3, 0x7632));
+      }
+      dst[c] = n;
+    }
+  }
+}
+
 // ---------------------------------------------------- trainable head --
 // hg[m, d] = bf16(coeff[m] * H[m, d]): the B operand of the dW GEMM (the row
 // cotangent enters along K, so it is folded into the rows of H).

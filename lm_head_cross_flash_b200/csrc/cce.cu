@@ -28,6 +28,12 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_pairs{1};  // 2-CTA (cta_group::2) tiles for dense heads
+// 4/8-bit heads: 0 = choose, 1 = dequantise inside the GEMM, 2 = staged chunks
+std::atomic<int> g_qstage{0};
+// Staged dequantisation pays off once several row tiles reuse each weight:
+// at least this many 128-row tiles, and chunks of at least this many rows.
+constexpr int64_t kStageMinRowTiles = 8;
+constexpr int64_t kStageMinRows = 8192;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -78,12 +84,13 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
   PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM,
-  PK_PREFIX, PK_DW, PK_N
+  PK_PREFIX, PK_DW, PK_DEQ, PK_N
 };
 const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
                                       "bwd_dh_gemm",   "selftest",     "dh_split_sum",
-                                      "prefix_gather_scatter", "bwd_dw_gemm"};
+                                      "prefix_gather_scatter", "bwd_dw_gemm",
+                                      "dequant_chunk"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -247,6 +254,8 @@ struct Layout {
   size_t g = 0, tile_skip = 0, row_skip = 0;
   size_t dh_part = 0;                      // K-split partial dH buffers
   size_t hg = 0;                           // coeff * H (bf16), trainable head
+  size_t wq = 0;                           // staged fp16 chunk of a 4/8-bit head
+  bool staged = false;
   int64_t vc = 0;                          // backward vocab chunk
   int ksplit = 1;
   size_t total = 0;
@@ -262,18 +271,21 @@ int sm_count_guess() {
   return 148;
 }
 
-// K split of the dH GEMM: the smallest S in 1..4 whose tile count fills the
+// K split of the dH GEMM: the smallest S whose tile count fills the
 // persistent grid's last wave best (each split needs its own fp32 partial
-// buffer, summed once at the end).  Every chunk has at least 4 K steps, so
-// every split gets at least one.
+// buffer, summed once at the end).  S goes up to 4, or up to the number of
+// splits that fill the grid once when there are few tiles (small M: the
+// GEMM then streams W at full bandwidth; the buffers are small).  A split
+// that gets no K steps of a narrow chunk only zeroes its buffer.
 int choose_ksplit(int64_t tiles, int sms) {
   auto eff = [&](int S) {
     const double w = double(tiles) * S / sms;
     return w / std::ceil(w);
   };
+  const int smax = int(std::max<int64_t>(4, std::min<int64_t>(32, sms / std::max<int64_t>(1, tiles))));
   int best = 1;
   double be = eff(1);
-  for (int S = 2; S <= 4; ++S)
+  for (int S = 2; S <= smax; ++S)
     if (eff(S) > be + 0.03) {
       best = S;
       be = eff(S);
@@ -284,18 +296,19 @@ int choose_ksplit(int64_t tiles, int sms) {
 // Dense heads run the S and dH GEMMs on CTA pairs unless switched off, or
 // unless padding the rows to 256-row pair tiles would add more than an eighth
 // to the 128-row tiles' work (M <= 128: a single row tile, HBM-bound on W).
-bool pairs_wanted(int64_t M, const cce_head* W) {
-  if (g_pairs.load() == 0 || W->format != CCE_W_DENSE) return false;
+bool pairs_wanted(int64_t M, const cce_head* W, bool staged = false) {
+  if (g_pairs.load() == 0 || (W->format != CCE_W_DENSE && !staged)) return false;
   const int64_t n128 = ceil_div(M, BM);
   return n128 >= 2 && 8 * (2 * ceil_div(M, 2 * BM) - n128) <= n128;
 }
 
-int ksplit_for(int64_t M, const cce_head* W, int sms) {
-  if (pairs_wanted(M, W)) return choose_ksplit(ceil_div(M, 2 * BM) * ceil_div(W->D, BN), sms / 2);
+int ksplit_for(int64_t M, const cce_head* W, int sms, bool staged = false) {
+  if (pairs_wanted(M, W, staged)) return choose_ksplit(ceil_div(M, 2 * BM) * ceil_div(W->D, BN), sms / 2);
   return choose_ksplit(ceil_div(M, BM) * ceil_div(W->D, BN), sms);
 }
 
-Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ksplit = 1) {
+Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ksplit = 1,
+                   bool staged = false) {
   Layout L;
   const int64_t cols = ceil_div(W->V, BN);
   const int64_t n_rt = ceil_div(M, BM);
@@ -321,8 +334,12 @@ Layout make_layout(int64_t M, cce_dtype h, const cce_head* W, int64_t vc, int ks
     L.hs = s; s += align_up(size_t(M) * 3 * W->D * 2);
     L.ws = s; s += align_up(size_t(W->V) * 3 * W->D * 2);
   } else if (W->format != CCE_W_DENSE) {
-    L.hs = s; s += align_up(size_t(M) * W->D * 2);  // fp16, K-permuted rows
+    L.hs = s; s += align_up(size_t(M) * W->D * 2);  // fp16 rows (K-permuted unless staged)
+    if (staged) {
+      L.wq = s; s += align_up(size_t(vc) * W->D * 2);  // fp16 [vc, D] head chunk
+    }
   }
+  L.staged = staged && W->format != CCE_W_DENSE;
   L.vc = vc;
   L.total = s;
   return L;
@@ -346,16 +363,74 @@ int64_t default_vc(int64_t M, const cce_head* W) {
 
 // Widest chunk whose layout fits in ws_bytes (0 if even the narrowest
 // does not fit).
-int64_t fit_vc(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes, int ksplit) {
+int64_t fit_vc(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes, int ksplit,
+              bool staged = false) {
   const int64_t vmax = ceil_div(W->V, BN) * BN;
-  if (make_layout(M, h, W, BN, ksplit).total > ws_bytes) return 0;
+  if (make_layout(M, h, W, BN, ksplit, staged).total > ws_bytes) return 0;
   int64_t lo = 1, hi = vmax / BN;
   while (lo < hi) {
     const int64_t mid = (lo + hi + 1) / 2;
-    if (make_layout(M, h, W, mid * BN, ksplit).total <= ws_bytes) lo = mid;
+    if (make_layout(M, h, W, mid * BN, ksplit, staged).total <= ws_bytes) lo = mid;
     else hi = mid - 1;
   }
   return lo * BN;
+}
+
+// A 4/8-bit head is dequantised chunk by chunk into fp16 in the workspace
+// (then the dense GEMMs run on it) when enough row tiles reuse each weight.
+bool q_stage_wanted(int64_t M, const cce_head* W) {
+  if (W->format == CCE_W_DENSE) return false;
+  const int mode = g_qstage.load();
+  return mode == 2 || (mode == 0 && ceil_div(M, BM) >= kStageMinRowTiles);
+}
+
+// Smallest staged chunk worth its launches (the whole head if it is smaller).
+int64_t stage_min_rows(const cce_head* W) {
+  return std::min<int64_t>(kStageMinRows, ceil_div(W->V, BN) * BN);
+}
+
+// How one forward call runs for a workspace size: staged chunks of vq rows
+// (4/8-bit heads at large M), else a single launch over the vocabulary.
+struct FwdPlan {
+  bool staged = false;
+  int64_t vq = 0;
+  Layout L;
+};
+FwdPlan plan_forward(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes) {
+  FwdPlan p;
+  p.staged = q_stage_wanted(M, W);
+  if (p.staged && (p.vq = fit_vc(M, h, W, ws_bytes, 1, true)) < stage_min_rows(W))
+    p.staged = false;
+  p.L = p.staged ? make_layout(M, h, W, p.vq, 1, true) : make_layout(M, h, W, BN);
+  if (!p.staged) p.vq = ceil_div(W->V, BN) * BN;
+  return p;
+}
+
+// How one backward call runs: the G'' chunk vc, the K split of the dH GEMM
+// (fewer splits when the workspace cannot hold their buffers), staging of a
+// 4/8-bit head (only with chunks of stage_min_rows or more), and whether the
+// split is the one CTA pairs were sized for.  vc == 0: workspace too small.
+struct BwdPlan {
+  bool staged = false;
+  int ksplit = 1;
+  int64_t vc = 0;
+  bool pairs = false;
+  Layout L;
+};
+BwdPlan plan_backward(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes) {
+  BwdPlan p;
+  p.staged = q_stage_wanted(M, W);
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    p.ksplit = ksplit_for(M, W, sm_count_guess(), p.staged);
+    while ((p.vc = fit_vc(M, h, W, ws_bytes, p.ksplit, p.staged)) == 0 && p.ksplit > 1)
+      --p.ksplit;
+    if (!p.staged || p.vc >= stage_min_rows(W)) break;
+    p.staged = false;
+  }
+  p.pairs = pairs_wanted(M, W, p.staged) &&
+            p.ksplit == ksplit_for(M, W, sm_count_guess(), p.staged);
+  if (p.vc > 0) p.L = make_layout(M, h, W, p.vc, p.ksplit, p.staged);
+  return p;
 }
 
 uint32_t* status_word(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
@@ -410,6 +485,7 @@ void launch_tc(int qb, int64_t tiles, int sms, cudaStream_t st, const CUtensorMa
 // and B (head) with their K extents.
 struct Operands {
   int qb;          // 4 / 8: quantised head, B is dequantised in-kernel, A is fp16
+  int stage_qb = 0;  // 4 / 8: quantised head staged as fp16 chunks in b
   const void* a;   // [M, ka] 16-bit
   const void* b;   // [V, kb] 16-bit (dense heads)
   int64_t k;       // contraction length used by the S GEMM
@@ -423,6 +499,27 @@ cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_hea
                             const Layout& L, void* ws, cudaStream_t st, Operands* op) {
   const int64_t D = W->D;
   op->qb = W->format == CCE_W_AFFINE_Q4_G64 ? 4 : W->format == CCE_W_AFFINE_Q8_G64 ? 8 : 0;
+  op->stage_qb = 0;
+  if (op->qb && L.staged) {
+    // fp16 rows in natural order; B is the fp16 chunk staged by stage_chunk
+    uint4* h16 = reinterpret_cast<uint4*>(static_cast<char*>(ws) + L.hs);
+    {
+      ProfScope ps(PK_SPLIT, st);
+      h_to_f16_perm_kernel<0><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+    }
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    op->stage_qb = op->qb;
+    op->qb = 0;
+    op->a = h16;
+    op->b = static_cast<char*>(ws) + L.wq;
+    op->k = D;
+    op->ld_a = D;
+    op->ld_b = D;
+    op->bf16 = false;
+    op->d_pass_off = 0;
+    op->npass_dh = 1;
+    return CCE_OK;
+  }
   if (op->qb) {
     uint4* h16 = reinterpret_cast<uint4*>(static_cast<char*>(ws) + L.hs);
     {
@@ -474,6 +571,26 @@ cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_hea
   return CCE_OK;
 }
 
+// Dequantise head rows [v0, v0 + rows) of a staged 4/8-bit head into the
+// fp16 chunk buffer (op.b).
+cce_status stage_chunk(const Operands& op, const cce_head* W, int64_t v0, int64_t rows,
+                       int sms, cudaStream_t st) {
+  const int64_t units = rows * (W->D / 64);
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, 256), 8 * sms)));
+  const auto* qw = static_cast<const uint32_t*>(W->w);
+  const auto* sc = static_cast<const uint16_t*>(W->scales);
+  const auto* bi = static_cast<const uint16_t*>(W->biases);
+  uint4* out = static_cast<uint4*>(const_cast<void*>(op.b));
+  {
+    ProfScope ps(PK_DEQ, st);
+    if (op.stage_qb == 4)
+      dequant_rows_f16_kernel<4><<<grid, 256, 0, st>>>(qw, sc, bi, v0, rows, int(W->D), out);
+    else
+      dequant_rows_f16_kernel<8><<<grid, 256, 0, st>>>(qw, sc, bi, v0, rows, int(W->D), out);
+  }
+  return launch_ok();
+}
+
 }  // namespace
 
 // ========================================================================
@@ -498,16 +615,42 @@ void cce_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? kDefaultWait
 
 void cce_set_cta_pairs(int on) { g_pairs.store(on != 0 ? 1 : 0); }
 
+void cce_set_quant_staging(int mode) { g_qstage.store(mode == 1 || mode == 2 ? mode : 0); }
+
+cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
+                          cce_plan* out) {
+  if (out == nullptr || M <= 0 || M > (int64_t(1) << 30)) return CCE_ERR_INVALID_ARGUMENT;
+  if (h_dtype != CCE_F32 && h_dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
+  const cce_status s = check_head(W, h_dtype);
+  if (s != CCE_OK) return s;
+  std::memset(out, 0, sizeof(*out));
+  const FwdPlan f = plan_forward(M, h_dtype, W, ws_bytes);
+  const BwdPlan b = plan_backward(M, h_dtype, W, ws_bytes);
+  out->fwd_ok = f.L.total <= ws_bytes;
+  out->fwd_chunk = f.vq;
+  out->fwd_staged = f.staged;
+  out->fwd_cta_pairs = pairs_wanted(M, W, f.staged);
+  out->bwd_ok = b.vc > 0;
+  out->bwd_chunk = b.vc;
+  out->bwd_ksplit = b.ksplit;
+  out->bwd_staged = b.staged;
+  out->bwd_cta_pairs = b.vc > 0 && b.pairs;
+  return CCE_OK;
+}
+
 int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
 
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
-  return make_layout(M, h_dtype, W, default_vc(M, W), ksplit_for(M, W, sm_count_guess())).total;
+  const bool staged = q_stage_wanted(M, W);
+  return make_layout(M, h_dtype, W, default_vc(M, W),
+                     ksplit_for(M, W, sm_count_guess(), staged), staged)
+      .total;
 }
 
 size_t cce_workspace_min_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
-  return make_layout(M, h_dtype, W, BN, ksplit_for(M, W, sm_count_guess())).total;
+  return make_layout(M, h_dtype, W, BN, 1).total;  // narrowest chunk, no K split
 }
 
 cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_head* W,
@@ -520,7 +663,11 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   if (!aligned16(H) || !aligned16(ws)) return CCE_ERR_INVALID_ARGUMENT;
   cce_status s = check_head(W, h_dtype);
   if (s != CCE_OK) return s;
-  const Layout L = make_layout(M, h_dtype, W, BN);
+  // A staged 4/8-bit head takes the widest fp16 chunk the workspace holds.
+  const FwdPlan plan = plan_forward(M, h_dtype, W, ws_bytes);
+  const bool staged = plan.staged;
+  const int64_t vq = plan.vq;
+  const Layout& L = plan.L;
   if (L.total > ws_bytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
   int sms = 0;
   if ((s = device_info(&sms)) != CCE_OK) return s;
@@ -536,11 +683,11 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   float* part_m = blockmax != nullptr ? blockmax : reinterpret_cast<float*>(wsc + L.part_m);
   float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
 
-  const int max_pairs = pairs_wanted(M, W) ? device_pairs() : 0;
-  const bool pairs = max_pairs > 0;
+  const int max_pairs = pairs_wanted(M, W, staged) ? device_pairs() : 0;
+  const bool pairs = max_pairs > 0;  // forward tiles need no K split
   CUtensorMap ma, mb;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
-  if (op.qb) mb = ma;  // unused: B is dequantised in-kernel
+  if (op.qb || staged) mb = ma;  // in-kernel dequantisation / set per staged chunk
   else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN))
     return CCE_ERR_CUDA;
 
@@ -569,20 +716,34 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   a.softcap = W->softcap;
   a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
   a.n_rt128 = int(n_rt);
-  {
+  // One launch over the whole vocabulary, or one per staged chunk.
+  const int64_t step = staged ? vq : cols * BN;
+  for (int64_t v0 = 0; v0 < V; v0 += step) {
+    const int64_t w = std::min<int64_t>(step, V - v0);
+    const int64_t ct_n = ceil_div(w, BN);
+    TileArgs ac = a;
+    if (staged) {
+      if ((s = stage_chunk(op, W, v0, w, sms, st)) != CCE_OK) return s;
+      if (!make_map(&mb, op.b, false, op.k, w, op.ld_b, BK, pairs ? BN / 2 : BN))
+        return CCE_ERR_CUDA;
+      ac.n_ct = int(ct_n);
+      ac.b_row0 = int(v0);
+      ac.b_shift = int(v0);
+      ac.ct_off = int(v0 / BN);
+    }
     ProfScope ps(PK_LSE, st);
     if (pairs) {
-      TileArgs a2 = a;
+      TileArgs a2 = ac;
       a2.n_rt = int(ceil_div(M, 2 * BM));
-      a2.group_rt = std::max(1, a.group_rt / 2);
-      if (launch_tc_pairs<Mode::kLse>(int64_t(a2.n_rt) * cols, max_pairs, st, ma, mb, ma, ma,
+      a2.group_rt = std::max(1, ac.group_rt / 2);
+      if (launch_tc_pairs<Mode::kLse>(int64_t(a2.n_rt) * ct_n, max_pairs, st, ma, mb, ma, ma,
                                       a2) != cudaSuccess)
         return CCE_ERR_CUDA;
     } else {
-      launch_tc<Mode::kLse>(op.qb, n_rt * cols, sms, st, ma, mb, ma, ma, a);
+      launch_tc<Mode::kLse>(op.qb, n_rt * ct_n, sms, st, ma, mb, ma, ma, ac);
     }
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
-  if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
 
   const int rows_per_block = 8;
   {
@@ -728,11 +889,14 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   if (s != CCE_OK) return s;
   // K split of the dH GEMM; fall back to fewer splits if the workspace
   // cannot hold their partial buffers.
-  int ksplit = ksplit_for(M, W, sm_count_guess());
-  int64_t vc = 0;
-  while ((vc = fit_vc(M, h_dtype, W, ws_bytes, ksplit)) == 0 && ksplit > 1) --ksplit;
-  if (vc == 0) return CCE_ERR_WORKSPACE_TOO_SMALL;
-  const Layout L = make_layout(M, h_dtype, W, vc, ksplit);
+  // A staged 4/8-bit head needs chunks of stage_min_rows at least; else the
+  // GEMMs dequantise in-kernel.
+  const BwdPlan plan = plan_backward(M, h_dtype, W, ws_bytes);
+  if (plan.vc == 0) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  const bool staged = plan.staged;
+  const int ksplit = plan.ksplit;
+  const int64_t vc = plan.vc;
+  const Layout& L = plan.L;
   int sms = 0;
   if ((s = device_info(&sms)) != CCE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -761,11 +925,11 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   }
 
   CUtensorMap ma, mb, mg, mw, mgs, md0, md1;
-  const int max_pairs = pairs_wanted(M, W) ? device_pairs() : 0;
-  const bool pairs = max_pairs > 0 && ksplit == ksplit_for(M, W, sm_count_guess());
+  const int max_pairs = plan.pairs ? device_pairs() : 0;
+  const bool pairs = max_pairs > 0;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
-  if (op.qb) {
-    mb = ma;  // unused: B is dequantised in-kernel
+  if (op.qb || staged) {
+    mb = ma;  // B is dequantised in-kernel, or mapped per staged chunk
     mw = ma;
   } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN) ||
              !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK)) {
@@ -844,8 +1008,15 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   for (int64_t v0 = 0; v0 < V; v0 += vc) {
     const int64_t w = std::min<int64_t>(vc, V - v0);
     const int64_t ct_n = ceil_div(w, BN);
+    if (staged) {
+      if ((s = stage_chunk(op, W, v0, w, sms, st)) != CCE_OK) return s;
+      if (!make_map(&mb, op.b, false, op.k, w, op.ld_b, BK, pairs ? BN / 2 : BN) ||
+          !make_map(&mw, op.b, false, op.ld_b, w, op.ld_b, 64, BK))
+        return CCE_ERR_CUDA;
+    }
     // G' = onehot - softmax for this chunk
     TileArgs ag = a;
+    ag.b_shift = staged ? int(v0) : 0;
     ag.n_ct = int(ct_n);
     ag.nk = int(op.k / BK);
     ag.npass = 1;
@@ -884,6 +1055,7 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
     ad.npass = op.npass_dh;
     ad.b_pass_off = int(op.d_pass_off);
     ad.b_row0 = int(v0);
+    ad.b_shift = staged ? int(v0) : 0;
     ad.first_chunk = v0 == 0 ? 1 : 0;
     {
       ProfScope ps(PK_DH, st);

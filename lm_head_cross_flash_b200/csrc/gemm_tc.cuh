@@ -73,6 +73,7 @@ struct TileArgs {
   int npass;     // passes over K (kDh: hi/lo halves of a split f32 head)
   int b_pass_off;  // kDh: B inner-coordinate offset of pass 1
   int b_row0;    // kLse/kGrad: first vocab row of this launch; kDh: chunk v0
+  int b_shift;   // B tensor-map row of vocab row v is v - b_shift (a staged chunk)
   int V;
   int D;
   int fmt;       // operand format: 0 = f16, 1 = bf16
@@ -119,7 +120,9 @@ __host__ __device__ constexpr int q8_pos(int e) {
   return (e & 4) + ((e & 3) == 1 ? 2 : (e & 3) == 2 ? 1 : (e & 3));
 }
 template <int QB>
-__host__ __device__ constexpr int qpos(int e) { return QB == 8 ? q8_pos(e) : q4_pos(e); }
+__host__ __device__ constexpr int qpos(int e) {
+  return QB == 8 ? q8_pos(e) : QB == 4 ? q4_pos(e) : e;
+}
 
 // 8-bit variant: 16 packed words (element 4c+j = byte j of word c).
 __device__ __forceinline__ void dequant_group64_q8(const uint4 (&wv)[4], uint16_t sbits,
@@ -202,9 +205,11 @@ __device__ __forceinline__ TileCoord tile_coord(const TileArgs& a, int t) {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
-// 0 = compute, 1 = write zeros only, 2 = nothing.
+// 0 = compute, 1 = write zeros only, 2 = nothing.  s: the K split of a kDh
+// tile; a split left without K steps (a chunk narrower than the split count)
+// only zeroes its buffer on the first chunk.
 template <Mode MODE>
-__device__ __forceinline__ int tile_kind(const TileArgs& a, int rt, int ct) {
+__device__ __forceinline__ int tile_kind(const TileArgs& a, int rt, int ct, int s = 0) {
   if (MODE == Mode::kLse || MODE == Mode::kDw) return 0;
   const bool rs = a.row_skip != nullptr && a.row_skip[rt] != 0;
   if (MODE == Mode::kGrad) {
@@ -212,21 +217,21 @@ __device__ __forceinline__ int tile_kind(const TileArgs& a, int rt, int ct) {
     if (a.tile_skip != nullptr && a.tile_skip[rt * a.skip_ld + a.ct_off + ct]) return 1;
     return 0;
   }
-  if (rs) return a.first_chunk ? 1 : 2;
+  if (rs || (s + 1) * a.nk / a.ksplit == s * a.nk / a.ksplit) return a.first_chunk ? 1 : 2;
   return 0;
 }
 
 // Kind of a pair tile (two 128-row halves): computed when either half is.
 template <Mode MODE>
-__device__ __forceinline__ int pair_kind(const TileArgs& a, int rt2, int ct) {
-  const int k0 = tile_kind<MODE>(a, 2 * rt2, ct);
-  const int k1 = 2 * rt2 + 1 < a.n_rt128 ? tile_kind<MODE>(a, 2 * rt2 + 1, ct) : 2;
+__device__ __forceinline__ int pair_kind(const TileArgs& a, int rt2, int ct, int s) {
+  const int k0 = tile_kind<MODE>(a, 2 * rt2, ct, s);
+  const int k1 = 2 * rt2 + 1 < a.n_rt128 ? tile_kind<MODE>(a, 2 * rt2 + 1, ct, s) : 2;
   return (k0 == 0 || k1 == 0) ? 0 : 1;
 }
 
 template <Mode MODE, bool C2>
-__device__ __forceinline__ int launch_kind(const TileArgs& a, int rt, int ct) {
-  return C2 ? pair_kind<MODE>(a, rt, ct) : tile_kind<MODE>(a, rt, ct);
+__device__ __forceinline__ int launch_kind(const TileArgs& a, int rt, int ct, int s) {
+  return C2 ? pair_kind<MODE>(a, rt, ct, s) : tile_kind<MODE>(a, rt, ct, s);
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, int fmt) {
@@ -364,7 +369,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       const uint64_t keep = l2_policy_evict_last();
       for (int t = tile0; t < ntiles && ok; t += tstride) {
         const TileCoord tc = tile_coord<MODE>(a, t);
-        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct) != 0) continue;
+        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct, tc.s) != 0) continue;
         const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
         const int ksteps = nks * a.npass;
         for (int kk = 0; kk < ksteps; ++kk) {
@@ -387,11 +392,11 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                 tma_load_2d_pair(sB + j * (64 * BK * 2), &tmB, bar,
                                  tc.ct * BN + static_cast<int>(rank) * (BN / 2) + j * 64 +
                                      pass * a.b_pass_off,
-                                 a.b_row0 + k * BK, keep);
+                                 a.b_row0 - a.b_shift + k * BK, keep);
             } else {
               tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, keep);
               tma_load_2d_pair(sB, &tmB, bar, k * BK,
-                               a.b_row0 + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
+                               a.b_row0 - a.b_shift + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
                                l2_policy_evict_normal());
             }
           } else if (QB) {
@@ -419,11 +424,11 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             for (int j = 0; j < BN / 64; ++j)
               tma_load_2d_hint(sB + j * (64 * BK * 2), &tmB, &full[stage],
                                tc.ct * BN + j * 64 + pass * a.b_pass_off,
-                               a.b_row0 + k * BK, keep);
+                               a.b_row0 - a.b_shift + k * BK, keep);
           } else {
             mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
             tma_load_2d_hint(sA, &tmA, &full[stage], k * BK, tc.rt * BM, keep);
-            tma_load_2d(sB, &tmB, &full[stage], k * BK, a.b_row0 + tc.ct * BN);
+            tma_load_2d(sB, &tmB, &full[stage], k * BK, a.b_row0 - a.b_shift + tc.ct * BN);
           }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       bool ok = true;
       for (int t = tile0; t < ntiles && ok; t += tstride) {
         const TileCoord tc = tile_coord<MODE>(a, t);
-        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct) != 0) continue;
+        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct, tc.s) != 0) continue;
         const int ksteps =
             ((tc.s + 1) * a.nk / nsplit - tc.s * a.nk / nsplit) * a.npass;
         const int b = acc & 1;
@@ -563,7 +568,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     };
     for (int t = tile0; t < ntiles && ok; t += tstride) {
       const TileCoord tc = tile_coord<MODE>(a, t);
-      if (tile_kind<MODE>(a, tc.rt, tc.ct) != 0) continue;
+      if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
       const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
       Unit c0 = load(tc, kb, dq);
       for (int kk = 0; kk < nks; ++kk) {
@@ -628,9 +633,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       const int rt = C2 ? tc.rt * 2 + static_cast<int>(rank) : tc.rt, ct = tc.ct;
       float* const dh_buf =
           tc.s == 0 ? a.dh : a.dh_part + static_cast<size_t>(tc.s - 1) * a.M * a.D;
-      const int kind_launch = launch_kind<MODE, C2>(a, tc.rt, ct);
+      const int kind_launch = launch_kind<MODE, C2>(a, tc.rt, ct, tc.s);
       const int kind = !C2 ? kind_launch
-                           : (rt < a.n_rt128 ? tile_kind<MODE>(a, rt, ct) : 2);
+                           : (rt < a.n_rt128 ? tile_kind<MODE>(a, rt, ct, tc.s) : 2);
       const int row = rt * BM + rin;
       const bool live = row < a.M;
       if (C2 && kind_launch == 0 && kind != 0) {

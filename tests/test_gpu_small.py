@@ -406,3 +406,92 @@ def test_cta_pairs_match_single_cta(cfg, split, D, V):
     W = oracle_W(wl)
     ologp, olse, _ = O.head_forward(wl.H, W, wl.labels)
     assert np.max(np.abs(lp1 - ologp)) <= TOL_LOGP
+
+
+def _staged_two_chunk_ws(M, hd, head, V):
+    """Smallest workspace (in steps of 64 vocab rows) on which both passes run
+    staged fp16 chunks and neither fits the vocabulary in one chunk."""
+    lo = cce.workspace_min_bytes(M, hd, head)
+    step = 64 * (2 * M + 2 * head.D)
+    for i in range(1, 20000):
+        p = cce.cce_query_plan(M, hd, head, lo + i * step)
+        if p["bwd_staged"] and p["fwd_staged"]:
+            assert p["fwd_chunk"] < V and p["bwd_chunk"] < V, p
+            return lo + i * step
+    raise AssertionError("no workspace gives staged chunks")
+
+
+@pytest.mark.parametrize("wformat", ["q4g64", "q8g64"])
+@pytest.mark.parametrize("split,D,V,cap", [((40, 45, 44), 128, 20000, 0.0),
+                                           ((100, 150, 262), 256, 30001, 0.0),
+                                           ((300, 400, 400), 192, 18000, 30.0)])
+def test_quant_staging_modes(wformat, split, D, V, cap):
+    """4/8-bit heads dequantised in the GEMM (mode 1) and staged as fp16
+    chunks (mode 2, on a workspace where both passes take two chunks or more)
+    both match the oracle, and match each other to accumulation order (the
+    fp16 weights are the same)."""
+    wl = S.make_custom(4, M_split=split, D=D, V=V, wformat=wformat)
+    H, head, labels = upload(wl)
+    head.softcap = cap
+    hd = cce.h_dtype(H)
+    g = torch.from_numpy(S.random_cotangent(wl)).cuda()
+    f = dict(device="cuda", dtype=torch.float32)
+    outs = {}
+    for mode in (1, 2):
+        cce.cce_set_quant_staging(mode)
+        try:
+            ws_bytes = _staged_two_chunk_ws(wl.M, hd, head, V) if mode == 2 else None
+            ws = cce.alloc_workspace(wl.M, hd, head, nbytes=ws_bytes)
+            logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+            dH = torch.empty(wl.M, wl.D, **f)
+            cce.cce_profile_enable(True)
+            cce.cce_forward(H, head, labels, logp, lse, None, None, ws)
+            cce.cce_backward_dh(H, head, labels, lse, g, 0.0, None, dH, None, ws)
+            torch.cuda.synchronize()
+            prof = cce.cce_profile_read()
+        finally:
+            cce.cce_profile_enable(False)
+            cce.cce_set_quant_staging(0)
+        assert cce.cce_device_status(ws) == 0
+        n_deq = prof.get("dequant_chunk", (0.0, 0))[1]
+        if mode == 1:
+            assert n_deq == 0
+        else:
+            assert n_deq >= 4  # two or more chunks in each of the two passes
+        outs[mode] = (logp.cpu().numpy(), lse.cpu().numpy(), dH.cpu().numpy())
+    W = oracle_W(wl)
+    ologp, olse, _ = O.head_forward(wl.H, W, wl.labels, softcap=cap)
+    want = O.head_dh(wl.H, W, wl.labels, g.cpu().numpy(), olse, softcap=cap)
+    for mode in (1, 2):
+        lp, ls, dh = outs[mode]
+        assert np.max(np.abs(lp - ologp)) <= TOL_LOGP
+        assert np.max(np.abs(ls - olse)) <= TOL_LOGP
+        assert rel_fro(dh, want) <= TOL_DH
+    assert np.max(np.abs(outs[1][0] - outs[2][0])) <= 1e-4
+    assert rel_fro(outs[2][2], outs[1][2]) <= 1e-3
+
+
+@pytest.mark.parametrize("extra_kb", [0, 300, 600])
+def test_small_m_many_k_splits(extra_kb):
+    """M = 64 gives one dH tile per d-tile, so the dH GEMM splits K up to 32
+    ways.  Workspaces between the minimum and a few chunks wide make vocab
+    chunks whose last one is narrower than the split count (splits without K
+    steps); dH must still match the oracle and the wide-workspace result."""
+    wl = S.make_custom(2, M_split=(8, 28, 28), D=256, V=5000)
+    (H, head, labels, ws), logp, lse, _, _ = _forward(wl)
+    g = torch.from_numpy(S.random_cotangent(wl)).cuda()
+    lse_t = torch.from_numpy(lse).cuda()
+    d1 = torch.empty(wl.M, wl.D, device="cuda")
+    cce.cce_backward_dh(H, head, labels, lse_t, g, 0.0, None, d1, None, ws)
+    hd = cce.h_dtype(H)
+    nbytes = cce.workspace_min_bytes(wl.M, hd, head) + 31 * wl.M * wl.D * 4 + extra_kb * 1024
+    small = cce.alloc_workspace(wl.M, hd, head, nbytes=nbytes)
+    d2 = torch.empty(wl.M, wl.D, device="cuda")
+    cce.cce_backward_dh(H, head, labels, lse_t, g, 0.0, None, d2, None, small)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0 and cce.cce_device_status(small) == 0
+    W = oracle_W(wl)
+    want = O.head_dh(wl.H, W, wl.labels, g.cpu().numpy(), O.head_forward(wl.H, W, wl.labels)[1])
+    assert rel_fro(d1.cpu().numpy(), want) <= TOL_DH
+    assert rel_fro(d2.cpu().numpy(), want) <= TOL_DH
+    assert rel_fro(d2.cpu().numpy(), d1.cpu().numpy()) < 1e-5

@@ -144,3 +144,47 @@ def test_objective_rejects_bad_arguments(lib):
         assert lib.pref_loss_from_logps(a, a, 20, lay, ctypes.byref(obj), a, a, 4096, None) == 1
         assert lib.pref_grad_coeffs(a, a, 20, lay, ctypes.byref(obj), a, a, 4096, None) == 1
     assert lib.pref_loss_from_logps(a, a, 20, lay, None, a, a, 4096, None) == 1
+
+
+def test_query_plan_chunks_splits_and_staging(lib):
+    """The host-side planner: forward/backward chunking, the dH K split,
+    CTA pairs and staged dequantisation follow the workspace and M."""
+    big = _head(V=262144, D=2048)
+    ws = lib.cce_workspace_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
+    p = cce.cce_query_plan(8192, cce.CCE_BF16, big, ws)
+    assert p["fwd_ok"] and p["bwd_ok"] and not p["fwd_staged"] and not p["bwd_staged"]
+    assert p["fwd_chunk"] == 262144          # one forward launch over V
+    assert 256 <= p["bwd_chunk"] < 262144 and p["bwd_chunk"] % 256 == 0
+    assert 1 <= p["bwd_ksplit"] <= 4 and p["fwd_cta_pairs"] and p["bwd_cta_pairs"]
+    # a wider workspace gives wider backward chunks
+    p2 = cce.cce_query_plan(8192, cce.CCE_BF16, big, 4 * ws)
+    assert p2["bwd_chunk"] > p["bwd_chunk"]
+    # the minimum workspace (sized for a 256-wide chunk and no K split; the
+    # forward's statistics may leave the backward room for a wider chunk)
+    lo = lib.cce_workspace_min_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
+    p3 = cce.cce_query_plan(8192, cce.CCE_BF16, big, lo)
+    assert p3["fwd_ok"] and p3["bwd_ok"] and p3["bwd_chunk"] >= 256 and p3["bwd_ksplit"] == 1
+    p4 = cce.cce_query_plan(8192, cce.CCE_BF16, big, lo - 1)
+    assert not p4["fwd_ok"] and not p4["bwd_ok"]
+    # small M: few dH tiles, so the K split goes past 4 to fill the grid;
+    # M <= 128 runs single-CTA tiles
+    small = cce.cce_query_plan(64, cce.CCE_BF16, big,
+                               lib.cce_workspace_bytes(64, cce.CCE_BF16, ctypes.byref(big)))
+    assert small["bwd_ksplit"] > 4 and not small["bwd_cta_pairs"]
+
+
+def test_query_plan_quant_staging(lib):
+    q4 = cce._Head(cce.CCE_W_AFFINE_Q4_G64, cce.CCE_BF16, 128256, 4096, 4096, 4096, 4096)
+    try:
+        for mode, M, want in [(0, 32768, 1), (0, 512, 0), (1, 32768, 0), (2, 512, 1)]:
+            cce.cce_set_quant_staging(mode)
+            ws = lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(q4))
+            p = cce.cce_query_plan(M, cce.CCE_BF16, q4, ws)
+            assert p["fwd_staged"] == want and p["bwd_staged"] == want, (mode, M, p)
+            assert p["bwd_cta_pairs"] == want  # in-kernel dequantisation is single-CTA
+            # the minimum workspace always runs (staging falls back to in-kernel)
+            lo = lib.cce_workspace_min_bytes(M, cce.CCE_BF16, ctypes.byref(q4))
+            pl = cce.cce_query_plan(M, cce.CCE_BF16, q4, lo)
+            assert pl["fwd_ok"] and pl["bwd_ok"] and not pl["bwd_staged"]
+    finally:
+        cce.cce_set_quant_staging(0)
