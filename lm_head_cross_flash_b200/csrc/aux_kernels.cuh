@@ -279,50 +279,53 @@ __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
 // ---------------------------------------------- staged dequantisation --
 // fp16 rows [rows, D] of a 4- or 8-bit affine head, vocab rows v0 .. v0+rows,
 // in natural column order: w = q * scale + bias per group of 64 along D.  The
-// values are those the in-kernel dequantiser produces (same fp16 fma), only
-// the K-interleaved pairs it emits are put back in order with byte permutes.
-// One thread per (row, group): 32 (4-bit) or 64 (8-bit) bytes in, 128 out.
+// values are those the in-kernel dequantiser produces (the same fp16 ops on
+// the same bits: 0x6400 | q is 1024 + q, subtract 1024, one fma), only laid
+// out in order.  One thread per 8 weights (one 4-bit word or two 8-bit
+// words): a warp reads 128 or 256 contiguous bytes and writes 512.
 template <int QB>
 __global__ void dequant_rows_f16_kernel(const uint32_t* __restrict__ qw,
                                         const uint16_t* __restrict__ scales,
                                         const uint16_t* __restrict__ biases, int64_t v0,
                                         int64_t rows, int D, uint4* __restrict__ out) {
   static_assert(QB == 4 || QB == 8, "4- or 8-bit heads");
+  const int64_t n8 = rows * (D / 8);  // 8-weight units
   const int gpr = D / 64;
-  const int64_t units = rows * gpr;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = u / gpr;
-    const int g = static_cast<int>(u - r * gpr);
+  const __half2 k1024 = __float2half2_rn(1024.f);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / (D / 8);
+    const int c8 = static_cast<int>(i - r * (D / 8));  // 8-weight unit within the row
     const int64_t v = v0 + r;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        qw + static_cast<size_t>(v) * (D / (32 / QB)) + static_cast<size_t>(g) * (2 * QB));
-    const uint16_t sc = __ldg(scales + static_cast<size_t>(v) * gpr + g);
-    const uint16_t bi = __ldg(biases + static_cast<size_t>(v) * gpr + g);
-    uint4 h[8];
-    if constexpr (QB == 8) {
-      uint4 wv[4];
+    const size_t gi = static_cast<size_t>(v) * gpr + c8 / 8;
+    const __half2 s2 =
+        __float2half2_rn(__uint_as_float(static_cast<uint32_t>(__ldg(scales + gi)) << 16));
+    const __half2 b2 =
+        __float2half2_rn(__uint_as_float(static_cast<uint32_t>(__ldg(biases + gi)) << 16));
+    uint32_t t[4];
+    if constexpr (QB == 4) {
+      // element j = bits 4j..4j+3: the half pairs come out as (e_i, e_i+4)
+      const uint32_t w = __ldg(qw + static_cast<size_t>(v) * (D / 8) + c8);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) wv[i] = __ldg(src + i);
-      dequant_group64_q8(wv, sc, bi, h);
-    } else {
-      dequant_group64(__ldg(src), __ldg(src + 1), sc, bi, h);
-    }
-    uint4* dst = out + (static_cast<size_t>(r) * D + static_cast<size_t>(g) * 64) / 8;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      // 4-bit: halves (e0,e4) (e1,e5) (e2,e6) (e3,e7); 8-bit: (e0,e2) (e1,e3)
-      // (e4,e6) (e5,e7).  Natural order is (e0,e1) (e2,e3) (e4,e5) (e6,e7).
-      const uint32_t t0 = h[c].x, t1 = h[c].y, t2 = h[c].z, t3 = h[c].w;
-      uint4 n;
-      if constexpr (QB == 4) {
-        n = make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t2, t3, 0x5410),
-                       __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x7632));
-      } else {
-        n = make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632),
-                       __byte_perm(t2, t3, 0x5410), __byte_perm(t2, t3, 0x7632));
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t x = ((w >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
+        __half2 h = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, b2);
+        t[k] = *reinterpret_cast<uint32_t*>(&h);
       }
-      dst[c] = n;
+      out[i] = make_uint4(__byte_perm(t[0], t[1], 0x5410), __byte_perm(t[2], t[3], 0x5410),
+                          __byte_perm(t[0], t[1], 0x7632), __byte_perm(t[2], t[3], 0x7632));
+    } else {
+      // element j of a word = byte j: pairs (e0,e2) (e1,e3) per word
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(qw + static_cast<size_t>(v) * (D / 4)) + c8);
+      const uint32_t ws[2] = {w.x, w.y};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t x = ((ws[k >> 1] >> (8 * (k & 1))) & 0x00FF00FFu) | 0x64006400u;
+        __half2 h = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, b2);
+        t[k] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      out[i] = make_uint4(__byte_perm(t[0], t[1], 0x5410), __byte_perm(t[0], t[1], 0x7632),
+                          __byte_perm(t[2], t[3], 0x5410), __byte_perm(t[2], t[3], 0x7632));
     }
   }
 }

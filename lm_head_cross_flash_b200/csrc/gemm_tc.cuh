@@ -176,8 +176,8 @@ __device__ __forceinline__ void dequant_group64(const uint4& wa, const uint4& wb
 // `group_rt` (sized so a group of H rows stays in L2); inside a group the row
 // tile is fastest, so the CTAs in flight share one vocab tile of W, and the
 // group sweeps the whole vocabulary before the next group starts.  kDh:
-// d-tile fastest, then K split, then row tile, so the CTAs in flight share a
-// G' row tile.
+// d-tile fastest, then row tile, then K split, so the CTAs in flight share a
+// G'' row tile and one K range of the W chunk.
 struct TileCoord {
   int rt, ct, s;
 };
@@ -186,10 +186,13 @@ template <Mode MODE>
 __device__ __forceinline__ TileCoord tile_coord(const TileArgs& a, int t) {
   TileCoord c;
   if (MODE == Mode::kDh || MODE == Mode::kDw) {
-    c.ct = t % a.n_ct;
-    const int r = t / a.n_ct;
-    c.s = r % a.ksplit;
-    c.rt = r / a.ksplit;
+    // K split outermost: the tiles in flight stream the same K range of the
+    // W chunk (one wave reads 1/ksplit of it), row tiles share G'' rows.
+    const int per_s = a.n_ct * a.n_rt;
+    c.s = t / per_s;
+    const int r = t - c.s * per_s;
+    c.ct = r % a.n_ct;
+    c.rt = r / a.n_ct;
   } else {
     const int per_group = a.group_rt * a.n_ct;
     const int grp = t / per_group;
