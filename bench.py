@@ -70,13 +70,18 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The sources that decide the tensor-core kernels' memory traffic: the kernel
+# template and its PTX wrappers, and the host code that picks tiles, chunks
+# and launch shapes.
+TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "cce.cu")
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     src = os.path.join(ROOT, "lm_head_cross_flash_b200", "csrc")
-    for n in sorted(os.listdir(src)):
-        if n.endswith((".cu", ".cuh")):
-            with open(os.path.join(src, n), "rb") as f:
-                h.update(n.encode() + f.read())
+    for n in TRAFFIC_SOURCES:
+        with open(os.path.join(src, n), "rb") as f:
+            h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
 
 

@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "gemm_tc.cuh"
 
 namespace cce {
@@ -289,43 +291,58 @@ __global__ void dequant_rows_f16_kernel(const uint32_t* __restrict__ qw,
                                         const uint16_t* __restrict__ biases, int64_t v0,
                                         int64_t rows, int D, uint4* __restrict__ out) {
   static_assert(QB == 4 || QB == 8, "4- or 8-bit heads");
+  using Word = typename std::conditional<QB == 4, uint32_t, uint2>::type;
+  constexpr int U = 4;  // units per thread in flight (loads issued before use)
   const int64_t n8 = rows * (D / 8);  // 8-weight units
-  const int gpr = D / 64;
+  const int upr = D / 8, gpr = D / 64;
   const __half2 k1024 = __float2half2_rn(1024.f);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / (D / 8);
-    const int c8 = static_cast<int>(i - r * (D / 8));  // 8-weight unit within the row
-    const int64_t v = v0 + r;
-    const size_t gi = static_cast<size_t>(v) * gpr + c8 / 8;
-    const __half2 s2 =
-        __float2half2_rn(__uint_as_float(static_cast<uint32_t>(__ldg(scales + gi)) << 16));
-    const __half2 b2 =
-        __float2half2_rn(__uint_as_float(static_cast<uint32_t>(__ldg(biases + gi)) << 16));
-    uint32_t t[4];
-    if constexpr (QB == 4) {
-      // element j = bits 4j..4j+3: the half pairs come out as (e_i, e_i+4)
-      const uint32_t w = __ldg(qw + static_cast<size_t>(v) * (D / 8) + c8);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < n8;
+       i0 += U * stride) {
+    Word w[U];
+    uint16_t sb[U], bb[U];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t x = ((w >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
-        __half2 h = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, b2);
-        t[k] = *reinterpret_cast<uint32_t*>(&h);
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < n8) {
+        const int64_t r = i / upr;
+        const int c8 = static_cast<int>(i - r * upr);
+        const int64_t v = v0 + r;
+        const size_t gi = static_cast<size_t>(v) * gpr + c8 / 8;
+        w[u] = __ldg(reinterpret_cast<const Word*>(qw + static_cast<size_t>(v) * (D / (32 / QB))) + c8);
+        sb[u] = __ldg(scales + gi);
+        bb[u] = __ldg(biases + gi);
       }
-      out[i] = make_uint4(__byte_perm(t[0], t[1], 0x5410), __byte_perm(t[2], t[3], 0x5410),
-                          __byte_perm(t[0], t[1], 0x7632), __byte_perm(t[2], t[3], 0x7632));
-    } else {
-      // element j of a word = byte j: pairs (e0,e2) (e1,e3) per word
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(qw + static_cast<size_t>(v) * (D / 4)) + c8);
-      const uint32_t ws[2] = {w.x, w.y};
+    }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t x = ((ws[k >> 1] >> (8 * (k & 1))) & 0x00FF00FFu) | 0x64006400u;
-        __half2 h = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, b2);
-        t[k] = *reinterpret_cast<uint32_t*>(&h);
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= n8) break;
+      const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sb[u]) << 16));
+      const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bb[u]) << 16));
+      uint32_t t[4];
+      if constexpr (QB == 4) {
+        // element j = bits 4j..4j+3: the half pairs come out as (e_k, e_k+4)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t x = ((w[u] >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
+          __half2 h = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, b2);
+          t[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        out[i] = make_uint4(__byte_perm(t[0], t[1], 0x5410), __byte_perm(t[2], t[3], 0x5410),
+                            __byte_perm(t[0], t[1], 0x7632), __byte_perm(t[2], t[3], 0x7632));
+      } else {
+        // element j of a word = byte j: pairs (e0,e2) (e1,e3) per word
+        const uint32_t ws[2] = {w[u].x, w[u].y};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t x = ((ws[k >> 1] >> (8 * (k & 1))) & 0x00FF00FFu) | 0x64006400u;
+          __half2 h = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, b2);
+          t[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        out[i] = make_uint4(__byte_perm(t[0], t[1], 0x5410), __byte_perm(t[0], t[1], 0x7632),
+                            __byte_perm(t[2], t[3], 0x5410), __byte_perm(t[2], t[3], 0x7632));
       }
-      out[i] = make_uint4(__byte_perm(t[0], t[1], 0x5410), __byte_perm(t[0], t[1], 0x7632),
-                          __byte_perm(t[2], t[3], 0x5410), __byte_perm(t[2], t[3], 0x7632));
     }
   }
 }

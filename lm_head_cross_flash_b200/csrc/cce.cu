@@ -576,7 +576,7 @@ cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_hea
 cce_status stage_chunk(const Operands& op, const cce_head* W, int64_t v0, int64_t rows,
                        int sms, cudaStream_t st) {
   const int64_t units = rows * (W->D / 8);
-  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, 256), 16 * sms)));
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, 256 * 4), 8 * sms)));
   const auto* qw = static_cast<const uint32_t*>(W->w);
   const auto* sc = static_cast<const uint16_t*>(W->scales);
   const auto* bi = static_cast<const uint16_t*>(W->biases);

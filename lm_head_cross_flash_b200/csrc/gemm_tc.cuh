@@ -11,15 +11,27 @@
 //           (ORPO design 0.0.6, fused-head spec, "Backward".)
 //   kDh   : dH[:, d-tile] (+)= coeff * (G'[:, chunk] . W[chunk, d-tile]),
 //           fp32 accumulation in TMEM and across chunks.
+//   kDw   : dW[chunk rows, d-tile] = -(G'^T . coeff*H) (trainable head),
+//           both operands MN-major.
 //
 // Roles (192 threads): warp 0 issues TMA loads into a 4-stage shared-memory
 // ring; warp 1 owns the TMEM allocation and issues tcgen05.mma (M=128,
 // N=256, K=16) into one of two 256-column fp32 accumulators; warps 2-5 drain
 // the accumulator with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)..+31,
 // i.e. one row per thread) and run the epilogue, overlapping the MMA of the
-// next tile.  Tiles are assigned round-robin over a grid of at most one CTA
-// per SM; consecutive tile ids share the column tile (vocab or d), so the CTAs
-// in flight stream the same W tiles from L2.
+// next tile.  A quantised head (QB = 4 or 8) adds 8 warps that dequantise
+// the B half of every stage.  Tiles are assigned round-robin over a grid of
+// at most one CTA per SM, in the order tile_coord gives (below), so the CTAs
+// in flight share the operand that should stay in L2.
+//
+// C2 = true runs the same roles on clusters of two CTAs (one TPC) computing
+// a 256x256 tile per pair with tcgen05.mma.cta_group::2 (M=256): each CTA
+// loads its own 128 rows of A and one half of B into a 6-stage ring of 32 KB
+// stages, both CTAs' copies complete on the leader CTA's full barrier, only
+// the leader issues MMAs, and tcgen05.commit with a CTA mask signals both
+// CTAs' stage-free and accumulator-full barriers.  Each CTA drains its own
+// 128 TMEM lanes; the leader's accumulator-empty barrier counts both CTAs'
+// epilogue threads.  No copy is multicast.
 #pragma once
 
 #include <cuda_bf16.h>
