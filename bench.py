@@ -52,9 +52,10 @@ def parse_args(argv=None):
                    help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
     p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
                    help="1: 2-CTA (cta_group::2) tiles where they apply; 0: single-CTA tiles")
-    p.add_argument("--sweep", choices=["small_m"], default=None,
-                   help="small_m: the W-stream (HBM-bound) regime, M in {64, 128, 256} at "
-                        "D=2048, V=262144; one JSON line per M")
+    p.add_argument("--sweep", choices=["small_m", "small_m_q4"], default=None,
+                   help="the W-stream (HBM-bound) regime, M in {64, 128, 256}, one JSON "
+                        "line per M: small_m at D=2048, V=262144 (bf16 head); small_m_q4 "
+                        "at D=4096, V=128256 (4-bit head, dequantised in the GEMMs)")
     return p.parse_args(argv)
 
 
@@ -381,6 +382,10 @@ def run_ours(args):
 
     peaks, peaks_src = load_peaks()
     flop_step = 6.0 * wl.M * wl.V * wl.D
+    # executed work: every row in the forward, rows with a nonzero cotangent
+    # in the two backward GEMMs (the response scope zeroes the prompt rows)
+    m_b = int((buf.coeff != 0).sum().item())
+    flop_exec = 2.0 * wl.M * wl.V * wl.D + 4.0 * m_b * wl.V * wl.D
     tflops = flop_step / (ms_step / 1e3) / 1e12
     # roofline of the dominant kernel kind (largest summed time)
     per_kind_flops = {"fwd_lse_gemm": 2.0 * wl.M * wl.V * wl.D,  # per step
@@ -427,6 +432,9 @@ def run_ours(args):
                    "cta_pairs": bool(args.cta_pairs),
                    "quant_staging": ["choose", "in-kernel", "staged"][args.quant_staging]},
         "tflops": tflops,
+        "executed": {"rows_backward": m_b, "tflop_per_step": flop_exec / 1e12,
+                     "tflops": flop_exec / (ms_step / 1e3) / 1e12,
+                     "note": "2*M*V*D + 4*M_b*V*D; skipped vocab tiles (skip_tiles) not subtracted"},
         "pct_bf16_peak": {"sustained": 100.0 * tflops / peak_s,
                           "burst": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
                           "source": peaks_src},
@@ -447,14 +455,16 @@ def run_ours(args):
 
 # ------------------------------------------------------ small-M sweep --
 
-def run_small_m(args):
-    """Forward and backward of the head at M = 64, 128, 256 (D = 2,048,
-    V = 262,144, bf16, flat H): the regime where streaming W from HBM bounds
-    the time.  Achieved GB/s counts the method's minimum bytes: W once per
-    pass, H in, dH out and the per-row / per-block statistics.  This
-    implementation's backward reads W twice (the G'' recompute and the dH
-    contraction are separate GEMMs) and moves G'' through HBM; those bytes are
-    reported as design_bytes."""
+def run_small_m(args, quant=False):
+    """Forward and backward of the head at M = 64, 128, 256: the regime where
+    streaming W from HBM bounds the time.  bf16 head: D = 2,048, V = 262,144,
+    flat H.  quant: the 4-bit head of the long-context workload (D = 4,096,
+    V = 128,256, groups of 64), dequantised inside the GEMMs.  Achieved GB/s
+    counts the method's minimum bytes: W once per pass (as stored: 16 or 4.25
+    bits per weight), H in, dH out and the per-row / per-block statistics.
+    This implementation's backward reads W twice (the G'' recompute and the
+    dH contraction are separate GEMMs) and moves G'' through HBM; those bytes
+    are reported as design_bytes."""
     import torch
 
     from lm_head_cross_flash_b200 import cce
@@ -467,7 +477,10 @@ def run_small_m(args):
     for M in (64, 128, 256):
         P = M // 8
         Rc = (M - P) // 2
-        wl = S.make_custom(2, M_split=(P, Rc, M - P - Rc), D=2048, V=262144)
+        if quant:
+            wl = S.make_custom(4, M_split=(P, Rc, M - P - Rc))
+        else:
+            wl = S.make_custom(2, M_split=(P, Rc, M - P - Rc), D=2048, V=262144)
         H, head, labels = cce.upload_workload(wl, dev)
         buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head, dev)
         stream = torch.cuda.current_stream(dev)
@@ -502,13 +515,14 @@ def run_small_m(args):
         st = cce.cce_device_status(buf.ws)
         if st != 0:
             raise RuntimeError(f"device status {st} in the small-M sweep (M={M})")
-        wbytes = 2.0 * wl.V * wl.D
+        wbytes = (wl.V * wl.D / 2.0 + 2 * 2.0 * wl.V * wl.D / 64) if quant else 2.0 * wl.V * wl.D
         cols = cce.blockmax_cols(wl.V)
         stats = 4.0 * M * cols + 4.0 * 4 * M
         fwd_bytes = wbytes + 2.0 * M * wl.D + stats
         bwd_bytes = wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 3 * 4.0 * M
         bwd_design = 2 * wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 2 * 2.0 * M * wl.V
-        line = {"sweep": "small_m", "M": M, "D": wl.D, "V": wl.V, "dtype": "bf16",
+        line = {"sweep": "small_m_q4" if quant else "small_m", "M": M, "D": wl.D, "V": wl.V,
+                "dtype": "f16 (4-bit head dequantised in-kernel)" if quant else "bf16",
                 "steps": args.steps, "fwd_ms": t_f, "bwd_ms": t_b,
                 "fwd_gbs": fwd_bytes / (t_f / 1e3) / 1e9,
                 "bwd_gbs": bwd_bytes / (t_b / 1e3) / 1e9,
@@ -519,7 +533,7 @@ def run_small_m(args):
                 "bwd_design_gbs": bwd_design / (t_b / 1e3) / 1e9,
                 "tokens_per_s": M / ((t_f + t_b) / 1e3),
                 "hbm_peak_gbs": hbm, "peak_source": f"{peaks_src} hbm_gbs (MEASURED_PEAKS.json)",
-                "l2": "W (1.07 GB) larger than L2; no flush"}
+                "l2": f"W ({wbytes / 1e9:.2f} GB as stored) larger than the 126 MB L2; no flush"}
         lines.append(line)
         del buf, H, head, labels
         torch.cuda.empty_cache()
@@ -577,8 +591,8 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
-    if args.sweep == "small_m":
-        for line in run_small_m(args):
+    if args.sweep in ("small_m", "small_m_q4"):
+        for line in run_small_m(args, quant=args.sweep == "small_m_q4"):
             print(json.dumps(line), flush=True)
         return
     out = run_reference(args) if args.impl == "reference" else run_ours(args)
