@@ -192,7 +192,7 @@ cce_status device_info(int* sms) {
     const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
     bool ok = true;
 #define CCE_SET_SMEM(MODE, QB) \
-    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, QB>, attr, smem_bytes<MODE, false, QB>()) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, QB>, attr, smem_bytes<MODE>()) == cudaSuccess;
     CCE_SET_SMEM(Mode::kLse, 0) CCE_SET_SMEM(Mode::kGrad, 0) CCE_SET_SMEM(Mode::kDh, 0)
     CCE_SET_SMEM(Mode::kLse, 4) CCE_SET_SMEM(Mode::kGrad, 4) CCE_SET_SMEM(Mode::kDh, 4)
     CCE_SET_SMEM(Mode::kLse, 8) CCE_SET_SMEM(Mode::kGrad, 8) CCE_SET_SMEM(Mode::kDh, 8)
@@ -471,10 +471,10 @@ void launch_tc(int qb, int64_t tiles, int sms, cudaStream_t st, const CUtensorMa
                const CUtensorMap& mb, const CUtensorMap& mc, const CUtensorMap& mc2,
                const TileArgs& args) {
   if (qb == 4)
-    cce_tc_kernel<MODE, 4><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE, false, 4>(), st>>>(
+    cce_tc_kernel<MODE, 4><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
         ma, mb, mc, mc2, args);
   else if (qb == 8)
-    cce_tc_kernel<MODE, 8><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE, false, 8>(), st>>>(
+    cce_tc_kernel<MODE, 8><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
         ma, mb, mc, mc2, args);
   else
     cce_tc_kernel<MODE, 0><<<grid_for(tiles, sms), NUM_THREADS, smem_bytes<MODE>(), st>>>(

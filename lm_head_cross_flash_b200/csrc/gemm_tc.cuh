@@ -67,23 +67,10 @@ __host__ __device__ constexpr int staging_buf_bytes() {
 constexpr int STAGES2 = 6;
 constexpr int B_HALF_BYTES = (BN / 2) * BK * 2;
 constexpr int STAGE2_BYTES = A_BYTES + B_HALF_BYTES;
-// Quantised heads (QB = 4 or 8) dequantise B in-kernel: 2 operand stages,
-// plus a per-thread prefetch ring of the packed weights (q_ring_depth steps
-// of one (row, group) unit, 32 or 64 bytes, per dequantisation thread) kept
-// full with cp.async, so each thread has several units in flight.
-constexpr int STAGES_Q = 2;
-template <int QB>
-__host__ __device__ constexpr int q_unit_bytes() { return QB == 8 ? 64 : 32; }
-template <int QB>
-__host__ __device__ constexpr int q_ring_depth() { return QB == 8 ? 5 : 9; }
-template <int QB>
-__host__ __device__ constexpr int q_ring_bytes() {
-  return QB ? q_ring_depth<QB>() * 32 * DQ_WARPS * q_unit_bytes<QB>() : 0;
-}
-template <Mode MODE, bool C2 = false, int QB = 0>
+template <Mode MODE, bool C2 = false>
 __host__ __device__ constexpr int smem_bytes() {
-  return (C2 ? STAGES2 * STAGE2_BYTES : (QB ? STAGES_Q : STAGES) * STAGE_BYTES) +
-         q_ring_bytes<QB>() + 4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
+  return (C2 ? STAGES2 * STAGE2_BYTES : STAGES * STAGE_BYTES) +
+         4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
@@ -325,7 +312,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
   static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
   static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
-  constexpr int NST = C2 ? STAGES2 : (QB ? STAGES_Q : STAGES);
+  constexpr int NST = C2 ? STAGES2 : STAGES;
   constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES;
   // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
   // rank 0 (the leader) issues the MMAs for both; each CTA loads its own
@@ -339,8 +326,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t* qring = base + NST * SBYTES;  // quantised heads: packed-weight prefetch
-  uint8_t* staging = qring + q_ring_bytes<QB>();
+  uint8_t* staging = base + NST * SBYTES;
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
   uint64_t* empty = full + NST;
@@ -547,22 +533,22 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
     }
   } else if (QB && warp >= DQ_WARP0) {
-    // ------------------------------------------ 4/8-bit dequantisation --
+    // --------------------------------------------- 4-bit dequantisation --
     // 256 threads fill the B half of every stage: 256 (row, group) units of
-    // 64 weights per K step, one per thread.  A thread's packed words for the
-    // next q_ring_depth - 1 units are already on their way into its slots of
-    // the prefetch ring (cp.async); scale and bias come through L1 (16
-    // consecutive groups of a row share a sector).  Each unit is dequantised
-    // to fp16 and written in the 128-byte-swizzled layout the TMA would
-    // produce (16-byte chunk c of row r at c ^ (r & 7)).
-    constexpr int PQ = q_ring_depth<QB>();
-    constexpr int QU = q_unit_bytes<QB>();
-    constexpr int NV = QU / 16;  // 16-byte vectors per unit
+    // 64 weights per K step, one per thread, read from global memory (words,
+    // scale, bias), dequantised to fp16 and written in the 128-byte-swizzled
+    // layout the TMA would produce (16-byte chunk c of row r at c ^ (r & 7)).
     const int dq = threadIdx.x - DQ_WARP0 * 32;
     const int gpr = a.D / 64;  // groups per head row
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    constexpr int NV = QB == 8 ? 4 : 2;  // 16-byte vectors per (row, group)
+    struct Unit {
+      uint4 w[NV];
+      uint16_t sc, bi;
+      bool valid;
+    };
     // unit u of K step k of tile tc: source row, group and smem offset
     auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& off) {
       if (MODE == Mode::kDh) {
@@ -576,95 +562,68 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         off = u * 128;
       }
     };
-    // The (tile, K step) units this CTA dequantises, in order.
-    struct Cursor {
-      int t, kk, kb, nks;
-      TileCoord tc;
-    };
-    auto settle = [&](Cursor& c) {  // move to the first computed tile at or after c.t
-      for (; c.t < ntiles; c.t += tstride) {
-        c.tc = tile_coord<MODE>(a, c.t);
-        if (tile_kind<MODE>(a, c.tc.rt, c.tc.ct, c.tc.s) != 0) continue;
-        c.kb = c.tc.s * a.nk / nsplit;
-        c.nks = (c.tc.s + 1) * a.nk / nsplit - c.kb;
-        if (c.nks > 0) break;
-      }
-      c.kk = 0;
-    };
-    auto advance = [&](Cursor& c) {
-      if (++c.kk == c.nks) {
-        c.t += tstride;
-        settle(c);
-      }
-    };
-    // slot-major ring: the 256 threads' units of one slot are contiguous
-    auto slot_ptr = [&](int slot) { return qring + (slot * 256 + dq) * QU; };
-    auto issue = [&](const Cursor& c, int slot) {  // one commit group per call
-      if (c.t < ntiles) {
-        int v, g, off;
-        locate(c.tc, c.kb + c.kk, dq, v, g, off);
-        if (v < a.V && g < gpr) {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(
-              a.q_w + static_cast<size_t>(v) * (a.D / (32 / (QB ? QB : 4))) + g * (2 * QB));
+    auto load = [&](const TileCoord& tc, int k, int u) {
+      Unit x;
+      int v, g, off;
+      locate(tc, k, u, v, g, off);
+      x.valid = v < a.V && g < gpr;
+      if (x.valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            a.q_w + static_cast<size_t>(v) * (a.D / (32 / (QB ? QB : 4))) + g * (2 * QB));
 #pragma unroll
-          for (int i = 0; i < NV; ++i) cp_async_16(smem_u32(slot_ptr(slot) + 16 * i), src + 16 * i);
+        for (int i = 0; i < NV; ++i) x.w[i] = __ldg(src + i);
+        x.sc = __ldg(a.q_scale + static_cast<size_t>(v) * gpr + g);
+        x.bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
+      } else {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) x.w[i] = make_uint4(0, 0, 0, 0);
+        x.sc = x.bi = 0;
+      }
+      return x;
+    };
+    for (int t = tile0; t < ntiles && ok; t += tstride) {
+      const TileCoord tc = tile_coord<MODE>(a, t);
+      if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
+      const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
+      Unit c0 = load(tc, kb, dq);
+      for (int kk = 0; kk < nks; ++kk) {
+        Unit n0;
+        if (kk + 1 < nks) n0 = load(tc, kb + kk + 1, dq);
+        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
         }
-      }
-      cp_async_commit();
-    };
-    Cursor use{tile0, 0, 0, 0, TileCoord{}};
-    settle(use);
-    Cursor pre = use;
-    for (int i = 0; i < PQ - 1; ++i) {
-      issue(pre, i);
-      if (pre.t < ntiles) advance(pre);
-    }
-    int slot_use = 0, slot_pre = PQ - 1;
-    while (use.t < ntiles) {
-      issue(pre, slot_pre);
-      if (pre.t < ntiles) advance(pre);
-      slot_pre = slot_pre + 1 == PQ ? 0 : slot_pre + 1;
-      if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
-        ok = false;
-        break;
-      }
-      cp_async_wait<PQ - 1>();  // this unit's words have landed
-      uint8_t* sB = base + stage * SBYTES + A_BYTES;
-      {
-        int v, g, off;
-        locate(use.tc, use.kb + use.kk, dq, v, g, off);
-        const int r = MODE == Mode::kDh ? (dq & 63) : dq;
-        uint4 out[8];
-        if (v < a.V && g < gpr) {
-          uint4 w[NV];
+        uint8_t* sB = base + stage * SBYTES + A_BYTES;
+        {
+          const Unit& x = c0;
+          const int u = dq;
+          int v, g, off;
+          locate(tc, kb + kk, u, v, g, off);
+          const int r = MODE == Mode::kDh ? (u & 63) : u;
+          uint4 out[8];
+          if (x.valid) {
+            if constexpr (QB == 8)
+              dequant_group64_q8(x.w, x.sc, x.bi, out);
+            else
+              dequant_group64(x.w[0], x.w[QB == 8 ? 0 : 1], x.sc, x.bi, out);
+          } else {
 #pragma unroll
-          for (int i = 0; i < NV; ++i)
-            w[i] = *reinterpret_cast<const uint4*>(slot_ptr(slot_use) + 16 * i);
-          const uint16_t sc = __ldg(a.q_scale + static_cast<size_t>(v) * gpr + g);
-          const uint16_t bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
-          if constexpr (QB == 8)
-            dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sc, bi, out);
-          else
-            dequant_group64(w[0], w[NV - 1], sc, bi, out);
-        } else {
+            for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
+          }
 #pragma unroll
-          for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(sB + off + ((c ^ (r & 7)) << 4)) = out[c];
         }
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(sB + off + ((c ^ (r & 7)) << 4)) = out[c];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == NST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        c0 = n0;
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[stage]);
-      if (++stage == NST) {
-        stage = 0;
-        phase ^= 1u;
-      }
-      slot_use = slot_use + 1 == PQ ? 0 : slot_use + 1;
-      advance(use);
     }
-    cp_async_wait<0>();  // no copy into this CTA's ring is left in flight
     if (!ok) {
       set_status(a.status, ST_TIMEOUT);
       *abort_flag = 1;
