@@ -151,6 +151,18 @@ bool make_map_ex(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int ra
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed 4/8-bit head as bytes [V, D*qb/8] for the in-kernel dequantisers:
+// box {box_bytes, box_rows}, no swizzle, zero fill past the last row.
+bool make_packed_map(CUtensorMap* m, const cce_head* W, int qb, uint32_t box_bytes,
+                     uint32_t box_rows) {
+  const uint64_t row_bytes = uint64_t(W->D) * qb / 8;
+  const uint64_t dims[2] = {row_bytes, uint64_t(W->V)};
+  const uint64_t strides[1] = {row_bytes};
+  const uint32_t box[2] = {box_bytes, box_rows};
+  return make_map_ex(m, W->w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 // --------------------------------------------------------- device facts --
 struct DevInfo {
   int sms = 0;
@@ -192,7 +204,7 @@ cce_status device_info(int* sms) {
     const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
     bool ok = true;
 #define CCE_SET_SMEM(MODE, QB) \
-    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, QB>, attr, smem_bytes<MODE>()) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, QB>, attr, smem_bytes<MODE, false, QB>()) == cudaSuccess;
     CCE_SET_SMEM(Mode::kLse, 0) CCE_SET_SMEM(Mode::kGrad, 0) CCE_SET_SMEM(Mode::kDh, 0)
     CCE_SET_SMEM(Mode::kLse, 4) CCE_SET_SMEM(Mode::kGrad, 4) CCE_SET_SMEM(Mode::kDh, 4)
     CCE_SET_SMEM(Mode::kLse, 8) CCE_SET_SMEM(Mode::kGrad, 8) CCE_SET_SMEM(Mode::kDh, 8)
@@ -471,10 +483,10 @@ void launch_tc(int qb, int64_t tiles, int sms, cudaStream_t st, const CUtensorMa
                const CUtensorMap& mb, const CUtensorMap& mc, const CUtensorMap& mc2,
                const TileArgs& args) {
   if (qb == 4)
-    cce_tc_kernel<MODE, 4><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
+    cce_tc_kernel<MODE, 4><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE, false, 4>(), st>>>(
         ma, mb, mc, mc2, args);
   else if (qb == 8)
-    cce_tc_kernel<MODE, 8><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE>(), st>>>(
+    cce_tc_kernel<MODE, 8><<<grid_for(tiles, sms), NUM_THREADS_Q4, smem_bytes<MODE, false, 8>(), st>>>(
         ma, mb, mc, mc2, args);
   else
     cce_tc_kernel<MODE, 0><<<grid_for(tiles, sms), NUM_THREADS, smem_bytes<MODE>(), st>>>(
@@ -687,8 +699,12 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   const bool pairs = max_pairs > 0;  // forward tiles need no K split
   CUtensorMap ma, mb;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
-  if (op.qb || staged) mb = ma;  // in-kernel dequantisation / set per staged chunk
-  else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN))
+  if (op.qb) {
+    // kLse: one group of 64 weights of 256 rows per K step
+    if (!make_packed_map(&mb, W, op.qb, 64 * op.qb / 8, BN)) return CCE_ERR_CUDA;
+  } else if (staged) {
+    mb = ma;  // set per staged chunk
+  } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN))
     return CCE_ERR_CUDA;
 
   TileArgs a;
@@ -928,8 +944,13 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   const int max_pairs = plan.pairs ? device_pairs() : 0;
   const bool pairs = max_pairs > 0;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
-  if (op.qb || staged) {
-    mb = ma;  // B is dequantised in-kernel, or mapped per staged chunk
+  if (op.qb) {
+    // packed tiles: kGrad as the forward, kDh 64 rows x 256 columns per K step
+    if (!make_packed_map(&mb, W, op.qb, 64 * op.qb / 8, BN) ||
+        !make_packed_map(&mw, W, op.qb, BN * op.qb / 8, BK))
+      return CCE_ERR_CUDA;
+  } else if (staged) {
+    mb = ma;  // mapped per staged chunk
     mw = ma;
   } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN) ||
              !make_map(&mw, op.b, op.bf16, op.ld_b, V, op.ld_b, 64, BK)) {

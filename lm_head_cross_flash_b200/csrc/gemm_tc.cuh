@@ -67,9 +67,18 @@ __host__ __device__ constexpr int staging_buf_bytes() {
 constexpr int STAGES2 = 6;
 constexpr int B_HALF_BYTES = (BN / 2) * BK * 2;
 constexpr int STAGE2_BYTES = A_BYTES + B_HALF_BYTES;
-template <Mode MODE, bool C2 = false>
+// Quantised heads (QB = 4 or 8) dequantise B in-kernel.  Each of their 3
+// stages also holds the packed weights of its B tile, brought in by TMA
+// (kLse/kGrad: 256 rows x one group of 64; kDh: 64 rows x 256 columns).
+constexpr int STAGES_Q = 3;
+template <Mode MODE, int QB>
+__host__ __device__ constexpr int pk_bytes() {
+  return MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8);
+}
+template <Mode MODE, bool C2 = false, int QB = 0>
 __host__ __device__ constexpr int smem_bytes() {
-  return (C2 ? STAGES2 * STAGE2_BYTES : STAGES * STAGE_BYTES) +
+  return (C2 ? STAGES2 * STAGE2_BYTES
+             : QB ? STAGES_Q * (STAGE_BYTES + pk_bytes<MODE, QB>()) : STAGES * STAGE_BYTES) +
          4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
@@ -312,8 +321,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
   static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
   static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
-  constexpr int NST = C2 ? STAGES2 : STAGES;
-  constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES;
+  constexpr int NST = C2 ? STAGES2 : (QB ? STAGES_Q : STAGES);
+  constexpr int PKB = QB ? pk_bytes<MODE, QB>() : 0;  // packed B tile per stage
+  constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES + PKB;
   // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
   // rank 0 (the leader) issues the MMAs for both; each CTA loads its own
   // 128 rows of A and its half of B and drains its own 128 TMEM lanes.
@@ -330,7 +340,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
   uint64_t* empty = full + NST;
-  uint64_t* acc_full = empty + NST;
+  uint64_t* pk_full = empty + NST;  // packed tile landed (quantised heads)
+  uint64_t* acc_full = pk_full + NST;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -345,6 +356,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], QB ? 1 + DQ_WARPS : 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&pk_full[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -415,7 +427,15 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                                l2_policy_evict_normal());
             }
           } else if (QB) {
-            // B comes from the dequantisation warps.
+            // B comes from the dequantisation warps, which read the packed
+            // tile (tmB: the packed head as bytes [V, D*QB/8]) from the stage.
+            uint8_t* sP = sA + STAGE_BYTES;
+            mbar_arrive_expect_tx(&pk_full[stage], PKB);
+            if (MODE == Mode::kDh)
+              tma_load_2d(sP, &tmB, &pk_full[stage], tc.ct * (BN * QB / 8), a.b_row0 + k * BK);
+            else
+              tma_load_2d(sP, &tmB, &pk_full[stage], k * (64 * QB / 8),
+                          a.b_row0 + tc.ct * BN);
             mbar_arrive_expect_tx(&full[stage], A_BYTES);
             if (MODE == Mode::kDh)
               tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
@@ -462,9 +482,12 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       // cluster barrier keeps both CTAs alive until then).
       if (!C2 || rank == 0)
         for (int s = 0; s < NST; ++s)
-          if (issued_mask & (1u << s))
+          if (issued_mask & (1u << s)) {
+            if (QB)
+              wait_bounded(&pk_full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS, nullptr);
             wait_bounded(&full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS,
                          nullptr);
+          }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
@@ -533,87 +556,98 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
     }
   } else if (QB && warp >= DQ_WARP0) {
-    // --------------------------------------------- 4-bit dequantisation --
+    // ------------------------------------------ 4/8-bit dequantisation --
     // 256 threads fill the B half of every stage: 256 (row, group) units of
-    // 64 weights per K step, one per thread, read from global memory (words,
-    // scale, bias), dequantised to fp16 and written in the 128-byte-swizzled
-    // layout the TMA would produce (16-byte chunk c of row r at c ^ (r & 7)).
+    // 64 weights per K step, one per thread.  The packed words come from the
+    // stage (TMA, pk_full); scale and bias from global memory, fetched one
+    // unit ahead (kLse/kGrad: 8 groups of a row at once when rows are 16-byte
+    // aligned).  Each unit is dequantised to fp16 and written in the
+    // 128-byte-swizzled layout the TMA would produce (16-byte chunk c of row
+    // r at c ^ (r & 7)).
+    constexpr int QU = 64 * (QB ? QB : 4) / 8;  // packed bytes per unit
+    constexpr int NV = QU / 16;
     const int dq = threadIdx.x - DQ_WARP0 * 32;
     const int gpr = a.D / 64;  // groups per head row
+    const bool vec8 = MODE != Mode::kDh && (gpr % 8) == 0 &&
+                      ((reinterpret_cast<uintptr_t>(a.q_scale) |
+                        reinterpret_cast<uintptr_t>(a.q_bias)) & 15u) == 0;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    constexpr int NV = QB == 8 ? 4 : 2;  // 16-byte vectors per (row, group)
-    struct Unit {
-      uint4 w[NV];
-      uint16_t sc, bi;
-      bool valid;
-    };
-    // unit u of K step k of tile tc: source row, group and smem offset
-    auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& off) {
+    // unit u of K step k of tile tc: source row, group, offset of its packed
+    // words in the stage's packed tile, and of its fp16 output in B.  kDh:
+    // the 4 groups of a row are adjacent threads (their scales share a
+    // sector).
+    auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& pk, int& off) {
       if (MODE == Mode::kDh) {
-        const int r = u & 63, j = u >> 6;
+        const int r = u >> 2, j = u & 3;
         v = a.b_row0 + k * BK + r;
         g = tc.ct * (BN / 64) + j;
+        pk = r * (BN * QB / 8) + j * QU;
         off = j * (64 * BK * 2) + r * 128;
       } else {
         v = a.b_row0 + tc.ct * BN + u;
         g = k;
+        pk = u * QU;
         off = u * 128;
       }
     };
-    auto load = [&](const TileCoord& tc, int k, int u) {
-      Unit x;
-      int v, g, off;
-      locate(tc, k, u, v, g, off);
-      x.valid = v < a.V && g < gpr;
-      if (x.valid) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            a.q_w + static_cast<size_t>(v) * (a.D / (32 / (QB ? QB : 4))) + g * (2 * QB));
-#pragma unroll
-        for (int i = 0; i < NV; ++i) x.w[i] = __ldg(src + i);
-        x.sc = __ldg(a.q_scale + static_cast<size_t>(v) * gpr + g);
-        x.bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
+    const int r_sw = MODE == Mode::kDh ? (dq >> 2) : dq;  // row for the swizzle
+    uint4 sv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);  // 8 groups (vec8)
+    int vec_row = -1, vec_g0 = -1;
+    auto scale_bias = [&](int v, int g, uint16_t& sc, uint16_t& bi) {
+      if (vec8) {
+        const int g0 = g & ~7;
+        if (v != vec_row || g0 != vec_g0) {
+          sv = __ldg(reinterpret_cast<const uint4*>(a.q_scale + static_cast<size_t>(v) * gpr + g0));
+          bv = __ldg(reinterpret_cast<const uint4*>(a.q_bias + static_cast<size_t>(v) * gpr + g0));
+          vec_row = v;
+          vec_g0 = g0;
+        }
+        const int q = (g & 7) >> 1;
+        const uint32_t ws = q == 0 ? sv.x : q == 1 ? sv.y : q == 2 ? sv.z : sv.w;
+        const uint32_t wb = q == 0 ? bv.x : q == 1 ? bv.y : q == 2 ? bv.z : bv.w;
+        sc = static_cast<uint16_t>((g & 1) ? ws >> 16 : ws & 0xFFFFu);
+        bi = static_cast<uint16_t>((g & 1) ? wb >> 16 : wb & 0xFFFFu);
       } else {
-#pragma unroll
-        for (int i = 0; i < NV; ++i) x.w[i] = make_uint4(0, 0, 0, 0);
-        x.sc = x.bi = 0;
+        sc = __ldg(a.q_scale + static_cast<size_t>(v) * gpr + g);
+        bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
       }
-      return x;
     };
     for (int t = tile0; t < ntiles && ok; t += tstride) {
       const TileCoord tc = tile_coord<MODE>(a, t);
       if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
       const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
-      Unit c0 = load(tc, kb, dq);
       for (int kk = 0; kk < nks; ++kk) {
-        Unit n0;
-        if (kk + 1 < nks) n0 = load(tc, kb + kk + 1, dq);
-        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
+        int v, g, pk, off;
+        locate(tc, kb + kk, dq, v, g, pk, off);
+        const bool valid = v < a.V && g < gpr;
+        uint16_t sc = 0, bi = 0;
+        if (valid) scale_bias(v, g, sc, bi);
+        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag) ||
+            !wait_bounded(&pk_full[stage], phase, a.wait_ns, abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t* sB = base + stage * SBYTES + A_BYTES;
-        {
-          const Unit& x = c0;
-          const int u = dq;
-          int v, g, off;
-          locate(tc, kb + kk, u, v, g, off);
-          const int r = MODE == Mode::kDh ? (u & 63) : u;
-          uint4 out[8];
-          if (x.valid) {
-            if constexpr (QB == 8)
-              dequant_group64_q8(x.w, x.sc, x.bi, out);
-            else
-              dequant_group64(x.w[0], x.w[QB == 8 ? 0 : 1], x.sc, x.bi, out);
-          } else {
+        uint8_t* sA = base + stage * SBYTES;
+        uint8_t* sB = sA + A_BYTES;
+        const uint8_t* sP = sA + STAGE_BYTES;
+        uint4 out[8];
+        if (valid) {
+          uint4 w[NV];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
-          }
+          for (int i = 0; i < NV; ++i) w[i] = *reinterpret_cast<const uint4*>(sP + pk + 16 * i);
+          if constexpr (QB == 8)
+            dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sc, bi, out);
+          else
+            dequant_group64(w[0], w[NV - 1], sc, bi, out);
+        } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(sB + off + ((c ^ (r & 7)) << 4)) = out[c];
+          for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
         }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(sB + off + ((c ^ (r_sw & 7)) << 4)) = out[c];
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[stage]);
@@ -621,7 +655,6 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           stage = 0;
           phase ^= 1u;
         }
-        c0 = n0;
       }
     }
     if (!ok) {
