@@ -68,33 +68,36 @@ __host__ __device__ constexpr int staging_buf_bytes() {
 constexpr int STAGES2 = 6;
 constexpr int B_HALF_BYTES = (BN / 2) * BK * 2;
 constexpr int STAGE2_BYTES = A_BYTES + B_HALF_BYTES;
-// Quantised heads (QB = 4 or 8) dequantise B in-kernel from packed tiles
-// (kLse/kGrad: 256 rows x one group of 64; kDh: 64 rows x 256 columns per K
-// step) that a producer warp of their own streams by TMA into a ring that
-// runs ahead of the 3 operand stages: the packed weights come from HBM, so
-// their latency must not sit on the operand stages' round trip.  The ring
-// takes what shared memory is left, up to 8 steps.
-constexpr int STAGES_Q = 3;
+// Quantised heads (QB = 4 or 8) dequantise B in-kernel.  Their stages are
+// three separate rings: A tiles (TMA; as many as fit, up to 8, so the L2
+// round trip of H is hidden), B tiles written by the dequantisation warps (2),
+// and the packed weights of each B tile (kLse/kGrad: 256 rows x one group of
+// 64; kDh: 64 rows x 256 columns), which a producer warp of their own streams
+// from HBM by TMA (4).
 constexpr int SMEM_LIMIT = 232448;  // bytes of dynamic shared memory per block
+constexpr int BAR_BYTES = 512;      // mbarriers, TMEM slot, abort flag
+constexpr int QB_NB = 2;
+constexpr int QB_NPK = 4;
 template <Mode MODE, int QB>
 __host__ __device__ constexpr int pk_bytes() {
   return MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8);
 }
 template <Mode MODE, int QB>
-__host__ __device__ constexpr int pk_stages() {
+__host__ __device__ constexpr int qa_stages() {
   return QB == 0 ? 0
-                 : ((SMEM_LIMIT - 1024 - 256 - STAGES_Q * STAGE_BYTES -
-                     4 * 2 * staging_buf_bytes<MODE>()) / pk_bytes<MODE, QB>() > 8
+                 : ((SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * B_BYTES - QB_NPK * pk_bytes<MODE, QB>() -
+                     4 * 2 * staging_buf_bytes<MODE>()) / A_BYTES > 8
                         ? 8
-                        : (SMEM_LIMIT - 1024 - 256 - STAGES_Q * STAGE_BYTES -
-                           4 * 2 * staging_buf_bytes<MODE>()) / pk_bytes<MODE, QB>());
+                        : (SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * B_BYTES -
+                           QB_NPK * pk_bytes<MODE, QB>() - 4 * 2 * staging_buf_bytes<MODE>()) /
+                              A_BYTES);
 }
 template <Mode MODE, bool C2 = false, int QB = 0>
 __host__ __device__ constexpr int smem_bytes() {
   return (C2 ? STAGES2 * STAGE2_BYTES
-             : QB ? STAGES_Q * STAGE_BYTES + pk_stages<MODE, QB>() * pk_bytes<MODE, QB>()
+             : QB ? qa_stages<MODE, QB>() * A_BYTES + QB_NB * B_BYTES + QB_NPK * pk_bytes<MODE, QB>()
                   : STAGES * STAGE_BYTES) +
-         4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
+         4 * 2 * staging_buf_bytes<MODE>() + 1024 + BAR_BYTES;
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
@@ -336,11 +339,13 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
   static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
   static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
-  constexpr int NST = C2 ? STAGES2 : (QB ? STAGES_Q : STAGES);
-  constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES;
+  // Stages of the operand ring (quantised heads: A only; B has its own ring).
+  constexpr int NST = C2 ? STAGES2 : (QB ? qa_stages<MODE, QB>() : STAGES);
+  constexpr int SBYTES = C2 ? STAGE2_BYTES : (QB ? A_BYTES : STAGE_BYTES);
+  constexpr int NB = QB ? QB_NB : 0;                  // dequantised B ring
   constexpr int PKB = QB ? pk_bytes<MODE, QB>() : 0;  // one packed B tile
-  constexpr int NPK = QB ? pk_stages<MODE, QB>() : 0;  // packed ring depth
-  static_assert(!QB || NPK >= 2, "packed ring needs two stages");
+  constexpr int NPK = QB ? QB_NPK : 0;                 // packed ring depth
+  static_assert(!QB || NST >= 3, "quantised heads need 3 A stages at least");
   static_assert(smem_bytes<MODE, C2, QB>() <= SMEM_LIMIT, "shared memory");
   // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
   // rank 0 (the leader) issues the MMAs for both; each CTA loads its own
@@ -354,12 +359,15 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t* pk_ring = base + NST * SBYTES;  // quantised heads: packed tiles
+  uint8_t* b_ring = base + NST * SBYTES;    // quantised heads: dequantised B
+  uint8_t* pk_ring = b_ring + NB * B_BYTES;  // quantised heads: packed tiles
   uint8_t* staging = pk_ring + NPK * PKB;
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
   uint64_t* empty = full + NST;
-  uint64_t* pk_full = empty + NST;      // packed tile landed (quantised heads)
+  uint64_t* b_full = empty + NST;       // B tile written by all dequant warps
+  uint64_t* b_empty = b_full + NB;      // B tile consumed by the MMAs
+  uint64_t* pk_full = b_empty + NB;     // packed tile landed (quantised heads)
   uint64_t* pk_empty = pk_full + NPK;   // packed tile read by all dequant warps
   uint64_t* acc_full = pk_empty + NPK;
   uint64_t* acc_empty = acc_full + 2;
@@ -374,8 +382,12 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], QB ? 1 + DQ_WARPS : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < NB; ++s) {
+      mbar_init(&b_full[s], DQ_WARPS);
+      mbar_init(&b_empty[s], 1);
     }
     for (int s = 0; s < NPK; ++s) {
       mbar_init(&pk_full[s], 1);
@@ -506,8 +518,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_f16(C2 ? 2 * BM : BM, BN, a.fmt, MODE == Mode::kDw,
                                        MODE == Mode::kDh || MODE == Mode::kDw);
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, bst = 0;
+      uint32_t phase = 0, bph = 0;
       int acc = 0;
       bool ok = true;
       for (int t = tile0; t < ntiles && ok; t += tstride) {
@@ -524,13 +536,14 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kk = 0; kk < ksteps; ++kk) {
-          if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
+          if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag) ||
+              (QB && !wait_bounded(&b_full[bst], bph, a.wait_ns, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sA = smem_u32(base + stage * SBYTES);
-          const uint32_t sB = sA + A_BYTES;
+          const uint32_t sB = QB ? smem_u32(b_ring + bst * B_BYTES) : sA + A_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             const uint64_t ad = MODE == Mode::kDw
@@ -548,6 +561,13 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           // the stage is free in both CTAs once these MMAs have read it
           if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
           else umma_commit(&empty[stage]);
+          if (QB) {
+            umma_commit(&b_empty[bst]);
+            if (++bst == NB) {
+              bst = 0;
+              bph ^= 1u;
+            }
+          }
           if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
@@ -625,8 +645,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     const bool vec8 = MODE != Mode::kDh && (gpr % 8) == 0 &&
                       ((reinterpret_cast<uintptr_t>(a.q_scale) |
                         reinterpret_cast<uintptr_t>(a.q_bias)) & 15u) == 0;
-    int stage = 0, ps = 0;
-    uint32_t phase = 0, pph = 0;
+    int bst = 0, ps = 0;
+    uint32_t bph = 0, pph = 0;
     bool ok = true;
     // unit u of K step k of tile tc: source row, group, offset of its packed
     // words in the packed tile, and of its fp16 output in B.  kDh: the 4
@@ -677,27 +697,16 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         const bool valid = v < a.V && g < gpr;
         uint16_t sc = 0, bi = 0;
         if (valid) scale_bias(v, g, sc, bi);
-        uint4 w[NV];
         if (!wait_bounded(&pk_full[ps], pph, a.wait_ns, abort_flag)) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int i = 0; i < NV; ++i)
-          w[i] = *reinterpret_cast<const uint4*>(pk_ring + ps * PKB + pk + 16 * i);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pk_empty[ps]);
-        if (++ps == NPK) {
-          ps = 0;
-          pph ^= 1u;
-        }
-        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sB = base + stage * SBYTES + A_BYTES;
         uint4 out[8];
         if (valid) {
+          uint4 w[NV];
+#pragma unroll
+          for (int i = 0; i < NV; ++i)
+            w[i] = *reinterpret_cast<const uint4*>(pk_ring + ps * PKB + pk + 16 * i);
           if constexpr (QB == 8)
             dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sc, bi, out);
           else
@@ -706,15 +715,30 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
         }
+        // The slot may be refilled (TMA, async proxy) once every warp is done
+        // with it: the values computed above hold the loaded words, and the
+        // proxy fence orders these generic reads before the refill.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pk_empty[ps]);
+        if (++ps == NPK) {
+          ps = 0;
+          pph ^= 1u;
+        }
+        if (!wait_bounded(&b_empty[bst], bph ^ 1u, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sB = b_ring + bst * B_BYTES;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(sB + off + ((c ^ (r_sw & 7)) << 4)) = out[c];
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == NST) {
-          stage = 0;
-          phase ^= 1u;
+        if (lane == 0) mbar_arrive(&b_full[bst]);
+        if (++bst == NB) {
+          bst = 0;
+          bph ^= 1u;
         }
       }
     }
