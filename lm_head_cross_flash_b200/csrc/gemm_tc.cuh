@@ -78,24 +78,25 @@ constexpr int SMEM_LIMIT = 232448;  // bytes of dynamic shared memory per block
 constexpr int BAR_BYTES = 512;      // mbarriers, TMEM slot, abort flag
 constexpr int QB_NB = 2;
 constexpr int QB_NPK = 4;
-template <Mode MODE, int QB>
+// On CTA pairs (C2) each CTA holds half of B and of its packed tile.
+template <Mode MODE, int QB, bool C2 = false>
 __host__ __device__ constexpr int pk_bytes() {
-  return MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8);
+  return (MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8)) / (C2 ? 2 : 1);
 }
-template <Mode MODE, int QB>
+template <Mode MODE, int QB, bool C2 = false>
+__host__ __device__ constexpr int qa_free() {
+  return SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * (C2 ? B_HALF_BYTES : B_BYTES) -
+         QB_NPK * pk_bytes<MODE, QB, C2>() - 4 * 2 * staging_buf_bytes<MODE>();
+}
+template <Mode MODE, int QB, bool C2 = false>
 __host__ __device__ constexpr int qa_stages() {
-  return QB == 0 ? 0
-                 : ((SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * B_BYTES - QB_NPK * pk_bytes<MODE, QB>() -
-                     4 * 2 * staging_buf_bytes<MODE>()) / A_BYTES > 8
-                        ? 8
-                        : (SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * B_BYTES -
-                           QB_NPK * pk_bytes<MODE, QB>() - 4 * 2 * staging_buf_bytes<MODE>()) /
-                              A_BYTES);
+  return QB == 0 ? 0 : (qa_free<MODE, QB, C2>() / A_BYTES > 8 ? 8 : qa_free<MODE, QB, C2>() / A_BYTES);
 }
 template <Mode MODE, bool C2 = false, int QB = 0>
 __host__ __device__ constexpr int smem_bytes() {
-  return (C2 ? STAGES2 * STAGE2_BYTES
-             : QB ? qa_stages<MODE, QB>() * A_BYTES + QB_NB * B_BYTES + QB_NPK * pk_bytes<MODE, QB>()
+  return (QB ? qa_stages<MODE, QB, C2>() * A_BYTES + QB_NB * (C2 ? B_HALF_BYTES : B_BYTES) +
+                   QB_NPK * pk_bytes<MODE, QB, C2>()
+             : C2 ? STAGES2 * STAGE2_BYTES
                   : STAGES * STAGE_BYTES) +
          4 * 2 * staging_buf_bytes<MODE>() + 1024 + BAR_BYTES;
 }
@@ -163,49 +164,30 @@ __host__ __device__ constexpr int qpos(int e) {
   return QB == 8 ? q8_pos(e) : QB == 4 ? q4_pos(e) : e;
 }
 
-// 8-bit variant: 16 packed words (element 4c+j = byte j of word c).
-__device__ __forceinline__ void dequant_group64_q8(const uint4 (&wv)[4], uint16_t sbits,
-                                                   uint16_t bbits, uint4 (&out)[8]) {
+// Dequantise NCH consecutive 8-weight chunks of a group of 64: w = q * scale
+// + bias, rounded once to fp16 (fma.rn.f16x2 on q, scale, bias, all exact in
+// fp16); q comes from the bit pattern 0x6400 | q = 1024 + q in fp16.  Chunk c
+// is word c of a 4-bit group (element 8c+j = bits 4j..4j+3) or words 2c, 2c+1
+// of an 8-bit group (element 4w+j = byte j of word w).  out[c] holds the 8
+// fp16 values of chunk c in qpos<QB> order: (e0,e4) (e1,e5) (e2,e6) (e3,e7)
+// for 4-bit, (e0,e2) (e1,e3) (e4,e6) (e5,e7) for 8-bit.
+template <int QB, int NCH>
+__device__ __forceinline__ void dequant_chunks(const uint32_t* words, uint16_t sbits,
+                                               uint16_t bbits, uint4 (&out)[NCH]) {
   const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
   const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bbits) << 16));
   const __half2 k1024 = __float2half2_rn(1024.f);
-  const uint32_t words[16] = {wv[0].x, wv[0].y, wv[0].z, wv[0].w, wv[1].x, wv[1].y,
-                              wv[1].z, wv[1].w, wv[2].x, wv[2].y, wv[2].z, wv[2].w,
-                              wv[3].x, wv[3].y, wv[3].z, wv[3].w};
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < NCH; ++c) {
     uint32_t t[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t x = ((words[2 * c + (i >> 1)] >> (8 * (i & 1))) & 0x00FF00FFu) | 0x64006400u;
-      __half2 h = *reinterpret_cast<const __half2*>(&x);
-      h = __hfma2(__hsub2(h, k1024), s2, b2);
-      t[i] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    out[c] = make_uint4(t[0], t[1], t[2], t[3]);
-  }
-}
-
-// Dequantise the 64 weights of one (row, group): w = q * scale + bias, with
-// q read from 8 packed words (element 8c+j = bits 4j..4j+3 of word c) and
-// the result rounded once to fp16 (fma.rn.f16x2 on q, scale, bias, all exact
-// in fp16).  q comes from the bit pattern 0x6400 | q = 1024 + q in fp16.
-// out[c] holds the 8 fp16 values of word c in q4_pos order.
-__device__ __forceinline__ void dequant_group64(const uint4& wa, const uint4& wb, uint16_t sbits,
-                                                uint16_t bbits, uint4 (&out)[8]) {
-  const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
-  const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bbits) << 16));
-  const __half2 k1024 = __float2half2_rn(1024.f);
-  const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t t[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t x = ((words[c] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
-      __half2 h = *reinterpret_cast<const __half2*>(&x);
-      h = __hfma2(__hsub2(h, k1024), s2, b2);
-      t[i] = *reinterpret_cast<uint32_t*>(&h);
+      const uint32_t x =
+          QB == 8 ? ((words[2 * c + (i >> 1)] >> (8 * (i & 1))) & 0x00FF00FFu) | 0x64006400u
+                  : ((words[c] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
+      __half2 hh = *reinterpret_cast<const __half2*>(&x);
+      hh = __hfma2(__hsub2(hh, k1024), s2, b2);
+      t[i] = *reinterpret_cast<uint32_t*>(&hh);
     }
     out[c] = make_uint4(t[0], t[1], t[2], t[3]);
   }
@@ -337,14 +319,14 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC,
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
-  static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
   static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
   // Stages of the operand ring (quantised heads: A only; B has its own ring).
-  constexpr int NST = C2 ? STAGES2 : (QB ? qa_stages<MODE, QB>() : STAGES);
-  constexpr int SBYTES = C2 ? STAGE2_BYTES : (QB ? A_BYTES : STAGE_BYTES);
-  constexpr int NB = QB ? QB_NB : 0;                  // dequantised B ring
-  constexpr int PKB = QB ? pk_bytes<MODE, QB>() : 0;  // one packed B tile
-  constexpr int NPK = QB ? QB_NPK : 0;                 // packed ring depth
+  constexpr int NST = QB ? qa_stages<MODE, QB, C2>() : (C2 ? STAGES2 : STAGES);
+  constexpr int SBYTES = QB ? A_BYTES : (C2 ? STAGE2_BYTES : STAGE_BYTES);
+  constexpr int NB = QB ? QB_NB : 0;                       // dequantised B ring
+  constexpr int BBYTES = C2 ? B_HALF_BYTES : B_BYTES;      // this CTA's B tile
+  constexpr int PKB = QB ? pk_bytes<MODE, QB, C2>() : 0;  // this CTA's packed tile
+  constexpr int NPK = QB ? QB_NPK : 0;                      // packed ring depth
   static_assert(!QB || NST >= 3, "quantised heads need 3 A stages at least");
   static_assert(smem_bytes<MODE, C2, QB>() <= SMEM_LIMIT, "shared memory");
   // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
@@ -360,7 +342,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   uint8_t* b_ring = base + NST * SBYTES;    // quantised heads: dequantised B
-  uint8_t* pk_ring = b_ring + NB * B_BYTES;  // quantised heads: packed tiles
+  uint8_t* pk_ring = b_ring + NB * BBYTES;  // quantised heads: packed tiles
   uint8_t* staging = pk_ring + NPK * PKB;
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
@@ -386,7 +368,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < NB; ++s) {
-      mbar_init(&b_full[s], DQ_WARPS);
+      mbar_init(&b_full[s], (C2 ? 2 : 1) * DQ_WARPS);  // the leader's counts both CTAs
       mbar_init(&b_empty[s], 1);
     }
     for (int s = 0; s < NPK; ++s) {
@@ -447,19 +429,23 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * SBYTES);
             const int arow = (tc.rt * 2 + static_cast<int>(rank)) * BM;
+            // (quantised heads: A only, B comes from the dequantisation warps)
             if (MODE == Mode::kDh) {
               tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, l2_policy_evict_normal());
+              if (!QB) {
 #pragma unroll
-              for (int j = 0; j < BN / 128; ++j)
-                tma_load_2d_pair(sB + j * (64 * BK * 2), &tmB, bar,
-                                 tc.ct * BN + static_cast<int>(rank) * (BN / 2) + j * 64 +
-                                     pass * a.b_pass_off,
-                                 a.b_row0 - a.b_shift + k * BK, keep);
+                for (int j = 0; j < BN / 128; ++j)
+                  tma_load_2d_pair(sB + j * (64 * BK * 2), &tmB, bar,
+                                   tc.ct * BN + static_cast<int>(rank) * (BN / 2) + j * 64 +
+                                       pass * a.b_pass_off,
+                                   a.b_row0 - a.b_shift + k * BK, keep);
+              }
             } else {
               tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, keep);
-              tma_load_2d_pair(sB, &tmB, bar, k * BK,
-                               a.b_row0 - a.b_shift + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
-                               l2_policy_evict_normal());
+              if (!QB)
+                tma_load_2d_pair(sB, &tmB, bar, k * BK,
+                                 a.b_row0 - a.b_shift + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
+                                 l2_policy_evict_normal());
             }
           } else if (QB) {
             // B comes from the dequantisation warps.
@@ -541,9 +527,10 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             ok = false;
             break;
           }
+          if (C2 && QB) fence_acq_rel_cluster();  // the peer's B half is visible
           tc_fence_after();
           const uint32_t sA = smem_u32(base + stage * SBYTES);
-          const uint32_t sB = QB ? smem_u32(b_ring + bst * B_BYTES) : sA + A_BYTES;
+          const uint32_t sB = QB ? smem_u32(b_ring + bst * BBYTES) : sA + A_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             const uint64_t ad = MODE == Mode::kDw
@@ -562,7 +549,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
           else umma_commit(&empty[stage]);
           if (QB) {
-            umma_commit(&b_empty[bst]);
+            if constexpr (C2) umma_commit2_mc(&b_empty[bst], 0x3);
+            else umma_commit(&b_empty[bst]);
             if (++bst == NB) {
               bst = 0;
               bph ^= 1u;
@@ -598,7 +586,7 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       bool ok = true;
       for (int t = tile0; t < ntiles && ok; t += tstride) {
         const TileCoord tc = tile_coord<MODE>(a, t);
-        if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
+        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct, tc.s) != 0) continue;
         const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
         for (int kk = 0; kk < nks; ++kk) {
           if (!wait_bounded(&pk_empty[ps], pph ^ 1u, a.wait_ns, abort_flag)) {
@@ -607,12 +595,14 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           }
           const int k = kb + kk;
           mbar_arrive_expect_tx(&pk_full[ps], PKB);
+          // this CTA's half of the B tile on pairs (columns, resp. rows)
           if (MODE == Mode::kDh)
-            tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps], tc.ct * (BN * QB / 8),
+            tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps],
+                        tc.ct * (BN * QB / 8) + static_cast<int>(rank) * (BN / 2 * QB / 8),
                         a.b_row0 + k * BK);
           else
             tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps], k * (64 * QB / 8),
-                        a.b_row0 + tc.ct * BN);
+                        a.b_row0 + tc.ct * BN + static_cast<int>(rank) * (BN / 2));
           issued_mask |= 1u << ps;
           issued_phase = (issued_phase & ~(1u << ps)) | (pph << ps);
           if (++ps == NPK) {
@@ -631,15 +621,18 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     }
   } else if (QB && warp >= DQ_WARP0) {
     // ------------------------------------------ 4/8-bit dequantisation --
-    // 256 threads fill the B half of every stage: 256 (row, group) units of
-    // 64 weights per K step, one per thread.  The packed words come from the
-    // packed ring (released as soon as every warp has read them); scale and
-    // bias from global memory (kLse/kGrad: 8 groups of a row per 16-byte
-    // load when rows are 16-byte aligned).  Each unit is dequantised to fp16
-    // and written in the 128-byte-swizzled layout the TMA would produce
-    // (16-byte chunk c of row r at c ^ (r & 7)).
+    // 256 threads fill this CTA's B tile of every K step.  Single CTA: 256
+    // (row, group) units of 64 weights, one per thread.  Pair: this CTA's
+    // half of B holds 128 units, so each thread takes half a unit (32
+    // weights, 4 of its 8 16-byte chunks).  The packed words come from the
+    // packed ring (a slot is released after use, behind a proxy fence: its
+    // refill is an async-proxy write); scale and bias from global memory
+    // (kLse/kGrad: 8 groups of a row per 16-byte load when rows are 16-byte
+    // aligned).  The fp16 result is written in the 128-byte-swizzled layout
+    // the TMA would produce (16-byte chunk c of row r at c ^ (r & 7)).
     constexpr int QU = 64 * (QB ? QB : 4) / 8;  // packed bytes per unit
-    constexpr int NV = QU / 16;
+    constexpr int NCH = C2 ? 4 : 8;             // 16-byte output chunks per thread
+    constexpr int NV = QU * NCH / 8 / 16;       // 16-byte packed vectors per thread
     const int dq = threadIdx.x - DQ_WARP0 * 32;
     const int gpr = a.D / 64;  // groups per head row
     const bool vec8 = MODE != Mode::kDh && (gpr % 8) == 0 &&
@@ -648,24 +641,31 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     int bst = 0, ps = 0;
     uint32_t bph = 0, pph = 0;
     bool ok = true;
-    // unit u of K step k of tile tc: source row, group, offset of its packed
-    // words in the packed tile, and of its fp16 output in B.  kDh: the 4
-    // groups of a row are adjacent threads (their scales share a sector).
-    auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& pk, int& off) {
+    // This thread's part of K step k of tile tc: source row v and group g,
+    // the offset of its packed words in the packed tile, its output row r in
+    // B (for the swizzle), the offset of that row, and its first chunk c0.
+    // kDh: the groups of a row sit in adjacent threads (their scales share a
+    // sector).
+    const int h = C2 ? (dq & 1) : 0;  // half of the unit (pairs)
+    const int c0 = h * NCH;
+    auto locate = [&](const TileCoord& tc, int k, int& v, int& g, int& pk, int& r, int& off) {
       if (MODE == Mode::kDh) {
-        const int r = u >> 2, j = u & 3;
+        constexpr int GW = C2 ? 2 : 4;  // groups of this CTA's B columns
+        const int u = C2 ? (dq >> 1) : dq;
+        r = u / GW;
+        const int j = u % GW;
         v = a.b_row0 + k * BK + r;
-        g = tc.ct * (BN / 64) + j;
-        pk = r * (BN * QB / 8) + j * QU;
+        g = tc.ct * (BN / 64) + static_cast<int>(rank) * GW * (C2 ? 1 : 0) + j;
+        pk = r * (GW * QU) + j * QU + h * (QU / 2);
         off = j * (64 * BK * 2) + r * 128;
       } else {
-        v = a.b_row0 + tc.ct * BN + u;
+        r = C2 ? (dq >> 1) : dq;
+        v = a.b_row0 + tc.ct * BN + static_cast<int>(rank) * (BN / 2) + r;
         g = k;
-        pk = u * QU;
-        off = u * 128;
+        pk = r * QU + h * (QU / 2);
+        off = r * 128;
       }
     };
-    const int r_sw = MODE == Mode::kDh ? (dq >> 2) : dq;  // row for the swizzle
     uint4 sv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);  // 8 groups (vec8)
     int vec_row = -1, vec_g0 = -1;
     auto scale_bias = [&](int v, int g, uint16_t& sc, uint16_t& bi) {
@@ -687,13 +687,15 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
       }
     };
+    // the leader's b_full counts both CTAs' dequantisation warps
+    const uint32_t bfull_leader = C2 ? mapa_shared(smem_u32(&b_full[0]), 0) : 0u;
     for (int t = tile0; t < ntiles && ok; t += tstride) {
       const TileCoord tc = tile_coord<MODE>(a, t);
-      if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
+      if (launch_kind<MODE, C2>(a, tc.rt, tc.ct, tc.s) != 0) continue;
       const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
       for (int kk = 0; kk < nks; ++kk) {
-        int v, g, pk, off;
-        locate(tc, kb + kk, dq, v, g, pk, off);
+        int v, g, pk, r, off;
+        locate(tc, kb + kk, v, g, pk, r, off);
         const bool valid = v < a.V && g < gpr;
         uint16_t sc = 0, bi = 0;
         if (valid) scale_bias(v, g, sc, bi);
@@ -701,19 +703,16 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           ok = false;
           break;
         }
-        uint4 out[8];
+        uint4 out[NCH];
         if (valid) {
           uint4 w[NV];
 #pragma unroll
           for (int i = 0; i < NV; ++i)
             w[i] = *reinterpret_cast<const uint4*>(pk_ring + ps * PKB + pk + 16 * i);
-          if constexpr (QB == 8)
-            dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sc, bi, out);
-          else
-            dequant_group64(w[0], w[NV - 1], sc, bi, out);
+          dequant_chunks<QB, NCH>(reinterpret_cast<const uint32_t*>(w), sc, bi, out);
         } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < NCH; ++c) out[c] = make_uint4(0, 0, 0, 0);
         }
         // The slot may be refilled (TMA, async proxy) once every warp is done
         // with it: the values computed above hold the loaded words, and the
@@ -729,13 +728,16 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           ok = false;
           break;
         }
-        uint8_t* sB = b_ring + bst * B_BYTES;
+        uint8_t* sB = b_ring + bst * BBYTES;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(sB + off + ((c ^ (r_sw & 7)) << 4)) = out[c];
+        for (int c = 0; c < NCH; ++c)
+          *reinterpret_cast<uint4*>(sB + off + (((c0 + c) ^ (r & 7)) << 4)) = out[c];
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&b_full[bst]);
+        if (lane == 0) {
+          if constexpr (C2) mbar_arrive_cluster(bfull_leader + static_cast<uint32_t>(bst * 8));
+          else mbar_arrive(&b_full[bst]);
+        }
         if (++bst == NB) {
           bst = 0;
           bph ^= 1u;

@@ -378,26 +378,33 @@ def test_trainable_head_rejects_quantised_heads():
     assert e.value.status == 2
 
 
-@pytest.mark.parametrize("cfg,split,D,V", [(1, (40, 45, 44), 128, 257),
-                                           (2, (100, 150, 262), 256, 4097),
-                                           (1, (300, 400, 500), 512, 3000),
-                                           (1, (300, 400, 400), 448, 2000),
-                                           (0, (8, 60, 188), 64, 300),
-                                           (0, (40, 100, 116), 256, 1000)])
-def test_cta_pairs_match_single_cta(cfg, split, D, V):
+@pytest.mark.parametrize("cfg,split,D,V,wformat", [(1, (40, 45, 44), 128, 257, None),
+                                                   (2, (100, 150, 262), 256, 4097, None),
+                                                   (1, (300, 400, 500), 512, 3000, None),
+                                                   (1, (300, 400, 400), 448, 2000, None),
+                                                   (0, (8, 60, 188), 64, 300, None),
+                                                   (0, (40, 100, 116), 256, 1000, None),
+                                                   (4, (40, 45, 44), 192, 3000, "q4g64"),
+                                                   (4, (300, 400, 400), 512, 5000, "q4g64"),
+                                                   (4, (40, 45, 44), 128, 3000, "q8g64"),
+                                                   (4, (100, 150, 262), 320, 5000, "q8g64")])
+def test_cta_pairs_match_single_cta(cfg, split, D, V, wformat):
     """The 2-CTA (cta_group::2) tiles and the single-CTA tiles agree, and both
     match the oracle.  Row counts are ones that take pairs (at least two
     128-row tiles, at most an eighth of padding): 129, 512, 1200, 1100 (nine
     row tiles, the last pair half empty) and 256 rows; K depths from 2 to 12
-    steps of 64 wrap the 6-stage ring."""
-    wl = S.make_custom(cfg, M_split=split, D=D, V=V)
+    steps of 64 wrap the 6-stage ring.  The 4- and 8-bit heads run with the
+    in-kernel dequantisation (each CTA of a pair fills its half of B)."""
+    wl = S.make_custom(cfg, M_split=split, D=D, V=V, wformat=wformat)
     outs = []
     for pairs in (True, False):
         cce.cce_set_cta_pairs(pairs)
+        cce.cce_set_quant_staging(1)
         try:
             _, _, _, buf, st = run_pass(wl)
         finally:
             cce.cce_set_cta_pairs(True)
+            cce.cce_set_quant_staging(0)
         assert st == 0
         outs.append((buf.logp.cpu().numpy(), buf.lse.cpu().numpy(), buf.dH.cpu().numpy()))
     (lp1, ls1, d1), (lp0, ls0, d0) = outs
