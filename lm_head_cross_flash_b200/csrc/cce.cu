@@ -170,12 +170,12 @@ struct DevInfo {
   bool attrs = false;
 };
 
-template <Mode MODE, int QB = 0>
+template <Mode MODE>
 int max_pairs_of() {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);
-  cfg.blockDim = dim3(QB ? NUM_THREADS_Q4 : NUM_THREADS);
-  cfg.dynamicSmemBytes = smem_bytes<MODE, true, QB>();
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<MODE, true>();
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
@@ -184,7 +184,7 @@ int max_pairs_of() {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, cce_tc_kernel<MODE, QB, true>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, cce_tc_kernel<MODE, 0, true>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -210,21 +210,13 @@ cce_status device_info(int* sms) {
     CCE_SET_SMEM(Mode::kLse, 8) CCE_SET_SMEM(Mode::kGrad, 8) CCE_SET_SMEM(Mode::kDh, 8)
     CCE_SET_SMEM(Mode::kDw, 0)
 #undef CCE_SET_SMEM
-#define CCE_SET_SMEM2(MODE, QB) \
-    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, QB, true>, attr, smem_bytes<MODE, true, QB>()) == cudaSuccess;
-    CCE_SET_SMEM2(Mode::kLse, 0) CCE_SET_SMEM2(Mode::kGrad, 0) CCE_SET_SMEM2(Mode::kDh, 0)
-    CCE_SET_SMEM2(Mode::kLse, 4) CCE_SET_SMEM2(Mode::kGrad, 4) CCE_SET_SMEM2(Mode::kDh, 4)
-    CCE_SET_SMEM2(Mode::kLse, 8) CCE_SET_SMEM2(Mode::kGrad, 8) CCE_SET_SMEM2(Mode::kDh, 8)
+#define CCE_SET_SMEM2(MODE) \
+    ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, 0, true>, attr, smem_bytes<MODE, true>()) == cudaSuccess;
+    CCE_SET_SMEM2(Mode::kLse) CCE_SET_SMEM2(Mode::kGrad) CCE_SET_SMEM2(Mode::kDh)
 #undef CCE_SET_SMEM2
-    if (ok) {
-      const int dense = std::min(max_pairs_of<Mode::kLse>(),
-                                 std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
-      const int q4 = std::min(max_pairs_of<Mode::kLse, 4>(),
-                              std::min(max_pairs_of<Mode::kGrad, 4>(), max_pairs_of<Mode::kDh, 4>()));
-      const int q8 = std::min(max_pairs_of<Mode::kLse, 8>(),
-                              std::min(max_pairs_of<Mode::kGrad, 8>(), max_pairs_of<Mode::kDh, 8>()));
-      d.pairs = std::min(dense, std::min(q4, q8));
-    }
+    if (ok)
+      d.pairs = std::min(max_pairs_of<Mode::kLse>(),
+                         std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
     if (!ok)
       return CCE_ERR_CUDA;
     d.attrs = true;
@@ -317,8 +309,7 @@ int choose_ksplit(int64_t tiles, int sms) {
 // unless padding the rows to 256-row pair tiles would add more than an eighth
 // to the 128-row tiles' work (M <= 128: a single row tile, HBM-bound on W).
 bool pairs_wanted(int64_t M, const cce_head* W, bool staged = false) {
-  (void)staged;  // dense, staged and in-kernel-dequantised heads all run pairs
-  if (g_pairs.load() == 0) return false;
+  if (g_pairs.load() == 0 || (W->format != CCE_W_DENSE && !staged)) return false;
   const int64_t n128 = ceil_div(M, BM);
   return n128 >= 2 && 8 * (2 * ceil_div(M, 2 * BM) - n128) <= n128;
 }
@@ -465,15 +456,15 @@ int grid_for(int64_t tiles, int sms) {
 }
 
 // Launch a tensor-core step on CTA pairs (clusters of two, cta_group::2).
-template <Mode MODE, int QB = 0>
+template <Mode MODE>
 cudaError_t launch_tc_pairs(int64_t pair_tiles, int max_pairs, cudaStream_t st,
                             const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                             const CUtensorMap& mc2, const TileArgs& args) {
   cudaLaunchConfig_t cfg = {};
   const int pairs = int(std::max<int64_t>(1, std::min<int64_t>(pair_tiles, max_pairs)));
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(QB ? NUM_THREADS_Q4 : NUM_THREADS);
-  cfg.dynamicSmemBytes = smem_bytes<MODE, true, QB>();
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<MODE, true>();
   cfg.stream = st;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -482,18 +473,7 @@ cudaError_t launch_tc_pairs(int64_t pair_tiles, int max_pairs, cudaStream_t st,
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, cce_tc_kernel<MODE, QB, true>, ma, mb, mc, mc2, args);
-}
-
-// CTA-pair launch of the instantiation for a head read in-kernel with qb
-// bits per weight (0: a 16-bit operand).
-template <Mode MODE>
-cudaError_t launch_pairs(int qb, int64_t pair_tiles, int max_pairs, cudaStream_t st,
-                         const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
-                         const CUtensorMap& mc2, const TileArgs& args) {
-  if (qb == 4) return launch_tc_pairs<MODE, 4>(pair_tiles, max_pairs, st, ma, mb, mc, mc2, args);
-  if (qb == 8) return launch_tc_pairs<MODE, 8>(pair_tiles, max_pairs, st, ma, mb, mc, mc2, args);
-  return launch_tc_pairs<MODE, 0>(pair_tiles, max_pairs, st, ma, mb, mc, mc2, args);
+  return cudaLaunchKernelEx(&cfg, cce_tc_kernel<MODE, 0, true>, ma, mb, mc, mc2, args);
 }
 
 // Launch one tensor-core step; a quantised head adds the dequantisation
@@ -720,9 +700,8 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   CUtensorMap ma, mb;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
   if (op.qb) {
-    // kLse: one group of 64 weights of 256 rows (128 per CTA of a pair) per K step
-    if (!make_packed_map(&mb, W, op.qb, 64 * op.qb / 8, pairs ? BN / 2 : BN))
-      return CCE_ERR_CUDA;
+    // kLse: one group of 64 weights of 256 rows per K step
+    if (!make_packed_map(&mb, W, op.qb, 64 * op.qb / 8, BN)) return CCE_ERR_CUDA;
   } else if (staged) {
     mb = ma;  // set per staged chunk
   } else if (!make_map(&mb, op.b, op.bf16, op.k, V, op.ld_b, BK, pairs ? BN / 2 : BN))
@@ -773,8 +752,8 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
       TileArgs a2 = ac;
       a2.n_rt = int(ceil_div(M, 2 * BM));
       a2.group_rt = std::max(1, ac.group_rt / 2);
-      if (launch_pairs<Mode::kLse>(op.qb, int64_t(a2.n_rt) * ct_n, max_pairs, st, ma, mb, ma,
-                                   ma, a2) != cudaSuccess)
+      if (launch_tc_pairs<Mode::kLse>(int64_t(a2.n_rt) * ct_n, max_pairs, st, ma, mb, ma, ma,
+                                      a2) != cudaSuccess)
         return CCE_ERR_CUDA;
     } else {
       launch_tc<Mode::kLse>(op.qb, n_rt * ct_n, sms, st, ma, mb, ma, ma, ac);
@@ -966,10 +945,9 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   const bool pairs = max_pairs > 0;
   if (!make_map(&ma, op.a, op.bf16, op.k, M, op.ld_a, BK, BM)) return CCE_ERR_CUDA;
   if (op.qb) {
-    // packed tiles: kGrad as the forward, kDh 64 rows x 256 columns per K
-    // step (pairs: each CTA its half of the rows, resp. columns)
-    if (!make_packed_map(&mb, W, op.qb, 64 * op.qb / 8, pairs ? BN / 2 : BN) ||
-        !make_packed_map(&mw, W, op.qb, (pairs ? BN / 2 : BN) * op.qb / 8, BK))
+    // packed tiles: kGrad as the forward, kDh 64 rows x 256 columns per K step
+    if (!make_packed_map(&mb, W, op.qb, 64 * op.qb / 8, BN) ||
+        !make_packed_map(&mw, W, op.qb, BN * op.qb / 8, BK))
       return CCE_ERR_CUDA;
   } else if (staged) {
     mb = ma;  // mapped per staged chunk
@@ -1082,8 +1060,8 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
         TileArgs a2 = ag;
         a2.n_rt = int(n_rt2);
         a2.group_rt = std::max(1, ag.group_rt / 2);
-        if (launch_pairs<Mode::kGrad>(op.qb, n_rt2 * ct_n, max_pairs, st, ma, mb, mgs, mgs,
-                                      a2) != cudaSuccess)
+        if (launch_tc_pairs<Mode::kGrad>(n_rt2 * ct_n, max_pairs, st, ma, mb, mgs, mgs, a2) !=
+            cudaSuccess)
           return CCE_ERR_CUDA;
       } else {
         launch_tc<Mode::kGrad>(op.qb, n_rt * ct_n, sms, st, ma, mb, mgs, mgs, ag);
@@ -1105,8 +1083,8 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
       if (pairs) {
         TileArgs a2 = ad;
         a2.n_rt = int(n_rt2);
-        if (launch_pairs<Mode::kDh>(op.qb, n_rt2 * n_dt * ksplit, max_pairs, st, mg, mw, md0,
-                                    md1, a2) != cudaSuccess)
+        if (launch_tc_pairs<Mode::kDh>(n_rt2 * n_dt * ksplit, max_pairs, st, mg, mw, md0, md1,
+                                       a2) != cudaSuccess)
           return CCE_ERR_CUDA;
       } else {
         launch_tc<Mode::kDh>(op.qb, n_rt * n_dt * ksplit, sms, st, mg, mw, md0, md1, ad);

@@ -50,9 +50,8 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;     // TMA, MMA, 4 epilogue warps
 constexpr int DQ_WARPS = 8;          // dequantisation warps (4-bit head), 2 per SMSP
+constexpr int NUM_THREADS_Q4 = NUM_THREADS + 32 * DQ_WARPS;
 constexpr int DQ_WARP0 = 6;
-constexpr int PK_WARP = DQ_WARP0 + DQ_WARPS;  // packed-weight TMA producer
-constexpr int NUM_THREADS_Q4 = NUM_THREADS + 32 * DQ_WARPS + 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2, kDw = 3 };
 
@@ -68,37 +67,19 @@ __host__ __device__ constexpr int staging_buf_bytes() {
 constexpr int STAGES2 = 6;
 constexpr int B_HALF_BYTES = (BN / 2) * BK * 2;
 constexpr int STAGE2_BYTES = A_BYTES + B_HALF_BYTES;
-// Quantised heads (QB = 4 or 8) dequantise B in-kernel.  Their stages are
-// three separate rings: A tiles (TMA; as many as fit, up to 8, so the L2
-// round trip of H is hidden), B tiles written by the dequantisation warps (2),
-// and the packed weights of each B tile (kLse/kGrad: 256 rows x one group of
-// 64; kDh: 64 rows x 256 columns), which a producer warp of their own streams
-// from HBM by TMA (4).
-constexpr int SMEM_LIMIT = 232448;  // bytes of dynamic shared memory per block
-constexpr int BAR_BYTES = 512;      // mbarriers, TMEM slot, abort flag
-constexpr int QB_NB = 2;
-constexpr int QB_NPK = 4;
-// On CTA pairs (C2) each CTA holds half of B and of its packed tile.
-template <Mode MODE, int QB, bool C2 = false>
+// Quantised heads (QB = 4 or 8) dequantise B in-kernel.  Each of their 3
+// stages also holds the packed weights of its B tile, brought in by TMA
+// (kLse/kGrad: 256 rows x one group of 64; kDh: 64 rows x 256 columns).
+constexpr int STAGES_Q = 3;
+template <Mode MODE, int QB>
 __host__ __device__ constexpr int pk_bytes() {
-  return (MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8)) / (C2 ? 2 : 1);
-}
-template <Mode MODE, int QB, bool C2 = false>
-__host__ __device__ constexpr int qa_free() {
-  return SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * (C2 ? B_HALF_BYTES : B_BYTES) -
-         QB_NPK * pk_bytes<MODE, QB, C2>() - 4 * 2 * staging_buf_bytes<MODE>();
-}
-template <Mode MODE, int QB, bool C2 = false>
-__host__ __device__ constexpr int qa_stages() {
-  return QB == 0 ? 0 : (qa_free<MODE, QB, C2>() / A_BYTES > 8 ? 8 : qa_free<MODE, QB, C2>() / A_BYTES);
+  return MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8);
 }
 template <Mode MODE, bool C2 = false, int QB = 0>
 __host__ __device__ constexpr int smem_bytes() {
-  return (QB ? qa_stages<MODE, QB, C2>() * A_BYTES + QB_NB * (C2 ? B_HALF_BYTES : B_BYTES) +
-                   QB_NPK * pk_bytes<MODE, QB, C2>()
-             : C2 ? STAGES2 * STAGE2_BYTES
-                  : STAGES * STAGE_BYTES) +
-         4 * 2 * staging_buf_bytes<MODE>() + 1024 + BAR_BYTES;
+  return (C2 ? STAGES2 * STAGE2_BYTES
+             : QB ? STAGES_Q * (STAGE_BYTES + pk_bytes<MODE, QB>()) : STAGES * STAGE_BYTES) +
+         4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
@@ -164,30 +145,49 @@ __host__ __device__ constexpr int qpos(int e) {
   return QB == 8 ? q8_pos(e) : QB == 4 ? q4_pos(e) : e;
 }
 
-// Dequantise NCH consecutive 8-weight chunks of a group of 64: w = q * scale
-// + bias, rounded once to fp16 (fma.rn.f16x2 on q, scale, bias, all exact in
-// fp16); q comes from the bit pattern 0x6400 | q = 1024 + q in fp16.  Chunk c
-// is word c of a 4-bit group (element 8c+j = bits 4j..4j+3) or words 2c, 2c+1
-// of an 8-bit group (element 4w+j = byte j of word w).  out[c] holds the 8
-// fp16 values of chunk c in qpos<QB> order: (e0,e4) (e1,e5) (e2,e6) (e3,e7)
-// for 4-bit, (e0,e2) (e1,e3) (e4,e6) (e5,e7) for 8-bit.
-template <int QB, int NCH>
-__device__ __forceinline__ void dequant_chunks(const uint32_t* words, uint16_t sbits,
-                                               uint16_t bbits, uint4 (&out)[NCH]) {
+// 8-bit variant: 16 packed words (element 4c+j = byte j of word c).
+__device__ __forceinline__ void dequant_group64_q8(const uint4 (&wv)[4], uint16_t sbits,
+                                                   uint16_t bbits, uint4 (&out)[8]) {
   const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
   const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bbits) << 16));
   const __half2 k1024 = __float2half2_rn(1024.f);
+  const uint32_t words[16] = {wv[0].x, wv[0].y, wv[0].z, wv[0].w, wv[1].x, wv[1].y,
+                              wv[1].z, wv[1].w, wv[2].x, wv[2].y, wv[2].z, wv[2].w,
+                              wv[3].x, wv[3].y, wv[3].z, wv[3].w};
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
+  for (int c = 0; c < 8; ++c) {
     uint32_t t[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t x =
-          QB == 8 ? ((words[2 * c + (i >> 1)] >> (8 * (i & 1))) & 0x00FF00FFu) | 0x64006400u
-                  : ((words[c] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
-      __half2 hh = *reinterpret_cast<const __half2*>(&x);
-      hh = __hfma2(__hsub2(hh, k1024), s2, b2);
-      t[i] = *reinterpret_cast<uint32_t*>(&hh);
+      const uint32_t x = ((words[2 * c + (i >> 1)] >> (8 * (i & 1))) & 0x00FF00FFu) | 0x64006400u;
+      __half2 h = *reinterpret_cast<const __half2*>(&x);
+      h = __hfma2(__hsub2(h, k1024), s2, b2);
+      t[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    out[c] = make_uint4(t[0], t[1], t[2], t[3]);
+  }
+}
+
+// Dequantise the 64 weights of one (row, group): w = q * scale + bias, with
+// q read from 8 packed words (element 8c+j = bits 4j..4j+3 of word c) and
+// the result rounded once to fp16 (fma.rn.f16x2 on q, scale, bias, all exact
+// in fp16).  q comes from the bit pattern 0x6400 | q = 1024 + q in fp16.
+// out[c] holds the 8 fp16 values of word c in q4_pos order.
+__device__ __forceinline__ void dequant_group64(const uint4& wa, const uint4& wb, uint16_t sbits,
+                                                uint16_t bbits, uint4 (&out)[8]) {
+  const __half2 s2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
+  const __half2 b2 = __float2half2_rn(__uint_as_float(static_cast<uint32_t>(bbits) << 16));
+  const __half2 k1024 = __float2half2_rn(1024.f);
+  const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t x = ((words[c] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
+      __half2 h = *reinterpret_cast<const __half2*>(&x);
+      h = __hfma2(__hsub2(h, k1024), s2, b2);
+      t[i] = *reinterpret_cast<uint32_t*>(&h);
     }
     out[c] = make_uint4(t[0], t[1], t[2], t[3]);
   }
@@ -319,16 +319,11 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC,
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
+  static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
   static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
-  // Stages of the operand ring (quantised heads: A only; B has its own ring).
-  constexpr int NST = QB ? qa_stages<MODE, QB, C2>() : (C2 ? STAGES2 : STAGES);
-  constexpr int SBYTES = QB ? A_BYTES : (C2 ? STAGE2_BYTES : STAGE_BYTES);
-  constexpr int NB = QB ? QB_NB : 0;                       // dequantised B ring
-  constexpr int BBYTES = C2 ? B_HALF_BYTES : B_BYTES;      // this CTA's B tile
-  constexpr int PKB = QB ? pk_bytes<MODE, QB, C2>() : 0;  // this CTA's packed tile
-  constexpr int NPK = QB ? QB_NPK : 0;                      // packed ring depth
-  static_assert(!QB || NST >= 3, "quantised heads need 3 A stages at least");
-  static_assert(smem_bytes<MODE, C2, QB>() <= SMEM_LIMIT, "shared memory");
+  constexpr int NST = C2 ? STAGES2 : (QB ? STAGES_Q : STAGES);
+  constexpr int PKB = QB ? pk_bytes<MODE, QB>() : 0;  // packed B tile per stage
+  constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES + PKB;
   // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
   // rank 0 (the leader) issues the MMAs for both; each CTA loads its own
   // 128 rows of A and its half of B and drains its own 128 TMEM lanes.
@@ -341,17 +336,12 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t* b_ring = base + NST * SBYTES;    // quantised heads: dequantised B
-  uint8_t* pk_ring = b_ring + NB * BBYTES;  // quantised heads: packed tiles
-  uint8_t* staging = pk_ring + NPK * PKB;
+  uint8_t* staging = base + NST * SBYTES;
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
   uint64_t* empty = full + NST;
-  uint64_t* b_full = empty + NST;       // B tile written by all dequant warps
-  uint64_t* b_empty = b_full + NB;      // B tile consumed by the MMAs
-  uint64_t* pk_full = b_empty + NB;     // packed tile landed (quantised heads)
-  uint64_t* pk_empty = pk_full + NPK;   // packed tile read by all dequant warps
-  uint64_t* acc_full = pk_empty + NPK;
+  uint64_t* pk_full = empty + NST;  // packed tile landed (quantised heads)
+  uint64_t* acc_full = pk_full + NST;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -364,16 +354,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], QB ? 1 + DQ_WARPS : 1);
       mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < NB; ++s) {
-      mbar_init(&b_full[s], (C2 ? 2 : 1) * DQ_WARPS);  // the leader's counts both CTAs
-      mbar_init(&b_empty[s], 1);
-    }
-    for (int s = 0; s < NPK; ++s) {
       mbar_init(&pk_full[s], 1);
-      mbar_init(&pk_empty[s], DQ_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -429,26 +412,30 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * SBYTES);
             const int arow = (tc.rt * 2 + static_cast<int>(rank)) * BM;
-            // (quantised heads: A only, B comes from the dequantisation warps)
             if (MODE == Mode::kDh) {
               tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, l2_policy_evict_normal());
-              if (!QB) {
 #pragma unroll
-                for (int j = 0; j < BN / 128; ++j)
-                  tma_load_2d_pair(sB + j * (64 * BK * 2), &tmB, bar,
-                                   tc.ct * BN + static_cast<int>(rank) * (BN / 2) + j * 64 +
-                                       pass * a.b_pass_off,
-                                   a.b_row0 - a.b_shift + k * BK, keep);
-              }
+              for (int j = 0; j < BN / 128; ++j)
+                tma_load_2d_pair(sB + j * (64 * BK * 2), &tmB, bar,
+                                 tc.ct * BN + static_cast<int>(rank) * (BN / 2) + j * 64 +
+                                     pass * a.b_pass_off,
+                                 a.b_row0 - a.b_shift + k * BK, keep);
             } else {
               tma_load_2d_pair(sA, &tmA, bar, k * BK, arow, keep);
-              if (!QB)
-                tma_load_2d_pair(sB, &tmB, bar, k * BK,
-                                 a.b_row0 - a.b_shift + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
-                                 l2_policy_evict_normal());
+              tma_load_2d_pair(sB, &tmB, bar, k * BK,
+                               a.b_row0 - a.b_shift + tc.ct * BN + static_cast<int>(rank) * (BN / 2),
+                               l2_policy_evict_normal());
             }
           } else if (QB) {
-            // B comes from the dequantisation warps.
+            // B comes from the dequantisation warps, which read the packed
+            // tile (tmB: the packed head as bytes [V, D*QB/8]) from the stage.
+            uint8_t* sP = sA + STAGE_BYTES;
+            mbar_arrive_expect_tx(&pk_full[stage], PKB);
+            if (MODE == Mode::kDh)
+              tma_load_2d(sP, &tmB, &pk_full[stage], tc.ct * (BN * QB / 8), a.b_row0 + k * BK);
+            else
+              tma_load_2d(sP, &tmB, &pk_full[stage], k * (64 * QB / 8),
+                          a.b_row0 + tc.ct * BN);
             mbar_arrive_expect_tx(&full[stage], A_BYTES);
             if (MODE == Mode::kDh)
               tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
@@ -495,17 +482,20 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       // cluster barrier keeps both CTAs alive until then).
       if (!C2 || rank == 0)
         for (int s = 0; s < NST; ++s)
-          if (issued_mask & (1u << s))
+          if (issued_mask & (1u << s)) {
+            if (QB)
+              wait_bounded(&pk_full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS, nullptr);
             wait_bounded(&full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS,
                          nullptr);
+          }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_f16(C2 ? 2 * BM : BM, BN, a.fmt, MODE == Mode::kDw,
                                        MODE == Mode::kDh || MODE == Mode::kDw);
-      int stage = 0, bst = 0;
-      uint32_t phase = 0, bph = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       int acc = 0;
       bool ok = true;
       for (int t = tile0; t < ntiles && ok; t += tstride) {
@@ -522,15 +512,13 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kk = 0; kk < ksteps; ++kk) {
-          if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag) ||
-              (QB && !wait_bounded(&b_full[bst], bph, a.wait_ns, abort_flag))) {
+          if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
             ok = false;
             break;
           }
-          if (C2 && QB) fence_acq_rel_cluster();  // the peer's B half is visible
           tc_fence_after();
           const uint32_t sA = smem_u32(base + stage * SBYTES);
-          const uint32_t sB = QB ? smem_u32(b_ring + bst * BBYTES) : sA + A_BYTES;
+          const uint32_t sB = sA + A_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             const uint64_t ad = MODE == Mode::kDw
@@ -548,14 +536,6 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           // the stage is free in both CTAs once these MMAs have read it
           if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
           else umma_commit(&empty[stage]);
-          if (QB) {
-            if constexpr (C2) umma_commit2_mc(&b_empty[bst], 0x3);
-            else umma_commit(&b_empty[bst]);
-            if (++bst == NB) {
-              bst = 0;
-              bph ^= 1u;
-            }
-          }
           if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
@@ -575,97 +555,44 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       else umma_commit(drain);
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
     }
-  } else if (QB && warp == PK_WARP) {
-    // -------------------------------------------- packed-weight producer --
-    // Streams the packed B tile of every K step (tmB: the packed head as
-    // bytes [V, D*QB/8]) into the packed ring, as far ahead as the ring
-    // allows, independently of the operand stages.
-    if (lane == 0) {
-      int ps = 0;
-      uint32_t pph = 0, issued_mask = 0, issued_phase = 0;
-      bool ok = true;
-      for (int t = tile0; t < ntiles && ok; t += tstride) {
-        const TileCoord tc = tile_coord<MODE>(a, t);
-        if (launch_kind<MODE, C2>(a, tc.rt, tc.ct, tc.s) != 0) continue;
-        const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
-        for (int kk = 0; kk < nks; ++kk) {
-          if (!wait_bounded(&pk_empty[ps], pph ^ 1u, a.wait_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int k = kb + kk;
-          mbar_arrive_expect_tx(&pk_full[ps], PKB);
-          // this CTA's half of the B tile on pairs (columns, resp. rows)
-          if (MODE == Mode::kDh)
-            tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps],
-                        tc.ct * (BN * QB / 8) + static_cast<int>(rank) * (BN / 2 * QB / 8),
-                        a.b_row0 + k * BK);
-          else
-            tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps], k * (64 * QB / 8),
-                        a.b_row0 + tc.ct * BN + static_cast<int>(rank) * (BN / 2));
-          issued_mask |= 1u << ps;
-          issued_phase = (issued_phase & ~(1u << ps)) | (pph << ps);
-          if (++ps == NPK) {
-            ps = 0;
-            pph ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        set_status(a.status, ST_TIMEOUT);
-        *abort_flag = 1;
-      }
-      for (int s2 = 0; s2 < NPK; ++s2)  // every issued copy lands before exit
-        if (issued_mask & (1u << s2))
-          wait_bounded(&pk_full[s2], (issued_phase >> s2) & 1u, DRAIN_LIMIT_NS, nullptr);
-    }
   } else if (QB && warp >= DQ_WARP0) {
     // ------------------------------------------ 4/8-bit dequantisation --
-    // 256 threads fill this CTA's B tile of every K step.  Single CTA: 256
-    // (row, group) units of 64 weights, one per thread.  Pair: this CTA's
-    // half of B holds 128 units, so each thread takes half a unit (32
-    // weights, 4 of its 8 16-byte chunks).  The packed words come from the
-    // packed ring (a slot is released after use, behind a proxy fence: its
-    // refill is an async-proxy write); scale and bias from global memory
-    // (kLse/kGrad: 8 groups of a row per 16-byte load when rows are 16-byte
-    // aligned).  The fp16 result is written in the 128-byte-swizzled layout
-    // the TMA would produce (16-byte chunk c of row r at c ^ (r & 7)).
+    // 256 threads fill the B half of every stage: 256 (row, group) units of
+    // 64 weights per K step, one per thread.  The packed words come from the
+    // stage (TMA, pk_full); scale and bias from global memory, fetched one
+    // unit ahead (kLse/kGrad: 8 groups of a row at once when rows are 16-byte
+    // aligned).  Each unit is dequantised to fp16 and written in the
+    // 128-byte-swizzled layout the TMA would produce (16-byte chunk c of row
+    // r at c ^ (r & 7)).
     constexpr int QU = 64 * (QB ? QB : 4) / 8;  // packed bytes per unit
-    constexpr int NCH = C2 ? 4 : 8;             // 16-byte output chunks per thread
-    constexpr int NV = QU * NCH / 8 / 16;       // 16-byte packed vectors per thread
+    constexpr int NV = QU / 16;
     const int dq = threadIdx.x - DQ_WARP0 * 32;
     const int gpr = a.D / 64;  // groups per head row
     const bool vec8 = MODE != Mode::kDh && (gpr % 8) == 0 &&
                       ((reinterpret_cast<uintptr_t>(a.q_scale) |
                         reinterpret_cast<uintptr_t>(a.q_bias)) & 15u) == 0;
-    int bst = 0, ps = 0;
-    uint32_t bph = 0, pph = 0;
+    int stage = 0;
+    uint32_t phase = 0;
     bool ok = true;
-    // This thread's part of K step k of tile tc: source row v and group g,
-    // the offset of its packed words in the packed tile, its output row r in
-    // B (for the swizzle), the offset of that row, and its first chunk c0.
-    // kDh: the groups of a row sit in adjacent threads (their scales share a
+    // unit u of K step k of tile tc: source row, group, offset of its packed
+    // words in the stage's packed tile, and of its fp16 output in B.  kDh:
+    // the 4 groups of a row are adjacent threads (their scales share a
     // sector).
-    const int h = C2 ? (dq & 1) : 0;  // half of the unit (pairs)
-    const int c0 = h * NCH;
-    auto locate = [&](const TileCoord& tc, int k, int& v, int& g, int& pk, int& r, int& off) {
+    auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& pk, int& off) {
       if (MODE == Mode::kDh) {
-        constexpr int GW = C2 ? 2 : 4;  // groups of this CTA's B columns
-        const int u = C2 ? (dq >> 1) : dq;
-        r = u / GW;
-        const int j = u % GW;
+        const int r = u >> 2, j = u & 3;
         v = a.b_row0 + k * BK + r;
-        g = tc.ct * (BN / 64) + static_cast<int>(rank) * GW * (C2 ? 1 : 0) + j;
-        pk = r * (GW * QU) + j * QU + h * (QU / 2);
+        g = tc.ct * (BN / 64) + j;
+        pk = r * (BN * QB / 8) + j * QU;
         off = j * (64 * BK * 2) + r * 128;
       } else {
-        r = C2 ? (dq >> 1) : dq;
-        v = a.b_row0 + tc.ct * BN + static_cast<int>(rank) * (BN / 2) + r;
+        v = a.b_row0 + tc.ct * BN + u;
         g = k;
-        pk = r * QU + h * (QU / 2);
-        off = r * 128;
+        pk = u * QU;
+        off = u * 128;
       }
     };
+    const int r_sw = MODE == Mode::kDh ? (dq >> 2) : dq;  // row for the swizzle
     uint4 sv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);  // 8 groups (vec8)
     int vec_row = -1, vec_g0 = -1;
     auto scale_bias = [&](int v, int g, uint16_t& sc, uint16_t& bi) {
@@ -687,60 +614,46 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         bi = __ldg(a.q_bias + static_cast<size_t>(v) * gpr + g);
       }
     };
-    // the leader's b_full counts both CTAs' dequantisation warps
-    const uint32_t bfull_leader = C2 ? mapa_shared(smem_u32(&b_full[0]), 0) : 0u;
     for (int t = tile0; t < ntiles && ok; t += tstride) {
       const TileCoord tc = tile_coord<MODE>(a, t);
-      if (launch_kind<MODE, C2>(a, tc.rt, tc.ct, tc.s) != 0) continue;
+      if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
       const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
       for (int kk = 0; kk < nks; ++kk) {
-        int v, g, pk, r, off;
-        locate(tc, kb + kk, v, g, pk, r, off);
+        int v, g, pk, off;
+        locate(tc, kb + kk, dq, v, g, pk, off);
         const bool valid = v < a.V && g < gpr;
         uint16_t sc = 0, bi = 0;
         if (valid) scale_bias(v, g, sc, bi);
-        if (!wait_bounded(&pk_full[ps], pph, a.wait_ns, abort_flag)) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag) ||
+            !wait_bounded(&pk_full[stage], phase, a.wait_ns, abort_flag)) {
           ok = false;
           break;
         }
-        uint4 out[NCH];
+        uint8_t* sA = base + stage * SBYTES;
+        uint8_t* sB = sA + A_BYTES;
+        const uint8_t* sP = sA + STAGE_BYTES;
+        uint4 out[8];
         if (valid) {
           uint4 w[NV];
 #pragma unroll
-          for (int i = 0; i < NV; ++i)
-            w[i] = *reinterpret_cast<const uint4*>(pk_ring + ps * PKB + pk + 16 * i);
-          dequant_chunks<QB, NCH>(reinterpret_cast<const uint32_t*>(w), sc, bi, out);
+          for (int i = 0; i < NV; ++i) w[i] = *reinterpret_cast<const uint4*>(sP + pk + 16 * i);
+          if constexpr (QB == 8)
+            dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sc, bi, out);
+          else
+            dequant_group64(w[0], w[NV - 1], sc, bi, out);
         } else {
 #pragma unroll
-          for (int c = 0; c < NCH; ++c) out[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
         }
-        // The slot may be refilled (TMA, async proxy) once every warp is done
-        // with it: the values computed above hold the loaded words, and the
-        // proxy fence orders these generic reads before the refill.
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pk_empty[ps]);
-        if (++ps == NPK) {
-          ps = 0;
-          pph ^= 1u;
-        }
-        if (!wait_bounded(&b_empty[bst], bph ^ 1u, a.wait_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sB = b_ring + bst * BBYTES;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          *reinterpret_cast<uint4*>(sB + off + (((c0 + c) ^ (r & 7)) << 4)) = out[c];
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(sB + off + ((c ^ (r_sw & 7)) << 4)) = out[c];
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          if constexpr (C2) mbar_arrive_cluster(bfull_leader + static_cast<uint32_t>(bst * 8));
-          else mbar_arrive(&b_full[bst]);
-        }
-        if (++bst == NB) {
-          bst = 0;
-          bph ^= 1u;
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == NST) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
     }

@@ -394,7 +394,8 @@ def test_cta_pairs_match_single_cta(cfg, split, D, V, wformat):
     128-row tiles, at most an eighth of padding): 129, 512, 1200, 1100 (nine
     row tiles, the last pair half empty) and 256 rows; K depths from 2 to 12
     steps of 64 wrap the 6-stage ring.  The 4- and 8-bit heads run with the
-    in-kernel dequantisation (each CTA of a pair fills its half of B)."""
+    in-kernel dequantisation, which stays on single-CTA tiles: both settings
+    must give the same results."""
     wl = S.make_custom(cfg, M_split=split, D=D, V=V, wformat=wformat)
     outs = []
     for pairs in (True, False):
