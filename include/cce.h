@@ -38,6 +38,9 @@
  * - Labels: y < 0 marks an ignored row (logp = 0, no loss term, dH row
  *   exactly 0; lse is still computed).  y >= V is an error.
  * - Tensor-core path requirements: D % 64 == 0; 16-byte aligned pointers.
+ * - Size limits: M <= 2^30, V <= 2^30, D <= 2^16, and the kernels' tile count
+ *   ceil(M/128) * max(ceil(V/256), 32*ceil(D/256)) below 2^31; larger
+ *   problems return CCE_ERR_UNSUPPORTED (split them by rows).
  */
 #ifndef CCE_H_
 #define CCE_H_

@@ -258,6 +258,15 @@ cce_status check_head(const cce_head* W, cce_dtype h_dtype) {
   return CCE_ERR_INVALID_ARGUMENT;
 }
 
+// The kernels number their tiles with 32-bit ints: ceil(M/128) row tiles
+// times the vocab tiles (forward, recompute) or the d-tiles of every K split
+// (dH, at most 32 splits) must stay below 2^31.
+bool tiles_fit(int64_t M, const cce_head* W) {
+  const int64_t n_rt = (M + 127) / 128;
+  const int64_t per_row = std::max<int64_t>((W->V + 255) / 256, 32 * ((W->D + 255) / 256));
+  return n_rt * per_row < (int64_t(1) << 31) - 1;
+}
+
 // ------------------------------------------------------ workspace layout --
 struct Layout {
   size_t status = 0;
@@ -635,6 +644,7 @@ cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_
   if (h_dtype != CCE_F32 && h_dtype != CCE_BF16) return CCE_ERR_INVALID_ARGUMENT;
   const cce_status s = check_head(W, h_dtype);
   if (s != CCE_OK) return s;
+  if (!tiles_fit(M, W)) return CCE_ERR_UNSUPPORTED;
   std::memset(out, 0, sizeof(*out));
   const FwdPlan f = plan_forward(M, h_dtype, W, ws_bytes);
   const BwdPlan b = plan_backward(M, h_dtype, W, ws_bytes);
@@ -675,6 +685,7 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   if (!aligned16(H) || !aligned16(ws)) return CCE_ERR_INVALID_ARGUMENT;
   cce_status s = check_head(W, h_dtype);
   if (s != CCE_OK) return s;
+  if (!tiles_fit(M, W)) return CCE_ERR_UNSUPPORTED;
   // A staged 4/8-bit head takes the widest fp16 chunk the workspace holds.
   const FwdPlan plan = plan_forward(M, h_dtype, W, ws_bytes);
   const bool staged = plan.staged;
@@ -903,6 +914,7 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   if (!aligned16(H) || !aligned16(ws) || !aligned16(dH)) return CCE_ERR_INVALID_ARGUMENT;
   cce_status s = check_head(W, h_dtype);
   if (s != CCE_OK) return s;
+  if (!tiles_fit(M, W)) return CCE_ERR_UNSUPPORTED;
   // K split of the dH GEMM; fall back to fewer splits if the workspace
   // cannot hold their partial buffers.
   // A staged 4/8-bit head needs chunks of stage_min_rows at least; else the

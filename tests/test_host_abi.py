@@ -188,3 +188,20 @@ def test_query_plan_quant_staging(lib):
             assert pl["fwd_ok"] and pl["bwd_ok"] and not pl["bwd_staged"]
     finally:
         cce.cce_set_quant_staging(0)
+
+
+def test_oversized_tile_counts_are_rejected(lib):
+    """Shapes whose tile count would overflow the kernels' 32-bit tile ids
+    are refused before anything is launched."""
+    big = _head(V=1 << 30, D=2048)
+    f = ctypes.c_void_p(4096)
+    M = 1 << 30
+    st = lib.cce_forward(f, cce.CCE_BF16, M, ctypes.byref(big), f, f, f, None, None, f,
+                         1 << 40, None)
+    assert cce.STATUS_NAMES[st] == "CCE_ERR_UNSUPPORTED"
+    out = cce._Plan()
+    assert lib.cce_query_plan(M, cce.CCE_BF16, ctypes.byref(big), 1 << 40,
+                              ctypes.byref(out)) == 2
+    # the same head at a modest M is accepted by the planner
+    assert lib.cce_query_plan(8192, cce.CCE_BF16, ctypes.byref(big), 1 << 40,
+                              ctypes.byref(out)) == 0
