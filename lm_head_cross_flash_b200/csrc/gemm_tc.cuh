@@ -20,7 +20,7 @@
 // the accumulator with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)..+31,
 // i.e. one row per thread) and run the epilogue, overlapping the MMA of the
 // next tile.  A quantised head (QB = 4 or 8) adds 8 warps that dequantise
-// the B half of every stage.  Tiles are assigned round-robin over a grid of
+// the B half of every stage (3 stages, each also holding the packed B tile).  Tiles are assigned round-robin over a grid of
 // at most one CTA per SM, in the order tile_coord gives (below), so the CTAs
 // in flight share the operand that should stay in L2.
 //
