@@ -52,6 +52,10 @@ def parse_args(argv=None):
                    help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
     p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
                    help="1: 2-CTA (cta_group::2) tiles where they apply; 0: single-CTA tiles")
+    p.add_argument("--graph", action="store_true",
+                   help="time replays of the head pass captured as one CUDA graph (for the "
+                        "launch-bound small workloads); per-kernel times then come from as "
+                        "many profiled direct passes after the timed region")
     p.add_argument("--sweep", choices=["small_m", "small_m_q4"], default=None,
                    help="the W-stream (HBM-bound) regime, M in {64, 128, 256}, one JSON "
                         "line per M: small_m at D=2048, V=262144 (bf16 head); small_m_q4 "
@@ -259,10 +263,15 @@ def run_ours(args):
         cce.orpo_head_pass(H, head, labels, wl.layout_tuple, wl.lam, wl.scope, wl.filter_eps,
                            wl.block_skip, buf, stream)
 
+    run_step = step
+    if args.graph:
+        run_step = cce.HeadPassGraph(H, head, labels, wl.layout_tuple, wl.lam, wl.scope,
+                                     wl.filter_eps, wl.block_skip, buf).replay
+
     sampler = ClockSampler(gpu_uuid(dev))
     sampler.start()
     for _ in range(max(3, args.warmup)):
-        step()
+        run_step()
     torch.cuda.synchronize(dev)
     st = cce.cce_device_status(buf.ws)
     if st != 0:
@@ -271,17 +280,22 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    cce.cce_profile_enable(True)
+    cce.cce_profile_enable(not args.graph)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        run_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     ms_total = e0.elapsed_time(e1)
+    if args.graph:  # kernel times of the same work, from direct passes
+        cce.cce_profile_enable(True)
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize(dev)
     prof = cce.cce_profile_read()
     cce.cce_profile_enable(False)
     sampler.stop()
@@ -430,6 +444,7 @@ def run_ours(args):
                    "l2": "inputs larger than L2 (W is 1.07 GB, L2 126 MB); no flush",
                    "workspace_bytes": int(buf.ws.numel()),
                    "cta_pairs": bool(args.cta_pairs),
+                   "cuda_graph": bool(args.graph),
                    "quant_staging": ["choose", "in-kernel", "staged"][args.quant_staging]},
         "tflops": tflops,
         "executed": {"rows_backward": m_b, "tflop_per_step": flop_exec / 1e12,

@@ -329,6 +329,34 @@ def orpo_head_pass(H, head: Head, labels, layout, lam, sft_scope, filter_eps,
                     buf.blockmax if block_skip else None, buf.dH, buf.skip, buf.ws, stream)
 
 
+class HeadPassGraph:
+    """``orpo_head_pass`` captured once into a CUDA graph and replayed.
+
+    The library allocates nothing and never synchronises inside a call, and
+    every launch goes to the stream it is given, so the whole pass (forward,
+    merge, loss, cotangent, backward) is one graph.  The graph keeps the
+    addresses of ``H``, ``labels`` and ``buf``: copy each step's inputs into
+    those tensors, then ``replay()``.  The settings read at capture time
+    (CTA pairs, quantised-head staging, the wait limit) are frozen into the
+    graph.  Profiling must be off while capturing.
+    """
+
+    def __init__(self, H, head: Head, labels, layout, lam, sft_scope, filter_eps,
+                 block_skip: bool, buf: HeadBuffers):
+        self.args = (H, head, labels, layout, lam, sft_scope, filter_eps, block_skip, buf)
+        side = torch.cuda.Stream(device=H.device)
+        side.wait_stream(torch.cuda.current_stream(H.device))
+        with torch.cuda.stream(side):  # first call outside the capture: one-time setup
+            orpo_head_pass(*self.args, stream=side)
+        torch.cuda.current_stream(H.device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            orpo_head_pass(*self.args, stream=torch.cuda.current_stream(H.device))
+
+    def replay(self):
+        self.graph.replay()
+
+
 def upload_workload(wl, device="cuda"):
     """Device tensors (H, Head, labels) of a ``synthetic.Workload``."""
     import numpy as np

@@ -503,3 +503,32 @@ def test_small_m_many_k_splits(extra_kb):
     assert rel_fro(d1.cpu().numpy(), want) <= TOL_DH
     assert rel_fro(d2.cpu().numpy(), want) <= TOL_DH
     assert rel_fro(d2.cpu().numpy(), d1.cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("cfg,split,D,V", [(0, (32, 96, 128), 256, 4096),
+                                           (1, (100, 150, 262), 256, 3000),
+                                           (4, (40, 45, 44), 128, 2000)])
+def test_head_pass_graph_replay(cfg, split, D, V):
+    """The whole head pass captured in a CUDA graph and replayed gives the
+    same results, bit for bit, as direct calls, also after new inputs are
+    copied into the captured tensors."""
+    wl = S.make_custom(cfg, M_split=split, D=D, V=V)
+    H, head, labels = upload(wl)
+    hd = cce.h_dtype(H)
+    direct = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+    graphed = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+    args = (wl.layout_tuple, wl.lam, wl.scope, wl.filter_eps, wl.block_skip)
+    g = cce.HeadPassGraph(H, head, labels, *args, graphed)
+    for step in range(2):
+        if step == 1:  # new inputs into the captured tensors
+            H.copy_(torch.roll(H, shifts=1, dims=0))
+            labels.copy_(torch.roll(labels, shifts=3))
+        g.replay()
+        cce.orpo_head_pass(H, head, labels, *args, direct)
+        torch.cuda.synchronize()
+        assert cce.cce_device_status(graphed.ws) == 0
+        assert cce.cce_device_status(direct.ws) == 0
+        for name in ("logp", "lse", "out8", "coeff", "dH"):
+            a = getattr(graphed, name).cpu().numpy()
+            b = getattr(direct, name).cpu().numpy()
+            assert np.array_equal(a, b), (step, name)
