@@ -19,9 +19,8 @@
 // N=256, K=16) into one of two 256-column fp32 accumulators; warps 2-5 drain
 // the accumulator with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)..+31,
 // i.e. one row per thread) and run the epilogue, overlapping the MMA of the
-// next tile.  A quantised head (QB = 4 or 8) adds 8 warps that dequantise B
-// and a warp that streams the packed weights (separate rings for A, packed
-// and fp16 B tiles; see below).  Tiles are assigned round-robin over a grid of
+// next tile.  A quantised head (QB = 4 or 8) adds 8 warps that dequantise
+// the B half of every stage (3 stages, each also holding the packed B tile).  Tiles are assigned round-robin over a grid of
 // at most one CTA per SM, in the order tile_coord gives (below), so the CTAs
 // in flight share the operand that should stay in L2.
 //
@@ -51,9 +50,8 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;     // TMA, MMA, 4 epilogue warps
 constexpr int DQ_WARPS = 8;          // dequantisation warps (4-bit head), 2 per SMSP
+constexpr int NUM_THREADS_Q4 = NUM_THREADS + 32 * DQ_WARPS;
 constexpr int DQ_WARP0 = 6;
-constexpr int PK_WARP = DQ_WARP0 + DQ_WARPS;  // packed-weight TMA producer
-constexpr int NUM_THREADS_Q4 = NUM_THREADS + 32 * DQ_WARPS + 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 enum class Mode : int { kLse = 0, kGrad = 1, kDh = 2, kDw = 3 };
 
@@ -69,36 +67,19 @@ __host__ __device__ constexpr int staging_buf_bytes() {
 constexpr int STAGES2 = 6;
 constexpr int B_HALF_BYTES = (BN / 2) * BK * 2;
 constexpr int STAGE2_BYTES = A_BYTES + B_HALF_BYTES;
-// Quantised heads (QB = 4 or 8) dequantise B in-kernel.  Their stages are
-// three separate rings: A tiles (TMA, from L2), packed B tiles (TMA, from HBM;
-// kLse/kGrad: 256 rows x one group of 64, kDh: 64 rows x 256 columns), both
-// fed well ahead since either round trip takes a few thousand cycles under
-// load, and 2 stages of fp16 B tiles written by the dequantisation warps.
-// The A and packed rings get the same depth: as deep as shared memory
-// allows, up to 8.
-constexpr int SMEM_LIMIT = 232448;  // bytes of dynamic shared memory per block
-constexpr int BAR_BYTES = 512;      // mbarriers, TMEM slot, abort flag
-constexpr int QB_NB = 2;
+// Quantised heads (QB = 4 or 8) dequantise B in-kernel.  Each of their 3
+// stages also holds the packed weights of its B tile, brought in by TMA
+// (kLse/kGrad: 256 rows x one group of 64; kDh: 64 rows x 256 columns).
+constexpr int STAGES_Q = 3;
 template <Mode MODE, int QB>
 __host__ __device__ constexpr int pk_bytes() {
   return MODE == Mode::kDh ? BK * (BN * QB / 8) : BN * (64 * QB / 8);
 }
-template <Mode MODE, int QB>
-__host__ __device__ constexpr int q_ring_depth() {
-  return QB == 0 ? 0
-                 : ((SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * B_BYTES - 4 * 2 * staging_buf_bytes<MODE>()) /
-                                (A_BYTES + pk_bytes<MODE, QB>()) > 8
-                        ? 8
-                        : (SMEM_LIMIT - 1024 - BAR_BYTES - QB_NB * B_BYTES -
-                           4 * 2 * staging_buf_bytes<MODE>()) /
-                              (A_BYTES + pk_bytes<MODE, QB>()));
-}
 template <Mode MODE, bool C2 = false, int QB = 0>
 __host__ __device__ constexpr int smem_bytes() {
   return (C2 ? STAGES2 * STAGE2_BYTES
-             : QB ? q_ring_depth<MODE, QB>() * (A_BYTES + pk_bytes<MODE, QB>()) + QB_NB * B_BYTES
-                  : STAGES * STAGE_BYTES) +
-         4 * 2 * staging_buf_bytes<MODE>() + 1024 + BAR_BYTES;
+             : QB ? STAGES_Q * (STAGE_BYTES + pk_bytes<MODE, QB>()) : STAGES * STAGE_BYTES) +
+         4 * 2 * staging_buf_bytes<MODE>() + 1024 + 256;
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
@@ -340,14 +321,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmC2, const TileArgs a) {
   static_assert(!(C2 && QB), "quantised heads run single-CTA tiles");
   static_assert(!(C2 && MODE == Mode::kDw), "the dW GEMM runs single-CTA tiles");
-  // Stages of the operand ring (quantised heads: A only; B has its own ring).
-  constexpr int NST = C2 ? STAGES2 : (QB ? q_ring_depth<MODE, QB>() : STAGES);
-  constexpr int SBYTES = C2 ? STAGE2_BYTES : (QB ? A_BYTES : STAGE_BYTES);
-  constexpr int NB = QB ? QB_NB : 0;                  // dequantised B ring
-  constexpr int PKB = QB ? pk_bytes<MODE, QB>() : 0;  // one packed B tile
-  constexpr int NPK = QB ? q_ring_depth<MODE, QB>() : 0;  // packed ring depth
-  static_assert(!QB || NST >= 3, "quantised heads need 3 A stages at least");
-  static_assert(smem_bytes<MODE, C2, QB>() <= SMEM_LIMIT, "shared memory");
+  constexpr int NST = C2 ? STAGES2 : (QB ? STAGES_Q : STAGES);
+  constexpr int PKB = QB ? pk_bytes<MODE, QB>() : 0;  // packed B tile per stage
+  constexpr int SBYTES = C2 ? STAGE2_BYTES : STAGE_BYTES + PKB;
   // With C2 the kernel runs as clusters of two CTAs (a pair on one TPC).
   // rank 0 (the leader) issues the MMAs for both; each CTA loads its own
   // 128 rows of A and its half of B and drains its own 128 TMEM lanes.
@@ -360,17 +336,12 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t* b_ring = base + NST * SBYTES;    // quantised heads: dequantised B
-  uint8_t* pk_ring = b_ring + NB * B_BYTES;  // quantised heads: packed tiles
-  uint8_t* staging = pk_ring + NPK * PKB;
+  uint8_t* staging = base + NST * SBYTES;
   uint64_t* full =
       reinterpret_cast<uint64_t*>(staging + 4 * 2 * staging_buf_bytes<MODE>());
   uint64_t* empty = full + NST;
-  uint64_t* b_full = empty + NST;       // B tile written by all dequant warps
-  uint64_t* b_empty = b_full + NB;      // B tile consumed by the MMAs
-  uint64_t* pk_full = b_empty + NB;     // packed tile landed (quantised heads)
-  uint64_t* pk_empty = pk_full + NPK;   // packed tile read by all dequant warps
-  uint64_t* acc_full = pk_empty + NPK;
+  uint64_t* pk_full = empty + NST;  // packed tile landed (quantised heads)
+  uint64_t* acc_full = pk_full + NST;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -383,16 +354,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], QB ? 1 + DQ_WARPS : 1);
       mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < NB; ++s) {
-      mbar_init(&b_full[s], DQ_WARPS);
-      mbar_init(&b_empty[s], 1);
-    }
-    for (int s = 0; s < NPK; ++s) {
       mbar_init(&pk_full[s], 1);
-      mbar_init(&pk_empty[s], DQ_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -463,7 +427,15 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
                                l2_policy_evict_normal());
             }
           } else if (QB) {
-            // B comes from the dequantisation warps.
+            // B comes from the dequantisation warps, which read the packed
+            // tile (tmB: the packed head as bytes [V, D*QB/8]) from the stage.
+            uint8_t* sP = sA + STAGE_BYTES;
+            mbar_arrive_expect_tx(&pk_full[stage], PKB);
+            if (MODE == Mode::kDh)
+              tma_load_2d(sP, &tmB, &pk_full[stage], tc.ct * (BN * QB / 8), a.b_row0 + k * BK);
+            else
+              tma_load_2d(sP, &tmB, &pk_full[stage], k * (64 * QB / 8),
+                          a.b_row0 + tc.ct * BN);
             mbar_arrive_expect_tx(&full[stage], A_BYTES);
             if (MODE == Mode::kDh)
               tma_load_2d(sA, &tmA, &full[stage], k * BK, tc.rt * BM);
@@ -510,17 +482,20 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       // cluster barrier keeps both CTAs alive until then).
       if (!C2 || rank == 0)
         for (int s = 0; s < NST; ++s)
-          if (issued_mask & (1u << s))
+          if (issued_mask & (1u << s)) {
+            if (QB)
+              wait_bounded(&pk_full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS, nullptr);
             wait_bounded(&full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS,
                          nullptr);
+          }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_f16(C2 ? 2 * BM : BM, BN, a.fmt, MODE == Mode::kDw,
                                        MODE == Mode::kDh || MODE == Mode::kDw);
-      int stage = 0, bst = 0;
-      uint32_t phase = 0, bph = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       int acc = 0;
       bool ok = true;
       for (int t = tile0; t < ntiles && ok; t += tstride) {
@@ -537,14 +512,13 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
         for (int kk = 0; kk < ksteps; ++kk) {
-          if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag) ||
-              (QB && !wait_bounded(&b_full[bst], bph, a.wait_ns, abort_flag))) {
+          if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sA = smem_u32(base + stage * SBYTES);
-          const uint32_t sB = QB ? smem_u32(b_ring + bst * B_BYTES) : sA + A_BYTES;
+          const uint32_t sB = sA + A_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             const uint64_t ad = MODE == Mode::kDw
@@ -562,13 +536,6 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
           // the stage is free in both CTAs once these MMAs have read it
           if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
           else umma_commit(&empty[stage]);
-          if (QB) {
-            umma_commit(&b_empty[bst]);
-            if (++bst == NB) {
-              bst = 0;
-              bph ^= 1u;
-            }
-          }
           if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
@@ -588,57 +555,15 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
       else umma_commit(drain);
       wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
     }
-  } else if (QB && warp == PK_WARP) {
-    // -------------------------------------------- packed-weight producer --
-    // Streams the packed B tile of every K step (tmB: the packed head as
-    // bytes [V, D*QB/8]) into the packed ring, as far ahead as the ring
-    // allows, independently of the operand stages.
-    if (lane == 0) {
-      int ps = 0;
-      uint32_t pph = 0, issued_mask = 0, issued_phase = 0;
-      bool ok = true;
-      for (int t = tile0; t < ntiles && ok; t += tstride) {
-        const TileCoord tc = tile_coord<MODE>(a, t);
-        if (tile_kind<MODE>(a, tc.rt, tc.ct, tc.s) != 0) continue;
-        const int kb = tc.s * a.nk / nsplit, nks = (tc.s + 1) * a.nk / nsplit - kb;
-        for (int kk = 0; kk < nks; ++kk) {
-          if (!wait_bounded(&pk_empty[ps], pph ^ 1u, a.wait_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int k = kb + kk;
-          mbar_arrive_expect_tx(&pk_full[ps], PKB);
-          if (MODE == Mode::kDh)
-            tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps], tc.ct * (BN * QB / 8),
-                        a.b_row0 + k * BK);
-          else
-            tma_load_2d(pk_ring + ps * PKB, &tmB, &pk_full[ps], k * (64 * QB / 8),
-                        a.b_row0 + tc.ct * BN);
-          issued_mask |= 1u << ps;
-          issued_phase = (issued_phase & ~(1u << ps)) | (pph << ps);
-          if (++ps == NPK) {
-            ps = 0;
-            pph ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        set_status(a.status, ST_TIMEOUT);
-        *abort_flag = 1;
-      }
-      for (int s2 = 0; s2 < NPK; ++s2)  // every issued copy lands before exit
-        if (issued_mask & (1u << s2))
-          wait_bounded(&pk_full[s2], (issued_phase >> s2) & 1u, DRAIN_LIMIT_NS, nullptr);
-    }
   } else if (QB && warp >= DQ_WARP0) {
     // ------------------------------------------ 4/8-bit dequantisation --
     // 256 threads fill the B half of every stage: 256 (row, group) units of
     // 64 weights per K step, one per thread.  The packed words come from the
-    // packed ring (released as soon as every warp has read them); scale and
-    // bias from global memory (kLse/kGrad: 8 groups of a row per 16-byte
-    // load when rows are 16-byte aligned).  Each unit is dequantised to fp16
-    // and written in the 128-byte-swizzled layout the TMA would produce
-    // (16-byte chunk c of row r at c ^ (r & 7)).
+    // stage (TMA, pk_full); scale and bias from global memory, fetched one
+    // unit ahead (kLse/kGrad: 8 groups of a row at once when rows are 16-byte
+    // aligned).  Each unit is dequantised to fp16 and written in the
+    // 128-byte-swizzled layout the TMA would produce (16-byte chunk c of row
+    // r at c ^ (r & 7)).
     constexpr int QU = 64 * (QB ? QB : 4) / 8;  // packed bytes per unit
     constexpr int NV = QU / 16;
     const int dq = threadIdx.x - DQ_WARP0 * 32;
@@ -646,12 +571,13 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
     const bool vec8 = MODE != Mode::kDh && (gpr % 8) == 0 &&
                       ((reinterpret_cast<uintptr_t>(a.q_scale) |
                         reinterpret_cast<uintptr_t>(a.q_bias)) & 15u) == 0;
-    int bst = 0, ps = 0;
-    uint32_t bph = 0, pph = 0;
+    int stage = 0;
+    uint32_t phase = 0;
     bool ok = true;
     // unit u of K step k of tile tc: source row, group, offset of its packed
-    // words in the packed tile, and of its fp16 output in B.  kDh: the 4
-    // groups of a row are adjacent threads (their scales share a sector).
+    // words in the stage's packed tile, and of its fp16 output in B.  kDh:
+    // the 4 groups of a row are adjacent threads (their scales share a
+    // sector).
     auto locate = [&](const TileCoord& tc, int k, int u, int& v, int& g, int& pk, int& off) {
       if (MODE == Mode::kDh) {
         const int r = u >> 2, j = u & 3;
@@ -698,16 +624,19 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         const bool valid = v < a.V && g < gpr;
         uint16_t sc = 0, bi = 0;
         if (valid) scale_bias(v, g, sc, bi);
-        if (!wait_bounded(&pk_full[ps], pph, a.wait_ns, abort_flag)) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag) ||
+            !wait_bounded(&pk_full[stage], phase, a.wait_ns, abort_flag)) {
           ok = false;
           break;
         }
+        uint8_t* sA = base + stage * SBYTES;
+        uint8_t* sB = sA + A_BYTES;
+        const uint8_t* sP = sA + STAGE_BYTES;
         uint4 out[8];
         if (valid) {
           uint4 w[NV];
 #pragma unroll
-          for (int i = 0; i < NV; ++i)
-            w[i] = *reinterpret_cast<const uint4*>(pk_ring + ps * PKB + pk + 16 * i);
+          for (int i = 0; i < NV; ++i) w[i] = *reinterpret_cast<const uint4*>(sP + pk + 16 * i);
           if constexpr (QB == 8)
             dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sc, bi, out);
           else
@@ -716,30 +645,15 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
         }
-        // The slot may be refilled (TMA, async proxy) once every warp is done
-        // with it: the values computed above hold the loaded words, and the
-        // proxy fence orders these generic reads before the refill.
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pk_empty[ps]);
-        if (++ps == NPK) {
-          ps = 0;
-          pph ^= 1u;
-        }
-        if (!wait_bounded(&b_empty[bst], bph ^ 1u, a.wait_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sB = b_ring + bst * B_BYTES;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(sB + off + ((c ^ (r_sw & 7)) << 4)) = out[c];
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&b_full[bst]);
-        if (++bst == NB) {
-          bst = 0;
-          bph ^= 1u;
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == NST) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
     }
