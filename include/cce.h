@@ -287,7 +287,7 @@ void cce_set_cta_pairs(int on);
 
 /* How the GEMMs read a 4- or 8-bit head (the dequantisation step of the
  * quantised-head design, Training design, MLX affine quantisation):
- *   0  choose (default): staged when M spans at least 8 row tiles of 128 and
+ *   0  choose (default): staged when M spans at least 2 row tiles of 128 and
  *      the workspace holds chunks of at least 8,192 head rows, else in-kernel;
  *   1  in-kernel: extra warps of the GEMM kernels dequantise each B tile into
  *      shared memory (reads 4.25 or 8.25 bits per weight; the small-M choice);

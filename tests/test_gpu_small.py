@@ -249,10 +249,19 @@ def test_objective_siblings_match_oracle(kind):
             assert np.allclose(coeff.cpu().numpy(), g, rtol=1e-6, atol=1e-12)
 
 
-@pytest.mark.parametrize("cfg,cap", [(1, 30.0), (2, 2.0), (4, 30.0), (0, 5.0)])
-def test_softcap_forward_and_backward(cfg, cap):
+@pytest.mark.parametrize("cfg,cap,qmode", [(1, 30.0, 0), (2, 2.0, 0), (4, 30.0, 1),
+                                           (4, 30.0, 2), (0, 5.0, 0)])
+def test_softcap_forward_and_backward(cfg, cap, qmode):
     """Gemma-style logit capping: capped logits in the forward, the
-    1 - tanh^2 factor in the backward."""
+    1 - tanh^2 factor in the backward (4-bit head: in-kernel and staged)."""
+    cce.cce_set_quant_staging(qmode)
+    try:
+        _softcap_case(cfg, cap)
+    finally:
+        cce.cce_set_quant_staging(0)
+
+
+def _softcap_case(cfg, cap):
     wl = S.make_custom(cfg, M_split=(60, 70, 80), D=128, V=1500)
     H, head, labels = upload(wl)
     head.softcap = cap
@@ -274,14 +283,23 @@ def test_softcap_forward_and_backward(cfg, cap):
     assert rel_fro(dH.cpu().numpy(), want) <= TOL_DH
 
 
+@pytest.mark.parametrize("qmode", [1, 2])
 @pytest.mark.parametrize("split,D,V,cap", [((40, 45, 44), 128, 257, 0.0),
                                            ((100, 150, 131), 256, 4097, 0.0),
                                            ((64, 200, 300), 320, 1000, 30.0)])
-def test_q8_head_forward_and_backward(split, D, V, cap):
-    """8-bit affine head (group 64), dequantised in-kernel."""
+def test_q8_head_forward_and_backward(split, D, V, cap, qmode):
+    """8-bit affine head (group 64), dequantised in-kernel (1) or staged (2)."""
     wl = S.make_custom(4, M_split=split, D=D, V=V, wformat="q8g64")
     H, head, labels = upload(wl)
     head.softcap = cap
+    cce.cce_set_quant_staging(qmode)
+    try:
+        _q8_pass_and_check(wl, H, head, labels, cap)
+    finally:
+        cce.cce_set_quant_staging(0)
+
+
+def _q8_pass_and_check(wl, H, head, labels, cap):
     ws = cce.alloc_workspace(wl.M, cce.h_dtype(H), head)
     f = dict(device="cuda", dtype=torch.float32)
     logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)

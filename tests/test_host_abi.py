@@ -176,7 +176,8 @@ def test_query_plan_chunks_splits_and_staging(lib):
 def test_query_plan_quant_staging(lib):
     q4 = cce._Head(cce.CCE_W_AFFINE_Q4_G64, cce.CCE_BF16, 128256, 4096, 4096, 4096, 4096)
     try:
-        for mode, M, want in [(0, 32768, 1), (0, 512, 0), (1, 32768, 0), (2, 512, 1)]:
+        for mode, M, want in [(0, 32768, 1), (0, 512, 1), (0, 128, 0), (1, 32768, 0),
+                              (2, 128, 1)]:
             cce.cce_set_quant_staging(mode)
             ws = lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(q4))
             p = cce.cce_query_plan(M, cce.CCE_BF16, q4, ws)
