@@ -287,8 +287,9 @@ void cce_set_cta_pairs(int on);
 
 /* How the GEMMs read a 4- or 8-bit head (the dequantisation step of the
  * quantised-head design, Training design, MLX affine quantisation):
- *   0  choose (default): staged when M spans at least 2 row tiles of 128 and
- *      the workspace holds chunks of at least 8,192 head rows, else in-kernel;
+ *   0  choose (default): staged when M spans at least 3 row tiles of 128 in
+ *      the forward, 2 in the backward, and the workspace holds chunks of at
+ *      least 8,192 head rows; else in-kernel;
  *   1  in-kernel: extra warps of the GEMM kernels dequantise each B tile into
  *      shared memory (reads 4.25 or 8.25 bits per weight; the small-M choice);
  *   2  staged: each vocabulary chunk is first dequantised once into an fp16

@@ -30,11 +30,13 @@ std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_pairs{1};  // 2-CTA (cta_group::2) tiles for dense heads
 // 4/8-bit heads: 0 = choose, 1 = dequantise inside the GEMM, 2 = staged chunks
 std::atomic<int> g_qstage{0};
-// Staged dequantisation pays off as soon as two row tiles reuse each weight
-// (measured on the 4-bit long-context head: a whole pass at M=192 takes
-// 1.22 ms staged against 1.49 ms in-kernel, at M=128 1.12 against 0.81), and
-// with chunks of at least this many rows.
-constexpr int64_t kStageMinRowTiles = 2;
+// Staged dequantisation pays off once enough row tiles reuse each weight;
+// measured on the 4-bit long-context head (D=4096, V=128,256): the backward
+// from 2 row tiles (M=192: 0.71 ms staged against 1.06 ms in-kernel), the
+// forward from 3 (M=256: 0.50 against 0.42; M=384: 0.61 against 0.64), with
+// chunks of at least this many rows.
+constexpr int64_t kStageMinRowTilesFwd = 3;
+constexpr int64_t kStageMinRowTilesBwd = 2;
 constexpr int64_t kStageMinRows = 8192;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -401,10 +403,11 @@ int64_t fit_vc(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes, int k
 
 // A 4/8-bit head is dequantised chunk by chunk into fp16 in the workspace
 // (then the dense GEMMs run on it) when enough row tiles reuse each weight.
-bool q_stage_wanted(int64_t M, const cce_head* W) {
+bool q_stage_wanted(int64_t M, const cce_head* W, bool forward) {
   if (W->format == CCE_W_DENSE) return false;
   const int mode = g_qstage.load();
-  return mode == 2 || (mode == 0 && ceil_div(M, BM) >= kStageMinRowTiles);
+  const int64_t min_tiles = forward ? kStageMinRowTilesFwd : kStageMinRowTilesBwd;
+  return mode == 2 || (mode == 0 && ceil_div(M, BM) >= min_tiles);
 }
 
 // Smallest staged chunk worth its launches (the whole head if it is smaller).
@@ -421,7 +424,7 @@ struct FwdPlan {
 };
 FwdPlan plan_forward(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes) {
   FwdPlan p;
-  p.staged = q_stage_wanted(M, W);
+  p.staged = q_stage_wanted(M, W, true);
   if (p.staged && (p.vq = fit_vc(M, h, W, ws_bytes, 1, true)) < stage_min_rows(W))
     p.staged = false;
   p.L = p.staged ? make_layout(M, h, W, p.vq, 1, true) : make_layout(M, h, W, BN);
@@ -442,7 +445,7 @@ struct BwdPlan {
 };
 BwdPlan plan_backward(int64_t M, cce_dtype h, const cce_head* W, size_t ws_bytes) {
   BwdPlan p;
-  p.staged = q_stage_wanted(M, W);
+  p.staged = q_stage_wanted(M, W, false);
   for (int attempt = 0; attempt < 2; ++attempt) {
     p.ksplit = ksplit_for(M, W, sm_count_guess(), p.staged);
     while ((p.vc = fit_vc(M, h, W, ws_bytes, p.ksplit, p.staged)) == 0 && p.ksplit > 1)
@@ -666,7 +669,7 @@ int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
 
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
-  const bool staged = q_stage_wanted(M, W);
+  const bool staged = q_stage_wanted(M, W, false);  // the backward stages first
   return make_layout(M, h_dtype, W, default_vc(M, W),
                      ksplit_for(M, W, sm_count_guess(), staged), staged)
       .total;

@@ -176,14 +176,14 @@ def test_query_plan_chunks_splits_and_staging(lib):
 def test_query_plan_quant_staging(lib):
     q4 = cce._Head(cce.CCE_W_AFFINE_Q4_G64, cce.CCE_BF16, 128256, 4096, 4096, 4096, 4096)
     try:
-        for mode, M, want in [(0, 32768, 1), (0, 512, 1), (0, 128, 0), (1, 32768, 0),
-                              (2, 128, 1)]:
+        for mode, M, fwd, bwd in [(0, 32768, 1, 1), (0, 512, 1, 1), (0, 256, 0, 1),
+                                  (0, 128, 0, 0), (1, 32768, 0, 0), (2, 128, 1, 1)]:
             cce.cce_set_quant_staging(mode)
             ws = lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(q4))
             p = cce.cce_query_plan(M, cce.CCE_BF16, q4, ws)
-            assert p["fwd_staged"] == want and p["bwd_staged"] == want, (mode, M, p)
+            assert p["fwd_staged"] == fwd and p["bwd_staged"] == bwd, (mode, M, p)
             # in-kernel dequantisation is single-CTA; so is M <= 128
-            assert p["bwd_cta_pairs"] == (want and M > 128)
+            assert p["bwd_cta_pairs"] == (bwd and M > 128)
             # the minimum workspace always runs (staging falls back to in-kernel)
             lo = lib.cce_workspace_min_bytes(M, cce.CCE_BF16, ctypes.byref(q4))
             pl = cce.cce_query_plan(M, cce.CCE_BF16, q4, lo)
