@@ -172,6 +172,32 @@ cce_status orpo_grad_coeffs(const float* logp, const int32_t* labels,
                             size_t ws_bytes, cce_stream_t stream);
 
 /*
+ * One pair split by rows over several processes (one per GPU).  The
+ * objective (Training design §1) reads the rows only through three segment
+ * means, i.e. through the sums and counts of logp over the labelled prompt,
+ * chosen and rejected rows, so the shards need one exchange of six numbers
+ * between the forward and the backward.  No counterpart on the pages.
+ *
+ * orpo_partial_sums: sums6 (device fp64 [6], 8-byte aligned) = (sum of logp
+ *   over the labelled prompt, chosen, rejected rows of this shard; the three
+ *   counts), for an all-reduce (sum) across the shards.
+ * orpo_from_sums: from the all-reduced sums6, the loss out8 (as in
+ *   orpo_loss_from_logps; nullable) and dL/dlogp coeff for this shard's rows
+ *   (nullable, not both null).  Identical across shards for out8.
+ * layout: this shard's rows in its own row numbering; a shard may hold no
+ *   chosen or rejected row (an empty pair-wide segment sets
+ *   CCE_ERR_EMPTY_SEGMENT in the status word, as the unsharded call).
+ * Otherwise as orpo_loss_from_logps / orpo_grad_coeffs.
+ */
+cce_status orpo_partial_sums(const float* logp, const int32_t* labels, int64_t M,
+                             const cce_layout* layout, double* sums6, void* ws,
+                             size_t ws_bytes, cce_stream_t stream);
+cce_status orpo_from_sums(const double* sums6, const int32_t* labels, int64_t M,
+                          const cce_layout* layout, double lambda, int sft_scope,
+                          double* out8, float* coeff, void* ws, size_t ws_bytes,
+                          cce_stream_t stream);
+
+/*
  * Objective siblings on the same log-prob engine (Training design §8.3
  * "Objective variants"; the UltraFeedback research notes §6.1-6.3):
  *   CCE_OBJ_ORPO        the ORPO loss above (lambda, sft_scope; beta, gamma

@@ -83,6 +83,13 @@ _SIGS = {
                                         ctypes.POINTER(_Layout), ctypes.c_double, ctypes.c_int,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]),
+    "orpo_partial_sums": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                         ctypes.POINTER(_Layout), ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_size_t, ctypes.c_void_p]),
+    "orpo_from_sums": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                      ctypes.POINTER(_Layout), ctypes.c_double, ctypes.c_int,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_size_t, ctypes.c_void_p]),
     "cce_backward_dh": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.POINTER(_Head),
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -266,6 +273,23 @@ def orpo_grad_coeffs(logp, labels, layout, lam, sft_scope, coeff, ws, stream=Non
     _check(st, "orpo_grad_coeffs")
 
 
+def orpo_partial_sums(logp, labels, layout, sums6, ws, stream=None):
+    """This shard's segment sums and counts (fp64 [6] on the device)."""
+    st = lib().orpo_partial_sums(_p(logp), _p(labels), logp.shape[0],
+                                 ctypes.byref(_layout(layout)), _p(sums6), _p(ws), ws.numel(),
+                                 _stream(stream))
+    _check(st, "orpo_partial_sums")
+
+
+def orpo_from_sums(sums6, labels, layout, lam, sft_scope, out8, coeff, ws, stream=None):
+    """Loss and this shard's dL/dlogp from the all-reduced segment sums."""
+    st = lib().orpo_from_sums(_p(sums6), _p(labels), labels.shape[0],
+                              ctypes.byref(_layout(layout)), float(lam),
+                              SCOPE.get(sft_scope, sft_scope), _p(out8), _p(coeff), _p(ws),
+                              ws.numel(), _stream(stream))
+    _check(st, "orpo_from_sums")
+
+
 def cce_backward_dh(H, head: Head, labels, lse, coeff, filter_eps, blockmax, dH,
                     skip_stats=None, ws=None, stream=None):
     st = lib().cce_backward_dh(_p(H), h_dtype(H), H.shape[0], ctypes.byref(head.c()),
@@ -327,6 +351,32 @@ def orpo_head_pass(H, head: Head, labels, layout, lam, sft_scope, filter_eps,
     orpo_grad_coeffs(buf.logp, labels, layout, lam, sft_scope, buf.coeff, buf.ws, stream)
     cce_backward_dh(H, head, labels, buf.lse, buf.coeff, filter_eps,
                     buf.blockmax if block_skip else None, buf.dH, buf.skip, buf.ws, stream)
+
+
+def orpo_head_pass_sharded(H, head: Head, labels, layout, lam, sft_scope, filter_eps,
+                           block_skip: bool, buf: HeadBuffers, group=None, stream=None):
+    """One pair split by rows over the processes of ``group`` (one per GPU):
+    this process holds some rows of each segment (``layout`` in its own row
+    numbering).  Forward, then one all-reduce of the six segment sums, then
+    the loss, this shard's cotangent and its dH rows.  The all-reduce runs on
+    the device for NCCL and through host memory for gloo."""
+    import torch.distributed as dist
+    s = torch.cuda.current_stream() if stream is None else stream
+    cce_forward(H, head, labels, buf.logp, buf.lse, buf.tgt, buf.blockmax, buf.ws, s)
+    sums = torch.zeros(6, dtype=torch.float64, device=H.device)
+    orpo_partial_sums(buf.logp, labels, layout, sums, buf.ws, s)
+    if dist.get_backend(group) == "nccl":
+        with torch.cuda.stream(s):
+            dist.all_reduce(sums, group=group)
+    else:
+        s.synchronize()
+        host = sums.cpu()
+        dist.all_reduce(host, group=group)
+        with torch.cuda.stream(s):
+            sums.copy_(host)
+    orpo_from_sums(sums, labels, layout, lam, sft_scope, buf.out8, buf.coeff, buf.ws, s)
+    cce_backward_dh(H, head, labels, buf.lse, buf.coeff, filter_eps,
+                    buf.blockmax if block_skip else None, buf.dH, buf.skip, buf.ws, s)
 
 
 class HeadPassGraph:

@@ -62,6 +62,12 @@ struct OrpoArgs {
   int want_coeff;
   int kind;                        // 0 ORPO, 1 SimPO, 2 ORPO + SimPO margin
   double beta, gamma;              // SimPO scale and target margin
+  // Row-sharded pairs: sums_out != null -> write the local segment sums
+  // (sum and count of logp per segment) and stop; sums_in != null -> take
+  // the segment sums from there (all-reduced over the shards) instead of
+  // summing the local rows.
+  const double* sums_in;
+  double* sums_out;
 };
 
 // log(1 - e^x), x < 0: two-branch form (Maechler 2012), fp64.
@@ -82,7 +88,7 @@ __global__ void __launch_bounds__(1024) orpo_kernel(
     float* __restrict__ coeff, uint32_t* status) {
   double s[3] = {0.0, 0.0, 0.0};
   double n[3] = {0.0, 0.0, 0.0};
-  for (int64_t m = threadIdx.x; m < M; m += blockDim.x) {
+  for (int64_t m = threadIdx.x; o.sums_in == nullptr && m < M; m += blockDim.x) {
     if (labels[m] < 0) continue;
     const double v = static_cast<double>(logp[m]);
     if (m >= o.pb && m < o.pe) { s[0] += v; n[0] += 1.0; }
@@ -106,8 +112,16 @@ __global__ void __launch_bounds__(1024) orpo_kernel(
   if (threadIdx.x == 0) {
     double t[6] = {0, 0, 0, 0, 0, 0};
     const int nw = (blockDim.x + 31) >> 5;
-    for (int w = 0; w < nw; ++w)
-      for (int i = 0; i < 6; ++i) t[i] += red[w][i];
+    if (o.sums_in != nullptr) {
+      for (int i = 0; i < 6; ++i) t[i] = o.sums_in[i];
+    } else {
+      for (int w = 0; w < nw; ++w)
+        for (int i = 0; i < 6; ++i) t[i] += red[w][i];
+    }
+    if (o.sums_out != nullptr) {
+      for (int i = 0; i < 6; ++i) o.sums_out[i] = t[i];
+      return;
+    }
     const double sP = t[0], sC = t[1], sR = t[2];
     const double nP = t[3], nC = t[4], nR = t[5];
     double res[8];
@@ -176,7 +190,7 @@ __global__ void __launch_bounds__(1024) orpo_kernel(
     sc[1] = cC;
     sc[2] = cR;
   }
-  if (!o.want_coeff) return;
+  if (!o.want_coeff || o.sums_out != nullptr) return;
   __syncthreads();
   const float cP = static_cast<float>(sc[0]);
   const float cC = static_cast<float>(sc[1]);

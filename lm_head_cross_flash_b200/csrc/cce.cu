@@ -239,6 +239,7 @@ int device_pairs() {
 
 // ------------------------------------------------------------ validation --
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
 cce_status check_head(const cce_head* W, cce_dtype h_dtype) {
   if (W == nullptr) return CCE_ERR_INVALID_ARGUMENT;
@@ -786,7 +787,9 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   return launch_ok();
 }
 
-static cce_status check_layout(const cce_layout* L, int64_t M) {
+// allow_empty: a shard of a row-sharded pair may hold no chosen or rejected
+// row; emptiness of the whole pair shows in the all-reduced counts instead.
+static cce_status check_layout(const cce_layout* L, int64_t M, bool allow_empty = false) {
   if (L == nullptr) return CCE_ERR_INVALID_ARGUMENT;
   const int64_t r[3][2] = {{L->prompt_begin, L->prompt_end},
                            {L->chosen_begin, L->chosen_end},
@@ -796,7 +799,8 @@ static cce_status check_layout(const cce_layout* L, int64_t M) {
     for (int j = 0; j < i; ++j)
       if (r[i][0] < r[j][1] && r[j][0] < r[i][1]) return CCE_ERR_INVALID_ARGUMENT;
   }
-  if (r[1][1] == r[1][0] || r[2][1] == r[2][0]) return CCE_ERR_INVALID_ARGUMENT;
+  if (!allow_empty && (r[1][1] == r[1][0] || r[2][1] == r[2][0]))
+    return CCE_ERR_INVALID_ARGUMENT;
   return CCE_OK;
 }
 
@@ -804,17 +808,24 @@ static cce_status orpo_common(const float* logp, const int32_t* labels, int64_t 
                               const cce_layout* layout, double lambda, int scope,
                               double* out8, float* coeff, void* ws, size_t ws_bytes,
                               cce_stream_t stream, int kind = 0, double beta = 1.0,
-                              double gamma = 0.0) {
-  if (logp == nullptr || labels == nullptr || ws == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+                              double gamma = 0.0, const double* sums_in = nullptr,
+                              double* sums_out = nullptr) {
+  if (labels == nullptr || ws == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  if (logp == nullptr && sums_in == nullptr) return CCE_ERR_INVALID_ARGUMENT;
   if (M <= 0 || M > (int64_t(1) << 31)) return CCE_ERR_INVALID_ARGUMENT;
   if (!(lambda >= 0.0) || lambda > 1e30) return CCE_ERR_INVALID_ARGUMENT;
   if (kind < 0 || kind > 2 || !(beta >= 0.0) || beta > 1e30 || !(std::fabs(gamma) <= 1e30))
     return CCE_ERR_INVALID_ARGUMENT;
   if (scope != CCE_SCOPE_FULL && scope != CCE_SCOPE_RESPONSE) return CCE_ERR_INVALID_ARGUMENT;
   if (ws_bytes < kStatusBytes || !aligned16(ws)) return CCE_ERR_WORKSPACE_TOO_SMALL;
-  cce_status s = check_layout(layout, M);
+  const bool sharded = sums_in != nullptr || sums_out != nullptr;
+  if ((sums_in != nullptr && !aligned8(sums_in)) || (sums_out != nullptr && !aligned8(sums_out)))
+    return CCE_ERR_INVALID_ARGUMENT;
+  cce_status s = check_layout(layout, M, sharded);
   if (s != CCE_OK) return s;
-  OrpoArgs o;
+  OrpoArgs o{};
+  o.sums_in = sums_in;
+  o.sums_out = sums_out;
   o.pb = layout->prompt_begin;
   o.pe = layout->prompt_end;
   o.cb = layout->chosen_begin;
@@ -850,6 +861,23 @@ cce_status orpo_grad_coeffs(const float* logp, const int32_t* labels, int64_t M,
   if (coeff == nullptr) return CCE_ERR_INVALID_ARGUMENT;
   return orpo_common(logp, labels, M, layout, lambda, sft_scope, nullptr, coeff, ws,
                      ws_bytes, stream);
+}
+
+cce_status orpo_partial_sums(const float* logp, const int32_t* labels, int64_t M,
+                             const cce_layout* layout, double* sums6, void* ws,
+                             size_t ws_bytes, cce_stream_t stream) {
+  if (sums6 == nullptr || logp == nullptr) return CCE_ERR_INVALID_ARGUMENT;
+  return orpo_common(logp, labels, M, layout, 0.0, CCE_SCOPE_FULL, nullptr, nullptr, ws,
+                     ws_bytes, stream, 0, 1.0, 0.0, nullptr, sums6);
+}
+
+cce_status orpo_from_sums(const double* sums6, const int32_t* labels, int64_t M,
+                          const cce_layout* layout, double lambda, int sft_scope,
+                          double* out8, float* coeff, void* ws, size_t ws_bytes,
+                          cce_stream_t stream) {
+  if (sums6 == nullptr || (out8 == nullptr && coeff == nullptr)) return CCE_ERR_INVALID_ARGUMENT;
+  return orpo_common(nullptr, labels, M, layout, lambda, sft_scope, out8, coeff, ws, ws_bytes,
+                     stream, 0, 1.0, 0.0, sums6, nullptr);
 }
 
 static cce_status objective_args(const cce_objective* obj) {
