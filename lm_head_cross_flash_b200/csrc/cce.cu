@@ -23,7 +23,10 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
-constexpr int64_t kDefaultChunkBytes = 256ll << 20;  // G' chunk, default
+// Default G'' chunk: 1 GiB.  Fewer, longer recompute/dH launches; at the long
+// pair (M=8192, V=262,144) 4 chunks instead of 16 make the step 2.7 % faster
+// for 0.73 GB more workspace (measured: 21.53 -> 20.95 ms).
+constexpr int64_t kDefaultChunkBytes = 1ll << 30;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
@@ -378,8 +381,9 @@ int group_rows(int64_t n_rt, int64_t k_elems) {
   return int(std::max<int64_t>(1, std::min<int64_t>(n_rt, (int64_t(48) << 20) / per)));
 }
 
-// Default G'' chunk: 256 MB, or four times dH when that is larger (every
-// chunk adds into dH once, so wider chunks save dH traffic when M*D is big).
+// Default G'' chunk: kDefaultChunkBytes, or four times dH when that is larger
+// (every chunk adds into dH once, so wider chunks save dH traffic when M*D is
+// big).
 int64_t default_vc(int64_t M, const cce_head* W) {
   const int64_t vmax = ceil_div(W->V, BN) * BN;
   const int64_t budget = std::max<int64_t>(kDefaultChunkBytes, 4 * M * W->D * 4);
