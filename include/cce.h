@@ -78,18 +78,21 @@ typedef enum {
   CCE_W_AFFINE_Q8_G64 = 2  /* w: uint32 [V, D/4]; element 4k+j of a row is byte
                               j of word k (low byte first); scales, biases as
                               for the 4-bit head.  Quantised heads compute in
-                              fp16 (H converted once; weights dequantised
-                              in-kernel and rounded once to fp16).           */
+                              fp16: H is converted once, and each weight is
+                              dequantised by this library's kernels (inside
+                              the GEMM, or into a staged fp16 chunk of the
+                              workspace; see cce_set_quant_staging) and
+                              rounded once to fp16.                          */
 } cce_wformat;
 
 /* The frozen head (host struct; device pointers inside). */
 typedef struct {
   cce_wformat format;
-  cce_dtype dtype;       /* dense: dtype of w; Q4: must be CCE_BF16 (scales) */
+  cce_dtype dtype;       /* dense: dtype of w; 4/8-bit: CCE_BF16 (scales) */
   int64_t V, D;
   const void* w;
-  const void* scales;    /* Q4 only, else NULL */
-  const void* biases;    /* Q4 only, else NULL */
+  const void* scales;    /* 4/8-bit heads only, else NULL (2-byte aligned) */
+  const void* biases;    /* 4/8-bit heads only, else NULL (2-byte aligned) */
   float softcap;         /* > 0: logits are softcap * tanh(h.W_v / softcap)
                             (Gemma-style final-logit capping; the backward
                             applies 1 - tanh^2); 0 = none */
@@ -243,6 +246,8 @@ cce_status pref_grad_coeffs(const float* logp, const int32_t* labels,
  * dH: fp32 [M, D] output, overwritten.
  * skip_stats: optional device uint64 [2] incremented by (skipped tiles,
  *   total tiles).
+ * ws: as for cce_forward; the backward takes vocab chunks as wide as it
+ *   allows (G'' of one chunk lives there), see cce_query_plan.
  */
 cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M,
                            const cce_head* W, const int32_t* labels,
