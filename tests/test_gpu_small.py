@@ -550,3 +550,48 @@ def test_head_pass_graph_replay(cfg, split, D, V):
             a = getattr(graphed, name).cpu().numpy()
             b = getattr(direct, name).cpu().numpy()
             assert np.array_equal(a, b), (step, name)
+
+
+def test_domain_and_empty_segments_are_reported():
+    """Device-side errors of the epilogue, reported through the status word:
+    a mean log-prob >= 0 (outside the domain of log1mexp), an all-ignored
+    batch, and empty segments reaching the sharded epilogue through zero
+    counts.  Outputs are NaN losses and zero cotangents; nothing traps."""
+    wl = S.make_custom(1, M_split=(4, 6, 6), D=64, V=300)
+    H, head, labels = upload(wl)
+    ws = cce.alloc_workspace(wl.M, cce.h_dtype(H), head)
+    f = dict(device="cuda", dtype=torch.float32)
+    out8 = torch.empty(8, dtype=torch.float64, device="cuda")
+    coeff = torch.empty(wl.M, **f)
+    # chosen rows with logp = 0: lw = 0, log1mexp undefined
+    logp = torch.full((wl.M,), -3.0, **f)
+    logp[4:10] = 0.0
+    y = labels.clamp(min=0)
+    cce.orpo_loss_from_logps(logp, y, wl.layout_tuple, 0.1, "full", out8, ws)
+    assert cce.cce_device_status(ws) == 8
+    assert torch.isnan(out8).all()
+    cce.orpo_grad_coeffs(logp, y, wl.layout_tuple, 0.1, "full", coeff, ws)
+    assert cce.cce_device_status(ws) == 8
+    assert torch.count_nonzero(coeff).item() == 0
+    # every label ignored: the forward is fine (logp = 0), the loss is not
+    lp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
+    none = torch.full_like(labels, -1)
+    cce.cce_forward(H, head, none, lp, lse, None, None, ws)
+    assert cce.cce_device_status(ws) == 0
+    assert torch.count_nonzero(lp).item() == 0 and torch.isfinite(lse).all()
+    cce.orpo_loss_from_logps(lp, none, wl.layout_tuple, 0.1, "full", out8, ws)
+    assert cce.cce_device_status(ws) == 7
+    # sharded epilogue: all-reduced counts of zero for the chosen segment
+    sums = torch.tensor([-3.0, 0.0, -12.0, 1.0, 0.0, 4.0], dtype=torch.float64,
+                        device="cuda")
+    cce.orpo_from_sums(sums, y, wl.layout_tuple, 0.1, "full", out8, coeff, ws)
+    assert cce.cce_device_status(ws) == 7
+    assert torch.isnan(out8).all()
+    # and the partial sums of a valid shard equal the host sums
+    logp = torch.linspace(-9.0, -1.0, wl.M, **f)
+    cce.orpo_partial_sums(logp, y, wl.layout_tuple, sums, ws)
+    torch.cuda.synchronize()
+    assert cce.cce_device_status(ws) == 0
+    lpn = logp.cpu().double().numpy()
+    want = [lpn[0:4].sum(), lpn[4:10].sum(), lpn[10:16].sum(), 4, 6, 6]
+    assert np.allclose(sums.cpu().numpy(), want, rtol=1e-12, atol=1e-12)
