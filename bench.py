@@ -283,14 +283,19 @@ def run_ours(args):
     cce.cce_profile_enable(not args.graph)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    # one event per step boundary as well, for the median and minimum step
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     e0.record(stream)
-    for _ in range(args.steps):
+    marks[0].record(stream)
+    for i in range(args.steps):
         run_step()
+        marks[i + 1].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     ms_total = e0.elapsed_time(e1)
+    step_ms = sorted(marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps))
     if args.graph:  # kernel times of the same work, from direct passes
         cce.cce_profile_enable(True)
         for _ in range(args.steps):
@@ -387,7 +392,9 @@ def run_ours(args):
         rps, cores, rows, dt = time_oracle(wl, args.cpu_seconds)
         cpu = {"value": rps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{rows} rows of the {wl.name} workload (forward logp/lse and dH per "
-                         f"row, float64, logits materialised per row block) in {dt:.1f} s"}
+                         f"row, float64, logits materialised per row block) in {dt:.1f} s",
+               "extrapolated_full_pass_s": wl.M / rps,
+               "extrapolated_note": "extrapolated: M rows at the sampled rate"}
 
     if world > 1:
         dist.destroy_process_group()
@@ -431,6 +438,8 @@ def run_ours(args):
         "steps": args.steps,
         "warmup": max(3, args.warmup),
         "ms_per_step": ms_step,
+        "step_ms": {"median": statistics.median(step_ms), "min": step_ms[0],
+                    "max": step_ms[-1], "note": "this rank, per-step CUDA events"},
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
