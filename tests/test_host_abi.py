@@ -209,3 +209,45 @@ def test_oversized_tile_counts_are_rejected(lib):
     # the same head at a modest M is accepted by the planner
     assert lib.cce_query_plan(8192, cce.CCE_BF16, ctypes.byref(big), 1 << 40,
                               ctypes.byref(out)) == 0
+
+
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=200, deadline=None)
+@given(M=st.integers(1, 70000), V=st.integers(1, 300000), D64=st.integers(1, 96),
+       fmt=st.sampled_from([cce.CCE_W_DENSE, cce.CCE_W_AFFINE_Q4_G64, cce.CCE_W_AFFINE_Q8_G64]),
+       frac=st.floats(0.0, 2.0))
+def test_planner_invariants(lib, M, V, D64, fmt, frac):
+    """For any shape and any workspace between the minimum and twice the
+    default, the planner's choices are consistent: both calls fit, chunks are
+    whole vocab tiles, K splits stay in range, staging and CTA pairs follow
+    their documented thresholds."""
+    D = 64 * D64
+    h = cce._Head(fmt, cce.CCE_BF16, V, D, 4096, 4096 if fmt else None, 4096 if fmt else None)
+    lo = lib.cce_workspace_min_bytes(M, cce.CCE_BF16, ctypes.byref(h))
+    hi = lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h))
+    assert 0 < lo <= hi
+    ws = int(lo + frac * (2 * hi - lo) / 2)
+    p = cce.cce_query_plan(M, cce.CCE_BF16, h, ws)
+    vmax = -(-V // 256) * 256
+    n_rt = -(-M // 128)
+    assert p["fwd_ok"] and p["bwd_ok"]
+    assert p["bwd_chunk"] % 256 == 0 and 256 <= p["bwd_chunk"] <= vmax
+    assert p["fwd_chunk"] % 256 == 0 and 256 <= p["fwd_chunk"] <= vmax
+    assert 1 <= p["bwd_ksplit"] <= 32
+    if fmt == cce.CCE_W_DENSE:
+        assert not p["fwd_staged"] and not p["bwd_staged"]
+        assert p["fwd_chunk"] == vmax  # one forward launch over the vocabulary
+    else:
+        assert not p["fwd_staged"] or n_rt >= 3
+        assert not p["bwd_staged"] or n_rt >= 2
+        if not p["fwd_staged"]:
+            assert p["fwd_chunk"] == vmax
+    if p["fwd_cta_pairs"] or p["bwd_cta_pairs"]:
+        assert M > 128
+    if fmt != cce.CCE_W_DENSE and not p["bwd_staged"]:
+        assert not p["bwd_cta_pairs"]  # in-kernel dequantisation is single-CTA
+    # the default workspace never needs a narrower chunk than the minimum one
+    pd = cce.cce_query_plan(M, cce.CCE_BF16, h, hi)
+    assert pd["bwd_chunk"] >= cce.cce_query_plan(M, cce.CCE_BF16, h, lo)["bwd_chunk"]
