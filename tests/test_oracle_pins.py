@@ -512,3 +512,72 @@ def test_head_dw_finite_differences(cap):
             fd = (O.orpo_head_loss(H, Wp, y, L, 0.4, "full", softcap=cap)
                   - O.orpo_head_loss(H, Wm, y, L, 0.4, "full", softcap=cap)) / (2 * h)
             assert dW[v, d] == pytest.approx(fd, rel=1e-6, abs=1e-9)
+
+
+# --------------------------------------------------------------------------
+# randomised: the whole oracle path against torch float64 autograd
+# --------------------------------------------------------------------------
+
+from hypothesis import given, settings, strategies as hst
+
+
+def _autograd_reference(torch, H, W, y, L, lam, scope, cap):
+    """Loss and dL/dH by autograd over materialised float64 logits (the
+    objective of Training design §1 written with torch primitives)."""
+    Ht = torch.tensor(H, dtype=torch.float64, requires_grad=True)
+    Wt = torch.tensor(W, dtype=torch.float64)
+    S = Ht @ Wt.T
+    if cap > 0:
+        S = cap * torch.tanh(S / cap)
+    yt = torch.tensor(np.maximum(y, 0), dtype=torch.long)
+    ok = torch.tensor(y >= 0)
+    lp = torch.where(ok, torch.log_softmax(S, dim=1).gather(1, yt[:, None])[:, 0],
+                     torch.zeros((), dtype=torch.float64))
+
+    def seg(b, e):
+        return lp[b:e][ok[b:e]].sum(), int(ok[b:e].sum())
+
+    sP, nP = seg(L.prompt_begin, L.prompt_end)
+    sC, nC = seg(L.chosen_begin, L.chosen_end)
+    sR, nR = seg(L.rejected_begin, L.rejected_end)
+    lw, lr = sC / nC, sR / nR
+    nll = -(sP + sC) / (nP + nC) if scope == "full" else -lw
+    z = (lw - lr) - (torch.log(-torch.expm1(lw)) - torch.log(-torch.expm1(lr)))
+    loss = nll - lam * torch.nn.functional.logsigmoid(z)
+    loss.backward()
+    return loss.item(), Ht.grad.numpy()
+
+
+@settings(max_examples=60, deadline=None)
+@given(P=hst.integers(1, 6), Rc=hst.integers(1, 6), Rr=hst.integers(1, 6),
+       D=hst.integers(1, 12), V=hst.integers(2, 40), lam=hst.floats(0.0, 2.0),
+       scope=hst.sampled_from(["full", "response"]), cap=hst.sampled_from([0.0, 3.0]),
+       order=hst.permutations([0, 1, 2]), seed=hst.integers(0, 2**31 - 1),
+       n_ignore=hst.integers(0, 3))
+def test_randomised_against_torch_autograd(P, Rc, Rr, D, V, lam, scope, cap, order, seed,
+                                           n_ignore):
+    """Random sizes, segment order, ignored rows, lambda, scope and softcap:
+    the oracle's loss and dH equal torch autograd through materialised
+    logits."""
+    torch = pytest.importorskip("torch")
+    g = np.random.default_rng(seed)
+    sizes = [P, Rc, Rr]
+    starts, b = [0, 0, 0], 0
+    for k in order:                     # segments laid out in a random order
+        starts[k] = b
+        b += sizes[k]
+    M = b
+    L = O.Layout(starts[0], starts[0] + P, starts[1], starts[1] + Rc, starts[2], starts[2] + Rr)
+    H = g.standard_normal((M, D))
+    W = g.standard_normal((V, D)) / math.sqrt(D)
+    y = g.integers(0, V, size=M).astype(np.int32)
+    keep = {L.chosen_begin, L.rejected_begin}   # one labelled row in each response
+    for r in g.choice(M, size=min(n_ignore, M), replace=False):
+        if int(r) not in keep:
+            y[r] = -1
+    want_loss, want_dH = _autograd_reference(torch, H, W, y, L, lam, scope, cap)
+    logp = O.head_forward(H, W, y, softcap=cap)[0]
+    o = O.orpo_loss_from_logps(logp, y, L, lam, scope)
+    assert o.loss == pytest.approx(want_loss, rel=1e-11, abs=1e-12)
+    dH = O.orpo_head_grad(H, W, y, L, lam, scope, softcap=cap)
+    assert np.allclose(dH, want_dH, rtol=1e-8, atol=1e-12)
