@@ -1321,11 +1321,13 @@ extern "C" cce_status cce_forward_noalloc(const void* H, int64_t M, const cce_he
   const int64_t V = W->V, D = W->D;
   const int64_t cols = ceil_div(V, BN);
   const int64_t n_rt = ceil_div(M, BM);
-  // scratch: status word | part_s [cols, M] | part_m [cols, M] | tgt [M]
+  // scratch: status word | part_s [cols, M] | part_m [cols, M] | tgt [M];
+  // part_m and tgt take room only when the caller did not pass blockmax or
+  // tgt_logit (those outputs are then written directly).
   const size_t o_s = kStatusBytes;
   const size_t o_m = o_s + align_up(size_t(cols) * M * 4);
-  const size_t o_t = o_m + align_up(size_t(cols) * M * 4);
-  const size_t need = o_t + align_up(size_t(M) * 4);
+  const size_t o_t = o_m + (blockmax != nullptr ? 0 : align_up(size_t(cols) * M * 4));
+  const size_t need = o_t + (tgt_logit != nullptr ? 0 : align_up(size_t(M) * 4));
   if (need > kNoallocBytes) return CCE_ERR_WORKSPACE_TOO_SMALL;
   int sms = 0;
   if ((s = device_info(&sms)) != CCE_OK) return s;

@@ -40,6 +40,7 @@ import numpy as np
 
 LAMBDA = 0.1
 VOCAB_TILE = 256  # tail rows of the vocab are sampled at this granularity
+ROW_TILE = 128    # per-tile sampling: one row in every block of this many rows
 
 CONFIGS = {
     0: dict(name="tiny_pair_fp32_M256_D256_V4096", P=32, Rc=96, Rr=128, D=256,
@@ -282,22 +283,27 @@ def _make(cfg_id, c, seed, threads) -> Workload:
 # sampling and synthetic cotangents
 # ----------------------------------------------------------------------------
 
-def sample_rows(wl: Workload, n_uniform: int = 48, seed: int = 7) -> np.ndarray:
+def sample_rows(wl: Workload, n_uniform: int = 48, seed: int = 7, per_tile: bool = False,
+                edge: int = 4) -> np.ndarray:
     """Stratified rows for sampled parity at full size.
 
-    Row 0; the first and last 4 rows of each segment; up to 8 rows whose
-    label falls in the last (possibly partial) vocab tile; ``n_uniform``
+    Row 0; the first and last ``edge`` rows of each segment; up to 8 rows
+    whose label falls in the last (possibly partial) vocab tile; with
+    ``per_tile`` one seeded row inside every 128-row tile; ``n_uniform``
     uniform rows.  Sorted and unique.
     """
     M = wl.M
     rows = {0}
     for b, e in ((0, wl.P), (wl.P, wl.P + wl.Rc), (wl.P + wl.Rc, M)):
-        rows.update(range(b, min(e, b + 4)))
-        rows.update(range(max(b, e - 4), e))
+        rows.update(range(b, min(e, b + edge)))
+        rows.update(range(max(b, e - edge), e))
     tail0 = ((wl.V - 1) // VOCAB_TILE) * VOCAB_TILE
     tail_rows = np.nonzero(wl.labels >= tail0)[0][:8]
     rows.update(int(r) for r in tail_rows)
     g = np.random.Generator(np.random.PCG64(seed))
+    if per_tile:
+        for t0 in range(0, M, ROW_TILE):
+            rows.add(int(t0 + g.integers(0, min(ROW_TILE, M - t0))))
     rows.update(int(r) for r in g.integers(0, M, size=n_uniform))
     return np.array(sorted(rows), dtype=np.int64)
 

@@ -40,7 +40,7 @@ at a time in float64:
   (Training design §5.6; ORPO design (0.0.6), "Mixed-precision quantized
   base").
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * Head-row layout: rows ``[prompt_begin, prompt_end)`` are prompt positions,
   ``[chosen_begin, chosen_end)`` the chosen response, ``[rejected_begin,

@@ -310,6 +310,59 @@ def test_filter_limits():
     assert errs[0] <= errs[1] <= errs[2]
 
 
+def _filter_boundary_case():
+    """One head row whose logits are (0, 0, -10, -10) through the first
+    coordinate of W, with lse taken as 0, so the softmax values the filter
+    sees are exactly (1, 1, e^-10, e^-10).  The second coordinate of W tags
+    each vocabulary column, so dH shows which terms were kept."""
+    W = np.array([[0.0, 1.0], [0.0, 2.0], [-10.0, 4.0], [-10.0, 8.0]])
+    H = np.array([[1.0, 0.0]])
+    y = np.array([2], dtype=np.int32)
+    return H, W, y, np.array([0.0])
+
+
+@pytest.mark.parametrize("eps", [1.0, 0.6])
+def test_filter_boundary_by_hand(eps):
+    """A term is dropped iff its softmax p < eps strictly, on p itself (not
+    on g*p), and the target column is always kept.  eps = 1: the columns
+    with p == eps stay.  eps = 0.6 with g = 0.5: |g*p| = 0.5 < eps <= p = 1,
+    so those columns stay too.  Column 3 (p = e^-10 < eps, not the target)
+    is dropped; column 2 is the target (p = e^-10, kept)."""
+    H, W, y, lse = _filter_boundary_case()
+    g = np.array([0.5])
+    e10 = math.exp(-10.0)
+    # kept terms: g * (onehot - p) = 0.5 * (-1, -1, 1 - e^-10, 0)
+    G = 0.5 * np.array([-1.0, -1.0, 1.0 - e10, 0.0])
+    want_dh = (G @ W)[None, :]
+    assert want_dh[0, 1] == pytest.approx(0.5 * (-3.0 + 4.0 * (1.0 - e10)), rel=1e-15)
+    got = O.head_dh(H, W, y, g, lse, filter_eps=eps)
+    assert np.allclose(got, want_dh, rtol=1e-15, atol=0.0)
+    # dW[v] = G_v * H: zero for the dropped column exactly
+    want_dw = G[:, None] * H[0][None, :]
+    got_w = O.head_dw(H, W, y, g, lse, filter_eps=eps)
+    assert np.allclose(got_w, want_dw, rtol=1e-15, atol=0.0)
+    assert np.all(got_w[3] == 0.0)
+    # without the filter every column contributes
+    G0 = 0.5 * np.array([-1.0, -1.0, 1.0 - e10, -e10])
+    assert np.allclose(O.head_dh(H, W, y, g, lse), (G0 @ W)[None, :], rtol=1e-15, atol=0.0)
+    assert np.allclose(O.head_dw(H, W, y, g, lse), G0[:, None] * H[0][None, :], rtol=1e-15,
+                       atol=0.0)
+
+
+def test_filter_just_above_p_drops_it():
+    """eps one ulp above p = 1 drops the two non-target columns with p = 1 as
+    well: only the target term g * (1 - e^-10) * W_y is left."""
+    H, W, y, lse = _filter_boundary_case()
+    g = np.array([0.5])
+    e10 = math.exp(-10.0)
+    eps = float(np.nextafter(1.0, 2.0))
+    want = 0.5 * (1.0 - e10) * W[2]
+    assert np.allclose(O.head_dh(H, W, y, g, lse, filter_eps=eps)[0], want, rtol=1e-15, atol=0)
+    got_w = O.head_dw(H, W, y, g, lse, filter_eps=eps)
+    assert np.all(got_w[[0, 1, 3]] == 0.0)
+    assert got_w[2] == pytest.approx(0.5 * (1.0 - e10) * H[0], rel=1e-15)
+
+
 # --------------------------------------------------------------------------
 # 4-bit affine head format
 # --------------------------------------------------------------------------
