@@ -119,7 +119,7 @@ def choose_peak(peaks: dict, src: str, clk: dict, timed_s: float) -> dict:
 # The sources that decide the tensor-core kernels' memory traffic: the kernel
 # template and its PTX wrappers, and the host code that picks tiles, chunks
 # and launch shapes.
-TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "cce.cu")
+TRAFFIC_SOURCES = ("gemm_tc.cuh", "fused_bwd.cuh", "ptx.cuh", "cce.cu")
 
 
 def source_hash() -> str:
@@ -452,7 +452,9 @@ def run_ours(args):
     # roofline of the dominant kernel kind (largest summed time)
     per_kind_flops = {"fwd_lse_gemm": 2.0 * wl.M * wl.V * wl.D,  # per step
                       "bwd_grad_gemm": 2.0 * wl.M * wl.V * wl.D,
-                      "bwd_dh_gemm": 2.0 * wl.M * wl.V * wl.D}
+                      "bwd_dh_gemm": 2.0 * wl.M * wl.V * wl.D,
+                      # recompute of the logits and the dH contraction, one kernel
+                      "bwd_fused": 4.0 * wl.M * wl.V * wl.D}
     kinds = {k: v for k, v in prof.items() if v[1] > 0}
     dom = max(kinds, key=lambda k: kinds[k][0])
     dom_ms, dom_n = kinds[dom]
@@ -535,9 +537,10 @@ def run_small_m(args, quant=False):
     V = 128,256, groups of 64), dequantised inside the GEMMs.  Achieved GB/s
     counts the method's minimum bytes: W once per pass (as stored: 16 or 4.25
     bits per weight), H in, dH out and the per-row / per-block statistics.
-    This implementation's backward reads W twice (the G'' recompute and the
-    dH contraction are separate GEMMs) and moves G'' through HBM; those bytes
-    are reported as design_bytes."""
+    design_bytes are the bytes the backward that ran must move: the fused
+    backward (dense bf16 heads) reads W from HBM once and adds its partial dH
+    buffers; the two-GEMM backward (4/8-bit heads) reads W twice and moves
+    G'' through HBM."""
     import torch
 
     from lm_head_cross_flash_b200 import cce
@@ -593,7 +596,12 @@ def run_small_m(args, quant=False):
         stats = 4.0 * M * cols + 4.0 * 4 * M
         fwd_bytes = wbytes + 2.0 * M * wl.D + stats
         bwd_bytes = wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 3 * 4.0 * M
-        bwd_design = 2 * wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 2 * 2.0 * M * wl.V
+        plan = cce.cce_query_plan(M, cce.h_dtype(H), head, buf.ws.numel())
+        if plan["bwd_fused"]:
+            nparts = plan["bwd_fused_buffers"] - 1
+            bwd_design = bwd_bytes + 3 * 4.0 * nparts * M * wl.D  # parts written, read; dH RMW
+        else:
+            bwd_design = 2 * wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 2 * 2.0 * M * wl.V
         line = {"sweep": "small_m_q4" if quant else "small_m", "M": M, "D": wl.D, "V": wl.V,
                 "dtype": "f16 (4-bit head dequantised in-kernel)" if quant else "bf16",
                 "steps": args.steps, "fwd_ms": t_f, "bwd_ms": t_b,
@@ -602,6 +610,7 @@ def run_small_m(args, quant=False):
                 "fwd_frac_hbm": fwd_bytes / (t_f / 1e3) / 1e9 / hbm,
                 "bwd_frac_hbm": bwd_bytes / (t_b / 1e3) / 1e9 / hbm,
                 "fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes,
+                "bwd_form": "fused" if plan["bwd_fused"] else "two GEMMs per vocab chunk",
                 "bwd_design_bytes": bwd_design,
                 "bwd_design_gbs": bwd_design / (t_b / 1e3) / 1e9,
                 "tokens_per_s": M / ((t_f + t_b) / 1e3),

@@ -64,7 +64,10 @@ typedef enum {
   CCE_ERR_LABEL_OUT_OF_RANGE = 5,  /* device: some y >= V                    */
   CCE_ERR_DEVICE_TIMEOUT = 6,      /* device: a bounded wait ran out          */
   CCE_ERR_EMPTY_SEGMENT = 7,       /* device: no labelled chosen/rejected row */
-  CCE_ERR_DOMAIN = 8               /* device: mean logp >= 0 (log1mexp)       */
+  CCE_ERR_DOMAIN = 8,              /* device: mean logp >= 0 (log1mexp)       */
+  CCE_ERR_FP16_RANGE = 9           /* device: a 4/8-bit head's fp16 path met a
+                                      hidden value |h| > 65504, or a scale or
+                                      bias outside the fp16 normal range        */
 } cce_status;
 
 typedef enum { CCE_F32 = 0, CCE_BF16 = 1 } cce_dtype;
@@ -82,7 +85,17 @@ typedef enum {
                               dequantised by this library's kernels (inside
                               the GEMM, or into a staged fp16 chunk of the
                               workspace; see cce_set_quant_staging) and
-                              rounded once to fp16.                          */
+                              rounded once to fp16.  fp16 holds these values
+                              exactly only for |h| <= 65504 and scales and
+                              biases that are 0 or of magnitude in
+                              [2^-14, 65504]; anything else completes but sets
+                              CCE_ERR_FP16_RANGE in the status word.  The
+                              coefficient tile G'' is fp16 on this path and is
+                              stored times 2^14 (|G''| <= 1), so softmax
+                              probabilities down to about 4e-12 stay normal
+                              or representable (a flat softmax over 128k
+                              entries is 5e-6); the dH step divides it out in
+                              fp32.                                           */
 } cce_wformat;
 
 /* The frozen head (host struct; device pointers inside). */
@@ -246,8 +259,18 @@ cce_status pref_grad_coeffs(const float* logp, const int32_t* labels,
  * dH: fp32 [M, D] output, overwritten.
  * skip_stats: optional device uint64 [2] incremented by (skipped tiles,
  *   total tiles).
- * ws: as for cce_forward; the backward takes vocab chunks as wide as it
- *   allows (G'' of one chunk lives there), see cce_query_plan.
+ * ws: as for cce_forward.  A dense bf16 head runs the fused backward: one
+ *   persistent kernel recomputes every vocab tile, forms the coefficient
+ *   tile from the TMEM accumulator and contracts it with W into a dH
+ *   accumulator held in TMEM for a whole sweep of the vocabulary; the
+ *   coefficient tiles pass between the CTAs sharing a row tile through a
+ *   small ring of tiles in ws (DEPTH rounds per group, tens of MB, L2-
+ *   resident), never as a whole.  ws then holds the block-skip plan, the
+ *   ring and its flags, and O(M*D) partial dH buffers when row tiles are
+ *   shared between groups (cce_workspace_bytes sizes it).  Other heads (fp32,
+ *   4/8-bit, or a workspace too small for the fused layout) run two GEMMs per
+ *   vocab chunk, G'' of one chunk living in ws (chunks as wide as ws allows,
+ *   see cce_query_plan).  Deterministic in both forms.
  */
 cce_status cce_backward_dh(const void* H, cce_dtype h_dtype, int64_t M,
                            const cce_head* W, const int32_t* labels,
@@ -332,6 +355,14 @@ void cce_set_cta_pairs(int on);
  * (staged falls back to in-kernel when the chunk would be too narrow). */
 void cce_set_quant_staging(int mode);
 
+/* Backward of dense bf16 heads: 0 choose (default: the fused kernel when
+ * ws holds its layout, else two GEMMs per vocab chunk), 1 the fused kernel
+ * only (CCE_ERR_WORKSPACE_TOO_SMALL when ws cannot hold its layout), 2 two
+ * GEMMs per vocab chunk.  Both forms give the same results to accumulation
+ * order.  Process-wide; any other value is taken as 0.  No counterpart on
+ * the pages: it selects between two schedules of the same backward. */
+void cce_set_backward_mode(int mode);
+
 /* The execution plan cce_forward and cce_backward_dh would take for this
  * problem and workspace size under the current settings (host-only: no
  * launch, no device memory; with no device visible the SM count is taken as
@@ -344,7 +375,12 @@ void cce_set_quant_staging(int mode);
  *   bwd_ksplit        K splits of the dH GEMM (fp32 partial buffers);
  *   *_staged          1 when a 4/8-bit head runs as staged fp16 chunks;
  *   *_cta_pairs       1 when the GEMMs are planned on CTA pairs (used if the
- *                     device can co-schedule them).
+ *                     device can co-schedule them);
+ *   bwd_fused         1 when the backward runs the fused kernel (bwd_chunk
+ *                     is then 0);
+ *   bwd_fused_groups  groups of CTAs (pairs) that each sweep a row tile;
+ *   bwd_fused_members CTAs (pairs) per group, one per 256 columns of dH;
+ *   bwd_fused_buffers dH buffers (1 + partial buffers in ws).
  * Returns CCE_ERR_INVALID_ARGUMENT / UNSUPPORTED as the calls would. */
 typedef struct {
   int fwd_ok, bwd_ok;
@@ -352,9 +388,24 @@ typedef struct {
   int bwd_ksplit;
   int fwd_staged, bwd_staged;
   int fwd_cta_pairs, bwd_cta_pairs;
+  int bwd_fused, bwd_fused_groups, bwd_fused_members, bwd_fused_buffers;
 } cce_plan;
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out);
+
+/* The work schedule of the fused backward for this problem under the current
+ * settings (host-only: no launch, no device memory).  A unit is one round of
+ * a group's sweep: a row tile (256 rows on CTA pairs, 128 on single CTAs)
+ * against C = ceil(D/256) vocab tiles.  For every unit, group by group and
+ * in the order each group runs them, six int32 go to out[6n .. 6n+5]: group,
+ * row tile, round, first unit of a segment (a run of units on one row tile),
+ * last unit of a segment, and the dH buffer the segment writes (0 = dH,
+ * b >= 1 = partial buffer b-1, summed into dH in buffer order).  Writes at
+ * most `cap` units (out may be NULL) and returns the total number of units,
+ * or -1 when the fused backward does not take the problem.  No counterpart
+ * on the pages; it exposes the partition for tests. */
+int64_t cce_query_fused_schedule(int64_t M, cce_dtype h_dtype, const cce_head* W,
+                                 int32_t* out, int64_t cap);
 
 /* Self-test of the timeout path: launches one CTA that waits, with the
  * current wait limit, on an mbarrier nothing arrives on.  The wait runs out,

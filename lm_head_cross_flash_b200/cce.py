@@ -27,7 +27,7 @@ STATUS_NAMES = {
     0: "CCE_OK", 1: "CCE_ERR_INVALID_ARGUMENT", 2: "CCE_ERR_UNSUPPORTED",
     3: "CCE_ERR_CUDA", 4: "CCE_ERR_WORKSPACE_TOO_SMALL",
     5: "CCE_ERR_LABEL_OUT_OF_RANGE", 6: "CCE_ERR_DEVICE_TIMEOUT",
-    7: "CCE_ERR_EMPTY_SEGMENT", 8: "CCE_ERR_DOMAIN",
+    7: "CCE_ERR_EMPTY_SEGMENT", 8: "CCE_ERR_DOMAIN", 9: "CCE_ERR_FP16_RANGE",
 }
 
 
@@ -63,7 +63,9 @@ class _Plan(ctypes.Structure):
                 ("fwd_chunk", ctypes.c_int64), ("bwd_chunk", ctypes.c_int64),
                 ("bwd_ksplit", ctypes.c_int),
                 ("fwd_staged", ctypes.c_int), ("bwd_staged", ctypes.c_int),
-                ("fwd_cta_pairs", ctypes.c_int), ("bwd_cta_pairs", ctypes.c_int)]
+                ("fwd_cta_pairs", ctypes.c_int), ("bwd_cta_pairs", ctypes.c_int),
+                ("bwd_fused", ctypes.c_int), ("bwd_fused_groups", ctypes.c_int),
+                ("bwd_fused_members", ctypes.c_int), ("bwd_fused_buffers", ctypes.c_int)]
 
 
 _lib = None
@@ -104,6 +106,10 @@ _SIGS = {
     "cce_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "cce_set_cta_pairs": (None, [ctypes.c_int]),
     "cce_set_quant_staging": (None, [ctypes.c_int]),
+    "cce_set_backward_mode": (None, [ctypes.c_int]),
+    "cce_query_fused_schedule": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int,
+                                                  ctypes.POINTER(_Head), ctypes.c_void_p,
+                                                  ctypes.c_int64]),
     "cce_query_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(_Head),
                                       ctypes.c_size_t, ctypes.POINTER(_Plan)]),
     "cce_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -477,6 +483,27 @@ def cce_set_cta_pairs(on: bool):
 def cce_set_quant_staging(mode: int):
     """0: choose; 1: dequantise inside the GEMMs; 2: staged fp16 chunks."""
     lib().cce_set_quant_staging(int(mode))
+
+
+def cce_set_backward_mode(mode: int):
+    """Dense bf16 heads: 0 choose; 1 the fused backward kernel; 2 two GEMMs
+    per vocab chunk."""
+    lib().cce_set_backward_mode(int(mode))
+
+
+def cce_query_fused_schedule(M: int, H_dtype: int, head: "Head | _Head"):
+    """The fused backward's units as an int32 array [n, 6] (group, row tile,
+    round, first, last, dH buffer), or None when the fused kernel does not
+    take the problem (host-only)."""
+    import numpy as np
+    h = head.c() if isinstance(head, Head) else head
+    n = lib().cce_query_fused_schedule(M, H_dtype, ctypes.byref(h), None, 0)
+    if n < 0:
+        return None
+    out = np.zeros((max(n, 1), 6), dtype=np.int32)
+    lib().cce_query_fused_schedule(M, H_dtype, ctypes.byref(h),
+                                   out.ctypes.data_as(ctypes.c_void_p), n)
+    return out[:n]
 
 
 def cce_query_plan(M: int, H_dtype: int, head: "Head | _Head", ws_bytes: int) -> dict:

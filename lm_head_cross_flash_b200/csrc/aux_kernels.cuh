@@ -277,7 +277,8 @@ __global__ void split_f32_kernel(const float* __restrict__ src, int64_t rows,
 // the dequantiser lays out the weights along K).  n8 = rows*D/8.
 template <int QB>
 __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
-                                     uint4* __restrict__ dst) {
+                                     uint4* __restrict__ dst, uint32_t* status) {
+  bool over = false;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint4 v = src[i];
@@ -286,10 +287,31 @@ __global__ void h_to_f16_perm_kernel(const uint4* __restrict__ src, int64_t n8,
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint32_t bits = (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-      h[qpos<QB>(e)] = __float2half_rn(__uint_as_float(bits << 16));
+      const float x = __uint_as_float(bits << 16);
+      // a finite bf16 value beyond the largest fp16 would become inf
+      over = over || (fabsf(x) > 65504.f && fabsf(x) <= 3.4e38f);
+      h[qpos<QB>(e)] = __float2half_rn(x);
     }
     dst[i] = *reinterpret_cast<const uint4*>(h);
   }
+  if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0) set_status(status, ST_FP16);
+}
+
+// Scales and biases of a 4/8-bit head feed fp16 arithmetic, which holds a
+// bf16 value exactly only inside the fp16 normal range: report any nonzero
+// one with |x| < 2^-14 or |x| > 65504 (one pass over both arrays).
+__global__ void sb_range_kernel(const uint16_t* __restrict__ scales,
+                                const uint16_t* __restrict__ biases, int64_t n,
+                                uint32_t* status) {
+  bool bad = false;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float s = fabsf(__uint_as_float(static_cast<uint32_t>(scales[i]) << 16));
+    const float b = fabsf(__uint_as_float(static_cast<uint32_t>(biases[i]) << 16));
+    bad = bad || (s != 0.f && (s < 6.103515625e-05f || s > 65504.f)) ||
+          (b != 0.f && (b < 6.103515625e-05f || b > 65504.f));
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) set_status(status, ST_FP16);
 }
 
 // ---------------------------------------------- staged dequantisation --

@@ -15,6 +15,7 @@
 
 #include "../../include/cce.h"
 #include "aux_kernels.cuh"
+#include "fused_bwd.cuh"
 #include "gemm_tc.cuh"
 
 using namespace cce;
@@ -33,6 +34,9 @@ std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_pairs{1};  // 2-CTA (cta_group::2) tiles for dense heads
 // 4/8-bit heads: 0 = choose, 1 = dequantise inside the GEMM, 2 = staged chunks
 std::atomic<int> g_qstage{0};
+// Backward of dense bf16 heads: 0 = choose, 1 = the fused kernel (recompute,
+// coefficient tile and dH in one kernel), 2 = the two GEMMs per vocab chunk
+std::atomic<int> g_bwd_mode{0};
 // Staged dequantisation pays off once enough row tiles reuse each weight;
 // measured on the 4-bit long-context head (D=4096, V=128,256): the backward
 // from 2 row tiles (M=192: 0.71 ms staged against 1.06 ms in-kernel), the
@@ -91,13 +95,14 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
   PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM,
-  PK_PREFIX, PK_DW, PK_DEQ, PK_N
+  PK_PREFIX, PK_DW, PK_DEQ, PK_FUSED, PK_FSUM, PK_N
 };
 const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
                                       "bwd_dh_gemm",   "selftest",     "dh_split_sum",
                                       "prefix_gather_scatter", "bwd_dw_gemm",
-                                      "dequant_chunk"};
+                                      "dequant_chunk", "bwd_fused",
+                                      "fused_part_sum"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -174,6 +179,8 @@ bool make_packed_map(CUtensorMap* m, const cce_head* W, int qb, uint32_t box_byt
 struct DevInfo {
   int sms = 0;
   int pairs = 0;  // CTA pairs (clusters of 2) resident at once, 0 = none
+  int fused_pairs = 0;  // fused backward: pairs / single CTAs resident at once
+  int fused_ctas = 0;
   bool attrs = false;
 };
 
@@ -192,6 +199,26 @@ int max_pairs_of() {
   cfg.numAttrs = 1;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, cce_tc_kernel<MODE, 0, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+// Clusters of two resident at once for the fused backward's pair kernel.
+int max_fused_pairs() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = FusedCfg<true>::SMEM;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fused_bwd_kernel<true>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -221,9 +248,22 @@ cce_status device_info(int* sms) {
     ok = ok && cudaFuncSetAttribute(cce_tc_kernel<MODE, 0, true>, attr, smem_bytes<MODE, true>()) == cudaSuccess;
     CCE_SET_SMEM2(Mode::kLse) CCE_SET_SMEM2(Mode::kGrad) CCE_SET_SMEM2(Mode::kDh)
 #undef CCE_SET_SMEM2
-    if (ok)
+    ok = ok &&
+         cudaFuncSetAttribute(fused_bwd_kernel<true>, attr, FusedCfg<true>::SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(fused_bwd_kernel<false>, attr, FusedCfg<false>::SMEM) == cudaSuccess;
+    if (ok) {
       d.pairs = std::min(max_pairs_of<Mode::kLse>(),
                          std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
+      d.fused_pairs = max_fused_pairs();
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_bwd_kernel<false>,
+                                                        NUM_THREADS, FusedCfg<false>::SMEM) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        per_sm = 0;
+      }
+      d.fused_ctas = per_sm * d.sms;
+    }
     if (!ok)
       return CCE_ERR_CUDA;
     d.attrs = true;
@@ -531,12 +571,22 @@ cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_hea
   const int64_t D = W->D;
   op->qb = W->format == CCE_W_AFFINE_Q4_G64 ? 4 : W->format == CCE_W_AFFINE_Q8_G64 ? 8 : 0;
   op->stage_qb = 0;
+  if (op->qb) {
+    // 4/8-bit heads compute in fp16: report scales or biases it cannot hold
+    const int64_t n = W->V * (D / 64);
+    ProfScope ps(PK_SPLIT, st);
+    sb_range_kernel<<<int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(n, 256), 1184))), 256, 0,
+                      st>>>(static_cast<const uint16_t*>(W->scales),
+                            static_cast<const uint16_t*>(W->biases), n, status_word(ws));
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
   if (op->qb && L.staged) {
     // fp16 rows in natural order; B is the fp16 chunk staged by stage_chunk
     uint4* h16 = reinterpret_cast<uint4*>(static_cast<char*>(ws) + L.hs);
     {
       ProfScope ps(PK_SPLIT, st);
-      h_to_f16_perm_kernel<0><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+      h_to_f16_perm_kernel<0><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16,
+                                                            status_word(ws));
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     op->stage_qb = op->qb;
@@ -556,9 +606,11 @@ cce_status prepare_operands(const void* H, cce_dtype h, int64_t M, const cce_hea
     {
       ProfScope ps(PK_SPLIT, st);
       if (op->qb == 4)
-        h_to_f16_perm_kernel<4><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+        h_to_f16_perm_kernel<4><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16,
+                                                            status_word(ws));
       else
-        h_to_f16_perm_kernel<8><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16);
+        h_to_f16_perm_kernel<8><<<1184, 256, 0, st>>>(static_cast<const uint4*>(H), M * D / 8, h16,
+                                                            status_word(ws));
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
     op->a = h16;
@@ -622,6 +674,192 @@ cce_status stage_chunk(const Operands& op, const cce_head* W, int64_t v0, int64_
   return launch_ok();
 }
 
+// ------------------------------------------------------- fused backward --
+// Fused-backward units (pairs or single CTAs) resident at once: the device's
+// figure, or the B200 figure where no device is visible (host-side planning).
+int fused_resident(bool c2) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 &&
+      device_info(&sms) == CCE_OK) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    return c2 ? g_dev[dev].fused_pairs : g_dev[dev].fused_ctas;
+  }
+  cudaGetLastError();
+  return c2 ? 74 : 148;
+}
+
+// How the fused backward runs: tile shape, groups of C members, the waves
+// and remainder partition of (row tile, round) units, the number of dH
+// buffers, and its workspace (block-skip plan, exchange flags, the G'' ring,
+// partial dH buffers).  ok = false: the problem is not one the fused kernel
+// takes (4/8-bit or fp32 heads, a trainable head, the mode switch set to the
+// two GEMMs, or D too wide for a group of resident units).
+struct FusedPlan {
+  bool ok = false;
+  bool c2 = false;
+  FusedArgs a{};
+  int nbuf = 1;
+  int64_t ring_rows = 0;
+  size_t tile_skip = 0, row_skip = 0, flags = 0, ring = 0, parts = 0, total = 0;
+};
+
+FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
+  FusedPlan f;
+  if (g_bwd_mode.load() == 2 || want_dw || h != CCE_BF16 || W->format != CCE_W_DENSE) return f;
+  const int64_t n128 = ceil_div(M, BM);
+  f.c2 = g_pairs.load() != 0 && n128 >= 2;
+  const int TH = f.c2 ? FusedCfg<true>::TH : FusedCfg<false>::TH;
+  const int BV = f.c2 ? FusedCfg<true>::BV : FusedCfg<false>::BV;
+  const int C = int(ceil_div(W->D, FB_DS));
+  const int G = fused_resident(f.c2) / C;
+  if (G < 1) return f;
+  FusedArgs& a = f.a;
+  a.M = int(M);
+  a.V = int(W->V);
+  a.D = int(W->D);
+  a.n_rt = int(ceil_div(M, TH));
+  a.n_rt128 = int(n128);
+  a.nk = int(ceil_div(W->D, BK));
+  a.C = C;
+  a.G = G;
+  a.n_vt = int(ceil_div(W->V, BV));
+  a.n_rounds = int(ceil_div(a.n_vt, C));
+  a.waves = a.n_rt / G;
+  a.rem = a.n_rt % G;
+  a.row_rem = int(std::min<int64_t>(M, int64_t(a.waves) * G * TH));
+  const int64_t T = int64_t(a.rem) * a.n_rounds;
+  a.Gr = int(std::min<int64_t>(G, T));
+  for (int i = 0; i < a.rem; ++i) {
+    const int gf = fb_group_of(int64_t(i) * a.n_rounds, T, a.Gr);
+    const int gl = fb_group_of(int64_t(i + 1) * a.n_rounds - 1, T, a.Gr);
+    f.nbuf = std::max(f.nbuf, gl - gf + 1);
+  }
+  f.ring_rows = int64_t(G) * FB_DEPTH * C * TH;
+  const int64_t cols = ceil_div(W->V, BN);
+  size_t o = kStatusBytes;
+  f.tile_skip = o; o += align_up(size_t(n128) * cols);
+  f.row_skip = o; o += align_up(size_t(n128));
+  f.flags = o; o += align_up(size_t(G) * FB_DEPTH * C * (2 + C) * 4);
+  f.ring = o; o += align_up(size_t(f.ring_rows) * BV * 2);
+  f.parts = o; o += align_up(size_t(f.nbuf - 1) * (M - a.row_rem) * W->D * 4);
+  // the forward's region shares the same bytes (it is dead by the backward)
+  f.total = std::max(o, make_layout(M, h, W, BN).total);
+  f.ok = true;
+  return f;
+}
+
+cce_status fused_backward(const FusedPlan& fp, const void* H, const cce_head* W,
+                          const int32_t* labels, const float* lse, const float* coeff,
+                          float filter_eps, const float* blockmax, float* dH,
+                          unsigned long long* skip_stats, void* ws, cudaStream_t st) {
+  int sms = 0;
+  cce_status s = device_info(&sms);
+  if (s != CCE_OK) return s;
+  char* wsc = static_cast<char*>(ws);
+  const FusedArgs& p = fp.a;
+  const int64_t M = p.M, V = p.V, D = p.D;
+  const int64_t cols = ceil_div(V, BN);
+  uint8_t* tile_skip = reinterpret_cast<uint8_t*>(wsc + fp.tile_skip);
+  uint8_t* row_skip = reinterpret_cast<uint8_t*>(wsc + fp.row_skip);
+  {
+    const int64_t units = int64_t(p.n_rt128) * cols;
+    const int wpb = 8;
+    ProfScope ps(PK_SKIP, st);
+    skip_plan_kernel<<<int(ceil_div(units, wpb)), wpb * 32, 0, st>>>(
+        filter_eps > 0.f ? blockmax : nullptr, lse, labels, coeff, int(M), int(cols),
+        p.n_rt128, filter_eps, tile_skip, row_skip, skip_stats);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+  const size_t flag_bytes = size_t(p.G) * FB_DEPTH * p.C * (2 + p.C) * 4;
+  if (cudaMemsetAsync(wsc + fp.flags, 0, flag_bytes, st) != cudaSuccess) return CCE_ERR_CUDA;
+
+  const int BV = fp.c2 ? FusedCfg<true>::BV : FusedCfg<false>::BV;
+  void* ring = wsc + fp.ring;
+  CUtensorMap mh, mwk, mwm, mgl, mgs, md0, md1;
+  if (!make_map(&mh, H, true, D, M, D, BK, BM) || !make_map(&mwk, W->w, true, D, V, D, BK, 128) ||
+      !make_map(&mwm, W->w, true, D, V, D, 64, BK) ||
+      !make_map(&mgl, ring, true, BV, fp.ring_rows, BV, BK, BM))
+    return CCE_ERR_CUDA;
+  {
+    const uint64_t gd[2] = {uint64_t(BV), uint64_t(fp.ring_rows)};
+    const uint64_t gs[1] = {uint64_t(BV) * 2};
+    const uint32_t gb[2] = {32, 32};
+    if (!make_map_ex(&mgs, ring, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, gd, gs, gb,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+      return CCE_ERR_CUDA;
+    const uint64_t dd[3] = {uint64_t(D), uint64_t(M), 1};
+    const uint64_t ds[2] = {uint64_t(D) * 4, uint64_t(M) * D * 4};
+    const uint32_t db[3] = {32, 32, 1};
+    if (!make_map_ex(&md0, dH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dd, ds, db,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return CCE_ERR_CUDA;
+    md1 = md0;
+    if (fp.nbuf > 1) {
+      const uint64_t mr = uint64_t(M - p.row_rem);
+      const uint64_t pd[3] = {uint64_t(D), mr, uint64_t(fp.nbuf - 1)};
+      const uint64_t ps[2] = {uint64_t(D) * 4, mr * D * 4};
+      if (!make_map_ex(&md1, wsc + fp.parts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, pd, ps, db,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+        return CCE_ERR_CUDA;
+    }
+  }
+  FusedArgs a = p;
+  a.wait_ns = g_wait_ns.load();
+  a.status = status_word(ws);
+  a.labels = labels;
+  a.lse = lse;
+  a.coeff = coeff;
+  a.filter_eps = filter_eps;
+  a.tile_skip = tile_skip;
+  a.skip_ld = int(cols);
+  a.row_skip = row_skip;
+  a.softcap = W->softcap;
+  a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
+  a.ready = reinterpret_cast<uint32_t*>(wsc + fp.flags);
+  a.consumed = a.ready + size_t(p.G) * FB_DEPTH * p.C * 2;
+  {
+    ProfScope ps(PK_FUSED, st);
+    const int members = a.G * a.C;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    if (fp.c2) {
+      cfg.gridDim = dim3(2 * members);
+      cfg.dynamicSmemBytes = FusedCfg<true>::SMEM;
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, fused_bwd_kernel<true>, mh, mwk, mwm, mgl, mgs, md0, md1, a) !=
+          cudaSuccess)
+        return CCE_ERR_CUDA;
+    } else {
+      cfg.gridDim = dim3(members);
+      cfg.dynamicSmemBytes = FusedCfg<false>::SMEM;
+      cfg.numAttrs = 0;
+      if (cudaLaunchKernelEx(&cfg, fused_bwd_kernel<false>, mh, mwk, mwm, mgl, mgs, md0, md1,
+                             a) != cudaSuccess)
+        return CCE_ERR_CUDA;
+    }
+  }
+  if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  if (fp.nbuf > 1) {
+    const int TH = fp.c2 ? FusedCfg<true>::TH : FusedCfg<false>::TH;
+    const int64_t n4 = (M - a.row_rem) * (D / 4);
+    ProfScope ps(PK_FSUM, st);
+    fused_sum_parts_kernel<<<int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(n4, 256),
+                                                                          4 * sms))),
+                             256, 0, st>>>(reinterpret_cast<float4*>(dH),
+                                           reinterpret_cast<const float4*>(wsc + fp.parts), a,
+                                           TH);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+  return CCE_OK;
+}
+
 }  // namespace
 
 // ========================================================================
@@ -638,6 +876,7 @@ const char* cce_status_string(cce_status s) {
     case CCE_ERR_DEVICE_TIMEOUT: return "CCE_ERR_DEVICE_TIMEOUT";
     case CCE_ERR_EMPTY_SEGMENT: return "CCE_ERR_EMPTY_SEGMENT";
     case CCE_ERR_DOMAIN: return "CCE_ERR_DOMAIN";
+    case CCE_ERR_FP16_RANGE: return "CCE_ERR_FP16_RANGE";
   }
   return "CCE_UNKNOWN_STATUS";
 }
@@ -647,6 +886,8 @@ void cce_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? kDefaultWait
 void cce_set_cta_pairs(int on) { g_pairs.store(on != 0 ? 1 : 0); }
 
 void cce_set_quant_staging(int mode) { g_qstage.store(mode == 1 || mode == 2 ? mode : 0); }
+
+void cce_set_backward_mode(int mode) { g_bwd_mode.store(mode == 1 || mode == 2 ? mode : 0); }
 
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out) {
@@ -667,13 +908,50 @@ cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_
   out->bwd_ksplit = b.ksplit;
   out->bwd_staged = b.staged;
   out->bwd_cta_pairs = b.vc > 0 && b.pairs;
+  const FusedPlan fp = plan_fused(M, h_dtype, W, false);
+  if (fp.ok && fp.total <= ws_bytes) {
+    out->bwd_ok = 1;
+    out->bwd_fused = 1;
+    out->bwd_chunk = 0;
+    out->bwd_ksplit = 1;
+    out->bwd_staged = 0;
+    out->bwd_cta_pairs = fp.c2 ? 1 : 0;
+    out->bwd_fused_groups = fp.a.G;
+    out->bwd_fused_members = fp.a.C;
+    out->bwd_fused_buffers = fp.nbuf;
+  }
   return CCE_OK;
+}
+
+int64_t cce_query_fused_schedule(int64_t M, cce_dtype h_dtype, const cce_head* W,
+                                 int32_t* out, int64_t cap) {
+  if (M <= 0 || M > (int64_t(1) << 30) || check_head(W, h_dtype) != CCE_OK) return -1;
+  const FusedPlan fp = plan_fused(M, h_dtype, W, false);
+  if (!fp.ok) return -1;
+  int64_t n = 0;
+  for (int g = 0; g < fp.a.G; ++g) {
+    const int nu = fb_units(fp.a, g);
+    for (int u = 0; u < nu; ++u, ++n) {
+      if (out == nullptr || n >= cap) continue;
+      const FUnit x = fb_unit(fp.a, g, u);
+      int32_t* o = out + 6 * n;
+      o[0] = g;
+      o[1] = x.r;
+      o[2] = x.j;
+      o[3] = x.first ? 1 : 0;
+      o[4] = x.last ? 1 : 0;
+      o[5] = x.buf;
+    }
+  }
+  return n;
 }
 
 int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
 
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
+  const FusedPlan fp = plan_fused(M, h_dtype, W, false);
+  if (fp.ok) return fp.total;
   const bool staged = q_stage_wanted(M, W, false);  // the backward stages first
   return make_layout(M, h_dtype, W, default_vc(M, W),
                      ksplit_for(M, W, sm_count_guess(), staged), staged)
@@ -952,6 +1230,15 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   cce_status s = check_head(W, h_dtype);
   if (s != CCE_OK) return s;
   if (!tiles_fit(M, W)) return CCE_ERR_UNSUPPORTED;
+  {
+    // Dense bf16 heads take the fused kernel when the workspace holds its
+    // (small) layout; the two GEMMs per vocab chunk cover the rest.
+    const FusedPlan fp = plan_fused(M, h_dtype, W, dW != nullptr);
+    if (fp.ok && fp.total <= ws_bytes)
+      return fused_backward(fp, H, W, labels, lse, coeff, filter_eps, blockmax, dH, skip_stats,
+                            ws, reinterpret_cast<cudaStream_t>(stream));
+    if (g_bwd_mode.load() == 1 && fp.ok) return CCE_ERR_WORKSPACE_TOO_SMALL;
+  }
   // K split of the dH GEMM; fall back to fewer splits if the workspace
   // cannot hold their partial buffers.
   // A staged 4/8-bit head needs chunks of stage_min_rows at least; else the
@@ -1258,6 +1545,7 @@ cce_status cce_device_status(void* ws, cce_stream_t stream) {
   if (word & ST_TIMEOUT) return CCE_ERR_DEVICE_TIMEOUT;
   if (word & ST_EMPTY) return CCE_ERR_EMPTY_SEGMENT;
   if (word & ST_DOMAIN) return CCE_ERR_DOMAIN;
+  if (word & ST_FP16) return CCE_ERR_FP16_RANGE;
   return CCE_OK;
 }
 

@@ -1,0 +1,662 @@
+// fused_bwd.cuh — the backward of the flash-CCE head as one persistent
+// kernel: every vocab tile of the logits is recomputed on the tensor cores,
+// turned into the coefficient tile G'' = softmax - onehot straight from the
+// TMEM accumulator, and contracted against the same vocab rows of W into a
+// dH accumulator that stays in TMEM for a whole sweep over the vocabulary.
+// (ORPO design 0.0.6, fused-head implementation spec, "Backward (recompute
+// vocab tiles from the saved LSE)": recompute, form g * (onehot - softmax),
+// accumulate dh, never form [M, V]; Training design §5.1, tier 4.)
+//
+// Why a group of CTAs, and what they exchange.  A row tile's dH is
+// rows x D fp32: 1 MB for 128 rows at D = 2048, four times a TMEM.  So each
+// CTA (or CTA pair) of a group of C = ceil(D / 256) owns the 256 d-columns
+// [256 p, 256 p + 256) of dH for the group's row tile, in 256 TMEM columns,
+// and the group sweeps the vocabulary in rounds of C vocab tiles.  In a round
+// member p recomputes the logits of vocab tile (round * C + p) (K = D), forms
+// its G'' tile and publishes it in a small ring of tiles in global memory
+// that stays in L2; then every member contracts all C published tiles of the
+// round with its own d-columns of W (K = C tiles of vocabulary).  The S GEMM
+// of one round overlaps the dH GEMM of the previous one, so a member's tensor
+// pipe never waits for the exchange.  G'' never exists as a whole: one ring
+// holds DEPTH rounds of tiles per group.
+//
+// Roles (192 threads, as in gemm_tc.cuh): warp 0 loads operand stages by
+// TMA (the S phase: H rows and W rows, both K-major; the dH phase: a G''
+// tile of the ring, K-major, and W as an MN-major operand); warp 1 issues
+// tcgen05.mma into the S accumulator(s) and the dH accumulator; warps 2-5
+// drain S, compute G'' (grad_chunk, the same arithmetic as the two-GEMM
+// path), stage it for TMA stores into the ring, and at the end of a row
+// tile's sweep drain dH, scale each row by -coeff and store it.
+//
+// C2 = true: clusters of two CTAs computing 256-row tiles with
+// tcgen05.mma.cta_group::2 (S: 256 x 256 vocab; dH: 256 x 256 d-columns),
+// each CTA loading its own 128 rows of A and half of B (as in gemm_tc.cuh).
+// C2 = false: single CTAs on 128-row tiles with 128-column vocab tiles and a
+// double-buffered S accumulator (used for at most one row tile, where the
+// path streams W from HBM and a narrower vocab tile halves the W held in L2
+// between a round's two reads).
+//
+// The exchange.  Ring slot (group, unit % DEPTH, member) is filled once per
+// DEPTH units.  Publisher: each epilogue warp waits until every member has
+// consumed the slot's previous fill (consumed[slot][member] >= fill), writes
+// its rows by TMA store, waits for the stores to complete, fences the async
+// proxy and adds 1 to ready[slot][half] with release semantics.  Consumer:
+// the producer warp waits for ready >= 4 (fill + 1) with acquire semantics,
+// fences the async proxy and loads the tile by TMA; once the tile has
+// landed (the leader's full barrier counts both CTAs of a pair) the MMA warp
+// stores consumed = fill + 1 (relaxed: the tile's reads are complete).  A tile that block skip (or the end of the
+// vocabulary) removes is neither computed nor loaded, but still advances
+// both counters, so the counts stay aligned.  Every wait is bounded; all
+// CTAs of the grid are resident at once (at most one CTA per SM, grid no
+// larger than the resident count).
+//
+// Partition of the work.  A unit is (row tile r, round j).  G groups take
+// the row tiles in waves (group g: r = w G + g), so that all groups sweep
+// the same rounds of W at the same time and W streams from HBM about once
+// per wave.  The rem = n_rt mod G row tiles left over are cut into
+// contiguous ranges of units, one per group: a row tile split between k
+// groups gives k partial dH slices (buffer 0 is dH itself, buffers 1.. are
+// in the workspace) that fused_sum_parts_kernel adds in a fixed order.
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace cce {
+
+constexpr int FB_DEPTH = 3;     // units in flight in the G'' ring of a group
+constexpr int FB_DS = 256;      // dH columns per member
+constexpr uint32_t FB_TMEM_COLS = 512;
+
+template <bool C2>
+struct FusedCfg {
+  static constexpr int TH = C2 ? 2 * BM : BM;        // rows of a tile
+  static constexpr int BV = C2 ? 256 : 128;          // vocab columns of an S tile
+  static constexpr int SB = C2 ? 1 : 2;              // S accumulators (TMEM columns [0, SB*BV))
+  static constexpr int DB = C2 ? FB_DS / 2 : FB_DS;  // d-columns of W each CTA loads (dH phase)
+  static constexpr int S_BYTES = A_BYTES + 128 * BK * 2;  // H 128 x 64 + W 128 x 64
+  static constexpr int D_BYTES = A_BYTES + BK * DB * 2;   // G'' 128 x 64 + W 64 x DB
+  static constexpr int STAGE = S_BYTES > D_BYTES ? S_BYTES : D_BYTES;
+  static constexpr int NST = C2 ? 6 : 4;
+  static constexpr int STAGING = 4 * 2 * 32 * 128;   // per epilogue warp two 4 KB blocks
+  static constexpr int SMEM = NST * STAGE + STAGING + 1024 + 256;
+};
+static_assert(FusedCfg<true>::SMEM <= 232448 && FusedCfg<false>::SMEM <= 232448,
+              "fused backward exceeds the shared memory of a CTA");
+
+struct FusedArgs {
+  int M, V, D;
+  int n_rt;       // row tiles of TH rows
+  int n_rt128;    // 128-row tiles (block-skip plan granularity)
+  int nk;         // K steps of BK over D
+  int C;          // members per group (d-slices of 256)
+  int G;          // groups in the waves
+  int Gr;         // groups sharing the remainder (<= G)
+  int n_vt;       // vocab tiles of BV
+  int n_rounds;   // ceil(n_vt / C)
+  int waves;      // n_rt / G
+  int rem;        // n_rt % G
+  int row_rem;    // first row of the remainder (waves * G * TH); partial
+                  // buffers hold rows [row_rem, M) only
+  uint64_t wait_ns;
+  uint32_t* status;
+  const int32_t* labels;
+  const float* lse;
+  const float* coeff;
+  float filter_eps;
+  const uint8_t* tile_skip;  // [n_rt128, skip_ld], 256-vocab blocks
+  int skip_ld;
+  const uint8_t* row_skip;   // [n_rt128]
+  float softcap;
+  float inv_cap;
+  uint32_t* ready;     // [G * DEPTH * C * 2]
+  uint32_t* consumed;  // [G * DEPTH * C * C]
+};
+
+// One unit of group g's sequence: row tile r, round j; first / last unit of
+// a segment (a run of units on one row tile), and the dH buffer the segment
+// writes.
+struct FUnit {
+  int r, j;
+  bool first, last;
+  int buf;
+};
+
+// Group containing unit e of the remainder's sequence (T units over Gr
+// groups, group g holding [g T / Gr, (g + 1) T / Gr)).
+__host__ __device__ __forceinline__ int fb_group_of(int64_t e, int64_t T, int Gr) {
+  return static_cast<int>(((e + 1) * Gr - 1) / T);
+}
+
+__host__ __device__ __forceinline__ int fb_units(const FusedArgs& a, int g) {
+  int n = a.waves * a.n_rounds;
+  if (g < a.Gr) {
+    const int64_t T = static_cast<int64_t>(a.rem) * a.n_rounds;
+    n += static_cast<int>((g + 1) * T / a.Gr - g * T / a.Gr);
+  }
+  return n;
+}
+
+__host__ __device__ __forceinline__ FUnit fb_unit(const FusedArgs& a, int g, int u) {
+  FUnit x;
+  const int full = a.waves * a.n_rounds;
+  if (u < full) {
+    const int w = u / a.n_rounds;
+    x.j = u - w * a.n_rounds;
+    x.r = w * a.G + g;
+    x.first = x.j == 0;
+    x.last = x.j == a.n_rounds - 1;
+    x.buf = 0;
+    return x;
+  }
+  const int64_t T = static_cast<int64_t>(a.rem) * a.n_rounds;
+  const int64_t lo = g * T / a.Gr, hi = (g + 1) * T / a.Gr;
+  const int64_t e = lo + (u - full);
+  const int i = static_cast<int>(e / a.n_rounds);
+  x.j = static_cast<int>(e - static_cast<int64_t>(i) * a.n_rounds);
+  x.r = a.waves * a.G + i;
+  x.first = (u == full) || x.j == 0;
+  x.last = (e == hi - 1) || x.j == a.n_rounds - 1;
+  x.buf = g - fb_group_of(static_cast<int64_t>(i) * a.n_rounds, T, a.Gr);
+  return x;
+}
+
+// Nothing to compute for (row tile r, vocab tile v): past the vocabulary,
+// or every 128-row half either past M, without a nonzero cotangent, or
+// block-skipped for the 256-wide vocabulary block holding v.
+template <bool C2>
+__device__ __forceinline__ bool fb_skip(const FusedArgs& a, int r, int v) {
+  if (v >= a.n_vt) return true;
+  const int b = C2 ? v : (v >> 1);
+  auto half = [&](int rt) -> bool {
+    if (rt >= a.n_rt128 || a.row_skip[rt]) return true;
+    return a.tile_skip != nullptr && a.tile_skip[static_cast<size_t>(rt) * a.skip_ld + b] != 0;
+  };
+  return C2 ? (half(2 * r) && half(2 * r + 1)) : half(r);
+}
+
+template <bool C2>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fused_bwd_kernel(const __grid_constant__ CUtensorMap tmH,   // H [M, D], box 64 x 128
+                     const __grid_constant__ CUtensorMap tmWk,  // W [V, D], box 64 x 128
+                     const __grid_constant__ CUtensorMap tmWm,  // W [V, D], box 64 x 64 (MN-major B)
+                     const __grid_constant__ CUtensorMap tmGl,  // ring [rows, BV], box 64 x 128
+                     const __grid_constant__ CUtensorMap tmGs,  // ring [rows, BV], box 32 x 32
+                     const __grid_constant__ CUtensorMap tmD0,  // dH [1, M, D] fp32
+                     const __grid_constant__ CUtensorMap tmD1,  // partial dH [nbuf-1, M-row_rem, D]
+                     const FusedArgs a) {
+  using F = FusedCfg<C2>;
+  const uint32_t rank = C2 ? cluster_ctarank() : 0u;
+  const int member_id = C2 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int g = member_id / a.C, p = member_id - (member_id / a.C) * a.C;
+
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  uint8_t* staging = base + F::NST * F::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + F::STAGING);
+  uint64_t* empty = full + F::NST;
+  uint64_t* s_full = empty + F::NST;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* dh_full = s_empty + 2;
+  uint64_t* dh_empty = dh_full + 1;
+  uint64_t* drain = dh_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_u = g < a.G ? fb_units(a, g) : 0;
+  constexpr int KV = F::BV / BK;  // K steps of one G'' tile in the dH phase
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < F::NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], (C2 ? 2 : 1) * 4 * 32);
+    }
+    mbar_init(dh_full, 1);
+    mbar_init(dh_empty, (C2 ? 2 : 1) * 4 * 32);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch_desc(&tmH);
+    tma_prefetch_desc(&tmWk);
+    tma_prefetch_desc(&tmWm);
+    tma_prefetch_desc(&tmGl);
+  }
+  if (warp == 1) {
+    if constexpr (C2) {
+      tmem_alloc2(tmem_slot, FB_TMEM_COLS);
+      tmem_relinquish2();
+    } else {
+      tmem_alloc(tmem_slot, FB_TMEM_COLS);
+      tmem_relinquish();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (C2) cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_dh = tmem_base + FB_DS;  // columns [256, 512)
+
+  auto slot_of = [&](int u, int q) { return (g * FB_DEPTH + u % FB_DEPTH) * a.C + q; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      const uint64_t keep = l2_policy_evict_last();
+      const uint64_t normal = l2_policy_evict_normal();
+      auto next_stage = [&](uint32_t bytes, uint8_t*& sA, uint8_t*& sB, uint32_t& bar) -> bool {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) return false;
+        sA = base + stage * F::STAGE;
+        sB = sA + A_BYTES;
+        if constexpr (C2) {
+          bar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
+        } else {
+          bar = smem_u32(&full[stage]);
+          mbar_arrive_expect_tx(&full[stage], bytes);
+        }
+        return true;
+      };
+      auto advance = [&]() {
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == F::NST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      for (int u = 0; u <= n_u && ok; ++u) {
+        if (u < n_u) {
+          const FUnit x = fb_unit(a, g, u);
+          const int v = x.j * a.C + p;
+          if (!fb_skip<C2>(a, x.r, v)) {
+            const int arow = x.r * F::TH + static_cast<int>(rank) * BM;
+            const int brow = v * F::BV + (C2 ? static_cast<int>(rank) * 128 : 0);
+            for (int k = 0; k < a.nk; ++k) {
+              uint8_t *sA, *sB;
+              uint32_t bar;
+              if (!next_stage(F::S_BYTES, sA, sB, bar)) {
+                ok = false;
+                break;
+              }
+              if constexpr (C2) {
+                tma_load_2d_pair(sA, &tmH, bar, k * BK, arow, keep);
+                tma_load_2d_pair(sB, &tmWk, bar, k * BK, brow, normal);
+              } else {
+                tma_load_2d_hint(sA, &tmH, &full[stage], k * BK, arow, keep);
+                tma_load_2d_hint(sB, &tmWk, &full[stage], k * BK, brow, normal);
+              }
+              advance();
+            }
+          }
+        }
+        if (u >= 1 && ok) {
+          const FUnit x = fb_unit(a, g, u - 1);
+          const uint32_t fill = static_cast<uint32_t>((u - 1) / FB_DEPTH);
+          for (int q = 0; q < a.C && ok; ++q) {
+            const int v = x.j * a.C + q;
+            if (fb_skip<C2>(a, x.r, v)) continue;
+            const int slot = slot_of(u - 1, q);
+            if (!wait_flag_geq(&a.ready[slot * 2 + static_cast<int>(rank)], 4u * (fill + 1u),
+                               a.wait_ns, abort_flag)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            const int grow = slot * F::TH + static_cast<int>(rank) * BM;
+            const int dcol = p * FB_DS + (C2 ? static_cast<int>(rank) * (FB_DS / 2) : 0);
+            for (int kv = 0; kv < KV; ++kv) {
+              uint8_t *sA, *sB;
+              uint32_t bar;
+              if (!next_stage(F::D_BYTES, sA, sB, bar)) {
+                ok = false;
+                break;
+              }
+              if constexpr (C2) {
+                tma_load_2d_pair(sA, &tmGl, bar, kv * BK, grow, normal);
+#pragma unroll
+                for (int jj = 0; jj < F::DB / 64; ++jj)
+                  tma_load_2d_pair(sB + jj * (64 * BK * 2), &tmWm, bar, dcol + jj * 64,
+                                   v * F::BV + kv * BK, normal);
+              } else {
+                tma_load_2d(sA, &tmGl, &full[stage], kv * BK, grow);
+#pragma unroll
+                for (int jj = 0; jj < F::DB / 64; ++jj)
+                  tma_load_2d(sB + jj * (64 * BK * 2), &tmWm, &full[stage], dcol + jj * 64,
+                              v * F::BV + kv * BK);
+              }
+              advance();
+            }
+          }
+        }
+      }
+      if (!ok) {
+        set_status(a.status, ST_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if (!C2 || rank == 0)
+        for (int s = 0; s < F::NST; ++s)
+          if (issued_mask & (1u << s))
+            wait_bounded(&full[s], (issued_phase >> s) & 1u, DRAIN_LIMIT_NS, nullptr);
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer --
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc_s = idesc_f16(F::TH, F::BV, 1, false, false);
+      const uint32_t idesc_d = idesc_f16(F::TH, FB_DS, 1, false, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int ns = 0, nseg = 0;
+      bool ok = true, dh_any = false;
+      for (int u = 0; u <= n_u && ok; ++u) {
+        if (u < n_u) {
+          const FUnit x = fb_unit(a, g, u);
+          if (!fb_skip<C2>(a, x.r, x.j * a.C + p)) {
+            const int sb = ns % F::SB;
+            if (!wait_bounded(&s_empty[sb], ((ns / F::SB) & 1) ^ 1u, a.wait_ns, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + sb * F::BV;
+            for (int kk = 0; kk < a.nk; ++kk) {
+              if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sA = smem_u32(base + stage * F::STAGE);
+              const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+              for (int j = 0; j < BK / 16; ++j) {
+                const uint64_t ad = sdesc_sw128(sA + j * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(sB + j * 32, 16, 1024);
+                if constexpr (C2) umma_f16_ss2(d_tmem, ad, bd, idesc_s, (kk | j) != 0 ? 1u : 0u);
+                else umma_f16_ss(d_tmem, ad, bd, idesc_s, (kk | j) != 0 ? 1u : 0u);
+              }
+              if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
+              else umma_commit(&empty[stage]);
+              if (++stage == F::NST) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+            if (!ok) break;
+            if constexpr (C2) umma_commit2_mc(&s_full[sb], 0x3);
+            else umma_commit(&s_full[sb]);
+            ++ns;
+          }
+        }
+        if (u >= 1) {
+          const FUnit x = fb_unit(a, g, u - 1);
+          const uint32_t fill = static_cast<uint32_t>((u - 1) / FB_DEPTH);
+          if (x.first) dh_any = false;
+          for (int q = 0; q < a.C && ok; ++q) {
+            const int slot = slot_of(u - 1, q);
+            uint32_t* cons = &a.consumed[slot * a.C + p];
+            if (fb_skip<C2>(a, x.r, x.j * a.C + q)) {
+              st_relaxed_gpu(cons, fill + 1u);
+              continue;
+            }
+            if (!dh_any) {
+              if (!wait_bounded(dh_empty, (nseg & 1) ^ 1u, a.wait_ns, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            for (int kv = 0; kv < KV; ++kv) {
+              if (!wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              // The whole tile has landed (in both CTAs of a pair): its ring
+              // slot may be refilled.  The reads are complete, so a relaxed
+              // store suffices; a release here would stall this thread, and
+              // with it the tensor pipe, on every tile.
+              if (kv == KV - 1) st_relaxed_gpu(cons, fill + 1u);
+              const uint32_t sA = smem_u32(base + stage * F::STAGE);
+              const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+              for (int j = 0; j < BK / 16; ++j) {
+                const uint64_t ad = sdesc_sw128(sA + j * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(sB + j * 16 * 128, 64 * BK * 2, 1024);
+                const uint32_t acc = (dh_any || kv != 0 || j != 0) ? 1u : 0u;
+                if constexpr (C2) umma_f16_ss2(tmem_dh, ad, bd, idesc_d, acc);
+                else umma_f16_ss(tmem_dh, ad, bd, idesc_d, acc);
+              }
+              if (kv == 0) dh_any = true;
+              if constexpr (C2) umma_commit2_mc(&empty[stage], 0x3);
+              else umma_commit(&empty[stage]);
+              if (++stage == F::NST) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+          }
+          if (ok && x.last && dh_any) {
+            if constexpr (C2) umma_commit2_mc(dh_full, 0x3);
+            else umma_commit(dh_full);
+            ++nseg;
+          }
+        }
+      }
+      if (!ok) {
+        set_status(a.status, ST_TIMEOUT);
+        *abort_flag = 1;
+      }
+      if constexpr (C2) umma_commit2_mc(drain, 0x1);
+      else umma_commit(drain);
+      wait_bounded(drain, 0, DRAIN_LIMIT_NS, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int quad = warp & 3;
+    const int rin = quad * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    uint8_t* const stage_base = staging + quad * 2 * (32 * 128);
+    uint32_t nstore = 0;
+    uint32_t s_empty_leader[2] = {0u, 0u}, dh_empty_leader = 0u;
+    if constexpr (C2) {
+      s_empty_leader[0] = mapa_shared(smem_u32(&s_empty[0]), 0);
+      s_empty_leader[1] = mapa_shared(smem_u32(&s_empty[1]), 0);
+      dh_empty_leader = mapa_shared(smem_u32(dh_empty), 0);
+    }
+    int ns = 0, nseg = 0;
+    bool ok = true;
+    // Staging per warp: 8 KB, four 2 KB slots for G'' blocks (the TMA store
+    // of a block may still be reading its slot while the next three are
+    // filled) or two 4 KB slots for fp32 dH blocks during a flush (which
+    // drains all pending reads before and after).
+    uint32_t ng = 0;
+    auto g_buf = [&]() -> uint8_t* {
+      uint8_t* sb = stage_base + (ng & 3) * (32 * 64);
+      if (lane == 0) bulk_wait_read<3>();
+      __syncwarp();
+      ++ng;
+      return sb;
+    };
+    auto staging_buf = [&]() -> uint8_t* {
+      uint8_t* sb = stage_base + (nstore & 1) * (32 * 128);
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      return sb;
+    };
+    // dH of a finished segment: -coeff * acc (or zeros when nothing was
+    // accumulated) as fp32 32x32 blocks into buffer x.buf.
+    auto flush = [&](const FUnit& x, bool any) {
+      const int row0 = x.r * F::TH + static_cast<int>(rank) * BM + quad * 32;
+      const int row = row0 + lane;
+      const float gc = row < a.M ? -a.coeff[row] : 0.f;
+      auto put = [&](int c, const uint32_t* r) {
+        uint8_t* sb = staging_buf();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 o = (r == nullptr || gc == 0.f)
+                               ? make_float4(0.f, 0.f, 0.f, 0.f)
+                               : make_float4(gc * u2f(r[4 * i]), gc * u2f(r[4 * i + 1]),
+                                             gc * u2f(r[4 * i + 2]), gc * u2f(r[4 * i + 3]));
+          *reinterpret_cast<float4*>(sb + lane * 128 + ((i ^ (lane & 7)) << 4)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (x.buf == 0)
+            tma_store_3d(&tmD0, sb, p * FB_DS + c * 32, row0, 0);
+          else
+            tma_store_3d(&tmD1, sb, p * FB_DS + c * 32, row0 - a.row_rem, x.buf - 1);
+          bulk_commit();
+        }
+        ++nstore;
+      };
+      const int nchunks = min(FB_DS / 32, (a.D - p * FB_DS + 31) / 32);
+      if (lane == 0) bulk_wait_read<0>();  // the G'' slots overlap the dH slots
+      __syncwarp();
+      if (any) {
+        if (!wait_bounded(dh_full, nseg & 1, a.wait_ns, abort_flag)) {
+          ok = false;
+          return;
+        }
+        tc_fence_after();
+        drain_chunks(tmem_dh + lane_addr, nchunks,
+                     [&](int c, const uint32_t (&r)[32]) { put(c, r); });
+        tc_fence_before();
+        if constexpr (C2) mbar_arrive_cluster(dh_empty_leader);
+        else mbar_arrive(dh_empty);
+        ++nseg;
+      } else {
+        for (int c = 0; c < nchunks; ++c) put(c, nullptr);
+      }
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+    };
+    bool seg_any = false, prev_any = false;
+    FUnit prev{};
+    for (int u = 0; u < n_u && ok; ++u) {
+      const FUnit x = fb_unit(a, g, u);
+      if (x.first) seg_any = false;
+      for (int q = 0; q < a.C; ++q) seg_any = seg_any || !fb_skip<C2>(a, x.r, x.j * a.C + q);
+      const int v = x.j * a.C + p;
+      const int slot = slot_of(u, p);
+      const uint32_t fill = static_cast<uint32_t>(u / FB_DEPTH);
+      uint32_t* rdy = &a.ready[slot * 2 + static_cast<int>(rank)];
+      if (!fb_skip<C2>(a, x.r, v)) {
+        const int sb = ns % F::SB;
+        if (!wait_bounded(&s_full[sb], (ns / F::SB) & 1, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // every member is done with this slot's previous fill
+        bool w_ok = true;
+        if (fill >= 1 && lane == 0) {
+          for (int c = 0; c < a.C && w_ok; ++c)
+            w_ok = wait_flag_geq(&a.consumed[slot * a.C + c], fill, a.wait_ns, abort_flag);
+          fence_proxy_async_global();
+        }
+        if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) {
+          ok = false;
+          break;
+        }
+        const int row = x.r * F::TH + static_cast<int>(rank) * BM + rin;
+        const bool live = row < a.M;
+        const int y = live ? a.labels[row] : -1;
+        const float nl = live ? -a.lse[row] * LOG2E : 0.f;
+        const int grow0 = slot * F::TH + static_cast<int>(rank) * BM + quad * 32;
+        drain_chunks(tmem_base + lane_addr + sb * F::BV, F::BV / 32,
+                     [&](int c, const uint32_t (&r)[32]) {
+                       uint32_t pk[16];
+                       grad_chunk(r, v * F::BV + c * 32, y, nl, a.filter_eps, a.V, a.softcap,
+                                  a.inv_cap, 1, pk);
+                       uint8_t* sbuf = g_buf();
+#pragma unroll
+                       for (int i = 0; i < 4; ++i)
+                         *reinterpret_cast<uint4*>(sbuf + lane * 64 +
+                                                   ((i ^ ((lane >> 1) & 3)) << 4)) =
+                             live ? make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2],
+                                               pk[4 * i + 3])
+                                  : make_uint4(0, 0, 0, 0);
+                       fence_proxy_async_smem();
+                       __syncwarp();
+                       if (lane == 0) {
+                         tma_store_2d(&tmGs, sbuf, c * 32, grow0);
+                         bulk_commit();
+                       }
+                     });
+        tc_fence_before();
+        if constexpr (C2) mbar_arrive_cluster(s_empty_leader[sb]);
+        else mbar_arrive(&s_empty[sb]);
+        ++ns;
+        if (lane == 0) {
+          bulk_wait<0>();  // the tile is in global memory (L2)
+          fence_proxy_async_global();
+          red_release_gpu_add(rdy, 1u);
+        }
+      } else if (lane == 0) {
+        red_release_gpu_add(rdy, 1u);
+      }
+      __syncwarp();
+      if (u >= 1 && prev.last) flush(prev, prev_any);
+      prev = x;
+      prev_any = seg_any;
+    }
+    if (ok && n_u > 0) flush(prev, prev_any);
+    if (!ok) {
+      set_status(a.status, ST_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (C2) cluster_sync_all();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    if constexpr (C2) tmem_dealloc2(tmem_base, FB_TMEM_COLS);
+    else tmem_dealloc(tmem_base, FB_TMEM_COLS);
+  }
+}
+
+// dH rows of the remainder row tiles += their partial buffers 1..k-1, in
+// buffer order (k = the number of groups that shared the row tile).  The
+// partial buffers hold rows [row_rem, M).
+__global__ void __launch_bounds__(256) fused_sum_parts_kernel(
+    float4* __restrict__ dh, const float4* __restrict__ parts, FusedArgs a, int TH) {
+  const int D4 = a.D / 4;
+  const int64_t n = static_cast<int64_t>(a.M - a.row_rem) * D4;
+  const int64_t T = static_cast<int64_t>(a.rem) * a.n_rounds;
+  for (int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; t < n;
+       t += int64_t(gridDim.x) * blockDim.x) {
+    const int m = a.row_rem + static_cast<int>(t / D4);
+    const int i = m / TH - a.waves * a.G;
+    const int gf = fb_group_of(static_cast<int64_t>(i) * a.n_rounds, T, a.Gr);
+    const int gl = fb_group_of(static_cast<int64_t>(i + 1) * a.n_rounds - 1, T, a.Gr);
+    const int64_t idx = static_cast<int64_t>(a.row_rem) * D4 + t;
+    float4 s = dh[idx];
+    for (int b = 1; b <= gl - gf; ++b) {
+      const float4 q = parts[static_cast<size_t>(b - 1) * n + t];
+      s.x += q.x;
+      s.y += q.y;
+      s.z += q.z;
+      s.w += q.w;
+    }
+    dh[idx] = s;
+  }
+}
+
+}  // namespace cce

@@ -83,6 +83,12 @@ __host__ __device__ constexpr int smem_bytes() {
 }
 constexpr int SMEM_BYTES = smem_bytes<Mode::kLse>();
 constexpr float LOG2E = 1.4426950408889634f;
+// fp16 G'' (4/8-bit heads) is stored times 2^14 so that the probabilities of
+// a flat softmax over a large vocabulary (about 5e-6 at V = 128k) stay out of
+// fp16 subnormals; |G''| <= 1 keeps it below 16,384.  The dH epilogue takes
+// the factor out again in fp32.  bf16 G'' is stored unscaled.
+constexpr float G16_SCALE = 16384.f;
+constexpr float G16_UNSCALE = 1.f / 16384.f;
 constexpr uint64_t DRAIN_LIMIT_NS = 1000000000ull;
 
 
@@ -279,6 +285,69 @@ __device__ __forceinline__ float tanh_ex2(float x) {
 // planner uses the same expression, so its decisions agree with the filter.
 __device__ __forceinline__ float softmax_p(float s, float nl) {
   return ex2_approx(fmaf(s, LOG2E, nl));
+}
+
+// G'' = softmax - onehot for the 32 vocabulary columns v0..v0+31 of one row
+// (label y, nl = -lse * log2 e), packed to 16 bits (fmt 1: bf16, else fp16).
+// Filter: a non-target term with p < eps is dropped.  Columns past V give 0.
+// fp16 values are scaled by G16_SCALE.
+// With a softcap the logits are cap * tanh(s / cap) and every term carries
+// 1 - tanh^2(s / cap).  Called by a whole warp (the fast-path test is
+// warp-uniform).  (ORPO design 0.0.6, fused-head spec, "Backward".)
+__device__ __forceinline__ void grad_chunk(const uint32_t (&r)[32], int v0, int y, float nl,
+                                           float eps, int V, float softcap, float inv_cap,
+                                           int fmt, uint32_t (&pk)[16]) {
+  const float gs = fmt == 1 ? 1.f : G16_SCALE;
+  const int tt = y - v0;
+  // Warp-uniform: a chunk inside the vocab with no label of this warp takes
+  // the short path (one FFMA + one ex2 per logit).
+  const bool slow =
+      (v0 + 32 > V) || __any_sync(0xffffffffu, static_cast<unsigned>(tt) < 32u);
+  if (softcap > 0.f) {
+    // capped logits; each term carries 1 - tanh^2(s / cap)
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      float g2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int v = v0 + j + h;
+        const float th = tanh_ex2(u2f(r[j + h]) * inv_cap);
+        float p = softmax_p(softcap * th, nl);
+        const bool tgt = (v == y);
+        if (p < eps && !tgt) p = 0.f;
+        g2[h] = v < V ? (tgt ? p - 1.f : p) * (1.f - th * th) : 0.f;
+      }
+      pk[j >> 1] = pack2(g2[0] * gs, g2[1] * gs, fmt);
+    }
+  } else if (!slow) {
+    if (eps > 0.f) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        float p0 = softmax_p(u2f(r[j]), nl), p1 = softmax_p(u2f(r[j + 1]), nl);
+        p0 = p0 < eps ? 0.f : p0;
+        p1 = p1 < eps ? 0.f : p1;
+        pk[j >> 1] = pack2(p0 * gs, p1 * gs, fmt);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; j += 2)
+        pk[j >> 1] = pack2(softmax_p(u2f(r[j]), nl) * gs, softmax_p(u2f(r[j + 1]), nl) * gs, fmt);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      float g2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int v = v0 + j + h;
+        float p = softmax_p(u2f(r[j + h]), nl);
+        const bool tgt = (v == y);
+        if (p < eps && !tgt) p = 0.f;
+        g2[h] = v < V ? (tgt ? p - 1.f : p) : 0.f;
+      }
+      pk[j >> 1] = pack2(g2[0] * gs, g2[1] * gs, fmt);
+    }
+  }
 }
 
 // Drains `nchunks` 32-column chunks of this warp's accumulator lanes through
@@ -796,58 +865,8 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         const float eps = a.filter_eps;
         const int vbase = a.b_row0 + ct * BN;
         drain_chunks(taddr, BN / 32, [&](int c, const uint32_t (&r)[32]) {
-          const int v0 = vbase + c * 32;
-          const int tt = y - v0;
-          // Warp-uniform: a chunk inside the vocab with no label of this warp
-          // takes the short path (one FFMA + one ex2 per logit).
-          const bool slow = (v0 + 32 > a.V) ||
-                            __any_sync(0xffffffffu, static_cast<unsigned>(tt) < 32u);
           uint32_t pk[16];
-          if (a.softcap > 0.f) {
-            // capped logits; each term carries 1 - tanh^2(s / cap)
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              float g2[2];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int v = v0 + j + h;
-                const float th = tanh_ex2(u2f(r[j + h]) * a.inv_cap);
-                float p = softmax_p(a.softcap * th, nl);
-                const bool tgt = (v == y);
-                if (p < eps && !tgt) p = 0.f;
-                g2[h] = v < a.V ? (tgt ? p - 1.f : p) * (1.f - th * th) : 0.f;
-              }
-              pk[j >> 1] = pack2(g2[0], g2[1], a.fmt);
-            }
-          } else if (!slow) {
-            if (eps > 0.f) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 2) {
-                float p0 = softmax_p(u2f(r[j]), nl), p1 = softmax_p(u2f(r[j + 1]), nl);
-                p0 = p0 < eps ? 0.f : p0;
-                p1 = p1 < eps ? 0.f : p1;
-                pk[j >> 1] = pack2(p0, p1, a.fmt);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; j += 2)
-                pk[j >> 1] = pack2(softmax_p(u2f(r[j]), nl), softmax_p(u2f(r[j + 1]), nl), a.fmt);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              float g2[2];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int v = v0 + j + h;
-                float p = softmax_p(u2f(r[j + h]), nl);
-                const bool tgt = (v == y);
-                if (p < eps && !tgt) p = 0.f;
-                g2[h] = v < a.V ? (tgt ? p - 1.f : p) : 0.f;
-              }
-              pk[j >> 1] = pack2(g2[0], g2[1], a.fmt);
-            }
-          }
+          grad_chunk(r, vbase + c * 32, y, nl, eps, a.V, a.softcap, a.inv_cap, a.fmt, pk);
           // Stage the 32x32 block in shared memory (64-byte swizzle: 16-byte
           // chunk i of row r sits at chunk i ^ ((r >> 1) & 3)) and let TMA
           // write it; rows past M are clipped by the tensor map.
@@ -870,7 +889,9 @@ __global__ void __launch_bounds__(QB ? NUM_THREADS_Q4 : NUM_THREADS, 1)
         if constexpr (C2) mbar_arrive_cluster(acc_empty_leader[b]);
         else mbar_arrive(&acc_empty[b]);
       } else {  // kDh: dH (+)= -coeff * (G'' . W);  kDw: dW[chunk] = -(G''^T . coeff*H)
-        const float g = MODE == Mode::kDw ? -1.f : (live ? -a.coeff[row] : 0.f);
+        const float g = MODE == Mode::kDw ? -1.f
+                        : live ? -a.coeff[row] * (a.fmt == 1 ? 1.f : G16_UNSCALE)
+                               : 0.f;
         const int dbase = ct * BN;
         const int nchunks = min(BN / 32, (a.D - dbase) / 32);
         const CUtensorMap* dmap = tc.s == 0 ? &tmC : &tmC2;

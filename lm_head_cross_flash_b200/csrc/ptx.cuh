@@ -18,6 +18,7 @@ enum : uint32_t {
   ST_TIMEOUT = 1u << 1,  // a bounded wait ran out
   ST_EMPTY = 1u << 2,    // an empty chosen or rejected segment
   ST_DOMAIN = 1u << 3,   // a mean log-prob >= 0 (log1mexp undefined)
+  ST_FP16 = 1u << 4,     // a value the fp16 path of 4/8-bit heads cannot hold
 };
 
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t bit) {
@@ -381,6 +382,45 @@ __device__ __forceinline__ void umma_commit2_mc(uint64_t* bar, uint16_t mask) {
       "[%0], %1;" ::"r"(smem_u32(bar)),
       "h"(mask)
       : "memory");
+}
+
+// ------------------------------------------- flags between CTAs (gpu scope) --
+// A counter in global memory that one CTA advances and others wait on.  The
+// data the counter guards moves through the async proxy (TMA), so both sides
+// put a proxy fence between the data and the flag.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// A store that orders nothing before it: enough to announce that a tile this
+// thread saw land (through an mbarrier) may be overwritten.
+__device__ __forceinline__ void st_relaxed_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's async-proxy accesses of global memory (TMA loads and
+// stores) against its generic-proxy accesses, in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Waits until *p >= target.  False when `limit_ns` elapsed or `*abort`
+// became non-zero first.
+__device__ __forceinline__ bool wait_flag_geq(const uint32_t* p, uint32_t target,
+                                              uint64_t limit_ns, const volatile int* abort) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
 }
 
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32).

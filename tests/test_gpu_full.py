@@ -3,13 +3,11 @@
 * tiny fp32 pair and small bf16 pair: the whole pass (logp, lse, loss,
   cotangent, dH) against the oracle on every row;
 * long bf16 pairs and the long-context 4-bit pair, through the real pass
-  (forward, ORPO epilogue, cotangent, backward): logp / lse on stratified
-  sampled rows (one in every 128-row tile, the segment edges, vocab-tail
-  labels, 200 uniform rows); the loss block and the whole cotangent vector
-  against the oracle's float64 epilogue applied to the device's logp vector
-  once the sampled rows pass (the oracle cannot afford every row of these
-  sizes, so this is a partial dependence on the device's logp); dH on the
-  sampled rows under those coefficients, against the UNFILTERED oracle;
+  (forward, ORPO epilogue, cotangent, backward): logp / lse on every row,
+  the loss and the cotangent against the oracle's own (its float64 forward
+  runs over every row); dH on stratified rows (one in every 128-row tile,
+  the segment edges, vocab-tail labels, 200 uniform rows) under the
+  oracle's cotangent, against the UNFILTERED oracle;
 * the same sizes under a seeded non-uniform cotangent; block skipping must
   not change a single bit of dH.
 """
@@ -50,36 +48,41 @@ def test_full_pass_every_row(cfg):
 
 
 @pytest.mark.parametrize("cfg", [2, 3, 4])
-def test_long_pair_real_pass_sampled(cfg):
+def test_long_pair_real_pass(cfg):
+    """The real pass at full size.  The oracle's float64 forward runs over
+    EVERY row (about 20 s at the long pair, 80 s at the long context on 16
+    host cores), so logp and lse are compared on every row and the loss and
+    the cotangent are the oracle's own; dH is compared on stratified rows
+    (one in every 128-row tile, segment edges, vocab-tail labels, 200
+    uniform rows) under the oracle's cotangent, against the UNFILTERED
+    oracle."""
     wl = S.make_workload(cfg)
     _, _, _, buf, st = run_pass(wl)
     assert st == 0
-    rows = S.sample_rows(wl, n_uniform=200, per_tile=True, edge=8)
-    assert len(np.unique(rows // 128)) == (wl.M + 127) // 128
     W = oracle_W(wl)
     L = oracle_layout(wl)
-    logp, lse, _ = O.head_forward(wl.H, W, wl.labels, rows=rows)
+    logp, lse, _ = O.head_forward(wl.H, W, wl.labels, block=256)
     d_logp = buf.logp.cpu().numpy()
-    assert np.max(np.abs(d_logp[rows] - logp)) <= TOL_LOGP
-    assert np.max(np.abs(buf.lse.cpu().numpy()[rows] - lse)) <= TOL_LOGP
+    e_logp = np.max(np.abs(d_logp - logp))
+    assert e_logp <= TOL_LOGP
+    assert np.max(np.abs(buf.lse.cpu().numpy() - lse)) <= TOL_LOGP
     assert np.all(d_logp[wl.labels < 0] == 0.0)
-    # the epilogue in float64 on the device's logp vector
-    o = O.orpo_loss_from_logps(d_logp, wl.labels, L, wl.lam, wl.scope)
+    o = O.orpo_loss_from_logps(logp, wl.labels, L, wl.lam, wl.scope)
     out8 = buf.out8.cpu().numpy()
-    want8 = np.array(o.as8())
-    assert abs(out8[0] - o.loss) <= TOL_LOSS * abs(o.loss)
-    assert np.allclose(out8, want8, rtol=1e-9, atol=1e-12), (out8, want8)
-    g = O.orpo_grad_coeffs(d_logp, wl.labels, L, wl.lam, wl.scope)
+    e_loss = abs(out8[0] - o.loss) / abs(o.loss)
+    assert e_loss <= TOL_LOSS
+    g = O.orpo_grad_coeffs(logp, wl.labels, L, wl.lam, wl.scope)
     d_coeff = buf.coeff.cpu().numpy().astype(np.float64)
-    assert np.max(np.abs(d_coeff - g)) <= 1e-6 * np.max(np.abs(g))
+    assert np.max(np.abs(d_coeff - g)) <= TOL_LOSS * np.max(np.abs(g))
     assert np.all(d_coeff[wl.labels < 0] == 0.0)
-    # dH under the real cotangent, against the unfiltered oracle
-    want = O.head_dh(wl.H, W, wl.labels, g, lse, rows=rows)
+    rows = S.sample_rows(wl, n_uniform=200, per_tile=True, edge=8)
+    assert len(np.unique(rows // 128)) == (wl.M + 127) // 128
+    want = O.head_dh(wl.H, W, wl.labels, g, lse[rows], rows=rows)
     got = buf.dH.cpu().numpy()[rows]
     err = rel_fro(got, want)
-    print(f"workload {cfg}: {len(rows)} rows, max|dlogp| "
-          f"{np.max(np.abs(d_logp[rows] - logp)):.2e}, loss {out8[0]:.9f}, "
-          f"sampled dH rel err {err:.3e}; skip tiles {buf.skip.cpu().tolist()}")
+    print(f"workload {cfg}: max|dlogp| {e_logp:.2e} over {wl.M} rows, loss {out8[0]:.9f} "
+          f"(rel err {e_loss:.2e}), dH rel err {err:.3e} on {len(rows)} rows; "
+          f"skip tiles {buf.skip.cpu().tolist()}")
     assert err <= TOL_DH
     assert np.all(got[wl.labels[rows] < 0] == 0.0)
 

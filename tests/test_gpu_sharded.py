@@ -94,3 +94,49 @@ def test_row_sharded_pair_matches_one_process():
         assert err < 1e-5, (rank, err)
     # every row of the pair is covered once
     assert sorted(np.concatenate([g[2] for g in got]).tolist()) == list(range(wl.M))
+
+
+def _nccl_worker(port, q):
+    """One rank of an NCCL process group on GPU 0: the device all-reduce of
+    the sharded pass runs on the caller's (non-default) stream."""
+    import datetime
+
+    import torch.distributed as dist
+    try:
+        torch.cuda.set_device(0)
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=60),
+                                device_id=torch.device("cuda", 0))
+        assert dist.get_backend() == "nccl"
+        wl = S.make_custom(2, M_split=SPLIT, D=D, V=V)
+        H, head, labels = cce.upload_workload(wl, "cuda")
+        ref = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head)
+        cce.orpo_head_pass(H, head, labels, wl.layout_tuple, wl.lam, wl.scope, 0.0, False, ref)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        buf = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, cce.h_dtype(H), head)
+        with torch.cuda.stream(side):
+            cce.orpo_head_pass_sharded(H, head, labels, wl.layout_tuple, wl.lam, wl.scope, 0.0,
+                                       False, buf, stream=side)
+        side.synchronize()
+        same = [torch.equal(getattr(buf, k), getattr(ref, k))
+                for k in ("logp", "lse", "out8", "coeff", "dH")]
+        q.put((cce.cce_device_status(buf.ws), same))
+        dist.destroy_process_group()
+    except Exception as e:  # pragma: no cover - reported to the parent
+        q.put((repr(e), None))
+
+
+def test_row_sharded_pair_nccl_branch_one_rank():
+    """The NCCL branch of the sharded pass (device all-reduce of the six
+    segment sums, ordered on the caller's stream) with a one-rank group on
+    one GPU: the same bits as the unsharded pass."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_nccl_worker, args=(_free_port(), q))
+    p.start()
+    st, same = q.get(timeout=300)
+    p.join(timeout=60)
+    assert st == 0, st
+    assert all(same), same

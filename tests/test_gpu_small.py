@@ -369,13 +369,21 @@ def test_trainable_head_dw(cfg, split, D, V, cap, eps):
     g[: split[0] // 2] = 0.0            # a run of zero-cotangent rows
     coeff = torch.from_numpy(g).cuda()
     dH1 = torch.empty(wl.M, wl.D, **f)
-    cce.cce_backward_dh(H, head, labels, lse, coeff, eps, None, dH1, None, ws)
+    dH0 = torch.empty(wl.M, wl.D, **f)
+    cce.cce_backward_dh(H, head, labels, lse, coeff, eps, None, dH0, None, ws)
+    cce.cce_set_backward_mode(2)   # the two GEMMs per chunk, as the dW call runs them
+    try:
+        cce.cce_backward_dh(H, head, labels, lse, coeff, eps, None, dH1, None, ws)
+    finally:
+        cce.cce_set_backward_mode(0)
     dH2 = torch.empty(wl.M, wl.D, **f)
     dW = torch.full((wl.V, wl.D), float("nan"), **f)
     cce.cce_backward_dh_dw(H, head, labels, lse, coeff, eps, None, dH2, dW, None, ws)
     torch.cuda.synchronize()
     assert cce.cce_device_status(ws) == 0
     assert torch.equal(dH1, dH2)
+    # the default backward (fused for dense bf16 heads) agrees to accumulation order
+    assert rel_fro(dH0.cpu().numpy(), dH1.cpu().numpy()) <= 1e-5
     W = oracle_W(wl)
     olse = O.head_forward(wl.H, W, wl.labels, softcap=cap)[1]
     want = O.head_dw(wl.H, W, wl.labels, g, olse, filter_eps=eps, softcap=cap)

@@ -6,6 +6,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from lm_head_cross_flash_b200 import build, cce
@@ -57,14 +59,25 @@ def _head(V=1000, D=128, dtype=cce.CCE_BF16, w=4096, fmt=cce.CCE_W_DENSE):
 
 def test_workspace_sizes_monotonic(lib):
     h = _head()
-    sz = [lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h)) for M in (1, 100, 1000, 5000)]
-    assert all(a <= b for a, b in zip(sz, sz[1:])) and sz[0] > 0
-    lo = lib.cce_workspace_min_bytes(1000, cce.CCE_BF16, ctypes.byref(h))
-    assert 0 < lo <= sz[2]
     big = _head(V=262144, D=2048)
-    # default workspace at the long pair: a 1 GiB G'' chunk and the K-split buffer,
-    # far below the 8.6 GB of fp32 logits it replaces
-    assert lib.cce_workspace_bytes(8192, cce.CCE_BF16, ctypes.byref(big)) < 1280 << 20
+    cce.cce_set_backward_mode(2)   # the two-GEMM backward's G'' chunk
+    try:
+        sz = [lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h))
+              for M in (1, 100, 1000, 5000)]
+        assert all(a <= b for a, b in zip(sz, sz[1:])) and sz[0] > 0
+        lo = lib.cce_workspace_min_bytes(1000, cce.CCE_BF16, ctypes.byref(h))
+        assert 0 < lo <= sz[2]
+        # default at the long pair: a 1 GiB G'' chunk and the K-split buffer,
+        # far below the 8.6 GB of fp32 logits it replaces
+        two = lib.cce_workspace_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
+        assert two < 1280 << 20
+    finally:
+        cce.cce_set_backward_mode(0)
+    # the fused backward needs no G'' chunk: the forward's statistics (67 MB
+    # at the long pair) bound it, plus the exchange ring and partial dH rows
+    fused = lib.cce_workspace_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
+    fwd_stats = 2 * 1024 * 8192 * 4
+    assert fwd_stats <= fused < 160 << 20 and fused < two / 6
     assert lib.cce_workspace_bytes(0, cce.CCE_BF16, ctypes.byref(h)) == 0
     bad = _head(D=96)
     assert lib.cce_workspace_bytes(10, cce.CCE_BF16, ctypes.byref(bad)) == 0
@@ -148,7 +161,14 @@ def test_objective_rejects_bad_arguments(lib):
     assert lib.pref_loss_from_logps(a, a, 20, lay, None, a, a, 4096, None) == 1
 
 
-def test_query_plan_chunks_splits_and_staging(lib):
+@pytest.fixture
+def two_gemm_backward():
+    cce.cce_set_backward_mode(2)
+    yield
+    cce.cce_set_backward_mode(0)
+
+
+def test_query_plan_chunks_splits_and_staging(lib, two_gemm_backward):
     """The host-side planner: forward/backward chunking, the dH K split,
     CTA pairs and staged dequantisation follow the workspace and M."""
     big = _head(V=262144, D=2048)
@@ -220,9 +240,17 @@ from hypothesis import given, settings, strategies as st
        frac=st.floats(0.0, 2.0))
 def test_planner_invariants(lib, M, V, D64, fmt, frac):
     """For any shape and any workspace between the minimum and twice the
-    default, the planner's choices are consistent: both calls fit, chunks are
-    whole vocab tiles, K splits stay in range, staging and CTA pairs follow
-    their documented thresholds."""
+    default, the two-GEMM backward planner's choices are consistent: both
+    calls fit, chunks are whole vocab tiles, K splits stay in range, staging
+    and CTA pairs follow their documented thresholds."""
+    cce.cce_set_backward_mode(2)
+    try:
+        _planner_invariants(lib, M, V, D64, fmt, frac)
+    finally:
+        cce.cce_set_backward_mode(0)
+
+
+def _planner_invariants(lib, M, V, D64, fmt, frac):
     D = 64 * D64
     h = cce._Head(fmt, cce.CCE_BF16, V, D, 4096, 4096 if fmt else None, 4096 if fmt else None)
     lo = lib.cce_workspace_min_bytes(M, cce.CCE_BF16, ctypes.byref(h))
@@ -251,3 +279,104 @@ def test_planner_invariants(lib, M, V, D64, fmt, frac):
     # the default workspace never needs a narrower chunk than the minimum one
     pd = cce.cce_query_plan(M, cce.CCE_BF16, h, hi)
     assert pd["bwd_chunk"] >= cce.cce_query_plan(M, cce.CCE_BF16, h, lo)["bwd_chunk"]
+
+
+# --------------------------------------------------------------------------
+# fused backward: plan and schedule (host-only)
+# --------------------------------------------------------------------------
+
+def test_fused_plan_choice(lib):
+    """Dense bf16 heads take the fused backward when the workspace holds its
+    layout; fp32 and 4-bit heads, a workspace below it, and mode 2 take the
+    two GEMMs.  Groups of ceil(D/256) members fill the resident units (74
+    CTA pairs or 148 CTAs on a B200)."""
+    big = _head(V=262144, D=2048)
+    ws = lib.cce_workspace_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
+    p = cce.cce_query_plan(8192, cce.CCE_BF16, big, ws)
+    assert p["bwd_ok"] and p["bwd_fused"] and p["bwd_chunk"] == 0 and p["bwd_cta_pairs"]
+    assert p["bwd_fused_members"] == 8 and p["bwd_fused_groups"] == 74 // 8
+    assert p["bwd_fused_buffers"] >= 2   # 32 pair tiles over 9 groups leave a remainder
+    small = cce.cce_query_plan(64, cce.CCE_BF16, big,
+                               lib.cce_workspace_bytes(64, cce.CCE_BF16, ctypes.byref(big)))
+    assert small["bwd_fused"] and not small["bwd_cta_pairs"]
+    assert small["bwd_fused_groups"] == 148 // 8
+    lo = lib.cce_workspace_min_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
+    if lo < ws:
+        assert not cce.cce_query_plan(8192, cce.CCE_BF16, big, lo)["bwd_fused"]
+    c1 = _head(V=73440, D=1536)
+    p1 = cce.cce_query_plan(2048, cce.CCE_BF16, c1,
+                            lib.cce_workspace_bytes(2048, cce.CCE_BF16, ctypes.byref(c1)))
+    assert p1["bwd_fused"] and p1["bwd_fused_members"] == 6 and p1["bwd_fused_groups"] == 12
+    f32 = cce._Head(cce.CCE_W_DENSE, cce.CCE_F32, 4096, 256, 4096, None, None)
+    pf = cce.cce_query_plan(256, cce.CCE_F32, f32,
+                            lib.cce_workspace_bytes(256, cce.CCE_F32, ctypes.byref(f32)))
+    assert pf["bwd_ok"] and not pf["bwd_fused"]
+    q4 = cce._Head(cce.CCE_W_AFFINE_Q4_G64, cce.CCE_BF16, 128256, 4096, 4096, 4096, 4096)
+    pq = cce.cce_query_plan(4096, cce.CCE_BF16, q4,
+                            lib.cce_workspace_bytes(4096, cce.CCE_BF16, ctypes.byref(q4)))
+    assert pq["bwd_ok"] and not pq["bwd_fused"]
+    assert cce.cce_query_fused_schedule(4096, cce.CCE_BF16, q4) is None
+    cce.cce_set_backward_mode(2)
+    try:
+        assert not cce.cce_query_plan(8192, cce.CCE_BF16, big, ws)["bwd_fused"]
+    finally:
+        cce.cce_set_backward_mode(0)
+
+
+def _check_schedule(M, V, D, sched, plan):
+    """Every (row tile, round) unit exactly once; a group's segments are runs
+    of consecutive rounds on one row tile, flagged first/last; the segments
+    of a row tile use dH buffers 0..k-1 once each, k <= the planned count;
+    in the waves, all groups run the same round at the same step."""
+    pairs = bool(plan["bwd_cta_pairs"])
+    TH, BV = (256, 256) if pairs else (128, 128)
+    C = -(-D // 256)
+    n_rt, n_rounds = -(-M // TH), -(-(-(-V // BV)) // C)
+    G = plan["bwd_fused_groups"]
+    assert plan["bwd_fused_members"] == C
+    assert len(sched) == n_rt * n_rounds
+    keys = sched[:, 1].astype(np.int64) * n_rounds + sched[:, 2]
+    assert np.array_equal(np.sort(keys), np.arange(n_rt * n_rounds))
+    bufs = {}
+    for g in range(G):
+        s = sched[sched[:, 0] == g]
+        k = 0
+        while k < len(s):
+            assert s[k, 3] == 1, (g, k)              # a segment opens
+            e = k
+            while s[e, 4] == 0:
+                e += 1
+                assert s[e, 1] == s[k, 1] and s[e, 2] == s[e - 1, 2] + 1 and s[e, 3] == 0
+            assert len(set(s[k:e + 1, 5])) == 1
+            bufs.setdefault(int(s[k, 1]), []).append(int(s[k, 5]))
+            k = e + 1
+        waves = n_rt // G
+        full = s[: waves * n_rounds]
+        assert np.array_equal(full[:, 2], np.tile(np.arange(n_rounds), waves))
+        assert np.array_equal(full[:, 1], np.repeat(np.arange(waves) * G + g, n_rounds))
+    for r, b in bufs.items():
+        assert sorted(b) == list(range(len(b))), (r, b)
+        assert len(b) <= plan["bwd_fused_buffers"]
+    assert max(len(b) for b in bufs.values()) == plan["bwd_fused_buffers"]
+
+
+@pytest.mark.parametrize("M,V,D", [(8192, 262144, 2048), (2048, 73440, 1536), (64, 262144, 2048),
+                                   (1, 300, 64), (300, 1000, 320), (32768, 128256, 4096),
+                                   (129, 4097, 256), (5000, 3000, 2048)])
+def test_fused_schedule_covers_every_unit_once(lib, M, V, D):
+    h = _head(V=V, D=D)
+    plan = cce.cce_query_plan(M, cce.CCE_BF16, h,
+                              lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h)))
+    assert plan["bwd_fused"]
+    _check_schedule(M, V, D, cce.cce_query_fused_schedule(M, cce.CCE_BF16, h), plan)
+
+
+@settings(max_examples=60, deadline=None)
+@given(M=st.integers(1, 20000), V=st.integers(1, 70000), D64=st.integers(1, 64))
+def test_fused_schedule_property(lib, M, V, D64):
+    D = 64 * D64
+    h = _head(V=V, D=D)
+    plan = cce.cce_query_plan(M, cce.CCE_BF16, h,
+                              lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h)))
+    assert plan["bwd_ok"] and plan["bwd_fused"]
+    _check_schedule(M, V, D, cce.cce_query_fused_schedule(M, cce.CCE_BF16, h), plan)
