@@ -461,7 +461,7 @@ def run_ours(args):
     launches_per_step = dom_n / args.steps
     peak_s = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_b = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    pk = choose_peak(peaks, peaks_src, clk, ms_max * args.steps / 1e3)
+    pk = choose_peak(peaks, peaks_src, clk, ms_max / 1e3)  # ms_max: the whole timed region
     if dom in per_kind_flops:
         achieved = per_kind_flops[dom] * args.steps / (dom_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": pk["peak"],

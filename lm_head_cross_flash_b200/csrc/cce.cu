@@ -218,7 +218,7 @@ int max_fused_pairs() {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, fused_bwd_kernel<true>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, fused_bwd_kernel<true, 128>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -249,14 +249,16 @@ cce_status device_info(int* sms) {
     CCE_SET_SMEM2(Mode::kLse) CCE_SET_SMEM2(Mode::kGrad) CCE_SET_SMEM2(Mode::kDh)
 #undef CCE_SET_SMEM2
     ok = ok &&
-         cudaFuncSetAttribute(fused_bwd_kernel<true>, attr, FusedCfg<true>::SMEM) == cudaSuccess &&
-         cudaFuncSetAttribute(fused_bwd_kernel<false>, attr, FusedCfg<false>::SMEM) == cudaSuccess;
+         cudaFuncSetAttribute(fused_bwd_kernel<true, 128>, attr, FusedCfg<true>::SMEM) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(fused_bwd_kernel<false, 128>, attr, FusedCfg<false, 128>::SMEM) ==
+             cudaSuccess;
     if (ok) {
       d.pairs = std::min(max_pairs_of<Mode::kLse>(),
                          std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
       d.fused_pairs = max_fused_pairs();
       int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_bwd_kernel<false>,
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_bwd_kernel<false, 128>,
                                                         NUM_THREADS, FusedCfg<false>::SMEM) !=
           cudaSuccess) {
         cudaGetLastError();
@@ -697,6 +699,7 @@ int fused_resident(bool c2) {
 struct FusedPlan {
   bool ok = false;
   bool c2 = false;
+  int bv = 256;  // vocab columns of an S tile
   FusedArgs a{};
   int nbuf = 1;
   int64_t ring_rows = 0;
@@ -709,8 +712,10 @@ FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
   const int64_t n128 = ceil_div(M, BM);
   f.c2 = g_pairs.load() != 0 && n128 >= 2;
   const int TH = f.c2 ? FusedCfg<true>::TH : FusedCfg<false>::TH;
-  const int BV = f.c2 ? FusedCfg<true>::BV : FusedCfg<false>::BV;
+  f.bv = f.c2 ? FusedCfg<true>::BV : FusedCfg<false>::BV;
+  const int BV = f.bv;
   const int C = int(ceil_div(W->D, FB_DS));
+  if (C > 32) return f;  // skip masks hold 32 members
   const int G = fused_resident(f.c2) / C;
   if (G < 1) return f;
   FusedArgs& a = f.a;
@@ -727,19 +732,31 @@ FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
   a.waves = a.n_rt / G;
   a.rem = a.n_rt % G;
   a.row_rem = int(std::min<int64_t>(M, int64_t(a.waves) * G * TH));
+  // remainder: bands of rem groups sharing rounds, then the leftover
   const int64_t T = int64_t(a.rem) * a.n_rounds;
-  a.Gr = int(std::min<int64_t>(G, T));
-  for (int i = 0; i < a.rem; ++i) {
-    const int gf = fb_group_of(int64_t(i) * a.n_rounds, T, a.Gr);
-    const int gl = fb_group_of(int64_t(i + 1) * a.n_rounds - 1, T, a.Gr);
-    f.nbuf = std::max(f.nbuf, gl - gf + 1);
+  a.nb = a.bw = a.lr = a.r0 = a.rl = 0;
+  if (a.rem > 0) {
+    if (T >= G) {
+      a.nb = G / a.rem;
+      const int r = G % a.rem;
+      if (r > 0) {
+        a.bw = int(T / G);
+        a.lr = r;
+        a.r0 = a.nb * a.bw;
+        a.rl = a.n_rounds - a.r0;
+      }
+    } else {
+      a.lr = int(T);
+      a.rl = a.n_rounds;
+    }
   }
+  for (int i = 0; i < a.rem; ++i) f.nbuf = std::max(f.nbuf, fb_slices(a, i));
   f.ring_rows = int64_t(G) * FB_DEPTH * C * TH;
   const int64_t cols = ceil_div(W->V, BN);
   size_t o = kStatusBytes;
   f.tile_skip = o; o += align_up(size_t(n128) * cols);
   f.row_skip = o; o += align_up(size_t(n128));
-  f.flags = o; o += align_up(size_t(G) * FB_DEPTH * C * (2 + C) * 4);
+  f.flags = o; o += align_up((size_t(G) * FB_DEPTH * C * (2 + C) + G) * 4);
   f.ring = o; o += align_up(size_t(f.ring_rows) * BV * 2);
   f.parts = o; o += align_up(size_t(f.nbuf - 1) * (M - a.row_rem) * W->D * 4);
   // the forward's region shares the same bytes (it is dead by the backward)
@@ -770,13 +787,14 @@ cce_status fused_backward(const FusedPlan& fp, const void* H, const cce_head* W,
         p.n_rt128, filter_eps, tile_skip, row_skip, skip_stats);
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
   }
-  const size_t flag_bytes = size_t(p.G) * FB_DEPTH * p.C * (2 + p.C) * 4;
+  const size_t flag_bytes = (size_t(p.G) * FB_DEPTH * p.C * (2 + p.C) + p.G) * 4;
   if (cudaMemsetAsync(wsc + fp.flags, 0, flag_bytes, st) != cudaSuccess) return CCE_ERR_CUDA;
 
-  const int BV = fp.c2 ? FusedCfg<true>::BV : FusedCfg<false>::BV;
+  const int BV = fp.bv;
   void* ring = wsc + fp.ring;
   CUtensorMap mh, mwk, mwm, mgl, mgs, md0, md1;
-  if (!make_map(&mh, H, true, D, M, D, BK, BM) || !make_map(&mwk, W->w, true, D, V, D, BK, 128) ||
+  if (!make_map(&mh, H, true, D, M, D, BK, BM) ||
+      !make_map(&mwk, W->w, true, D, V, D, BK, fp.c2 ? 128 : BV) ||
       !make_map(&mwm, W->w, true, D, V, D, 64, BK) ||
       !make_map(&mgl, ring, true, BV, fp.ring_rows, BV, BK, BM))
     return CCE_ERR_CUDA;
@@ -810,13 +828,15 @@ cce_status fused_backward(const FusedPlan& fp, const void* H, const cce_head* W,
   a.lse = lse;
   a.coeff = coeff;
   a.filter_eps = filter_eps;
-  a.tile_skip = tile_skip;
+  // the plan marks vocab blocks only with block skip (blockmax and a filter)
+  a.tile_skip = (filter_eps > 0.f && blockmax != nullptr) ? tile_skip : nullptr;
   a.skip_ld = int(cols);
   a.row_skip = row_skip;
   a.softcap = W->softcap;
   a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
   a.ready = reinterpret_cast<uint32_t*>(wsc + fp.flags);
   a.consumed = a.ready + size_t(p.G) * FB_DEPTH * p.C * 2;
+  a.progress = a.consumed + size_t(p.G) * FB_DEPTH * p.C * p.C;
   {
     ProfScope ps(PK_FUSED, st);
     const int members = a.G * a.C;
@@ -833,15 +853,15 @@ cce_status fused_backward(const FusedPlan& fp, const void* H, const cce_head* W,
       at[0].val.clusterDim.z = 1;
       cfg.attrs = at;
       cfg.numAttrs = 1;
-      if (cudaLaunchKernelEx(&cfg, fused_bwd_kernel<true>, mh, mwk, mwm, mgl, mgs, md0, md1, a) !=
-          cudaSuccess)
+      if (cudaLaunchKernelEx(&cfg, fused_bwd_kernel<true, 128>, mh, mwk, mwm, mgl, mgs, md0, md1,
+                             a) != cudaSuccess)
         return CCE_ERR_CUDA;
     } else {
       cfg.gridDim = dim3(members);
-      cfg.dynamicSmemBytes = FusedCfg<false>::SMEM;
       cfg.numAttrs = 0;
-      if (cudaLaunchKernelEx(&cfg, fused_bwd_kernel<false>, mh, mwk, mwm, mgl, mgs, md0, md1,
-                             a) != cudaSuccess)
+      cfg.dynamicSmemBytes = FusedCfg<false, 128>::SMEM;
+      if (cudaLaunchKernelEx(&cfg, fused_bwd_kernel<false, 128>, mh, mwk, mwm, mgl, mgs, md0,
+                             md1, a) != cudaSuccess)
         return CCE_ERR_CUDA;
     }
   }

@@ -32,9 +32,8 @@
 // tcgen05.mma.cta_group::2 (S: 256 x 256 vocab; dH: 256 x 256 d-columns),
 // each CTA loading its own 128 rows of A and half of B (as in gemm_tc.cuh).
 // C2 = false: single CTAs on 128-row tiles with 128-column vocab tiles and a
-// double-buffered S accumulator (used for at most one row tile, where the
-// path streams W from HBM and a narrower vocab tile halves the W held in L2
-// between a round's two reads).
+// double-buffered S accumulator (at most one row tile of 128, or CTA pairs
+// switched off).
 //
 // The exchange.  Ring slot (group, unit % DEPTH, member) is filled once per
 // DEPTH units.  Publisher: each epilogue warp waits until every member has
@@ -44,19 +43,21 @@
 // the producer warp waits for ready >= 4 (fill + 1) with acquire semantics,
 // fences the async proxy and loads the tile by TMA; once the tile has
 // landed (the leader's full barrier counts both CTAs of a pair) the MMA warp
-// stores consumed = fill + 1 (relaxed: the tile's reads are complete).  A tile that block skip (or the end of the
-// vocabulary) removes is neither computed nor loaded, but still advances
-// both counters, so the counts stay aligned.  Every wait is bounded; all
+// stores consumed = fill + 1 (relaxed: the tile's reads are complete).  A
+// tile that block skip (or the end of the vocabulary) removes is neither
+// computed nor loaded, but still advances both counters, so the counts stay
+// aligned.  Every wait is bounded; all
 // CTAs of the grid are resident at once (at most one CTA per SM, grid no
 // larger than the resident count).
 //
 // Partition of the work.  A unit is (row tile r, round j).  G groups take
 // the row tiles in waves (group g: r = w G + g), so that all groups sweep
 // the same rounds of W at the same time and W streams from HBM about once
-// per wave.  The rem = n_rt mod G row tiles left over are cut into
-// contiguous ranges of units, one per group: a row tile split between k
-// groups gives k partial dH slices (buffer 0 is dH itself, buffers 1.. are
-// in the workspace) that fused_sum_parts_kernel adds in a fixed order.
+// per wave.  The rem = n_rt mod G row tiles left over are cut into bands of
+// rounds (fb_unit) so that concurrent groups still share rounds: a row tile
+// split between k groups gives k partial dH slices (buffer 0 is dH itself,
+// buffers 1.. are in the workspace) that fused_sum_parts_kernel adds in a
+// fixed order.
 #pragma once
 
 #include "gemm_tc.cuh"
@@ -67,20 +68,25 @@ constexpr int FB_DEPTH = 3;     // units in flight in the G'' ring of a group
 constexpr int FB_DS = 256;      // dH columns per member
 constexpr uint32_t FB_TMEM_COLS = 512;
 
-template <bool C2>
+// BVS: vocab columns of a single-CTA S tile (CTA pairs use 256).  128 is
+// the one instantiated: 64-wide tiles at M = 64 halve the W held in L2
+// between a round's two reads but double the per-unit exchange overhead,
+// and measured slower (0.49 against 0.38 ms).
+template <bool C2, int BVS = 128>
 struct FusedCfg {
   static constexpr int TH = C2 ? 2 * BM : BM;        // rows of a tile
-  static constexpr int BV = C2 ? 256 : 128;          // vocab columns of an S tile
+  static constexpr int BV = C2 ? 256 : BVS;          // vocab columns of an S tile
   static constexpr int SB = C2 ? 1 : 2;              // S accumulators (TMEM columns [0, SB*BV))
   static constexpr int DB = C2 ? FB_DS / 2 : FB_DS;  // d-columns of W each CTA loads (dH phase)
-  static constexpr int S_BYTES = A_BYTES + 128 * BK * 2;  // H 128 x 64 + W 128 x 64
-  static constexpr int D_BYTES = A_BYTES + BK * DB * 2;   // G'' 128 x 64 + W 64 x DB
+  static constexpr int BR = C2 ? 128 : BV;           // W rows each CTA loads (S phase)
+  static constexpr int S_BYTES = A_BYTES + BR * BK * 2;  // H 128 x 64 + W BR x 64
+  static constexpr int D_BYTES = A_BYTES + BK * DB * 2;  // G'' 128 x 64 + W 64 x DB
   static constexpr int STAGE = S_BYTES > D_BYTES ? S_BYTES : D_BYTES;
   static constexpr int NST = C2 ? 6 : 4;
   static constexpr int STAGING = 4 * 2 * 32 * 128;   // per epilogue warp two 4 KB blocks
   static constexpr int SMEM = NST * STAGE + STAGING + 1024 + 256;
 };
-static_assert(FusedCfg<true>::SMEM <= 232448 && FusedCfg<false>::SMEM <= 232448,
+static_assert(FusedCfg<true>::SMEM <= 232448 && FusedCfg<false, 128>::SMEM <= 232448,
               "fused backward exceeds the shared memory of a CTA");
 
 struct FusedArgs {
@@ -88,9 +94,15 @@ struct FusedArgs {
   int n_rt;       // row tiles of TH rows
   int n_rt128;    // 128-row tiles (block-skip plan granularity)
   int nk;         // K steps of BK over D
-  int C;          // members per group (d-slices of 256)
+  int C;          // members per group (d-slices of 256), at most 32
   int G;          // groups in the waves
-  int Gr;         // groups sharing the remainder (<= G)
+  int nb;         // remainder bands: nb * rem groups, band b covering a round
+                  // range of every remainder row tile (0: no bands)
+  int bw;         // band width in rounds (0: split R evenly over nb bands)
+  int lr;         // groups of the leftover (after the bands) or of the whole
+                  // remainder when it has fewer units than groups
+  int r0;         // first round of the leftover
+  int rl;         // rounds of the leftover per remainder row tile
   int n_vt;       // vocab tiles of BV
   int n_rounds;   // ceil(n_vt / C)
   int waves;      // n_rt / G
@@ -110,7 +122,15 @@ struct FusedArgs {
   float inv_cap;
   uint32_t* ready;     // [G * DEPTH * C * 2]
   uint32_t* consumed;  // [G * DEPTH * C * C]
+  uint32_t* progress;  // [G]: units member 0 of each group has started
 };
+
+// Groups may run at most this many units ahead of the slowest group during
+// the waves: the groups then read the same rounds of W within a few units
+// of each other and share them in L2 (left alone they drift apart over a
+// wave, and each straggler streams W from HBM on its own).
+constexpr int FB_LEAD = 2;
+constexpr uint64_t FB_LEAD_WAIT_NS = 200000;  // a hint: give up after 0.2 ms
 
 // One unit of group g's sequence: row tile r, round j; first / last unit of
 // a segment (a run of units on one row tile), and the dH buffer the segment
@@ -121,17 +141,50 @@ struct FUnit {
   int buf;
 };
 
-// Group containing unit e of the remainder's sequence (T units over Gr
-// groups, group g holding [g T / Gr, (g + 1) T / Gr)).
-__host__ __device__ __forceinline__ int fb_group_of(int64_t e, int64_t T, int Gr) {
-  return static_cast<int>(((e + 1) * Gr - 1) / T);
+// The remainder (rem = n_rt mod G row tiles of R rounds) is cut so that
+// groups running at the same time share rounds of W:
+//  * nb = G / rem bands of rem groups; the group (b, i) takes remainder row
+//    tile i over band b's round range.  The groups of a band read the same
+//    rounds at the same time.  With G a multiple of rem the bands split R;
+//    otherwise each is bw = floor(rem R / G) rounds wide and
+//  * the leftover rounds [r0, R) of every remainder row tile (rem * rl units)
+//    go to the lr = G mod rem other groups as contiguous ranges of the
+//    sequence (tile, round); a tile may be shared by two or three of them.
+//  When the remainder has fewer units than groups, lr = its unit count and
+//  every unit is a leftover unit (nb = 0, r0 = 0, rl = R).
+// A remainder row tile gathers one dH slice per band and one per leftover
+// group that touches it: buffer b for band b, nb + k for the k-th leftover
+// group on the tile.
+
+// Leftover group containing leftover unit e (T units over lr groups, group
+// l holding [l T / lr, (l + 1) T / lr)).
+__host__ __device__ __forceinline__ int fb_group_of(int64_t e, int64_t T, int lr) {
+  return static_cast<int>(((e + 1) * lr - 1) / T);
+}
+
+// Round range [lo, hi) of band b.
+__host__ __device__ __forceinline__ void fb_band(const FusedArgs& a, int b, int& lo, int& hi) {
+  if (a.bw == 0) {
+    lo = b * a.n_rounds / a.nb;
+    hi = (b + 1) * a.n_rounds / a.nb;
+  } else {
+    lo = b * a.bw;
+    hi = lo + a.bw;
+  }
 }
 
 __host__ __device__ __forceinline__ int fb_units(const FusedArgs& a, int g) {
   int n = a.waves * a.n_rounds;
-  if (g < a.Gr) {
-    const int64_t T = static_cast<int64_t>(a.rem) * a.n_rounds;
-    n += static_cast<int>((g + 1) * T / a.Gr - g * T / a.Gr);
+  if (a.rem == 0) return n;
+  if (g < a.nb * a.rem) {
+    int lo, hi;
+    fb_band(a, g / a.rem, lo, hi);
+    return n + hi - lo;
+  }
+  const int l = g - a.nb * a.rem;
+  if (l < a.lr) {
+    const int64_t T = static_cast<int64_t>(a.rem) * a.rl;
+    n += static_cast<int>((l + 1) * T / a.lr - l * T / a.lr);
   }
   return n;
 }
@@ -148,33 +201,71 @@ __host__ __device__ __forceinline__ FUnit fb_unit(const FusedArgs& a, int g, int
     x.buf = 0;
     return x;
   }
-  const int64_t T = static_cast<int64_t>(a.rem) * a.n_rounds;
-  const int64_t lo = g * T / a.Gr, hi = (g + 1) * T / a.Gr;
-  const int64_t e = lo + (u - full);
-  const int i = static_cast<int>(e / a.n_rounds);
-  x.j = static_cast<int>(e - static_cast<int64_t>(i) * a.n_rounds);
+  const int t = u - full;
+  if (g < a.nb * a.rem) {
+    const int b = g / a.rem;
+    int lo, hi;
+    fb_band(a, b, lo, hi);
+    x.r = a.waves * a.G + (g - b * a.rem);
+    x.j = lo + t;
+    x.first = t == 0;
+    x.last = x.j == hi - 1;
+    x.buf = b;
+    return x;
+  }
+  const int l = g - a.nb * a.rem;
+  const int64_t T = static_cast<int64_t>(a.rem) * a.rl;
+  const int64_t lo = l * T / a.lr, hi = (l + 1) * T / a.lr;
+  const int64_t e = lo + t;
+  const int i = static_cast<int>(e / a.rl);
+  const int jj = static_cast<int>(e - static_cast<int64_t>(i) * a.rl);
   x.r = a.waves * a.G + i;
-  x.first = (u == full) || x.j == 0;
-  x.last = (e == hi - 1) || x.j == a.n_rounds - 1;
-  x.buf = g - fb_group_of(static_cast<int64_t>(i) * a.n_rounds, T, a.Gr);
+  x.j = a.r0 + jj;
+  x.first = t == 0 || jj == 0;
+  x.last = (e == hi - 1) || jj == a.rl - 1;
+  x.buf = a.nb + l - fb_group_of(static_cast<int64_t>(i) * a.rl, T, a.lr);
   return x;
 }
 
-// Nothing to compute for (row tile r, vocab tile v): past the vocabulary,
-// or every 128-row half either past M, without a nonzero cotangent, or
-// block-skipped for the 256-wide vocabulary block holding v.
-template <bool C2>
-__device__ __forceinline__ bool fb_skip(const FusedArgs& a, int r, int v) {
-  if (v >= a.n_vt) return true;
-  const int b = C2 ? v : (v >> 1);
-  auto half = [&](int rt) -> bool {
-    if (rt >= a.n_rt128 || a.row_skip[rt]) return true;
-    return a.tile_skip != nullptr && a.tile_skip[static_cast<size_t>(rt) * a.skip_ld + b] != 0;
-  };
-  return C2 ? (half(2 * r) && half(2 * r + 1)) : half(r);
+// dH slices a remainder row tile i gathers: one per band, and one per
+// leftover group touching it.
+__host__ __device__ __forceinline__ int fb_slices(const FusedArgs& a, int i) {
+  int k = a.nb;
+  if (a.lr > 0) {
+    const int64_t T = static_cast<int64_t>(a.rem) * a.rl;
+    k += fb_group_of(static_cast<int64_t>(i + 1) * a.rl - 1, T, a.lr) -
+         fb_group_of(static_cast<int64_t>(i) * a.rl, T, a.lr) + 1;
+  }
+  return k;
 }
 
-template <bool C2>
+// Tiles of round j with nothing to compute for row tile r, as bits q of a
+// mask (vocab tile j*C + q): past the vocabulary, or every 128-row half
+// either past M, without a nonzero cotangent, or block-skipped for the
+// 256-wide vocabulary block holding the tile.  Its loads are independent of
+// each other, and every role computes the mask of the next unit while it
+// works on the current one, so their latency stays off the issue path.
+template <bool C2, int BV>
+__device__ __forceinline__ uint32_t fb_mask(const FusedArgs& a, int r, int j) {
+  const int v0 = j * a.C;
+  uint32_t past = 0;
+  for (int q = 0; q < a.C; ++q)
+    if (v0 + q >= a.n_vt) past |= 1u << q;
+  auto half = [&](int rt) -> uint32_t {
+    if (rt >= a.n_rt128 || a.row_skip[rt]) return ~0u;
+    if (a.tile_skip == nullptr) return 0u;
+    const uint8_t* ts = a.tile_skip + static_cast<size_t>(rt) * a.skip_ld;
+    uint32_t m = 0;
+    for (int q = 0; q < a.C; ++q) {
+      const int v = v0 + q;
+      if (v < a.n_vt && ts[v / (256 / BV)] != 0) m |= 1u << q;
+    }
+    return m;
+  };
+  return past | (C2 ? (half(2 * r) & half(2 * r + 1)) : half(r));
+}
+
+template <bool C2, int BVS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fused_bwd_kernel(const __grid_constant__ CUtensorMap tmH,   // H [M, D], box 64 x 128
                      const __grid_constant__ CUtensorMap tmWk,  // W [V, D], box 64 x 128
@@ -184,7 +275,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      const __grid_constant__ CUtensorMap tmD0,  // dH [1, M, D] fp32
                      const __grid_constant__ CUtensorMap tmD1,  // partial dH [nbuf-1, M-row_rem, D]
                      const FusedArgs a) {
-  using F = FusedCfg<C2>;
+  using F = FusedCfg<C2, BVS>;
   const uint32_t rank = C2 ? cluster_ctarank() : 0u;
   const int member_id = C2 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
   const int g = member_id / a.C, p = member_id - (member_id / a.C) * a.C;
@@ -276,11 +367,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           phase ^= 1u;
         }
       };
+      uint32_t mk_prev = 0, mk_cur = 0;
+      if (n_u > 0) {
+        const FUnit x0 = fb_unit(a, g, 0);
+        mk_cur = fb_mask<C2, F::BV>(a, x0.r, x0.j);
+      }
       for (int u = 0; u <= n_u && ok; ++u) {
+        uint32_t mk_next = 0;
+        if (u + 1 < n_u) {
+          const FUnit xn = fb_unit(a, g, u + 1);
+          mk_next = fb_mask<C2, F::BV>(a, xn.r, xn.j);
+        }
+        if (u < n_u && p == 0 && rank == 0 && u < a.waves * a.n_rounds) {
+          st_relaxed_gpu(&a.progress[g], static_cast<uint32_t>(u));
+          if (u >= FB_LEAD) {
+            const uint32_t need = static_cast<uint32_t>(u - FB_LEAD);
+            const uint64_t t0 = globaltimer_ns();
+            for (int o = 0; o < a.G; ++o)
+              while (ld_relaxed_gpu(&a.progress[o]) < need &&
+                     globaltimer_ns() - t0 < FB_LEAD_WAIT_NS)
+                __nanosleep(128);
+          }
+        }
         if (u < n_u) {
           const FUnit x = fb_unit(a, g, u);
           const int v = x.j * a.C + p;
-          if (!fb_skip<C2>(a, x.r, v)) {
+          if (!((mk_cur >> p) & 1u)) {
             const int arow = x.r * F::TH + static_cast<int>(rank) * BM;
             const int brow = v * F::BV + (C2 ? static_cast<int>(rank) * 128 : 0);
             for (int k = 0; k < a.nk; ++k) {
@@ -306,7 +418,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fill = static_cast<uint32_t>((u - 1) / FB_DEPTH);
           for (int q = 0; q < a.C && ok; ++q) {
             const int v = x.j * a.C + q;
-            if (fb_skip<C2>(a, x.r, v)) continue;
+            if ((mk_prev >> q) & 1u) continue;
             const int slot = slot_of(u - 1, q);
             if (!wait_flag_geq(&a.ready[slot * 2 + static_cast<int>(rank)], 4u * (fill + 1u),
                                a.wait_ns, abort_flag)) {
@@ -340,6 +452,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+        mk_prev = mk_cur;
+        mk_cur = mk_next;
       }
       if (!ok) {
         set_status(a.status, ST_TIMEOUT);
@@ -359,10 +473,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int ns = 0, nseg = 0;
       bool ok = true, dh_any = false;
+      uint32_t mk_prev = 0, mk_cur = 0;
+      if (n_u > 0) {
+        const FUnit x0 = fb_unit(a, g, 0);
+        mk_cur = fb_mask<C2, F::BV>(a, x0.r, x0.j);
+      }
       for (int u = 0; u <= n_u && ok; ++u) {
+        uint32_t mk_next = 0;
+        if (u + 1 < n_u) {
+          const FUnit xn = fb_unit(a, g, u + 1);
+          mk_next = fb_mask<C2, F::BV>(a, xn.r, xn.j);
+        }
         if (u < n_u) {
-          const FUnit x = fb_unit(a, g, u);
-          if (!fb_skip<C2>(a, x.r, x.j * a.C + p)) {
+          if (!((mk_cur >> p) & 1u)) {
             const int sb = ns % F::SB;
             if (!wait_bounded(&s_empty[sb], ((ns / F::SB) & 1) ^ 1u, a.wait_ns, abort_flag)) {
               ok = false;
@@ -405,7 +528,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int q = 0; q < a.C && ok; ++q) {
             const int slot = slot_of(u - 1, q);
             uint32_t* cons = &a.consumed[slot * a.C + p];
-            if (fb_skip<C2>(a, x.r, x.j * a.C + q)) {
+            if ((mk_prev >> q) & 1u) {
               st_relaxed_gpu(cons, fill + 1u);
               continue;
             }
@@ -452,6 +575,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++nseg;
           }
         }
+        mk_prev = mk_cur;
+        mk_cur = mk_next;
       }
       if (!ok) {
         set_status(a.status, ST_TIMEOUT);
@@ -544,15 +669,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     bool seg_any = false, prev_any = false;
     FUnit prev{};
+    const uint32_t all_c = a.C >= 32 ? ~0u : ((1u << a.C) - 1u);
+    uint32_t mk_cur = 0;
+    if (n_u > 0) {
+      const FUnit x0 = fb_unit(a, g, 0);
+      mk_cur = fb_mask<C2, F::BV>(a, x0.r, x0.j);
+    }
     for (int u = 0; u < n_u && ok; ++u) {
+      uint32_t mk_next = 0;
+      if (u + 1 < n_u) {
+        const FUnit xn = fb_unit(a, g, u + 1);
+        mk_next = fb_mask<C2, F::BV>(a, xn.r, xn.j);
+      }
       const FUnit x = fb_unit(a, g, u);
       if (x.first) seg_any = false;
-      for (int q = 0; q < a.C; ++q) seg_any = seg_any || !fb_skip<C2>(a, x.r, x.j * a.C + q);
+      seg_any = seg_any || (mk_cur & all_c) != all_c;
       const int v = x.j * a.C + p;
       const int slot = slot_of(u, p);
       const uint32_t fill = static_cast<uint32_t>(u / FB_DEPTH);
       uint32_t* rdy = &a.ready[slot * 2 + static_cast<int>(rank)];
-      if (!fb_skip<C2>(a, x.r, v)) {
+      if (!((mk_cur >> p) & 1u)) {
         const int sb = ns % F::SB;
         if (!wait_bounded(&s_full[sb], (ns / F::SB) & 1, a.wait_ns, abort_flag)) {
           ok = false;
@@ -611,6 +747,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (u >= 1 && prev.last) flush(prev, prev_any);
       prev = x;
       prev_any = seg_any;
+      mk_cur = mk_next;
     }
     if (ok && n_u > 0) flush(prev, prev_any);
     if (!ok) {
@@ -639,16 +776,13 @@ __global__ void __launch_bounds__(256) fused_sum_parts_kernel(
     float4* __restrict__ dh, const float4* __restrict__ parts, FusedArgs a, int TH) {
   const int D4 = a.D / 4;
   const int64_t n = static_cast<int64_t>(a.M - a.row_rem) * D4;
-  const int64_t T = static_cast<int64_t>(a.rem) * a.n_rounds;
   for (int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; t < n;
        t += int64_t(gridDim.x) * blockDim.x) {
     const int m = a.row_rem + static_cast<int>(t / D4);
-    const int i = m / TH - a.waves * a.G;
-    const int gf = fb_group_of(static_cast<int64_t>(i) * a.n_rounds, T, a.Gr);
-    const int gl = fb_group_of(static_cast<int64_t>(i + 1) * a.n_rounds - 1, T, a.Gr);
+    const int k = fb_slices(a, m / TH - a.waves * a.G);
     const int64_t idx = static_cast<int64_t>(a.row_rem) * D4 + t;
     float4 s = dh[idx];
-    for (int b = 1; b <= gl - gf; ++b) {
+    for (int b = 1; b < k; ++b) {
       const float4 q = parts[static_cast<size_t>(b - 1) * n + t];
       s.x += q.x;
       s.y += q.y;

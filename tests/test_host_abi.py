@@ -354,6 +354,15 @@ def _check_schedule(M, V, D, sched, plan):
         full = s[: waves * n_rounds]
         assert np.array_equal(full[:, 2], np.tile(np.arange(n_rounds), waves))
         assert np.array_equal(full[:, 1], np.repeat(np.arange(waves) * G + g, n_rounds))
+    # the remainder's bands: groups of a band run the same rounds in step
+    rem = n_rt % G
+    if rem and rem * n_rounds >= G:
+        nb = G // rem
+        waves = n_rt // G
+        for band in range(nb):
+            seqs = [sched[sched[:, 0] == g][waves * n_rounds:, 2].tolist()
+                    for g in range(band * rem, (band + 1) * rem)]
+            assert all(q == seqs[0] for q in seqs), band
     for r, b in bufs.items():
         assert sorted(b) == list(range(len(b))), (r, b)
         assert len(b) <= plan["bwd_fused_buffers"]
