@@ -51,6 +51,9 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--workspace-mb", type=int, default=0,
                    help="workspace size (default: the library's default)")
+    p.add_argument("--backward-mode", type=int, choices=[0, 1, 2], default=0,
+                   help="dense bf16 heads: 0 choose, 1 the fused backward, 2 two GEMMs per "
+                        "vocab chunk")
     p.add_argument("--quant-staging", type=int, choices=[0, 1, 2], default=0,
                    help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
     p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
@@ -289,6 +292,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cce.cce_set_quant_staging(args.quant_staging)
+    cce.cce_set_backward_mode(args.backward_mode)
     cce.cce_set_cta_pairs(bool(args.cta_pairs))
 
     wl = S.make_workload(args.workload)
@@ -504,7 +508,8 @@ def run_ours(args):
                    "workspace_bytes": int(buf.ws.numel()),
                    "cta_pairs": bool(args.cta_pairs),
                    "cuda_graph": bool(args.graph),
-                   "quant_staging": ["choose", "in-kernel", "staged"][args.quant_staging]},
+                   "quant_staging": ["choose", "in-kernel", "staged"][args.quant_staging],
+                   "backward": ["choose", "fused", "two GEMMs"][args.backward_mode]},
         "tflops": tflops,
         "executed": {"rows_backward": m_b, "tflop_per_step": flop_exec / 1e12,
                      "tflops": flop_exec / (ms_step / 1e3) / 1e12,
@@ -547,6 +552,7 @@ def run_small_m(args, quant=False):
     from lm_head_cross_flash_b200 import synthetic as S
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    cce.cce_set_backward_mode(args.backward_mode)
     peaks, peaks_src = load_peaks()
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     lines = []

@@ -355,10 +355,12 @@ void cce_set_cta_pairs(int on);
  * (staged falls back to in-kernel when the chunk would be too narrow). */
 void cce_set_quant_staging(int mode);
 
-/* Backward of dense bf16 heads: 0 choose (default: the fused kernel when
- * ws holds its layout, else two GEMMs per vocab chunk), 1 the fused kernel
- * only (CCE_ERR_WORKSPACE_TOO_SMALL when ws cannot hold its layout), 2 two
- * GEMMs per vocab chunk.  Both forms give the same results to accumulation
+/* Backward of dense bf16 heads: 0 choose (default: the fused kernel from
+ * M = 1024 rows when ws holds its layout, where it measured at least as fast;
+ * else two GEMMs per vocab chunk), 1 the fused kernel at any M
+ * (CCE_ERR_WORKSPACE_TOO_SMALL when ws cannot hold its layout), 2 two GEMMs
+ * per vocab chunk.  cce_workspace_bytes sizes ws for the form the current
+ * setting takes.  Both forms give the same results to accumulation
  * order.  Process-wide; any other value is taken as 0.  No counterpart on
  * the pages: it selects between two schedules of the same backward. */
 void cce_set_backward_mode(int mode);

@@ -706,9 +706,22 @@ struct FusedPlan {
   size_t tile_skip = 0, row_skip = 0, flags = 0, ring = 0, parts = 0, total = 0;
 };
 
+// Choosing between the fused backward and the two GEMMs: below this many
+// rows the two GEMMs were faster on the same box (D = 2048, V = 262,144; ms):
+//   M      64     128    256    512    1024   2048   4096   8192
+//   fused  0.393  0.403  0.492  0.902  1.709  3.175  6.435  13.81
+//   two    0.344  0.361  0.485  0.857  1.712  3.380  6.962  13.60
+// (at small M the fused kernel's groups hold more W in flight than L2 keeps
+// between a round's two reads, so it reads W twice as well; at 8192 the two
+// are within 2 %, and the fused kernel needs 67 MB of workspace against
+// 1.17 GB).  D = 1536, V = 73,440: fused 1-4 % faster from M = 512.
+constexpr int64_t kFusedMinRows = 1024;
+
 FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
   FusedPlan f;
-  if (g_bwd_mode.load() == 2 || want_dw || h != CCE_BF16 || W->format != CCE_W_DENSE) return f;
+  const int mode = g_bwd_mode.load();
+  if (mode == 2 || want_dw || h != CCE_BF16 || W->format != CCE_W_DENSE) return f;
+  if (mode == 0 && M < kFusedMinRows) return f;
   const int64_t n128 = ceil_div(M, BM);
   f.c2 = g_pairs.load() != 0 && n128 >= 2;
   const int TH = f.c2 ? FusedCfg<true>::TH : FusedCfg<false>::TH;

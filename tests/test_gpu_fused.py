@@ -25,9 +25,15 @@ pytestmark = pytest.mark.gpu
 
 
 def _fwd(wl, ws_bytes=None):
+    """Forward, with a workspace sized for the fused backward at any M (the
+    default setting takes the fused kernel from 1,024 rows only)."""
     H, head, labels = upload(wl)
     hd = cce.h_dtype(H)
-    ws = cce.alloc_workspace(wl.M, hd, head, nbytes=ws_bytes)
+    cce.cce_set_backward_mode(1)
+    try:
+        ws = cce.alloc_workspace(wl.M, hd, head, nbytes=ws_bytes)
+    finally:
+        cce.cce_set_backward_mode(0)
     f = dict(device="cuda", dtype=torch.float32)
     logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
     bm = torch.empty(cce.blockmax_cols(wl.V), wl.M, **f)
@@ -69,7 +75,11 @@ CASES = [
 def test_fused_backward_matches_oracle_and_two_gemm(cfg, split, D, V):
     wl = S.make_custom(cfg, M_split=split, D=D, V=V)
     H, head, labels, ws, lse, _ = _fwd(wl)
-    plan = cce.cce_query_plan(wl.M, cce.h_dtype(H), head, ws.numel())
+    cce.cce_set_backward_mode(1)
+    try:
+        plan = cce.cce_query_plan(wl.M, cce.h_dtype(H), head, ws.numel())
+    finally:
+        cce.cce_set_backward_mode(0)
     assert plan["bwd_fused"], plan
     g = S.random_cotangent(wl)
     g[min(5, wl.M - 1):min(9, wl.M)] = 0.0
@@ -148,7 +158,11 @@ def test_fused_softcap(cap, split, D, V):
     H, head, labels = upload(wl)
     head = cce.Head(w=head.w, V=wl.V, D=wl.D, softcap=cap)
     hd = cce.h_dtype(H)
-    ws = cce.alloc_workspace(wl.M, hd, head)
+    cce.cce_set_backward_mode(1)
+    try:
+        ws = cce.alloc_workspace(wl.M, hd, head)
+    finally:
+        cce.cce_set_backward_mode(0)
     f = dict(device="cuda", dtype=torch.float32)
     logp, lse = torch.empty(wl.M, **f), torch.empty(wl.M, **f)
     cce.cce_forward(H, head, labels, logp, lse, None, None, ws)

@@ -162,6 +162,13 @@ def test_objective_rejects_bad_arguments(lib):
 
 
 @pytest.fixture
+def fused_backward():
+    cce.cce_set_backward_mode(1)
+    yield
+    cce.cce_set_backward_mode(0)
+
+
+@pytest.fixture
 def two_gemm_backward():
     cce.cce_set_backward_mode(2)
     yield
@@ -296,8 +303,18 @@ def test_fused_plan_choice(lib):
     assert p["bwd_ok"] and p["bwd_fused"] and p["bwd_chunk"] == 0 and p["bwd_cta_pairs"]
     assert p["bwd_fused_members"] == 8 and p["bwd_fused_groups"] == 74 // 8
     assert p["bwd_fused_buffers"] >= 2   # 32 pair tiles over 9 groups leave a remainder
-    small = cce.cce_query_plan(64, cce.CCE_BF16, big,
-                               lib.cce_workspace_bytes(64, cce.CCE_BF16, ctypes.byref(big)))
+    # below 1,024 rows the default takes the two GEMMs (measured faster there)
+    for M in (64, 512, 1023):
+        p0 = cce.cce_query_plan(M, cce.CCE_BF16, big,
+                                lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(big)))
+        assert p0["bwd_ok"] and not p0["bwd_fused"], M
+    assert cce.cce_query_plan(1024, cce.CCE_BF16, big, ws)["bwd_fused"]
+    cce.cce_set_backward_mode(1)   # the fused kernel at any M
+    try:
+        small = cce.cce_query_plan(64, cce.CCE_BF16, big,
+                                   lib.cce_workspace_bytes(64, cce.CCE_BF16, ctypes.byref(big)))
+    finally:
+        cce.cce_set_backward_mode(0)
     assert small["bwd_fused"] and not small["bwd_cta_pairs"]
     assert small["bwd_fused_groups"] == 148 // 8
     lo = lib.cce_workspace_min_bytes(8192, cce.CCE_BF16, ctypes.byref(big))
@@ -372,7 +389,7 @@ def _check_schedule(M, V, D, sched, plan):
 @pytest.mark.parametrize("M,V,D", [(8192, 262144, 2048), (2048, 73440, 1536), (64, 262144, 2048),
                                    (1, 300, 64), (300, 1000, 320), (32768, 128256, 4096),
                                    (129, 4097, 256), (5000, 3000, 2048)])
-def test_fused_schedule_covers_every_unit_once(lib, M, V, D):
+def test_fused_schedule_covers_every_unit_once(lib, M, V, D, fused_backward):
     h = _head(V=V, D=D)
     plan = cce.cce_query_plan(M, cce.CCE_BF16, h,
                               lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h)))
@@ -383,6 +400,14 @@ def test_fused_schedule_covers_every_unit_once(lib, M, V, D):
 @settings(max_examples=60, deadline=None)
 @given(M=st.integers(1, 20000), V=st.integers(1, 70000), D64=st.integers(1, 64))
 def test_fused_schedule_property(lib, M, V, D64):
+    cce.cce_set_backward_mode(1)
+    try:
+        _fused_schedule_property(lib, M, V, D64)
+    finally:
+        cce.cce_set_backward_mode(0)
+
+
+def _fused_schedule_property(lib, M, V, D64):
     D = 64 * D64
     h = _head(V=V, D=D)
     plan = cce.cce_query_plan(M, cce.CCE_BF16, h,
