@@ -264,7 +264,7 @@ cce_status pref_grad_coeffs(const float* logp, const int32_t* labels,
  *   tile from the TMEM accumulator and contracts it with W into a dH
  *   accumulator held in TMEM for a whole sweep of the vocabulary; the
  *   coefficient tiles pass between the CTAs sharing a row tile through a
- *   small ring of tiles in ws (DEPTH rounds per group, tens of MB, L2-
+ *   small ring of tiles in ws (two rounds per group, tens of MB, L2-
  *   resident), never as a whole.  ws then holds the block-skip plan, the
  *   ring and its flags, and O(M*D) partial dH buffers when row tiles are
  *   shared between groups (cce_workspace_bytes sizes it).  Other heads (fp32,

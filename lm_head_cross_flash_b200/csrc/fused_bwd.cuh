@@ -64,7 +64,11 @@
 
 namespace cce {
 
-constexpr int FB_DEPTH = 3;     // units in flight in the G'' ring of a group
+// Units in flight in the G'' ring of a group.  Two: a slot is rewritten two
+// units after it was filled, soon enough that its lines are still in L2 (a
+// three-deep ring had most of its tiles written back to HBM first: 3.3
+// against 1.5 GB of DRAM writes per launch at the long pair, 4 % slower).
+constexpr int FB_DEPTH = 2;
 constexpr int FB_DS = 256;      // dH columns per member
 constexpr uint32_t FB_TMEM_COLS = 512;
 
@@ -601,6 +605,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     int ns = 0, nseg = 0;
     bool ok = true;
+    const uint64_t ring_policy = l2_policy_evict_last();  // read by every member, then rewritten
     // Staging per warp: 8 KB, four 2 KB slots for G'' blocks (the TMA store
     // of a block may still be reading its slot while the next three are
     // filled) or two 4 KB slots for fp32 dH blocks during a flush (which
@@ -727,7 +732,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                        fence_proxy_async_smem();
                        __syncwarp();
                        if (lane == 0) {
-                         tma_store_2d(&tmGs, sbuf, c * 32, grow0);
+                         tma_store_2d_hint(&tmGs, sbuf, c * 32, grow0, ring_policy);
                          bulk_commit();
                        }
                      });

@@ -129,6 +129,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// tma_store_2d with an L2 eviction-priority hint.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* m, const void* src,
+                                                  int32_t c0, int32_t c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], "
+      "%4;" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
 // global[box] += shared[box] (element type of the tensor map), done in L2.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src,
                                                   int32_t c0, int32_t c1, int32_t c2) {
