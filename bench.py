@@ -51,9 +51,9 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--workspace-mb", type=int, default=0,
                    help="workspace size (default: the library's default)")
-    p.add_argument("--backward-mode", type=int, choices=[0, 1, 2], default=0,
-                   help="dense bf16 heads: 0 choose, 1 the fused backward, 2 two GEMMs per "
-                        "vocab chunk")
+    p.add_argument("--backward-mode", type=int, choices=[0, 1, 2, 3], default=0,
+                   help="dense bf16 heads: 0 choose, 1 the grouped fused backward, 2 two "
+                        "GEMMs per vocab chunk, 3 the sliced fused backward (M <= 64)")
     p.add_argument("--quant-staging", type=int, choices=[0, 1, 2], default=0,
                    help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
     p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
@@ -458,7 +458,8 @@ def run_ours(args):
                       "bwd_grad_gemm": 2.0 * wl.M * wl.V * wl.D,
                       "bwd_dh_gemm": 2.0 * wl.M * wl.V * wl.D,
                       # recompute of the logits and the dH contraction, one kernel
-                      "bwd_fused": 4.0 * wl.M * wl.V * wl.D}
+                      "bwd_fused": 4.0 * wl.M * wl.V * wl.D,
+                      "bwd_sliced": 4.0 * wl.M * wl.V * wl.D}
     kinds = {k: v for k, v in prof.items() if v[1] > 0}
     dom = max(kinds, key=lambda k: kinds[k][0])
     dom_ms, dom_n = kinds[dom]
@@ -509,7 +510,7 @@ def run_ours(args):
                    "cta_pairs": bool(args.cta_pairs),
                    "cuda_graph": bool(args.graph),
                    "quant_staging": ["choose", "in-kernel", "staged"][args.quant_staging],
-                   "backward": ["choose", "fused", "two GEMMs"][args.backward_mode]},
+                   "backward": ["choose", "fused", "two GEMMs", "sliced"][args.backward_mode]},
         "tflops": tflops,
         "executed": {"rows_backward": m_b, "tflop_per_step": flop_exec / 1e12,
                      "tflops": flop_exec / (ms_step / 1e3) / 1e12,
@@ -606,6 +607,9 @@ def run_small_m(args, quant=False):
         if plan["bwd_fused"]:
             nparts = plan["bwd_fused_buffers"] - 1
             bwd_design = bwd_bytes + 3 * 4.0 * nparts * M * wl.D  # parts written, read; dH RMW
+        elif plan["bwd_sliced"]:
+            # W once; one partial dH per cluster written and read back
+            bwd_design = bwd_bytes + 2 * 4.0 * plan["bwd_sliced_clusters"] * M * wl.D
         else:
             bwd_design = 2 * wbytes + 2.0 * M * wl.D + 4.0 * M * wl.D + 2 * 2.0 * M * wl.V
         line = {"sweep": "small_m_q4" if quant else "small_m", "M": M, "D": wl.D, "V": wl.V,
@@ -616,7 +620,8 @@ def run_small_m(args, quant=False):
                 "fwd_frac_hbm": fwd_bytes / (t_f / 1e3) / 1e9 / hbm,
                 "bwd_frac_hbm": bwd_bytes / (t_b / 1e3) / 1e9 / hbm,
                 "fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes,
-                "bwd_form": "fused" if plan["bwd_fused"] else "two GEMMs per vocab chunk",
+                "bwd_form": ("fused" if plan["bwd_fused"] else
+                             "sliced" if plan["bwd_sliced"] else "two GEMMs per vocab chunk"),
                 "bwd_design_bytes": bwd_design,
                 "bwd_design_gbs": bwd_design / (t_b / 1e3) / 1e9,
                 "tokens_per_s": M / ((t_f + t_b) / 1e3),

@@ -355,14 +355,24 @@ void cce_set_cta_pairs(int on);
  * (staged falls back to in-kernel when the chunk would be too narrow). */
 void cce_set_quant_staging(int mode);
 
-/* Backward of dense bf16 heads: 0 choose (default: the fused kernel from
- * M = 1024 rows when ws holds its layout, where it measured at least as fast;
- * else two GEMMs per vocab chunk), 1 the fused kernel at any M
- * (CCE_ERR_WORKSPACE_TOO_SMALL when ws cannot hold its layout), 2 two GEMMs
- * per vocab chunk.  cce_workspace_bytes sizes ws for the form the current
- * setting takes.  Both forms give the same results to accumulation
- * order.  Process-wide; any other value is taken as 0.  No counterpart on
- * the pages: it selects between two schedules of the same backward. */
+/* Backward of dense bf16 heads:
+ *   0  choose (default): the grouped fused kernel from M = 1024 rows when ws
+ *      holds its layout (where it measured at least as fast); else two GEMMs
+ *      per vocab chunk;
+ *   1  the grouped fused kernel at any M (CCE_ERR_WORKSPACE_TOO_SMALL when ws
+ *      cannot hold its layout);
+ *   2  two GEMMs per vocab chunk;
+ *   3  the sliced kernel (M <= 64, D <= 2048; CCE_ERR_UNSUPPORTED outside
+ *      that, CCE_ERR_WORKSPACE_TOO_SMALL when ws cannot hold its layout):
+ *      clusters of up to 8 CTAs, each owning 256 columns of D, sum their
+ *      partial logits through distributed shared memory, so W is read from
+ *      HBM once (at D = 2048, V = 262,144 and M <= 64 it measured 0.51 ms
+ *      against 0.344 ms for the two GEMMs, so 0 does not choose it).
+ * cce_workspace_bytes sizes ws for the form the current setting takes.  All
+ * forms give the same results to accumulation order (the sliced kernel sums
+ * the logits of its D slices in fp32 in a fixed order).  Process-wide; any
+ * other value is taken as 0.  No counterpart on the pages: it selects
+ * between schedules of the same backward. */
 void cce_set_backward_mode(int mode);
 
 /* The execution plan cce_forward and cce_backward_dh would take for this
@@ -382,7 +392,12 @@ void cce_set_backward_mode(int mode);
  *                     is then 0);
  *   bwd_fused_groups  groups of CTAs (pairs) that each sweep a row tile;
  *   bwd_fused_members CTAs (pairs) per group, one per 256 columns of dH;
- *   bwd_fused_buffers dH buffers (1 + partial buffers in ws).
+ *   bwd_fused_buffers dH buffers (1 + partial buffers in ws);
+ *   bwd_sliced        1 when the backward runs the sliced kernel (bwd_chunk
+ *                     and bwd_fused are then 0);
+ *   bwd_sliced_clusters  clusters it launches (each sweeps every
+ *                     bwd_sliced_clusters-th vocab tile of 128 rows);
+ *   bwd_sliced_ctas   CTAs per cluster, one per 256 columns of D.
  * Returns CCE_ERR_INVALID_ARGUMENT / UNSUPPORTED as the calls would. */
 typedef struct {
   int fwd_ok, bwd_ok;
@@ -391,6 +406,7 @@ typedef struct {
   int fwd_staged, bwd_staged;
   int fwd_cta_pairs, bwd_cta_pairs;
   int bwd_fused, bwd_fused_groups, bwd_fused_members, bwd_fused_buffers;
+  int bwd_sliced, bwd_sliced_clusters, bwd_sliced_ctas;
 } cce_plan;
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out);

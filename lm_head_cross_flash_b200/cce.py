@@ -65,7 +65,9 @@ class _Plan(ctypes.Structure):
                 ("fwd_staged", ctypes.c_int), ("bwd_staged", ctypes.c_int),
                 ("fwd_cta_pairs", ctypes.c_int), ("bwd_cta_pairs", ctypes.c_int),
                 ("bwd_fused", ctypes.c_int), ("bwd_fused_groups", ctypes.c_int),
-                ("bwd_fused_members", ctypes.c_int), ("bwd_fused_buffers", ctypes.c_int)]
+                ("bwd_fused_members", ctypes.c_int), ("bwd_fused_buffers", ctypes.c_int),
+                ("bwd_sliced", ctypes.c_int), ("bwd_sliced_clusters", ctypes.c_int),
+                ("bwd_sliced_ctas", ctypes.c_int)]
 
 
 _lib = None
@@ -486,8 +488,8 @@ def cce_set_quant_staging(mode: int):
 
 
 def cce_set_backward_mode(mode: int):
-    """Dense bf16 heads: 0 choose; 1 the fused backward kernel; 2 two GEMMs
-    per vocab chunk."""
+    """Dense bf16 heads: 0 choose; 1 the grouped fused backward kernel; 2 two
+    GEMMs per vocab chunk; 3 the sliced fused kernel (M <= 64, D <= 2048)."""
     lib().cce_set_backward_mode(int(mode))
 
 

@@ -16,6 +16,7 @@
 #include "../../include/cce.h"
 #include "aux_kernels.cuh"
 #include "fused_bwd.cuh"
+#include "slice_bwd.cuh"
 #include "gemm_tc.cuh"
 
 using namespace cce;
@@ -95,14 +96,15 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
   PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM,
-  PK_PREFIX, PK_DW, PK_DEQ, PK_FUSED, PK_FSUM, PK_N
+  PK_PREFIX, PK_DW, PK_DEQ, PK_FUSED, PK_FSUM, PK_SLICE, PK_SSUM, PK_N
 };
 const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
                                       "bwd_dh_gemm",   "selftest",     "dh_split_sum",
                                       "prefix_gather_scatter", "bwd_dw_gemm",
                                       "dequant_chunk", "bwd_fused",
-                                      "fused_part_sum"};
+                                      "fused_part_sum", "bwd_sliced",
+                                      "sliced_part_sum"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -181,6 +183,7 @@ struct DevInfo {
   int pairs = 0;  // CTA pairs (clusters of 2) resident at once, 0 = none
   int fused_pairs = 0;  // fused backward: pairs / single CTAs resident at once
   int fused_ctas = 0;
+  int slice_clusters[4] = {0, 0, 0, 0};  // sliced backward, clusters of 1, 2, 4, 8
   bool attrs = false;
 };
 
@@ -224,6 +227,36 @@ int max_fused_pairs() {
   }
   return n;
 }
+// The sliced backward's kernel for clusters of `ccl` CTAs.
+using SliceKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, SliceArgs);
+SliceKernel slice_kernel(int ccl) {
+  switch (ccl) {
+    case 1: return slice_bwd_kernel<1>;
+    case 2: return slice_bwd_kernel<2>;
+    case 4: return slice_bwd_kernel<4>;
+    default: return slice_bwd_kernel<8>;
+  }
+}
+// Clusters of `ccl` CTAs resident at once for the sliced backward.
+int max_slice_clusters(int ccl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ccl);
+  cfg.blockDim = dim3(SL_THREADS);
+  cfg.dynamicSmemBytes = SL_SMEM;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = ccl;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, slice_kernel(ccl), &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
 
@@ -252,7 +285,11 @@ cce_status device_info(int* sms) {
          cudaFuncSetAttribute(fused_bwd_kernel<true, 128>, attr, FusedCfg<true>::SMEM) ==
              cudaSuccess &&
          cudaFuncSetAttribute(fused_bwd_kernel<false, 128>, attr, FusedCfg<false, 128>::SMEM) ==
-             cudaSuccess;
+             cudaSuccess &&
+         cudaFuncSetAttribute(slice_bwd_kernel<1>, attr, SL_SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(slice_bwd_kernel<2>, attr, SL_SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(slice_bwd_kernel<4>, attr, SL_SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(slice_bwd_kernel<8>, attr, SL_SMEM) == cudaSuccess;
     if (ok) {
       d.pairs = std::min(max_pairs_of<Mode::kLse>(),
                          std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
@@ -265,6 +302,7 @@ cce_status device_info(int* sms) {
         per_sm = 0;
       }
       d.fused_ctas = per_sm * d.sms;
+      for (int i = 0; i < 4; ++i) d.slice_clusters[i] = max_slice_clusters(1 << i);
     }
     if (!ok)
       return CCE_ERR_CUDA;
@@ -720,7 +758,7 @@ constexpr int64_t kFusedMinRows = 1024;
 FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
   FusedPlan f;
   const int mode = g_bwd_mode.load();
-  if (mode == 2 || want_dw || h != CCE_BF16 || W->format != CCE_W_DENSE) return f;
+  if (mode == 2 || mode == 3 || want_dw || h != CCE_BF16 || W->format != CCE_W_DENSE) return f;
   if (mode == 0 && M < kFusedMinRows) return f;
   const int64_t n128 = ceil_div(M, BM);
   f.c2 = g_pairs.load() != 0 && n128 >= 2;
@@ -893,6 +931,133 @@ cce_status fused_backward(const FusedPlan& fp, const void* H, const cce_head* W,
   return CCE_OK;
 }
 
+
+// Clusters of `ccl` CTAs of the sliced backward resident at once (without a
+// device: 148 SMs over clusters of ccl).
+int slice_resident(int ccl) {
+  int dev = 0, sms = 0;
+  int i = 0;
+  while ((1 << i) < ccl) ++i;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 &&
+      device_info(&sms) == CCE_OK) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    return g_dev[dev].slice_clusters[i];
+  }
+  cudaGetLastError();
+  return 148 / ccl;
+}
+
+// How the sliced backward runs (slice_bwd.cuh): clusters of Ccl CTAs, one
+// 256-column slice of D each (Ccl the power of two covering D), the vocab
+// tiles dealt to the resident clusters in turn, and its workspace
+// (block-skip plan, one partial dH per cluster).  ok = false: the problem is
+// not one it takes (more than 64 rows, D above 2048, 4/8-bit or fp32
+// heads, a trainable head), or the mode switch is not 3.  The default does
+// not take it: at D = 2048, V = 262,144 it measured 0.51 ms at M = 64 (8 to
+// 64 rows alike) against 0.344 ms for the two GEMMs, which read W twice but
+// stream it at the HBM rate; the sliced kernel reads W once but its
+// exchange between the CTAs of a cluster, double-buffered as deep as shared
+// memory allows, holds each 128-row vocab tile to about 6,300 cycles.
+struct SlicePlan {
+  bool ok = false;
+  SliceArgs a{};
+  size_t tile_skip = 0, row_skip = 0, parts = 0, total = 0;
+};
+
+SlicePlan plan_slice(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
+  SlicePlan f;
+  const int mode = g_bwd_mode.load();
+  if (mode != 3 || want_dw || h != CCE_BF16 || W->format != CCE_W_DENSE) return f;
+  if (M > SL_MP || W->D > int64_t(SL_MAXC) * SL_DS) return f;
+  int ccl = 1;
+  while (ccl * SL_DS < W->D) ccl <<= 1;
+  const int n_vt = int(ceil_div(W->V, SL_BV));
+  const int ncl = std::min(slice_resident(ccl), n_vt);
+  if (ncl < 1) return f;
+  SliceArgs& a = f.a;
+  a.M = int(M);
+  a.V = int(W->V);
+  a.D = int(W->D);
+  a.Ccl = ccl;
+  a.n_cl = ncl;
+  a.n_vt = n_vt;
+  const int64_t cols = ceil_div(W->V, BN);
+  size_t o = kStatusBytes;
+  f.tile_skip = o; o += align_up(size_t(cols));
+  f.row_skip = o; o += align_up(1);
+  f.parts = o; o += align_up(size_t(ncl) * M * W->D * 4);
+  f.total = std::max(o, make_layout(M, h, W, BN).total);
+  f.ok = true;
+  return f;
+}
+
+cce_status slice_backward(const SlicePlan& sp, const void* H, const cce_head* W,
+                          const int32_t* labels, const float* lse, const float* coeff,
+                          float filter_eps, const float* blockmax, float* dH,
+                          unsigned long long* skip_stats, void* ws, cudaStream_t st) {
+  int sms = 0;
+  cce_status s = device_info(&sms);
+  if (s != CCE_OK) return s;
+  char* wsc = static_cast<char*>(ws);
+  const int64_t M = sp.a.M, V = sp.a.V, D = sp.a.D;
+  const int64_t cols = ceil_div(V, BN);
+  uint8_t* tile_skip = reinterpret_cast<uint8_t*>(wsc + sp.tile_skip);
+  uint8_t* row_skip = reinterpret_cast<uint8_t*>(wsc + sp.row_skip);
+  {
+    const int wpb = 8;
+    ProfScope ps(PK_SKIP, st);
+    skip_plan_kernel<<<int(ceil_div(cols, wpb)), wpb * 32, 0, st>>>(
+        filter_eps > 0.f ? blockmax : nullptr, lse, labels, coeff, int(M), int(cols), 1,
+        filter_eps, tile_skip, row_skip, skip_stats);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+  CUtensorMap mh, mws, mwd;
+  if (!make_map(&mh, H, true, D, M, D, 64, SL_MP) ||
+      !make_map(&mws, W->w, true, D, V, D, 64, SL_BV) ||
+      !make_map(&mwd, W->w, true, D, V, D, 64, 64))
+    return CCE_ERR_CUDA;
+  SliceArgs a = sp.a;
+  a.wait_ns = g_wait_ns.load();
+  a.status = status_word(ws);
+  a.labels = labels;
+  a.lse = lse;
+  a.coeff = coeff;
+  a.filter_eps = filter_eps;
+  // the plan marks vocab blocks only with block skip (blockmax and a filter)
+  a.tile_skip = (filter_eps > 0.f && blockmax != nullptr) ? tile_skip : nullptr;
+  a.row_skip = row_skip;
+  a.softcap = W->softcap;
+  a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
+  a.parts = reinterpret_cast<float*>(wsc + sp.parts);
+  {
+    ProfScope ps(PK_SLICE, st);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.n_cl * a.Ccl);
+    cfg.blockDim = dim3(SL_THREADS);
+    cfg.dynamicSmemBytes = SL_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = a.Ccl;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, slice_kernel(a.Ccl), mh, mws, mwd, a) != cudaSuccess)
+      return CCE_ERR_CUDA;
+  }
+  if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  {
+    const int64_t n4 = M * D / 4;
+    ProfScope ps(PK_SSUM, st);
+    slice_sum_kernel<<<int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(n4, 256), 4 * sms))),
+                       256, 0, st>>>(reinterpret_cast<float4*>(dH),
+                                     reinterpret_cast<const float4*>(a.parts), a.n_cl, n4);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
+  return CCE_OK;
+}
+
 }  // namespace
 
 // ========================================================================
@@ -920,7 +1085,7 @@ void cce_set_cta_pairs(int on) { g_pairs.store(on != 0 ? 1 : 0); }
 
 void cce_set_quant_staging(int mode) { g_qstage.store(mode == 1 || mode == 2 ? mode : 0); }
 
-void cce_set_backward_mode(int mode) { g_bwd_mode.store(mode == 1 || mode == 2 ? mode : 0); }
+void cce_set_backward_mode(int mode) { g_bwd_mode.store(mode >= 1 && mode <= 3 ? mode : 0); }
 
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out) {
@@ -953,6 +1118,21 @@ cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_
     out->bwd_fused_members = fp.a.C;
     out->bwd_fused_buffers = fp.nbuf;
   }
+  const SlicePlan sp = plan_slice(M, h_dtype, W, false);
+  if (sp.ok && sp.total <= ws_bytes) {
+    out->bwd_fused = 0;
+    out->bwd_fused_groups = 0;
+    out->bwd_fused_members = 0;
+    out->bwd_fused_buffers = 0;
+    out->bwd_ok = 1;
+    out->bwd_chunk = 0;
+    out->bwd_ksplit = 1;
+    out->bwd_staged = 0;
+    out->bwd_cta_pairs = 0;
+    out->bwd_sliced = 1;
+    out->bwd_sliced_clusters = sp.a.n_cl;
+    out->bwd_sliced_ctas = sp.a.Ccl;
+  }
   return CCE_OK;
 }
 
@@ -983,6 +1163,8 @@ int64_t cce_blockmax_cols(int64_t V) { return V <= 0 ? 0 : ceil_div(V, BN); }
 
 size_t cce_workspace_bytes(int64_t M, cce_dtype h_dtype, const cce_head* W) {
   if (M <= 0 || check_head(W, h_dtype) != CCE_OK) return 0;
+  const SlicePlan sp = plan_slice(M, h_dtype, W, false);
+  if (sp.ok) return sp.total;
   const FusedPlan fp = plan_fused(M, h_dtype, W, false);
   if (fp.ok) return fp.total;
   const bool staged = q_stage_wanted(M, W, false);  // the backward stages first
@@ -1264,8 +1446,16 @@ static cce_status backward_impl(const void* H, cce_dtype h_dtype, int64_t M, con
   if (s != CCE_OK) return s;
   if (!tiles_fit(M, W)) return CCE_ERR_UNSUPPORTED;
   {
-    // Dense bf16 heads take the fused kernel when the workspace holds its
-    // (small) layout; the two GEMMs per vocab chunk cover the rest.
+    // Dense bf16 heads take a fused kernel when the workspace holds its
+    // (small) layout: by default the grouped one from 1,024 rows (the
+    // sliced one only when mode 3 asks for it); the two GEMMs per vocab
+    // chunk cover the rest.
+    const SlicePlan sp = plan_slice(M, h_dtype, W, dW != nullptr);
+    if (sp.ok && sp.total <= ws_bytes)
+      return slice_backward(sp, H, W, labels, lse, coeff, filter_eps, blockmax, dH, skip_stats,
+                            ws, reinterpret_cast<cudaStream_t>(stream));
+    if (g_bwd_mode.load() == 3)
+      return sp.ok ? CCE_ERR_WORKSPACE_TOO_SMALL : CCE_ERR_UNSUPPORTED;
     const FusedPlan fp = plan_fused(M, h_dtype, W, dW != nullptr);
     if (fp.ok && fp.total <= ws_bytes)
       return fused_backward(fp, H, W, labels, lse, coeff, filter_eps, blockmax, dH, skip_stats,

@@ -307,7 +307,7 @@ def test_fused_plan_choice(lib):
     for M in (64, 512, 1023):
         p0 = cce.cce_query_plan(M, cce.CCE_BF16, big,
                                 lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(big)))
-        assert p0["bwd_ok"] and not p0["bwd_fused"], M
+        assert p0["bwd_ok"] and not p0["bwd_fused"] and not p0["bwd_sliced"], M
     assert cce.cce_query_plan(1024, cce.CCE_BF16, big, ws)["bwd_fused"]
     cce.cce_set_backward_mode(1)   # the fused kernel at any M
     try:
@@ -338,6 +338,41 @@ def test_fused_plan_choice(lib):
         assert not cce.cce_query_plan(8192, cce.CCE_BF16, big, ws)["bwd_fused"]
     finally:
         cce.cce_set_backward_mode(0)
+
+
+def _plan_in_mode(lib, mode, M, h, dtype=cce.CCE_BF16):
+    cce.cce_set_backward_mode(mode)
+    try:
+        ws = lib.cce_workspace_bytes(M, dtype, ctypes.byref(h))
+        return ws, cce.cce_query_plan(M, dtype, h, ws)
+    finally:
+        cce.cce_set_backward_mode(0)
+
+
+def test_sliced_plan_choice(lib):
+    """Mode 3 takes the sliced kernel up to 64 rows of a dense bf16 head with
+    D <= 2048: clusters of the power of two of 256-column slices covering D;
+    its workspace holds one partial dH per cluster.  The default and modes 1
+    and 2 never take it; fp32 and 4-bit heads, D above 2048 and more rows
+    are outside it."""
+    for D, ctas in ((64, 1), (256, 1), (320, 2), (1024, 4), (1536, 8), (2048, 8)):
+        h = _head(V=262144, D=D)
+        for M in (1, 17, 64):
+            ws, p = _plan_in_mode(lib, 3, M, h)
+            assert p["bwd_ok"] and p["bwd_sliced"] and not p["bwd_fused"], (D, M)
+            assert p["bwd_sliced_ctas"] == ctas and p["bwd_chunk"] == 0
+            n_cl = p["bwd_sliced_clusters"]
+            assert 1 <= n_cl <= 148 // ctas
+            assert ws >= n_cl * M * D * 4
+            for mode in (0, 1, 2):
+                assert not _plan_in_mode(lib, mode, M, h)[1]["bwd_sliced"], (mode, D, M)
+    for M in (65, 128):
+        assert not _plan_in_mode(lib, 3, M, _head(V=4096, D=2048))[1]["bwd_sliced"]
+    assert not _plan_in_mode(lib, 3, 64, _head(V=4096, D=2112))[1]["bwd_sliced"]
+    f32 = cce._Head(cce.CCE_W_DENSE, cce.CCE_F32, 4096, 256, 4096, None, None)
+    assert not _plan_in_mode(lib, 3, 64, f32, cce.CCE_F32)[1]["bwd_sliced"]
+    q4 = cce._Head(cce.CCE_W_AFFINE_Q4_G64, cce.CCE_BF16, 128256, 4096, 4096, 4096, 4096)
+    assert not _plan_in_mode(lib, 3, 64, q4)[1]["bwd_sliced"]
 
 
 def _check_schedule(M, V, D, sched, plan):
