@@ -785,7 +785,7 @@ FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
   a.row_rem = int(std::min<int64_t>(M, int64_t(a.waves) * G * TH));
   // remainder: bands of rem groups sharing rounds, then the leftover
   const int64_t T = int64_t(a.rem) * a.n_rounds;
-  a.nb = a.bw = a.lr = a.r0 = a.rl = 0;
+  a.nb = a.bw = a.lr = a.r0 = a.rl = a.ls = 0;
   if (a.rem > 0) {
     if (T >= G) {
       a.nb = G / a.rem;
@@ -795,6 +795,7 @@ FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
         a.lr = r;
         a.r0 = a.nb * a.bw;
         a.rl = a.n_rounds - a.r0;
+        a.ls = 1;  // r < rem: leftover groups take whole tiles first, in step
       }
     } else {
       a.lr = int(T);

@@ -107,6 +107,9 @@ struct FusedArgs {
                   // remainder when it has fewer units than groups
   int r0;         // first round of the leftover
   int rl;         // rounds of the leftover per remainder row tile
+  int ls;         // 1: leftover group l takes remainder row tile l whole (all
+                  // leftover groups in step), and only the other rem - lr
+                  // tiles are cut into ranges
   int n_vt;       // vocab tiles of BV
   int n_rounds;   // ceil(n_vt / C)
   int waves;      // n_rt / G
@@ -152,10 +155,15 @@ struct FUnit {
 //    rounds at the same time.  With G a multiple of rem the bands split R;
 //    otherwise each is bw = floor(rem R / G) rounds wide and
 //  * the leftover rounds [r0, R) of every remainder row tile (rem * rl units)
-//    go to the lr = G mod rem other groups as contiguous ranges of the
-//    sequence (tile, round); a tile may be shared by two or three of them.
+//    go to the lr = G mod rem other groups: leftover group l first takes
+//    remainder row tile l's leftover rounds whole, so the lr groups read the
+//    same rounds of W at the same time (ls = 1); the leftover rounds of
+//    tiles lr .. rem - 1 are then cut into contiguous ranges of the sequence
+//    (tile, round), one per leftover group; a tile may be shared by several
+//    of them.
 //  When the remainder has fewer units than groups, lr = its unit count and
-//  every unit is a leftover unit (nb = 0, r0 = 0, rl = R).
+//  every unit is a leftover unit (nb = 0, r0 = 0, rl = R, ls = 0: all of the
+//  remainder is cut into ranges).
 // A remainder row tile gathers one dH slice per band and one per leftover
 // group that touches it: buffer b for band b, nb + k for the k-th leftover
 // group on the tile.
@@ -177,6 +185,14 @@ __host__ __device__ __forceinline__ void fb_band(const FusedArgs& a, int b, int&
   }
 }
 
+// The leftover's ranged part: tiles [ls ? lr : 0, rem) of rl rounds each.
+__host__ __device__ __forceinline__ int fb_ranged_tile0(const FusedArgs& a) {
+  return a.ls ? a.lr : 0;
+}
+__host__ __device__ __forceinline__ int64_t fb_ranged_units(const FusedArgs& a) {
+  return static_cast<int64_t>(a.rem - fb_ranged_tile0(a)) * a.rl;
+}
+
 __host__ __device__ __forceinline__ int fb_units(const FusedArgs& a, int g) {
   int n = a.waves * a.n_rounds;
   if (a.rem == 0) return n;
@@ -187,8 +203,8 @@ __host__ __device__ __forceinline__ int fb_units(const FusedArgs& a, int g) {
   }
   const int l = g - a.nb * a.rem;
   if (l < a.lr) {
-    const int64_t T = static_cast<int64_t>(a.rem) * a.rl;
-    n += static_cast<int>((l + 1) * T / a.lr - l * T / a.lr);
+    const int64_t T = fb_ranged_units(a);
+    n += (a.ls ? a.rl : 0) + static_cast<int>((l + 1) * T / a.lr - l * T / a.lr);
   }
   return n;
 }
@@ -218,14 +234,25 @@ __host__ __device__ __forceinline__ FUnit fb_unit(const FusedArgs& a, int g, int
     return x;
   }
   const int l = g - a.nb * a.rem;
-  const int64_t T = static_cast<int64_t>(a.rem) * a.rl;
+  if (a.ls && t < a.rl) {
+    // remainder row tile l whole, in step with the other leftover groups
+    x.r = a.waves * a.G + l;
+    x.j = a.r0 + t;
+    x.first = t == 0;
+    x.last = t == a.rl - 1;
+    x.buf = a.nb;
+    return x;
+  }
+  const int tr = a.ls ? t - a.rl : t;
+  const int i0 = fb_ranged_tile0(a);
+  const int64_t T = fb_ranged_units(a);
   const int64_t lo = l * T / a.lr, hi = (l + 1) * T / a.lr;
-  const int64_t e = lo + t;
+  const int64_t e = lo + tr;
   const int i = static_cast<int>(e / a.rl);
   const int jj = static_cast<int>(e - static_cast<int64_t>(i) * a.rl);
-  x.r = a.waves * a.G + i;
+  x.r = a.waves * a.G + i0 + i;
   x.j = a.r0 + jj;
-  x.first = t == 0 || jj == 0;
+  x.first = tr == 0 || jj == 0;
   x.last = (e == hi - 1) || jj == a.rl - 1;
   x.buf = a.nb + l - fb_group_of(static_cast<int64_t>(i) * a.rl, T, a.lr);
   return x;
@@ -236,7 +263,10 @@ __host__ __device__ __forceinline__ FUnit fb_unit(const FusedArgs& a, int g, int
 __host__ __device__ __forceinline__ int fb_slices(const FusedArgs& a, int i) {
   int k = a.nb;
   if (a.lr > 0) {
-    const int64_t T = static_cast<int64_t>(a.rem) * a.rl;
+    const int i0 = fb_ranged_tile0(a);
+    if (i < i0) return k + 1;  // one leftover group takes it whole
+    const int64_t T = fb_ranged_units(a);
+    i -= i0;
     k += fb_group_of(static_cast<int64_t>(i + 1) * a.rl - 1, T, a.lr) -
          fb_group_of(static_cast<int64_t>(i) * a.rl, T, a.lr) + 1;
   }

@@ -415,6 +415,16 @@ def _check_schedule(M, V, D, sched, plan):
             seqs = [sched[sched[:, 0] == g][waves * n_rounds:, 2].tolist()
                     for g in range(band * rem, (band + 1) * rem)]
             assert all(q == seqs[0] for q in seqs), band
+        # then the leftover groups run the leftover rounds of one remainder
+        # row tile each, in step with each other
+        lr = G % rem
+        if lr:
+            bw = rem * n_rounds // G
+            rl = n_rounds - nb * bw
+            for g in range(nb * rem, nb * rem + lr):
+                s = sched[sched[:, 0] == g][waves * n_rounds:]
+                assert np.array_equal(s[:rl, 2], np.arange(nb * bw, n_rounds)), g
+                assert np.all(s[:rl, 1] == waves * G + g - nb * rem), g
     for r, b in bufs.items():
         assert sorted(b) == list(range(len(b))), (r, b)
         assert len(b) <= plan["bwd_fused_buffers"]
