@@ -544,9 +544,9 @@ def run_small_m(args, quant=False):
     counts the method's minimum bytes: W once per pass (as stored: 16 or 4.25
     bits per weight), H in, dH out and the per-row / per-block statistics.
     design_bytes are the bytes the backward that ran must move: the fused
-    backward (dense bf16 heads) reads W from HBM once and adds its partial dH
-    buffers; the two-GEMM backward (4/8-bit heads) reads W twice and moves
-    G'' through HBM."""
+    backwards (dense bf16 heads) read W from HBM once and add their partial
+    dH buffers; the two-GEMM backward reads W twice and moves G'' through
+    HBM.  With --backward-mode 3 (the sliced backward) only M = 64 runs."""
     import torch
 
     from lm_head_cross_flash_b200 import cce
@@ -558,6 +558,10 @@ def run_small_m(args, quant=False):
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     lines = []
     for M in (64, 128, 256):
+        if args.backward_mode == 3 and M > 64:
+            lines.append({"sweep": "small_m_q4" if quant else "small_m", "M": M,
+                          "skipped": "the sliced backward (mode 3) takes at most 64 rows"})
+            continue
         P = M // 8
         Rc = (M - P) // 2
         if quant:

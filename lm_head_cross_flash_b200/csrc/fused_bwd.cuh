@@ -135,8 +135,10 @@ struct FusedArgs {
 // Groups may run at most this many units ahead of the slowest group during
 // the waves: the groups then read the same rounds of W within a few units
 // of each other and share them in L2 (left alone they drift apart over a
-// wave, and each straggler streams W from HBM on its own).
-constexpr int FB_LEAD = 2;
+// wave, and each straggler streams W from HBM on its own).  Measured at the
+// long pair, three runs each on one box: a lead of 1 unit 13.05-13.24 ms per
+// launch, 2 units 13.30-13.44 ms, 4 units 13.39-13.92 ms.
+constexpr int FB_LEAD = 1;
 constexpr uint64_t FB_LEAD_WAIT_NS = 200000;  // a hint: give up after 0.2 ms
 
 // One unit of group g's sequence: row tile r, round j; first / last unit of
