@@ -1,0 +1,382 @@
+"""CPU models of the two fused backward kernels' synchronisation protocols.
+
+Each model replays, step by step, the waits and signals that every role of
+every CTA issues (the order the kernel code issues them in), over the
+library's own schedule where one exists, with random skip patterns, and
+checks that every role runs to the end: no deadlock.  The GPU waits are
+bounded, so a protocol error shows as a device timeout, not a hang; these
+models find such errors on the CPU first.  Planted mistakes (a wait one fill
+too far, a missing signal, a missing arm) must make the models stall, which
+shows that they can.
+
+* The grouped fused kernel (fused_bwd.cuh): per member, a producer, an MMA
+  issuer and the epilogue; a FIFO ring of operand stages shared by the
+  S-phase and dH-phase loads; the G'' exchange ring of DEPTH fills per
+  (group, member) with its ready and consumed counters; the S and dH
+  accumulator barriers.  The lead cap is a bounded hint, not a dependency,
+  and is left out.  A CTA pair runs as one member.
+* The sliced kernel (slice_bwd.cuh): per CTA of a cluster, the S and dH
+  loaders and MMA issuers, the drain warps and the reducer warps, with the
+  double-buffered partial (pfull, pempty), G'' (gfull, gempty) and S
+  accumulator (afull, aempty) barriers.  Barriers are phase objects: an
+  arrival or byte count lands in whatever phase is current, and the model
+  asserts it belongs to that phase's tile (so a sender that runs a phase
+  ahead is an error, as it would be on the GPU).
+"""
+
+import ctypes
+import random
+
+import pytest
+
+from lm_head_cross_flash_b200 import cce
+
+
+# --------------------------------------------------------------- machinery --
+def _run(procs, step):
+    """procs: list of (state, [op lists]).  Runs every op list as far as its
+    next op allows, until nothing moves.  Returns the list of stuck
+    (process, role, position, length)."""
+    pos = [[0] * len(lists) for _, lists in procs]
+    moved = True
+    while moved:
+        moved = False
+        for i, (st, lists) in enumerate(procs):
+            for r, ops in enumerate(lists):
+                while pos[i][r] < len(ops) and step(st, *ops[pos[i][r]]):
+                    pos[i][r] += 1
+                    moved = True
+    return [(i, r, pos[i][r], len(ops)) for i, (_, lists) in enumerate(procs)
+            for r, ops in enumerate(lists) if pos[i][r] < len(ops)]
+
+
+# ------------------------------------------------------ grouped fused kernel --
+FB_DEPTH = 2
+
+
+def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
+    lib = cce.lib()
+    h = cce._Head(cce.CCE_W_DENSE, cce.CCE_BF16, V, D, D, None, None)
+    cce.cce_set_backward_mode(1)
+    cce.cce_set_cta_pairs(pairs)
+    try:
+        plan = cce.cce_query_plan(M, cce.CCE_BF16, h,
+                                  lib.cce_workspace_bytes(M, cce.CCE_BF16, ctypes.byref(h)))
+        sched = cce.cce_query_fused_schedule(M, cce.CCE_BF16, h)
+    finally:
+        cce.cce_set_backward_mode(0)
+        cce.cce_set_cta_pairs(True)
+    assert plan["bwd_fused"]
+    C, G = plan["bwd_fused_members"], plan["bwd_fused_groups"]
+    c2 = bool(plan["bwd_cta_pairs"])
+    nk = -(-D // 64)                  # K steps of an S tile
+    kv = (256 if c2 else 128) // 64   # K steps of a dH tile
+    nst = 6 if c2 else 4              # operand stages
+    sbufs = 1 if c2 else 2            # S accumulators
+    rng = random.Random(seed)
+    skips = {}
+
+    def skip(r, v):
+        if (r, v) not in skips:
+            skips[(r, v)] = rng.random() < skip_prob
+        return skips[(r, v)]
+
+    units = {g: [tuple(int(x) for x in row[1:]) for row in sched[sched[:, 0] == g]]
+             for g in range(G)}
+    shared = {"ready": {}, "consumed": {}}
+    procs = []
+    for g in range(G):
+        U = units[g]
+        for p in range(C):
+            P, X, E = [], [], []
+            # producer: S loads of unit u, then the dH loads of unit u - 1
+            for u in range(len(U) + 1):
+                if u < len(U):
+                    r, j = U[u][0], U[u][1]
+                    if not skip(r, j * C + p):
+                        P += [("load",)] * nk
+                if u >= 1:
+                    r, j = U[u - 1][0], U[u - 1][1]
+                    fill = (u - 1) // FB_DEPTH
+                    for q in range(C):
+                        if skip(r, j * C + q):
+                            continue
+                        P.append(("wait_ready", (g, (u - 1) % FB_DEPTH, q), fill + 1))
+                        P += [("load",)] * kv
+            # MMA: S(u), then dH(u - 1)
+            ns = nseg = 0
+            dh_any = False
+            for u in range(len(U) + 1):
+                if u < len(U):
+                    r, j = U[u][0], U[u][1]
+                    if not skip(r, j * C + p):
+                        X.append(("wait_s_empty", ns))
+                        X += [("consume",)] * nk
+                        X.append(("s_full",))
+                        ns += 1
+                if u >= 1:
+                    r, j, first, last = U[u - 1][0], U[u - 1][1], U[u - 1][2], U[u - 1][3]
+                    fill = (u - 1) // FB_DEPTH
+                    if first:
+                        dh_any = False
+                    for q in range(C):
+                        key = (g, (u - 1) % FB_DEPTH, q, p)
+                        if skip(r, j * C + q):
+                            if bug != "no_consumed_on_skip":
+                                X.append(("set_consumed", key, fill + 1))
+                            continue
+                        if not dh_any:
+                            X.append(("wait_dh_empty", nseg))
+                        X += [("consume",)] * kv
+                        X.append(("set_consumed", key, fill + 1))
+                        dh_any = True
+                    if last and dh_any:
+                        X.append(("dh_full",))
+                        nseg += 1
+            # epilogue: publish G''(u) once every member consumed the slot's
+            # previous fill; flush a finished segment's dH
+            ns = nseg = 0
+            prev, seg_any, prev_any = None, False, False
+            for u in range(len(U)):
+                r, j, first = U[u][0], U[u][1], U[u][2]
+                if first:
+                    seg_any = False
+                seg_any = seg_any or any(not skip(r, j * C + q) for q in range(C))
+                fill = u // FB_DEPTH
+                if not skip(r, j * C + p):
+                    E.append(("wait_s_full", ns))
+                    need = fill + 1 if bug == "consumed_off_by_one" else fill
+                    if fill >= 1:
+                        for c in range(C):
+                            E.append(("wait_consumed", (g, u % FB_DEPTH, p, c), need))
+                    E.append(("s_empty",))
+                    ns += 1
+                E.append(("ready_add", (g, u % FB_DEPTH, p)))
+                if u >= 1 and prev[3] and prev_any:
+                    E += [("wait_dh_full", nseg), ("dh_empty",)]
+                    nseg += 1
+                prev, prev_any = U[u], seg_any
+            if prev is not None and prev_any:
+                E += [("wait_dh_full", nseg), ("dh_empty",)]
+            st = dict(ring=0, s_full=0, s_empty=0, dh_full=0, dh_empty=0)
+            procs.append((st, [P, X, E]))
+
+    def step(st, op, *arg):
+        if op == "load":
+            if st["ring"] >= nst:
+                return False
+            st["ring"] += 1
+            return True
+        if op == "consume":
+            if st["ring"] <= 0:
+                return False
+            st["ring"] -= 1
+            return True
+        if op == "wait_ready":
+            return shared["ready"].get(arg[0], 0) >= arg[1]
+        if op == "set_consumed":
+            shared["consumed"][arg[0]] = arg[1]
+            return True
+        if op == "wait_consumed":
+            return shared["consumed"].get(arg[0], 0) >= arg[1]
+        if op == "ready_add":
+            shared["ready"][arg[0]] = shared["ready"].get(arg[0], 0) + 1
+            return True
+        if op == "wait_s_empty":
+            return st["s_empty"] >= arg[0] - sbufs + 1
+        if op == "wait_s_full":
+            return st["s_full"] > arg[0]
+        if op == "wait_dh_empty":
+            return st["dh_empty"] >= arg[0]
+        if op == "wait_dh_full":
+            return st["dh_full"] > arg[0]
+        if op in ("s_full", "s_empty", "dh_full", "dh_empty"):
+            st[op] += 1
+            return True
+        raise ValueError(op)
+
+    return _run(procs, step)
+
+
+FUSED_SHAPES = [(8192, 16384, 2048, True), (300, 1000, 320, True), (64, 20000, 2048, False),
+                (5000, 3000, 2048, True), (2048, 7000, 1536, True), (1, 31, 64, False),
+                (129, 4097, 256, True), (900, 6000, 256, False)]
+
+
+@pytest.mark.parametrize("M,V,D,pairs", FUSED_SHAPES)
+@pytest.mark.parametrize("skip_prob", [0.0, 0.3, 0.9])
+def test_fused_protocol_runs_to_the_end(M, V, D, pairs, skip_prob):
+    assert _fused_model(M, V, D, skip_prob, seed=M + V, pairs=pairs) == []
+
+
+@pytest.mark.parametrize("bug,skip_prob", [("consumed_off_by_one", 0.0),
+                                           ("no_consumed_on_skip", 0.3)])
+def test_fused_protocol_model_catches_planted_mistakes(bug, skip_prob):
+    assert _fused_model(2048, 7000, 1536, skip_prob, seed=5, bug=bug) != []
+
+
+# ------------------------------------------------------------ sliced kernel --
+class _Phase:
+    """An mbarrier: a phase completes when `count` arrivals and the armed
+    bytes have all landed; arrivals and bytes tagged with the tile they
+    belong to, which must be the current phase's tile."""
+
+    def __init__(self, count, tiles):
+        self.count, self.tiles = count, tiles  # tiles: the tile of each phase, in order
+        self.phase, self.arrived, self.tx = 0, 0, 0
+
+    def cur(self):
+        return self.tiles[self.phase] if self.phase < len(self.tiles) else None
+
+    def _maybe_complete(self):
+        if self.arrived == self.count and self.tx == 0:
+            self.phase += 1
+            self.arrived = 0
+
+    def arrive(self, tile, expect=0):
+        assert tile == self.cur(), f"arrival for tile {tile} in the phase of tile {self.cur()}"
+        self.arrived += 1
+        self.tx += expect
+        self._maybe_complete()
+
+    def bytes(self, tile, n):
+        assert tile == self.cur(), f"bytes for tile {tile} in the phase of tile {self.cur()}"
+        self.tx -= n
+        self._maybe_complete()
+
+    def done(self, tile):
+        """Has the phase of `tile` completed?"""
+        return tile in self.tiles[:self.phase]
+
+
+class ProtocolError(AssertionError):
+    """A signal that would land in another tile's barrier phase."""
+
+
+def _sliced_model(n, ccl, ns=4, nd=2, nbuf=2, bug=None):
+    epi = 4
+    tiles_of = lambda b: list(range(b, n, nbuf))
+    ctas = []
+    for c in range(ccl):
+        st = dict(
+            sring=0, dring=0,
+            afull=[_Phase(1, tiles_of(b)) for b in range(nbuf)],
+            aempty=[_Phase(epi, tiles_of(b)) for b in range(nbuf)],
+            pfull=[_Phase(1, tiles_of(b)) for b in range(nbuf)],
+            pempty=[_Phase(ccl * epi, [k for k in tiles_of(b) if k + nbuf < n])
+                    for b in range(nbuf)],
+            gfull=[_Phase(1 + epi, tiles_of(b)) for b in range(nbuf)],
+            gempty=[_Phase(ccl, [k for k in tiles_of(b) if k + nbuf < n]) for b in range(nbuf)],
+            dhfull=_Phase(1, [0]))
+        ctas.append(st)
+    part = 1      # bytes one drain warp sends to one reducer per tile
+    grows = 1     # bytes one reducer warp copies to one peer per tile
+    for st in ctas:   # the first tiles' arms
+        for b in range(min(nbuf, n)):
+            st["pfull"][b].arrive(b, expect=ccl * epi * part)
+            st["gfull"][b].arrive(b, expect=(ccl - 1) * epi * grows)
+
+    procs = []
+    for c, st in enumerate(ctas):
+        sprod = [("sload",)] * (4 * n)
+        dprod = [("dload",)] * (4 * n)
+        smma, dmma = [], []
+        for k in range(n):
+            b = k % nbuf
+            if k >= nbuf:
+                smma.append(("wait", c, "aempty", b, k - nbuf))
+            smma += [("sconsume",)] * 4
+            smma.append(("arrive", c, "afull", b, k, 0))
+        for k in range(n):
+            b = k % nbuf
+            dmma.append(("wait", c, "gfull", b, k))
+            dmma += [("dconsume",)] * 4
+            if k + nbuf < n:
+                dmma += [("arrive", q, "gempty", b, k, 0) for q in range(ccl)]
+                if bug != "no_gfull_arm":
+                    dmma.append(("arrive", c, "gfull", b, k + nbuf, (ccl - 1) * epi * grows))
+        dmma.append(("arrive", c, "dhfull", 0, 0, 0))
+        roles = [sprod, dprod, smma, dmma]
+        for w in range(epi):   # drain warps
+            d = []
+            for j in range(n):
+                b = j % nbuf
+                d.append(("wait", c, "afull", b, j))
+                d.append(("arrive", c, "aempty", b, j, 0))
+                if j >= nbuf:
+                    d.append(("wait", c, "pempty", b, j - nbuf))
+                d += [("bytes", q, "pfull", b, j, part) for q in range(ccl)]
+            d.append(("wait", c, "dhfull", 0, 0))
+            roles.append(d)
+        for w in range(epi):   # reducer warps
+            r = []
+            for k in range(n):
+                b = k % nbuf
+                r.append(("wait", c, "pfull", b, k))
+                if k >= nbuf:
+                    r.append(("wait", c, "gempty", b, k - nbuf))
+                if k + nbuf < n:
+                    if w == 0:
+                        r.append(("arrive", c, "pfull", b, k + nbuf, ccl * epi * part))
+                    if bug != "no_pempty":
+                        r += [("arrive", q, "pempty", b, k, 0) for q in range(ccl)]
+                r += [("bytes", q, "gfull", b, k, grows) for q in range(ccl) if q != c]
+                r.append(("arrive", c, "gfull", b, k, 0))
+            roles.append(r)
+        procs.append((st, roles))
+
+    def step(st, op, *a):
+        if op == "sload":
+            if st["sring"] >= ns:
+                return False
+            st["sring"] += 1
+            return True
+        if op == "sconsume":
+            if st["sring"] <= 0:
+                return False
+            st["sring"] -= 1
+            return True
+        if op == "dload":
+            if st["dring"] >= nd:
+                return False
+            st["dring"] += 1
+            return True
+        if op == "dconsume":
+            if st["dring"] <= 0:
+                return False
+            st["dring"] -= 1
+            return True
+        cta, name, b, tile = a[0], a[1], a[2], a[3]
+        bar = ctas[cta][name] if name == "dhfull" else ctas[cta][name][b]
+        if op == "wait":
+            return bar.done(tile)
+        if bar.cur() != tile:
+            # the protocol must never signal ahead of the barrier's phase
+            raise ProtocolError(f"{op} for tile {tile} on {name}[{b}] of CTA {cta}, "
+                                f"whose current phase is tile {bar.cur()}")
+        if op == "arrive":
+            bar.arrive(tile, expect=a[4])
+        else:
+            bar.bytes(tile, a[4])
+        return True
+        raise ValueError(op)
+
+    return _run(procs, step)
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 7, 30])
+@pytest.mark.parametrize("ccl", [1, 2, 4, 8])
+def test_sliced_protocol_runs_to_the_end(n, ccl):
+    assert _sliced_model(n, ccl) == []
+
+
+@pytest.mark.parametrize("ns,nd,nbuf", [(2, 1, 2), (4, 4, 2), (1, 1, 2), (4, 2, 1), (4, 2, 3)])
+def test_sliced_protocol_other_depths(ns, nd, nbuf):
+    """Ring depths and buffer counts other than the kernel's (4, 2, 2) also
+    run to the end: nothing in the protocol relies on a particular depth."""
+    assert _sliced_model(9, 8, ns=ns, nd=nd, nbuf=nbuf) == []
+
+
+@pytest.mark.parametrize("bug", ["no_pempty", "no_gfull_arm"])
+def test_sliced_protocol_model_catches_planted_mistakes(bug):
+    assert _sliced_model(6, 4, bug=bug) != []
