@@ -170,10 +170,18 @@ struct FUnit {
 // group that touches it: buffer b for band b, nb + k for the k-th leftover
 // group on the tile.
 
-// Leftover group containing leftover unit e (T units over lr groups, group
-// l holding [l T / lr, (l + 1) T / lr)).
+// Ranges of the leftover: T units over lr groups, q = T / lr each and one
+// more for the first T mod lr groups, so the groups holding units (and the
+// groups touching any one row tile) are consecutive.  Group l holds
+// [fb_range_lo(l), fb_range_lo(l + 1)).
+__host__ __device__ __forceinline__ int64_t fb_range_lo(int64_t l, int64_t T, int lr) {
+  const int64_t q = T / lr, r = T % lr;
+  return l * q + (l < r ? l : r);
+}
+// Leftover group holding leftover unit e.
 __host__ __device__ __forceinline__ int fb_group_of(int64_t e, int64_t T, int lr) {
-  return static_cast<int>(((e + 1) * lr - 1) / T);
+  const int64_t q = T / lr, r = T % lr, big = r * (q + 1);
+  return static_cast<int>(e < big ? e / (q + 1) : r + (e - big) / q);
 }
 
 // Round range [lo, hi) of band b.
@@ -206,7 +214,7 @@ __host__ __device__ __forceinline__ int fb_units(const FusedArgs& a, int g) {
   const int l = g - a.nb * a.rem;
   if (l < a.lr) {
     const int64_t T = fb_ranged_units(a);
-    n += (a.ls ? a.rl : 0) + static_cast<int>((l + 1) * T / a.lr - l * T / a.lr);
+    n += (a.ls ? a.rl : 0) + static_cast<int>(fb_range_lo(l + 1, T, a.lr) - fb_range_lo(l, T, a.lr));
   }
   return n;
 }
@@ -248,7 +256,7 @@ __host__ __device__ __forceinline__ FUnit fb_unit(const FusedArgs& a, int g, int
   const int tr = a.ls ? t - a.rl : t;
   const int i0 = fb_ranged_tile0(a);
   const int64_t T = fb_ranged_units(a);
-  const int64_t lo = l * T / a.lr, hi = (l + 1) * T / a.lr;
+  const int64_t lo = fb_range_lo(l, T, a.lr), hi = fb_range_lo(l + 1, T, a.lr);
   const int64_t e = lo + tr;
   const int i = static_cast<int>(e / a.rl);
   const int jj = static_cast<int>(e - static_cast<int64_t>(i) * a.rl);

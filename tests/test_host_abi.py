@@ -433,7 +433,8 @@ def _check_schedule(M, V, D, sched, plan):
 
 @pytest.mark.parametrize("M,V,D", [(8192, 262144, 2048), (2048, 73440, 1536), (64, 262144, 2048),
                                    (1, 300, 64), (300, 1000, 320), (32768, 128256, 4096),
-                                   (129, 4097, 256), (5000, 3000, 2048)])
+                                   (129, 4097, 256), (5000, 3000, 2048),
+                                   (6145, 769, 64)])   # fewer ranged units than groups
 def test_fused_schedule_covers_every_unit_once(lib, M, V, D, fused_backward):
     h = _head(V=V, D=D)
     plan = cce.cce_query_plan(M, cce.CCE_BF16, h,
