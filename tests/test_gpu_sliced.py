@@ -170,3 +170,41 @@ def test_sliced_outside_its_range_is_refused():
         assert e.value.status == 2
     finally:
         cce.cce_set_backward_mode(0)
+
+
+@pytest.mark.parametrize("scope", ["full", "response"])
+def test_sliced_through_the_real_pass(scope):
+    """The whole head pass (forward, loss, cotangent, dH) with the sliced
+    backward, against the oracle; the response scope zeroes the prompt rows'
+    cotangent.  Then the same pass captured in a CUDA graph and replayed
+    gives the direct call's bits."""
+    wl = S.make_custom(2, M_split=(12, 24, 28), D=2048, V=9000)
+    wl.scope = scope
+    H, head, labels = upload(wl)
+    hd = cce.h_dtype(H)
+    cce.cce_set_backward_mode(3)
+    try:
+        direct = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+        graphed = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+        args = (wl.layout_tuple, wl.lam, wl.scope, wl.filter_eps, wl.block_skip)
+        cce.orpo_head_pass(H, head, labels, *args, direct)
+        g = cce.HeadPassGraph(H, head, labels, *args, graphed)
+        g.replay()
+        torch.cuda.synchronize()
+    finally:
+        cce.cce_set_backward_mode(0)
+    assert cce.cce_device_status(direct.ws) == 0
+    assert cce.cce_device_status(graphed.ws) == 0
+    W = oracle_W(wl)
+    L = O.Layout(*wl.layout_tuple)
+    ologp, olse, _ = O.head_forward(wl.H, W, wl.labels)
+    o = O.orpo_loss_from_logps(ologp, wl.labels, L, wl.lam, scope)
+    gc = O.orpo_grad_coeffs(ologp, wl.labels, L, wl.lam, scope)
+    odh = O.head_dh(wl.H, W, wl.labels, gc, olse)
+    out8 = direct.out8.cpu().numpy()
+    assert abs(out8[0] - o.loss) <= 1e-3 * abs(o.loss)
+    assert rel_fro(direct.coeff.cpu().numpy(), gc) <= 1e-5
+    assert rel_fro(direct.dH.cpu().numpy(), odh) <= TOL_DH
+    for name in ("logp", "lse", "out8", "coeff", "dH"):
+        assert np.array_equal(getattr(graphed, name).cpu().numpy(),
+                              getattr(direct, name).cpu().numpy()), name
