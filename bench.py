@@ -125,12 +125,43 @@ def choose_peak(peaks: dict, src: str, clk: dict, timed_s: float) -> dict:
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "fused_bwd.cuh", "ptx.cuh", "cce.cu")
 
 
-def source_hash() -> str:
-    h = hashlib.sha256()
+def strip_comments(text: str) -> str:
+    """C/C++ source without its comments and with whitespace collapsed, so
+    that a comment-only edit leaves the hash of the code unchanged (string
+    and character literals are kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def source_hash(read=None) -> str:
+    """Hash of the code (comments stripped) of TRAFFIC_SOURCES; `read(name)`
+    returns a file's text (default: the working tree)."""
     src = os.path.join(ROOT, "lm_head_cross_flash_b200", "csrc")
+    if read is None:
+        def read(n):
+            with open(os.path.join(src, n), encoding="utf-8") as f:
+                return f.read()
+    h = hashlib.sha256()
     for n in TRAFFIC_SOURCES:
-        with open(os.path.join(src, n), "rb") as f:
-            h.update(n.encode() + f.read())
+        h.update(n.encode() + strip_comments(read(n)).encode())
     return h.hexdigest()[:16]
 
 

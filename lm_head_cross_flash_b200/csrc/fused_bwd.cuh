@@ -16,9 +16,11 @@
 // its G'' tile and publishes it in a small ring of tiles in global memory
 // that stays in L2; then every member contracts all C published tiles of the
 // round with its own d-columns of W (K = C tiles of vocabulary).  The S GEMM
-// of one round overlaps the dH GEMM of the previous one, so a member's tensor
-// pipe never waits for the exchange.  G'' never exists as a whole: one ring
-// holds DEPTH rounds of tiles per group.
+// of one round is issued before the dH GEMM of the previous one, so the
+// exchange has a whole S GEMM to complete in before its tiles are needed
+// (what is left of the wait measured about 15 % of a unit at the long pair).
+// G'' never exists as a whole: one ring holds DEPTH rounds of tiles per
+// group.
 //
 // Roles (192 threads, as in gemm_tc.cuh): warp 0 loads operand stages by
 // TMA (the S phase: H rows and W rows, both K-major; the dH phase: a G''
