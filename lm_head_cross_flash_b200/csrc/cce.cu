@@ -741,7 +741,7 @@ struct FusedPlan {
   FusedArgs a{};
   int nbuf = 1;
   int64_t ring_rows = 0;
-  size_t tile_skip = 0, row_skip = 0, flags = 0, ring = 0, parts = 0, total = 0;
+  size_t tile_skip = 0, row_skip = 0, umask = 0, flags = 0, ring = 0, parts = 0, total = 0;
 };
 
 // Choosing between the fused backward and the two GEMMs: below this many
@@ -808,6 +808,7 @@ FusedPlan plan_fused(int64_t M, cce_dtype h, const cce_head* W, bool want_dw) {
   size_t o = kStatusBytes;
   f.tile_skip = o; o += align_up(size_t(n128) * cols);
   f.row_skip = o; o += align_up(size_t(n128));
+  f.umask = o; o += align_up(size_t(a.n_rt) * a.n_rounds * 4);
   f.flags = o; o += align_up((size_t(G) * FB_DEPTH * C * (2 + C) + G) * 4);
   f.ring = o; o += align_up(size_t(f.ring_rows) * BV * 2);
   f.parts = o; o += align_up(size_t(f.nbuf - 1) * (M - a.row_rem) * W->D * 4);
@@ -889,6 +890,19 @@ cce_status fused_backward(const FusedPlan& fp, const void* H, const cce_head* W,
   a.ready = reinterpret_cast<uint32_t*>(wsc + fp.flags);
   a.consumed = a.ready + size_t(p.G) * FB_DEPTH * p.C * 2;
   a.progress = a.consumed + size_t(p.G) * FB_DEPTH * p.C * p.C;
+  {
+    // every unit's skip mask, once, before the backward reads them
+    uint32_t* um = reinterpret_cast<uint32_t*>(wsc + fp.umask);
+    const int64_t units = int64_t(p.n_rt) * p.n_rounds;
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, 256), 4 * sms)));
+    ProfScope ps(PK_SKIP, st);
+    if (fp.c2)
+      fused_mask_kernel<true, FusedCfg<true>::BV><<<grid, 256, 0, st>>>(a, um);
+    else
+      fused_mask_kernel<false, FusedCfg<false, 128>::BV><<<grid, 256, 0, st>>>(a, um);
+    if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+    a.unit_mask = um;
+  }
   {
     ProfScope ps(PK_FUSED, st);
     const int members = a.G * a.C;

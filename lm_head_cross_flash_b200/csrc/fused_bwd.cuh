@@ -127,6 +127,7 @@ struct FusedArgs {
   const uint8_t* tile_skip;  // [n_rt128, skip_ld], 256-vocab blocks
   int skip_ld;
   const uint8_t* row_skip;   // [n_rt128]
+  const uint32_t* unit_mask;  // [n_rt, n_rounds]: fb_mask_of for every unit
   float softcap;
   float inv_cap;
   uint32_t* ready;     // [G * DEPTH * C * 2]
@@ -288,11 +289,10 @@ __host__ __device__ __forceinline__ int fb_slices(const FusedArgs& a, int i) {
 // Tiles of round j with nothing to compute for row tile r, as bits q of a
 // mask (vocab tile j*C + q): past the vocabulary, or every 128-row half
 // either past M, without a nonzero cotangent, or block-skipped for the
-// 256-wide vocabulary block holding the tile.  Its loads are independent of
-// each other, and every role computes the mask of the next unit while it
-// works on the current one, so their latency stays off the issue path.
+// 256-wide vocabulary block holding the tile.  fused_mask_kernel evaluates
+// it once per unit before the backward starts.
 template <bool C2, int BV>
-__device__ __forceinline__ uint32_t fb_mask(const FusedArgs& a, int r, int j) {
+__device__ __forceinline__ uint32_t fb_mask_of(const FusedArgs& a, int r, int j) {
   const int v0 = j * a.C;
   uint32_t past = 0;
   for (int q = 0; q < a.C; ++q)
@@ -309,6 +309,26 @@ __device__ __forceinline__ uint32_t fb_mask(const FusedArgs& a, int r, int j) {
     return m;
   };
   return past | (C2 ? (half(2 * r) & half(2 * r + 1)) : half(r));
+}
+
+// The skip mask of unit (r, j) for the kernel's roles: one word from the
+// table, loaded a unit before it is used.  (Evaluating fb_mask_of in the
+// roles themselves chained up to four L2 round trips onto every unit's
+// issue path: the long pair ran about 9 % slower with block skip on, even
+// when nothing was skipped.)
+__device__ __forceinline__ uint32_t fb_mask(const FusedArgs& a, int r, int j) {
+  return a.unit_mask[static_cast<size_t>(r) * a.n_rounds + j];
+}
+
+// unit_mask[r][j] = fb_mask_of(a, r, j) for every row tile and round.
+template <bool C2, int BV>
+__global__ void fused_mask_kernel(FusedArgs a, uint32_t* __restrict__ out) {
+  const int64_t n = static_cast<int64_t>(a.n_rt) * a.n_rounds;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / a.n_rounds);
+    out[i] = fb_mask_of<C2, BV>(a, r, static_cast<int>(i - static_cast<int64_t>(r) * a.n_rounds));
+  }
 }
 
 template <bool C2, int BVS>
@@ -416,13 +436,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t mk_prev = 0, mk_cur = 0;
       if (n_u > 0) {
         const FUnit x0 = fb_unit(a, g, 0);
-        mk_cur = fb_mask<C2, F::BV>(a, x0.r, x0.j);
+        mk_cur = fb_mask(a, x0.r, x0.j);
       }
       for (int u = 0; u <= n_u && ok; ++u) {
         uint32_t mk_next = 0;
         if (u + 1 < n_u) {
           const FUnit xn = fb_unit(a, g, u + 1);
-          mk_next = fb_mask<C2, F::BV>(a, xn.r, xn.j);
+          mk_next = fb_mask(a, xn.r, xn.j);
         }
         if (u < n_u && p == 0 && rank == 0 && u < a.waves * a.n_rounds) {
           st_relaxed_gpu(&a.progress[g], static_cast<uint32_t>(u));
@@ -522,13 +542,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t mk_prev = 0, mk_cur = 0;
       if (n_u > 0) {
         const FUnit x0 = fb_unit(a, g, 0);
-        mk_cur = fb_mask<C2, F::BV>(a, x0.r, x0.j);
+        mk_cur = fb_mask(a, x0.r, x0.j);
       }
       for (int u = 0; u <= n_u && ok; ++u) {
         uint32_t mk_next = 0;
         if (u + 1 < n_u) {
           const FUnit xn = fb_unit(a, g, u + 1);
-          mk_next = fb_mask<C2, F::BV>(a, xn.r, xn.j);
+          mk_next = fb_mask(a, xn.r, xn.j);
         }
         if (u < n_u) {
           if (!((mk_cur >> p) & 1u)) {
@@ -720,13 +740,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t mk_cur = 0;
     if (n_u > 0) {
       const FUnit x0 = fb_unit(a, g, 0);
-      mk_cur = fb_mask<C2, F::BV>(a, x0.r, x0.j);
+      mk_cur = fb_mask(a, x0.r, x0.j);
     }
     for (int u = 0; u < n_u && ok; ++u) {
       uint32_t mk_next = 0;
       if (u + 1 < n_u) {
         const FUnit xn = fb_unit(a, g, u + 1);
-        mk_next = fb_mask<C2, F::BV>(a, xn.r, xn.j);
+        mk_next = fb_mask(a, xn.r, xn.j);
       }
       const FUnit x = fb_unit(a, g, u);
       if (x.first) seg_any = false;
