@@ -199,3 +199,33 @@ def test_fused_workspace_too_small_is_reported():
     cce.cce_backward_dh(H, head, labels, lse, coeff, 0.0, None, dH, None, small)
     torch.cuda.synchronize()
     assert cce.cce_device_status(small) == 0
+
+
+@pytest.mark.parametrize("block_skip", [False, True])
+def test_fused_pass_graph_replay(block_skip):
+    """The whole head pass with the fused backward (the default from 1,024
+    rows) captured in a CUDA graph and replayed gives the direct call's
+    bits, also after new inputs are copied into the captured tensors; with
+    the filter and block skip on, too (the skip plan, the mask table and the
+    exchange counters are rebuilt inside the graph each replay)."""
+    wl = S.make_custom(1, M_split=(100, 500, 500), D=256, V=30000, alpha=12.0)
+    H, head, labels = upload(wl)
+    hd = cce.h_dtype(H)
+    direct = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+    graphed = cce.HeadBuffers.alloc(wl.M, wl.D, wl.V, hd, head)
+    assert cce.cce_query_plan(wl.M, hd, head, direct.ws.numel())["bwd_fused"]
+    eps = 1e-6 if block_skip else 0.0
+    args = (wl.layout_tuple, wl.lam, wl.scope, eps, block_skip)
+    g = cce.HeadPassGraph(H, head, labels, *args, graphed)
+    for step in range(2):
+        if step == 1:
+            H.copy_(torch.roll(H, shifts=1, dims=0))
+            labels.copy_(torch.roll(labels, shifts=3))
+        g.replay()
+        cce.orpo_head_pass(H, head, labels, *args, direct)
+        torch.cuda.synchronize()
+        assert cce.cce_device_status(graphed.ws) == 0
+        assert cce.cce_device_status(direct.ws) == 0
+        for name in ("logp", "lse", "out8", "coeff", "dH"):
+            assert np.array_equal(getattr(graphed, name).cpu().numpy(),
+                                  getattr(direct, name).cpu().numpy()), (step, name)
