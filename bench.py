@@ -54,6 +54,9 @@ def parse_args(argv=None):
     p.add_argument("--backward-mode", type=int, choices=[0, 1, 2, 3], default=0,
                    help="dense bf16 heads: 0 choose, 1 the grouped fused backward, 2 two "
                         "GEMMs per vocab chunk, 3 the sliced fused backward (M <= 64)")
+    p.add_argument("--forward-mode", type=int, choices=[0, 1], default=0,
+                   help="4/8-bit heads: 0 choose (the transposed small-M kernel up to 128 "
+                        "rows), 1 the tiled GEMM at every M")
     p.add_argument("--quant-staging", type=int, choices=[0, 1, 2], default=0,
                    help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
     p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
@@ -324,6 +327,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     cce.cce_set_quant_staging(args.quant_staging)
     cce.cce_set_backward_mode(args.backward_mode)
+    cce.cce_set_forward_mode(args.forward_mode)
     cce.cce_set_cta_pairs(bool(args.cta_pairs))
 
     wl = S.make_workload(args.workload)
@@ -585,6 +589,7 @@ def run_small_m(args, quant=False):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     cce.cce_set_backward_mode(args.backward_mode)
+    cce.cce_set_forward_mode(args.forward_mode)
     peaks, peaks_src = load_peaks()
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     lines = []
@@ -655,6 +660,8 @@ def run_small_m(args, quant=False):
                 "fwd_frac_hbm": fwd_bytes / (t_f / 1e3) / 1e9 / hbm,
                 "bwd_frac_hbm": bwd_bytes / (t_b / 1e3) / 1e9 / hbm,
                 "fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes,
+                "fwd_form": ("transposed small-M (head tile in TMEM)" if plan["fwd_q_small_m"]
+                             else "tiled GEMM"),
                 "bwd_form": ("fused" if plan["bwd_fused"] else
                              "sliced" if plan["bwd_sliced"] else "two GEMMs per vocab chunk"),
                 "bwd_design_bytes": bwd_design,

@@ -375,6 +375,23 @@ void cce_set_quant_staging(int mode);
  * between schedules of the same backward. */
 void cce_set_backward_mode(int mode);
 
+/* Which kernel the forward of a 4-bit or 8-bit head runs (dense heads and
+ * staged 4/8-bit heads are not affected):
+ *   0  choose: up to 128 head rows, with D a multiple of 512 and 16-byte
+ *      aligned scale and bias arrays, the transposed small-M kernel (the
+ *      logits as S^T = W_t H^T, the dequantised head tile written into
+ *      tensor memory as the MMA's A operand, H the shared-memory B operand
+ *      of N = M rounded up to 16, one CTA per SM over blocks of 256 vocab
+ *      rows); otherwise the tiled GEMM with in-kernel dequantisation;
+ *   1  the tiled GEMM with in-kernel dequantisation at every M.
+ * Both forms compute the same logits (the same fp16 weights and products,
+ * fp32 accumulation), so the results agree to accumulation order: the
+ * online softmax of the flash-CCE forward (ORPO design 0.0.6, fused-head
+ * implementation spec, "Forward") reduced over the vocabulary in another
+ * order.  Process-wide; any other value is taken as 0.  No counterpart on
+ * the pages: it selects between schedules of the same forward. */
+void cce_set_forward_mode(int mode);
+
 /* The execution plan cce_forward and cce_backward_dh would take for this
  * problem and workspace size under the current settings (host-only: no
  * launch, no device memory; with no device visible the SM count is taken as
@@ -397,7 +414,9 @@ void cce_set_backward_mode(int mode);
  *                     and bwd_fused are then 0);
  *   bwd_sliced_clusters  clusters it launches (each sweeps every
  *                     bwd_sliced_clusters-th vocab tile of 128 rows);
- *   bwd_sliced_ctas   CTAs per cluster, one per 256 columns of D.
+ *   bwd_sliced_ctas   CTAs per cluster, one per 256 columns of D;
+ *   fwd_q_small_m     1 when the forward of a 4/8-bit head runs the
+ *                     transposed small-M kernel (cce_set_forward_mode).
  * Returns CCE_ERR_INVALID_ARGUMENT / UNSUPPORTED as the calls would. */
 typedef struct {
   int fwd_ok, bwd_ok;
@@ -407,6 +426,7 @@ typedef struct {
   int fwd_cta_pairs, bwd_cta_pairs;
   int bwd_fused, bwd_fused_groups, bwd_fused_members, bwd_fused_buffers;
   int bwd_sliced, bwd_sliced_clusters, bwd_sliced_ctas;
+  int fwd_q_small_m;
 } cce_plan;
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out);

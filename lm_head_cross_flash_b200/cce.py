@@ -67,7 +67,7 @@ class _Plan(ctypes.Structure):
                 ("bwd_fused", ctypes.c_int), ("bwd_fused_groups", ctypes.c_int),
                 ("bwd_fused_members", ctypes.c_int), ("bwd_fused_buffers", ctypes.c_int),
                 ("bwd_sliced", ctypes.c_int), ("bwd_sliced_clusters", ctypes.c_int),
-                ("bwd_sliced_ctas", ctypes.c_int)]
+                ("bwd_sliced_ctas", ctypes.c_int), ("fwd_q_small_m", ctypes.c_int)]
 
 
 _lib = None
@@ -109,6 +109,7 @@ _SIGS = {
     "cce_set_cta_pairs": (None, [ctypes.c_int]),
     "cce_set_quant_staging": (None, [ctypes.c_int]),
     "cce_set_backward_mode": (None, [ctypes.c_int]),
+    "cce_set_forward_mode": (None, [ctypes.c_int]),
     "cce_query_fused_schedule": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int,
                                                   ctypes.POINTER(_Head), ctypes.c_void_p,
                                                   ctypes.c_int64]),
@@ -152,7 +153,7 @@ def cce_forward_noalloc(H, head: "Head", labels, logp, lse, tgt_logit=None, bloc
                                    _stream(stream))
     _check(st, "cce_forward_noalloc")
 
-PROFILE_KINDS = 16
+PROFILE_KINDS = 32
 
 
 def cce_profile_enable(on: bool):
@@ -165,7 +166,8 @@ def cce_profile_read() -> dict:
     ms = (ctypes.c_double * PROFILE_KINDS)()
     n = (ctypes.c_longlong * PROFILE_KINDS)()
     k = lib().cce_profile_read(ms, n, PROFILE_KINDS)
-    return {lib().cce_profile_kind_name(i).decode(): (ms[i], n[i]) for i in range(k)}
+    return {lib().cce_profile_kind_name(i).decode(): (ms[i], n[i])
+            for i in range(min(k, PROFILE_KINDS))}
 
 
 def lib():
@@ -491,6 +493,12 @@ def cce_set_backward_mode(mode: int):
     """Dense bf16 heads: 0 choose; 1 the grouped fused backward kernel; 2 two
     GEMMs per vocab chunk; 3 the sliced fused kernel (M <= 64, D <= 2048)."""
     lib().cce_set_backward_mode(int(mode))
+
+
+def cce_set_forward_mode(mode: int):
+    """4/8-bit heads: 0 choose (the transposed small-M kernel up to 128 head
+    rows); 1 the tiled GEMM with in-kernel dequantisation at every M."""
+    lib().cce_set_forward_mode(int(mode))
 
 
 def cce_query_fused_schedule(M: int, H_dtype: int, head: "Head | _Head"):

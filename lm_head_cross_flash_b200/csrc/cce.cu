@@ -17,6 +17,7 @@
 #include "aux_kernels.cuh"
 #include "fused_bwd.cuh"
 #include "slice_bwd.cuh"
+#include "qsmall_fwd.cuh"
 #include "gemm_tc.cuh"
 
 using namespace cce;
@@ -38,6 +39,7 @@ std::atomic<int> g_qstage{0};
 // Backward of dense bf16 heads: 0 = choose, 1 = the fused kernel (recompute,
 // coefficient tile and dH in one kernel), 2 = the two GEMMs per vocab chunk
 std::atomic<int> g_bwd_mode{0};
+std::atomic<int> g_fwd_mode{0};
 // Staged dequantisation pays off once enough row tiles reuse each weight;
 // measured on the 4-bit long-context head (D=4096, V=128,256): the backward
 // from 2 row tiles (M=192: 0.71 ms staged against 1.06 ms in-kernel), the
@@ -96,7 +98,7 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t cols,
 // bracketed by a CUDA event pair recorded on its own stream.
 enum ProfKind {
   PK_SPLIT = 0, PK_LSE, PK_MERGE, PK_ORPO, PK_SKIP, PK_GRAD, PK_DH, PK_SELFTEST, PK_DHSUM,
-  PK_PREFIX, PK_DW, PK_DEQ, PK_FUSED, PK_FSUM, PK_SLICE, PK_SSUM, PK_N
+  PK_PREFIX, PK_DW, PK_DEQ, PK_FUSED, PK_FSUM, PK_SLICE, PK_SSUM, PK_QFWD, PK_N
 };
 const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merge",
                                       "orpo_epilogue", "skip_plan",    "bwd_grad_gemm",
@@ -104,7 +106,7 @@ const char* const kProfNames[PK_N] = {"operand_prep",  "fwd_lse_gemm", "lse_merg
                                       "prefix_gather_scatter", "bwd_dw_gemm",
                                       "dequant_chunk", "bwd_fused",
                                       "fused_part_sum", "bwd_sliced",
-                                      "sliced_part_sum"};
+                                      "sliced_part_sum", "fwd_q_small_m"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -289,7 +291,9 @@ cce_status device_info(int* sms) {
          cudaFuncSetAttribute(slice_bwd_kernel<1>, attr, SL_SMEM) == cudaSuccess &&
          cudaFuncSetAttribute(slice_bwd_kernel<2>, attr, SL_SMEM) == cudaSuccess &&
          cudaFuncSetAttribute(slice_bwd_kernel<4>, attr, SL_SMEM) == cudaSuccess &&
-         cudaFuncSetAttribute(slice_bwd_kernel<8>, attr, SL_SMEM) == cudaSuccess;
+         cudaFuncSetAttribute(slice_bwd_kernel<8>, attr, SL_SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(qsmall_fwd_kernel<4>, attr, QsCfg<4>::SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(qsmall_fwd_kernel<8>, attr, QsCfg<8>::SMEM) == cudaSuccess;
     if (ok) {
       d.pairs = std::min(max_pairs_of<Mode::kLse>(),
                          std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
@@ -498,6 +502,14 @@ bool q_stage_wanted(int64_t M, const cce_head* W, bool forward) {
 // Smallest staged chunk worth its launches (the whole head if it is smaller).
 int64_t stage_min_rows(const cce_head* W) {
   return std::min<int64_t>(kStageMinRows, ceil_div(W->V, BN) * BN);
+}
+
+// The transposed small-M forward of a 4/8-bit head (qsmall_fwd.cuh): at
+// most 128 head rows, whole groups of 8 scales per 16-byte load (D a
+// multiple of 512, 16-byte aligned scale and bias rows), not staged.
+bool qsmall_wanted(int64_t M, const cce_head* W, bool staged) {
+  return g_fwd_mode.load() == 0 && W->format != CCE_W_DENSE && !staged && M <= QS_MAXM &&
+         W->D % 512 == 0 && aligned16(W->scales) && aligned16(W->biases);
 }
 
 // How one forward call runs for a workspace size: staged chunks of vq rows
@@ -1073,6 +1085,43 @@ cce_status slice_backward(const SlicePlan& sp, const void* H, const cce_head* W,
   return CCE_OK;
 }
 
+// Partials and target logits of the whole vocabulary from the transposed
+// small-M kernel: one CTA per SM over the 256-row vocab blocks.
+cce_status qsmall_forward(const Operands& op, const cce_head* W, int64_t M, int sms,
+                          cudaStream_t st, const int32_t* labels, float* part_m, float* part_s,
+                          float* tgt, uint32_t* status) {
+  const int Mp = int(std::max<int64_t>(16, ceil_div(M, 16) * 16));
+  CUtensorMap mp, mh;
+  if (!make_packed_map(&mp, W, op.qb, uint32_t(op.qb * 8), QS_BLK)) return CCE_ERR_CUDA;
+  if (!make_map(&mh, op.a, false, op.k, M, op.ld_a, 64, uint32_t(Mp))) return CCE_ERR_CUDA;
+  QsArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = int(M);
+  a.Mp = Mp;
+  a.V = int(W->V);
+  a.D = int(W->D);
+  a.nk = int(W->D / 64);
+  a.n_blk = int(ceil_div(W->V, QS_BLK));
+  a.nacc = Mp <= 64 ? 2 : 1;
+  a.wait_ns = g_wait_ns.load();
+  a.status = status;
+  a.labels = labels;
+  a.q_scale = static_cast<const uint16_t*>(W->scales);
+  a.q_bias = static_cast<const uint16_t*>(W->biases);
+  a.softcap = W->softcap;
+  a.inv_cap = W->softcap > 0.f ? 1.f / W->softcap : 0.f;
+  a.part_m = part_m;
+  a.part_s = part_s;
+  a.tgt = tgt;
+  const int grid = int(std::min<int64_t>(a.n_blk, sms));
+  ProfScope ps(PK_QFWD, st);
+  if (op.qb == 4)
+    qsmall_fwd_kernel<4><<<grid, QS_THREADS, QsCfg<4>::SMEM, st>>>(mp, mh, a);
+  else
+    qsmall_fwd_kernel<8><<<grid, QS_THREADS, QsCfg<8>::SMEM, st>>>(mp, mh, a);
+  return launch_ok();
+}
+
 }  // namespace
 
 // ========================================================================
@@ -1101,6 +1150,7 @@ void cce_set_cta_pairs(int on) { g_pairs.store(on != 0 ? 1 : 0); }
 void cce_set_quant_staging(int mode) { g_qstage.store(mode == 1 || mode == 2 ? mode : 0); }
 
 void cce_set_backward_mode(int mode) { g_bwd_mode.store(mode >= 1 && mode <= 3 ? mode : 0); }
+void cce_set_forward_mode(int mode) { g_fwd_mode.store(mode == 1 ? 1 : 0); }
 
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out) {
@@ -1116,6 +1166,8 @@ cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_
   out->fwd_chunk = f.vq;
   out->fwd_staged = f.staged;
   out->fwd_cta_pairs = pairs_wanted(M, W, f.staged);
+  out->fwd_q_small_m = qsmall_wanted(M, W, f.staged);
+  if (out->fwd_q_small_m) out->fwd_cta_pairs = 0;
   out->bwd_ok = b.vc > 0;
   out->bwd_chunk = b.vc;
   out->bwd_ksplit = b.ksplit;
@@ -1224,6 +1276,11 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   float* part_m = blockmax != nullptr ? blockmax : reinterpret_cast<float*>(wsc + L.part_m);
   float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
 
+  if (op.qb && qsmall_wanted(M, W, staged)) {
+    if ((s = qsmall_forward(op, W, M, sms, st, labels, part_m, part_s, tgt, status_word(ws))) !=
+        CCE_OK)
+      return s;
+  } else {
   const int max_pairs = pairs_wanted(M, W, staged) ? device_pairs() : 0;
   const bool pairs = max_pairs > 0;  // forward tiles need no K split
   CUtensorMap ma, mb;
@@ -1288,6 +1345,7 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
       launch_tc<Mode::kLse>(op.qb, n_rt * ct_n, sms, st, ma, mb, ma, ma, ac);
     }
     if (launch_ok() != CCE_OK) return CCE_ERR_CUDA;
+  }
   }
 
   const int rows_per_block = 8;
