@@ -375,6 +375,40 @@ def test_sliced_plan_choice(lib):
     assert not _plan_in_mode(lib, 3, 64, q4)[1]["bwd_sliced"]
 
 
+def test_q_small_m_forward_plan_choice(lib):
+    """The transposed small-M forward takes 4/8-bit heads with at most 128
+    rows, D a multiple of 512 and 16-byte aligned scales and biases, unless
+    forward mode 1 or forced staging is set; it never runs on CTA pairs."""
+    def q(fmt, D, sc=4096):
+        return cce._Head(fmt, cce.CCE_BF16, 128256, D, 4096, sc, sc)
+
+    def plan(M, h):
+        return cce.cce_query_plan(M, cce.CCE_BF16, h, 1 << 34)
+
+    for fmt in (cce.CCE_W_AFFINE_Q4_G64, cce.CCE_W_AFFINE_Q8_G64):
+        for D in (512, 1024, 4096):
+            for M in (1, 64, 128):
+                p = plan(M, q(fmt, D))
+                assert p["fwd_q_small_m"] == 1 and p["fwd_cta_pairs"] == 0, (fmt, D, M)
+                assert p["fwd_staged"] == 0
+            assert plan(129, q(fmt, D))["fwd_q_small_m"] == 0
+        for D in (64, 256, 576, 1088):
+            assert plan(64, q(fmt, D))["fwd_q_small_m"] == 0, D
+        assert plan(64, q(fmt, 4096, sc=4104))["fwd_q_small_m"] == 0  # scales not 16-byte aligned
+        cce.cce_set_forward_mode(1)
+        try:
+            assert plan(64, q(fmt, 4096))["fwd_q_small_m"] == 0
+        finally:
+            cce.cce_set_forward_mode(0)
+        cce.cce_set_quant_staging(2)
+        try:
+            p = plan(64, q(fmt, 4096))
+            assert p["fwd_staged"] == 1 and p["fwd_q_small_m"] == 0
+        finally:
+            cce.cce_set_quant_staging(0)
+    assert plan(64, _head(V=4096, D=4096))["fwd_q_small_m"] == 0  # dense heads
+
+
 def _check_schedule(M, V, D, sched, plan):
     """Every (row tile, round) unit exactly once; a group's segments are runs
     of consecutive rounds on one row tile, flagged first/last; the segments
