@@ -48,7 +48,11 @@
 // stores consumed = fill + 1 (relaxed: the tile's reads are complete).  A
 // tile that block skip (or the end of the vocabulary) removes is neither
 // computed nor loaded, but still advances both counters, so the counts stay
-// aligned.  Every wait is bounded; all
+// aligned; its publishers wait for the previous fill to be consumed before
+// adding 1, as for a computed tile.  ready counts 4 per fill in total, so
+// without that wait a fast warp's count for a skipped fill could stand in
+// for a slow warp's count of the fill before it, and the consumer would load
+// that fill before the slow warp's rows had landed.  Every wait is bounded; all
 // CTAs of the grid are resident at once (at most one CTA per SM, grid no
 // larger than the resident count).
 //
@@ -807,8 +811,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           fence_proxy_async_global();
           red_release_gpu_add(rdy, 1u);
         }
-      } else if (lane == 0) {
-        red_release_gpu_add(rdy, 1u);
+      } else {
+        // Nothing to publish, but this warp's count for the fill must not
+        // reach the slot's consumer before every warp's count for the fill
+        // before it: wait, as a publisher does, until that fill is consumed.
+        bool w_ok = true;
+        if (fill >= 1 && lane == 0)
+          for (int c = 0; c < a.C && w_ok; ++c)
+            w_ok = wait_flag_geq(&a.consumed[slot * a.C + c], fill, a.wait_ns, abort_flag);
+        if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) red_release_gpu_add(rdy, 1u);
       }
       __syncwarp();
       if (u >= 1 && prev.last) flush(prev, prev_any);

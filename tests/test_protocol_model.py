@@ -10,11 +10,16 @@ too far, a missing signal, a missing arm) must make the models stall, which
 shows that they can.
 
 * The grouped fused kernel (fused_bwd.cuh): per member, a producer, an MMA
-  issuer and the epilogue; a FIFO ring of operand stages shared by the
-  S-phase and dH-phase loads; the G'' exchange ring of DEPTH fills per
-  (group, member) with its ready and consumed counters; the S and dH
-  accumulator barriers.  The lead cap is a bounded hint, not a dependency,
-  and is left out.  A CTA pair runs as one member.
+  issuer and the four epilogue warps; a FIFO ring of operand stages shared
+  by the S-phase and dH-phase loads; the G'' exchange ring of DEPTH fills
+  per (group, member) with its ready and consumed counters (each warp adds
+  1 per fill, the consumer waits for 4 per fill); the S and dH accumulator
+  barriers.  Besides running to the end, the model checks safety: when a
+  consumer's wait for a fill passes, every warp's rows of that fill have
+  landed.  One epilogue warp can be made slow (it moves only when nothing
+  else can), which opens the windows a lagging warp leaves.  The lead cap is
+  a bounded hint, not a dependency, and is left out.  A CTA pair runs as one
+  member.
 * The sliced kernel (slice_bwd.cuh): per CTA of a cluster, the S and dH
   loaders and MMA issuers, the drain warps and the reducer warps, with the
   double-buffered partial (pfull, pempty), G'' (gfull, gempty) and S
@@ -33,19 +38,32 @@ from lm_head_cross_flash_b200 import cce
 
 
 # --------------------------------------------------------------- machinery --
-def _run(procs, step):
+def _run(procs, step, slow=()):
     """procs: list of (state, [op lists]).  Runs every op list as far as its
-    next op allows, until nothing moves.  Returns the list of stuck
-    (process, role, position, length)."""
+    next op allows, until nothing moves; the roles in `slow` ((process,
+    role) pairs) take one op at a time, and only when no other role can
+    move.  Returns the list of stuck (process, role, position, length)."""
     pos = [[0] * len(lists) for _, lists in procs]
-    moved = True
-    while moved:
+    slow = set(slow)
+    while True:
         moved = False
         for i, (st, lists) in enumerate(procs):
             for r, ops in enumerate(lists):
+                if (i, r) in slow:
+                    continue
                 while pos[i][r] < len(ops) and step(st, *ops[pos[i][r]]):
                     pos[i][r] += 1
                     moved = True
+        if moved:
+            continue
+        for i, r in sorted(slow):
+            ops = procs[i][1][r]
+            if pos[i][r] < len(ops) and step(procs[i][0], *ops[pos[i][r]]):
+                pos[i][r] += 1
+                moved = True
+                break
+        if not moved:
+            break
     return [(i, r, pos[i][r], len(ops)) for i, (_, lists) in enumerate(procs)
             for r, ops in enumerate(lists) if pos[i][r] < len(ops)]
 
@@ -54,7 +72,16 @@ def _run(procs, step):
 FB_DEPTH = 2
 
 
-def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
+EPI_WARPS = 4
+
+
+def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None, slow_warp=False):
+    """Stuck roles plus safety violations (empty: the protocol is sound on
+    this schedule and skip pattern).  bug: "consumed_off_by_one" (a
+    publisher waits one fill too far), "no_consumed_on_skip" (the MMA warp
+    does not release a skipped tile's slot), "skip_without_wait" (a warp
+    counts a skipped tile without waiting for the slot's previous fill to
+    be consumed)."""
     lib = cce.lib()
     h = cce._Head(cce.CCE_W_DENSE, cce.CCE_BF16, V, D, D, None, None)
     cce.cce_set_backward_mode(1)
@@ -83,7 +110,7 @@ def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
 
     units = {g: [tuple(int(x) for x in row[1:]) for row in sched[sched[:, 0] == g]]
              for g in range(G)}
-    shared = {"ready": {}, "consumed": {}}
+    shared = {"ready": {}, "consumed": {}, "landed": {}, "violations": []}
     procs = []
     for g in range(G):
         U = units[g]
@@ -133,33 +160,42 @@ def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
                     if last and dh_any:
                         X.append(("dh_full",))
                         nseg += 1
-            # epilogue: publish G''(u) once every member consumed the slot's
-            # previous fill; flush a finished segment's dH
-            ns = nseg = 0
-            prev, seg_any, prev_any = None, False, False
-            for u in range(len(U)):
-                r, j, first = U[u][0], U[u][1], U[u][2]
-                if first:
-                    seg_any = False
-                seg_any = seg_any or any(not skip(r, j * C + q) for q in range(C))
-                fill = u // FB_DEPTH
-                if not skip(r, j * C + p):
-                    E.append(("wait_s_full", ns))
-                    need = fill + 1 if bug == "consumed_off_by_one" else fill
-                    if fill >= 1:
+            # epilogue warps: publish their rows of G''(u) once every member
+            # consumed the slot's previous fill; flush a finished segment's dH
+            E = []
+            for w in range(EPI_WARPS):
+                Ew = []
+                ns = nseg = 0
+                prev, seg_any, prev_any = None, False, False
+                for u in range(len(U)):
+                    r, j, first = U[u][0], U[u][1], U[u][2]
+                    if first:
+                        seg_any = False
+                    seg_any = seg_any or any(not skip(r, j * C + q) for q in range(C))
+                    fill = u // FB_DEPTH
+                    slot = (g, u % FB_DEPTH, p)
+                    if not skip(r, j * C + p):
+                        Ew.append(("wait_s_full", ns))
+                        need = fill + 1 if bug == "consumed_off_by_one" else fill
+                        if fill >= 1:
+                            for c in range(C):
+                                Ew.append(("wait_consumed", (g, u % FB_DEPTH, p, c), need))
+                        Ew.append(("s_empty",))
+                        ns += 1
+                        Ew.append(("landed", slot, w, fill + 1))
+                    elif fill >= 1 and bug != "skip_without_wait":
                         for c in range(C):
-                            E.append(("wait_consumed", (g, u % FB_DEPTH, p, c), need))
-                    E.append(("s_empty",))
-                    ns += 1
-                E.append(("ready_add", (g, u % FB_DEPTH, p)))
-                if u >= 1 and prev[3] and prev_any:
-                    E += [("wait_dh_full", nseg), ("dh_empty",)]
-                    nseg += 1
-                prev, prev_any = U[u], seg_any
-            if prev is not None and prev_any:
-                E += [("wait_dh_full", nseg), ("dh_empty",)]
+                            Ew.append(("wait_consumed", (g, u % FB_DEPTH, p, c), fill))
+                    Ew.append(("ready_add", slot))
+                    if u >= 1 and prev[3] and prev_any:
+                        Ew += [("wait_dh_full", nseg), ("dh_empty",)]
+                        nseg += 1
+                    prev, prev_any = U[u], seg_any
+                if prev is not None and prev_any:
+                    Ew += [("wait_dh_full", nseg), ("dh_empty",)]
+                E.append(Ew)
             st = dict(ring=0, s_full=0, s_empty=0, dh_full=0, dh_empty=0)
-            procs.append((st, [P, X, E]))
+            procs.append((st, [P, X] + E))
 
     def step(st, op, *arg):
         if op == "load":
@@ -173,7 +209,16 @@ def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
             st["ring"] -= 1
             return True
         if op == "wait_ready":
-            return shared["ready"].get(arg[0], 0) >= arg[1]
+            if shared["ready"].get(arg[0], 0) < EPI_WARPS * arg[1]:
+                return False
+            late = [w for w in range(EPI_WARPS)
+                    if shared["landed"].get((arg[0], w), 0) < arg[1]]
+            if late:
+                shared["violations"].append(("read before landed", arg[0], arg[1], late))
+            return True
+        if op == "landed":
+            shared["landed"][(arg[0], arg[1])] = arg[2]
+            return True
         if op == "set_consumed":
             shared["consumed"][arg[0]] = arg[1]
             return True
@@ -183,11 +228,11 @@ def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
             shared["ready"][arg[0]] = shared["ready"].get(arg[0], 0) + 1
             return True
         if op == "wait_s_empty":
-            return st["s_empty"] >= arg[0] - sbufs + 1
+            return st["s_empty"] >= EPI_WARPS * (arg[0] - sbufs + 1)
         if op == "wait_s_full":
             return st["s_full"] > arg[0]
         if op == "wait_dh_empty":
-            return st["dh_empty"] >= arg[0]
+            return st["dh_empty"] >= EPI_WARPS * arg[0]
         if op == "wait_dh_full":
             return st["dh_full"] > arg[0]
         if op in ("s_full", "s_empty", "dh_full", "dh_empty"):
@@ -195,7 +240,8 @@ def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None):
             return True
         raise ValueError(op)
 
-    return _run(procs, step)
+    stuck = _run(procs, step, slow=[(0, 2)] if slow_warp else ())
+    return stuck + shared["violations"]
 
 
 FUSED_SHAPES = [(8192, 16384, 2048, True), (300, 1000, 320, True), (64, 20000, 2048, False),
@@ -213,6 +259,26 @@ def test_fused_protocol_runs_to_the_end(M, V, D, pairs, skip_prob):
                                            ("no_consumed_on_skip", 0.3)])
 def test_fused_protocol_model_catches_planted_mistakes(bug, skip_prob):
     assert _fused_model(2048, 7000, 1536, skip_prob, seed=5, bug=bug) != []
+
+
+@pytest.mark.parametrize("M,V,D,pairs", [(900, 60000, 256, False), (900, 20000, 256, False),
+                                         (300, 1000, 320, True), (2048, 7000, 1536, True),
+                                         (8192, 16384, 2048, True)])
+@pytest.mark.parametrize("skip_prob", [0.0, 0.3, 0.9])
+def test_fused_protocol_is_safe_with_a_slow_warp(M, V, D, pairs, skip_prob):
+    """One epilogue warp of group 0 moves only when nothing else can: no
+    consumer may load a fill before that warp's rows of it have landed."""
+    assert _fused_model(M, V, D, skip_prob, seed=M + V, pairs=pairs, slow_warp=True) == []
+
+
+def test_fused_protocol_model_catches_the_skipped_tile_race():
+    """A warp that counts a skipped tile without first waiting for the
+    slot's previous fill to be consumed lets its count stand in for a slow
+    warp's count of that fill: the consumer then loads the fill before the
+    slow warp's rows have landed (the model must report it)."""
+    found = _fused_model(900, 60000, 256, 0.5, seed=7, pairs=False, bug="skip_without_wait",
+                         slow_warp=True)
+    assert any(v[0] == "read before landed" for v in found), found[:3]
 
 
 # ------------------------------------------------------------ sliced kernel --
