@@ -319,7 +319,7 @@ class ProtocolError(AssertionError):
     """A signal that would land in another tile's barrier phase."""
 
 
-def _sliced_model(n, ccl, ns=4, nd=2, nbuf=2, bug=None):
+def _sliced_model(n, ccl, ns=4, nd=2, nbuf=2, bug=None, slow=()):
     epi = 4
     tiles_of = lambda b: list(range(b, n, nbuf))
     ctas = []
@@ -427,7 +427,7 @@ def _sliced_model(n, ccl, ns=4, nd=2, nbuf=2, bug=None):
         return True
         raise ValueError(op)
 
-    return _run(procs, step)
+    return _run(procs, step, slow=slow)
 
 
 @pytest.mark.parametrize("n", [0, 1, 2, 3, 4, 7, 30])
@@ -446,3 +446,16 @@ def test_sliced_protocol_other_depths(ns, nd, nbuf):
 @pytest.mark.parametrize("bug", ["no_pempty", "no_gfull_arm"])
 def test_sliced_protocol_model_catches_planted_mistakes(bug):
     assert _sliced_model(6, 4, bug=bug) != []
+
+
+SLICED_ROLES = 4 + 4 + 4   # loaders and MMA issuers, drain warps, reducer warps
+
+
+@pytest.mark.parametrize("n,ccl", [(5, 2), (9, 4), (7, 8), (6, 1)])
+def test_sliced_protocol_with_a_slow_role(n, ccl):
+    """Each role of the first and the last CTA in turn moves only when no
+    other role can: the protocol still runs to the end, and no arrival or
+    byte count lands in a phase that belongs to another tile."""
+    for c in sorted({0, ccl - 1}):
+        for r in range(SLICED_ROLES):
+            assert _sliced_model(n, ccl, slow=[(c, r)]) == [], (c, r)
