@@ -75,13 +75,15 @@ FB_DEPTH = 2
 EPI_WARPS = 4
 
 
-def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None, slow_warp=False):
+def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None, slow=()):
     """Stuck roles plus safety violations (empty: the protocol is sound on
     this schedule and skip pattern).  bug: "consumed_off_by_one" (a
     publisher waits one fill too far), "no_consumed_on_skip" (the MMA warp
     does not release a skipped tile's slot), "skip_without_wait" (a warp
     counts a skipped tile without waiting for the slot's previous fill to
-    be consumed)."""
+    be consumed).  slow: (process, role) pairs held back; a process is a
+    (group, member) in order, its roles the producer, the MMA issuer and
+    epilogue warps 0-3."""
     lib = cce.lib()
     h = cce._Head(cce.CCE_W_DENSE, cce.CCE_BF16, V, D, D, None, None)
     cce.cce_set_backward_mode(1)
@@ -240,7 +242,7 @@ def _fused_model(M, V, D, skip_prob, seed, pairs=True, bug=None, slow_warp=False
             return True
         raise ValueError(op)
 
-    stuck = _run(procs, step, slow=[(0, 2)] if slow_warp else ())
+    stuck = _run(procs, step, slow=slow)
     return stuck + shared["violations"]
 
 
@@ -268,7 +270,15 @@ def test_fused_protocol_model_catches_planted_mistakes(bug, skip_prob):
 def test_fused_protocol_is_safe_with_a_slow_warp(M, V, D, pairs, skip_prob):
     """One epilogue warp of group 0 moves only when nothing else can: no
     consumer may load a fill before that warp's rows of it have landed."""
-    assert _fused_model(M, V, D, skip_prob, seed=M + V, pairs=pairs, slow_warp=True) == []
+    assert _fused_model(M, V, D, skip_prob, seed=M + V, pairs=pairs, slow=[(0, 2)]) == []
+
+
+@pytest.mark.parametrize("role", range(6))
+def test_fused_protocol_with_each_role_held_back(role):
+    """The producer, the MMA issuer or one epilogue warp of group 0 held
+    back in turn, with block skip: still no deadlock and no early load."""
+    assert _fused_model(900, 60000, 256, 0.3, seed=11, pairs=False, slow=[(0, role)]) == []
+    assert _fused_model(2048, 7000, 1536, 0.3, seed=12, pairs=True, slow=[(0, role)]) == []
 
 
 def test_fused_protocol_model_catches_the_skipped_tile_race():
@@ -277,7 +287,7 @@ def test_fused_protocol_model_catches_the_skipped_tile_race():
     warp's count of that fill: the consumer then loads the fill before the
     slow warp's rows have landed (the model must report it)."""
     found = _fused_model(900, 60000, 256, 0.5, seed=7, pairs=False, bug="skip_without_wait",
-                         slow_warp=True)
+                         slow=[(0, 2)])
     assert any(v[0] == "read before landed" for v in found), found[:3]
 
 
