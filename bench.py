@@ -54,9 +54,10 @@ def parse_args(argv=None):
     p.add_argument("--backward-mode", type=int, choices=[0, 1, 2, 3], default=0,
                    help="dense bf16 heads: 0 choose, 1 the grouped fused backward, 2 two "
                         "GEMMs per vocab chunk, 3 the sliced fused backward (M <= 64)")
-    p.add_argument("--forward-mode", type=int, choices=[0, 1], default=0,
-                   help="4/8-bit heads: 0 choose (the transposed small-M kernel up to 128 "
-                        "rows), 1 the tiled GEMM at every M")
+    p.add_argument("--forward-mode", type=int, choices=[0, 1, 2], default=0,
+                   help="4/8-bit heads: 0 choose (a transposed small-M kernel up to 256 "
+                        "rows), 1 the tiled GEMM at every M, 2 the wide transposed form "
+                        "from 1 row")
     p.add_argument("--quant-staging", type=int, choices=[0, 1, 2], default=0,
                    help="4/8-bit heads: 0 choose, 1 dequantise in the GEMM, 2 staged fp16 chunks")
     p.add_argument("--cta-pairs", type=int, choices=[0, 1], default=1,
@@ -660,8 +661,9 @@ def run_small_m(args, quant=False):
                 "fwd_frac_hbm": fwd_bytes / (t_f / 1e3) / 1e9 / hbm,
                 "bwd_frac_hbm": bwd_bytes / (t_b / 1e3) / 1e9 / hbm,
                 "fwd_bytes": fwd_bytes, "bwd_bytes": bwd_bytes,
-                "fwd_form": ("transposed small-M (head tile in TMEM)" if plan["fwd_q_small_m"]
-                             else "tiled GEMM"),
+                "fwd_form": {0: "tiled GEMM", 1: "transposed small-M (head tile in TMEM)",
+                             2: "transposed, 128-row units (head tile in TMEM)"}[
+                                 plan["fwd_q_small_m"]],
                 "bwd_form": ("fused" if plan["bwd_fused"] else
                              "sliced" if plan["bwd_sliced"] else "two GEMMs per vocab chunk"),
                 "bwd_design_bytes": bwd_design,

@@ -377,13 +377,18 @@ void cce_set_backward_mode(int mode);
 
 /* Which kernel the forward of a 4-bit or 8-bit head runs (dense heads and
  * staged 4/8-bit heads are not affected):
- *   0  choose: up to 128 head rows, with D a multiple of 512 and 16-byte
- *      aligned scale and bias arrays, the transposed small-M kernel (the
+ *   0  choose: up to 240 head rows, with D a multiple of 512 and 16-byte
+ *      aligned scale and bias arrays, a transposed small-M kernel (the
  *      logits as S^T = W_t H^T, the dequantised head tile written into
  *      tensor memory as the MMA's A operand, H the shared-memory B operand
  *      of N = M rounded up to 16, one CTA per SM over blocks of 256 vocab
- *      rows); otherwise the tiled GEMM with in-kernel dequantisation;
- *   1  the tiled GEMM with in-kernel dequantisation at every M.
+ *      rows): up to 128 rows both 128-row halves of a block share each K
+ *      step, from 129 rows they run one after the other; otherwise the
+ *      tiled GEMM with in-kernel dequantisation;
+ *   1  the tiled GEMM with in-kernel dequantisation at every M;
+ *   2  the second transposed form for 1 to 256 rows (from 241 rows it
+ *      measured no faster than the tiled GEMM, whose 256-row tile costs the
+ *      same from 129 rows on).
  * Both forms compute the same logits (the same fp16 weights and products,
  * fp32 accumulation), so the results agree to accumulation order: the
  * online softmax of the flash-CCE forward (ORPO design 0.0.6, fused-head
@@ -415,8 +420,9 @@ void cce_set_forward_mode(int mode);
  *   bwd_sliced_clusters  clusters it launches (each sweeps every
  *                     bwd_sliced_clusters-th vocab tile of 128 rows);
  *   bwd_sliced_ctas   CTAs per cluster, one per 256 columns of D;
- *   fwd_q_small_m     1 when the forward of a 4/8-bit head runs the
- *                     transposed small-M kernel (cce_set_forward_mode).
+ *   fwd_q_small_m     the transposed small-M forward a 4/8-bit head runs
+ *                     (cce_set_forward_mode): 1 at most 128 head rows, 2
+ *                     129 to 240 (1 to 256 in mode 2); 0 the tiled GEMM.
  * Returns CCE_ERR_INVALID_ARGUMENT / UNSUPPORTED as the calls would. */
 typedef struct {
   int fwd_ok, bwd_ok;

@@ -496,8 +496,9 @@ def cce_set_backward_mode(mode: int):
 
 
 def cce_set_forward_mode(mode: int):
-    """4/8-bit heads: 0 choose (the transposed small-M kernel up to 128 head
-    rows); 1 the tiled GEMM with in-kernel dequantisation at every M."""
+    """4/8-bit heads: 0 choose (a transposed small-M kernel up to 240 head
+    rows); 1 the tiled GEMM with in-kernel dequantisation at every M; 2 the
+    transposed form of 129-240 rows for 1 to 256 rows."""
     lib().cce_set_forward_mode(int(mode))
 
 

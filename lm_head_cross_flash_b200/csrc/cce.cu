@@ -17,7 +17,7 @@
 #include "aux_kernels.cuh"
 #include "fused_bwd.cuh"
 #include "slice_bwd.cuh"
-#include "qsmall_fwd.cuh"
+#include "qwide_fwd.cuh"
 #include "gemm_tc.cuh"
 
 using namespace cce;
@@ -293,7 +293,9 @@ cce_status device_info(int* sms) {
          cudaFuncSetAttribute(slice_bwd_kernel<4>, attr, SL_SMEM) == cudaSuccess &&
          cudaFuncSetAttribute(slice_bwd_kernel<8>, attr, SL_SMEM) == cudaSuccess &&
          cudaFuncSetAttribute(qsmall_fwd_kernel<4>, attr, QsCfg<4>::SMEM) == cudaSuccess &&
-         cudaFuncSetAttribute(qsmall_fwd_kernel<8>, attr, QsCfg<8>::SMEM) == cudaSuccess;
+         cudaFuncSetAttribute(qsmall_fwd_kernel<8>, attr, QsCfg<8>::SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(qwide_fwd_kernel<4>, attr, QwCfg<4>::SMEM) == cudaSuccess &&
+         cudaFuncSetAttribute(qwide_fwd_kernel<8>, attr, QwCfg<8>::SMEM) == cudaSuccess;
     if (ok) {
       d.pairs = std::min(max_pairs_of<Mode::kLse>(),
                          std::min(max_pairs_of<Mode::kGrad>(), max_pairs_of<Mode::kDh>()));
@@ -504,12 +506,22 @@ int64_t stage_min_rows(const cce_head* W) {
   return std::min<int64_t>(kStageMinRows, ceil_div(W->V, BN) * BN);
 }
 
-// The transposed small-M forward of a 4/8-bit head (qsmall_fwd.cuh): at
-// most 128 head rows, whole groups of 8 scales per 16-byte load (D a
-// multiple of 512, 16-byte aligned scale and bias rows), not staged.
-bool qsmall_wanted(int64_t M, const cce_head* W, bool staged) {
-  return g_fwd_mode.load() == 0 && W->format != CCE_W_DENSE && !staged && M <= QS_MAXM &&
-         W->D % 512 == 0 && aligned16(W->scales) && aligned16(W->biases);
+// The transposed small-M forward of a 4/8-bit head, not staged, with whole
+// groups of 8 scales per 16-byte load (D a multiple of 512, 16-byte aligned
+// scale and bias rows): 1 = qsmall_fwd.cuh (at most 128 head rows), 2 =
+// qwide_fwd.cuh (129 to 240 by default; forward mode 2 takes it for 1 to
+// 256), 0 = the tiled GEMM.  The wide form's time grows with N = M rounded
+// up to 16 while the GEMM's 256-row tile costs the same from 129 to 256
+// rows: at D = 4,096, V = 128,256 the wide form took 0.403 ms at M = 200
+// against 0.439 ms, but 0.444 against 0.438 ms at M = 256.
+constexpr int64_t kQwideDefaultMaxM = 240;
+int qsmall_wanted(int64_t M, const cce_head* W, bool staged) {
+  const int mode = g_fwd_mode.load();
+  if (mode == 1 || W->format == CCE_W_DENSE || staged || W->D % 512 != 0 ||
+      !aligned16(W->scales) || !aligned16(W->biases) || M > QW_MAXM)
+    return 0;
+  if (mode == 2) return 2;
+  return M <= QS_MAXM ? 1 : M <= kQwideDefaultMaxM ? 2 : 0;
 }
 
 // How one forward call runs for a workspace size: staged chunks of vq rows
@@ -1087,12 +1099,13 @@ cce_status slice_backward(const SlicePlan& sp, const void* H, const cce_head* W,
 
 // Partials and target logits of the whole vocabulary from the transposed
 // small-M kernel: one CTA per SM over the 256-row vocab blocks.
-cce_status qsmall_forward(const Operands& op, const cce_head* W, int64_t M, int sms,
+cce_status qsmall_forward(const Operands& op, const cce_head* W, int64_t M, bool wide, int sms,
                           cudaStream_t st, const int32_t* labels, float* part_m, float* part_s,
                           float* tgt, uint32_t* status) {
   const int Mp = int(std::max<int64_t>(16, ceil_div(M, 16) * 16));
   CUtensorMap mp, mh;
-  if (!make_packed_map(&mp, W, op.qb, uint32_t(op.qb * 8), QS_BLK)) return CCE_ERR_CUDA;
+  if (!make_packed_map(&mp, W, op.qb, uint32_t(op.qb * 8), wide ? QW_UNIT : QS_BLK))
+    return CCE_ERR_CUDA;
   if (!make_map(&mh, op.a, false, op.k, M, op.ld_a, 64, uint32_t(Mp))) return CCE_ERR_CUDA;
   QsArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -1115,10 +1128,16 @@ cce_status qsmall_forward(const Operands& op, const cce_head* W, int64_t M, int 
   a.tgt = tgt;
   const int grid = int(std::min<int64_t>(a.n_blk, sms));
   ProfScope ps(PK_QFWD, st);
-  if (op.qb == 4)
+  if (wide) {
+    if (op.qb == 4)
+      qwide_fwd_kernel<4><<<grid, QW_THREADS, QwCfg<4>::SMEM, st>>>(mp, mh, a);
+    else
+      qwide_fwd_kernel<8><<<grid, QW_THREADS, QwCfg<8>::SMEM, st>>>(mp, mh, a);
+  } else if (op.qb == 4) {
     qsmall_fwd_kernel<4><<<grid, QS_THREADS, QsCfg<4>::SMEM, st>>>(mp, mh, a);
-  else
+  } else {
     qsmall_fwd_kernel<8><<<grid, QS_THREADS, QsCfg<8>::SMEM, st>>>(mp, mh, a);
+  }
   return launch_ok();
 }
 
@@ -1150,7 +1169,7 @@ void cce_set_cta_pairs(int on) { g_pairs.store(on != 0 ? 1 : 0); }
 void cce_set_quant_staging(int mode) { g_qstage.store(mode == 1 || mode == 2 ? mode : 0); }
 
 void cce_set_backward_mode(int mode) { g_bwd_mode.store(mode >= 1 && mode <= 3 ? mode : 0); }
-void cce_set_forward_mode(int mode) { g_fwd_mode.store(mode == 1 ? 1 : 0); }
+void cce_set_forward_mode(int mode) { g_fwd_mode.store(mode == 1 || mode == 2 ? mode : 0); }
 
 cce_status cce_query_plan(int64_t M, cce_dtype h_dtype, const cce_head* W, size_t ws_bytes,
                           cce_plan* out) {
@@ -1277,8 +1296,8 @@ cce_status cce_forward(const void* H, cce_dtype h_dtype, int64_t M, const cce_he
   float* tgt = tgt_logit != nullptr ? tgt_logit : reinterpret_cast<float*>(wsc + L.tgt);
 
   if (op.qb && qsmall_wanted(M, W, staged)) {
-    if ((s = qsmall_forward(op, W, M, sms, st, labels, part_m, part_s, tgt, status_word(ws))) !=
-        CCE_OK)
+    if ((s = qsmall_forward(op, W, M, qsmall_wanted(M, W, staged) == 2, sms, st, labels, part_m,
+                            part_s, tgt, status_word(ws))) != CCE_OK)
       return s;
   } else {
   const int max_pairs = pairs_wanted(M, W, staged) ? device_pairs() : 0;

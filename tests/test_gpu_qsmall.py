@@ -1,7 +1,8 @@
-"""GPU parity of the transposed small-M forward of 4/8-bit heads (at most 128
-head rows: the logits computed as S^T = W_t H^T with the dequantised head
-tile in tensor memory as the MMA's A operand) against the float64 oracle and
-against the tiled GEMM forward with in-kernel dequantisation (forward mode 1).
+"""GPU parity of the transposed small-M forwards of 4/8-bit heads (the
+logits computed as S^T = W_t H^T with the dequantised head tile in tensor
+memory as the MMA's A operand; the narrow form up to 128 head rows, the wide
+form of 128-row units up to 256) against the float64 oracle and against the
+tiled GEMM forward with in-kernel dequantisation (forward mode 1).
 
 Shapes cover 3 to 128 head rows (N = 16, 48, 64, 80, 128: one or two
 accumulator buffers, one to four 32-column chunks), D from 512 to 2048,
@@ -29,6 +30,7 @@ TOL_VS_GEMM = 2e-5
 
 
 def _forward(mode, H, head, labels, M, V):
+    """mode: 0 choose, 1 the tiled GEMM, 2 the wide transposed form."""
     f = dict(device="cuda", dtype=torch.float32)
     cce.cce_set_forward_mode(mode)
     try:
@@ -63,14 +65,32 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("wformat,split,D,V,cap", CASES)
-def test_q_small_m_forward_matches_oracle_and_gemm(wformat, split, D, V, cap):
+WIDE_CASES = [
+    ("q4g64", (40, 45, 44), 512, 4097, 0.0),       # M = 129: N = 144, five chunks
+    ("q8g64", (50, 70, 80), 1024, 3001, 0.0),      # M = 200: N = 208
+    ("q4g64", (60, 90, 90), 2048, 20000, 0.0),     # M = 240: N = 240, eight chunks
+    ("q4g64", (40, 80, 80), 512, 257, 30.0),       # softcap, a last block of one row
+    ("q8g64", (50, 80, 80), 512, 148 * 256 * 2 + 17, 0.0),  # 3 blocks per CTA
+]
+
+SMALL_IN_WIDE = [
+    ("q4g64", (1, 1, 1), 512, 31, 0.0),            # mode 2 from 3 rows: N = 16
+    ("q4g64", (20, 20, 24), 1024, 5000, 0.0),      # N = 64
+    ("q8g64", (40, 40, 48), 512, 9000, 0.0),       # N = 128
+    ("q4g64", (60, 98, 98), 2048, 20000, 0.0),     # M = 256: N = 256, eight full chunks
+]
+
+
+@pytest.mark.parametrize("mode,form,case", [(0, 1, c) for c in CASES] +
+                         [(0, 2, c) for c in WIDE_CASES] + [(2, 2, c) for c in SMALL_IN_WIDE])
+def test_q_small_m_forward_matches_oracle_and_gemm(mode, form, case):
+    wformat, split, D, V, cap = case
     wl = S.make_custom(4, M_split=split, D=D, V=V, wformat=wformat)
     H, head, labels = upload(wl)
     head.softcap = cap
     M = wl.M
-    plan, prof, logp, lse, tgt, bm = _forward(0, H, head, labels, M, V)
-    assert plan["fwd_q_small_m"] == 1 and plan["fwd_staged"] == 0, plan
+    plan, prof, logp, lse, tgt, bm = _forward(mode, H, head, labels, M, V)
+    assert plan["fwd_q_small_m"] == form and plan["fwd_staged"] == 0, plan
     assert prof.get("fwd_q_small_m", (0.0, 0))[1] == 1, prof
     assert prof.get("fwd_lse_gemm", (0.0, 0))[1] == 0, prof
     plan1, prof1, logp1, lse1, tgt1, bm1 = _forward(1, H, head, labels, M, V)
@@ -98,8 +118,8 @@ def test_q_small_m_forward_matches_oracle_and_gemm(wformat, split, D, V, cap):
 
 
 def test_q_small_m_not_taken_outside_its_range():
-    """129 rows, D not a multiple of 512, or forward mode 1: the GEMM form."""
-    for split, D in (((40, 45, 44), 512), ((20, 20, 24), 256)):
+    """257 rows, D not a multiple of 512, or forward mode 1: the GEMM form."""
+    for split, D in (((40, 110, 107), 512), ((20, 20, 24), 256)):
         wl = S.make_custom(4, M_split=split, D=D, V=3000, wformat="q4g64")
         H, head, labels = upload(wl)
         plan = cce.cce_query_plan(wl.M, cce.h_dtype(H), head, 1 << 34)

@@ -376,9 +376,12 @@ def test_sliced_plan_choice(lib):
 
 
 def test_q_small_m_forward_plan_choice(lib):
-    """The transposed small-M forward takes 4/8-bit heads with at most 128
-    rows, D a multiple of 512 and 16-byte aligned scales and biases, unless
-    forward mode 1 or forced staging is set; it never runs on CTA pairs."""
+    """A transposed small-M forward takes 4/8-bit heads with D a multiple of
+    512 and 16-byte aligned scales and biases: the narrow form (1) up to 128
+    rows, the wide form (2) from 129 to 240 (1 to 256 in forward mode 2);
+    neither in forward mode 1, with forced staging, past 240 rows (256 in
+    mode 2) or for
+    dense heads; never on CTA pairs."""
     def q(fmt, D, sc=4096):
         return cce._Head(fmt, cce.CCE_BF16, 128256, D, 4096, sc, sc)
 
@@ -387,17 +390,28 @@ def test_q_small_m_forward_plan_choice(lib):
 
     for fmt in (cce.CCE_W_AFFINE_Q4_G64, cce.CCE_W_AFFINE_Q8_G64):
         for D in (512, 1024, 4096):
-            for M in (1, 64, 128):
+            for M, form in ((1, 1), (64, 1), (128, 1), (129, 2), (200, 2), (240, 2), (241, 0),
+                            (256, 0)):
                 p = plan(M, q(fmt, D))
-                assert p["fwd_q_small_m"] == 1 and p["fwd_cta_pairs"] == 0, (fmt, D, M)
+                assert p["fwd_q_small_m"] == form and p["fwd_cta_pairs"] == 0, (fmt, D, M)
                 assert p["fwd_staged"] == 0
-            assert plan(129, q(fmt, D))["fwd_q_small_m"] == 0
+            assert plan(257, q(fmt, D))["fwd_q_small_m"] == 0
         for D in (64, 256, 576, 1088):
             assert plan(64, q(fmt, D))["fwd_q_small_m"] == 0, D
+            assert plan(200, q(fmt, D))["fwd_q_small_m"] == 0, D
         assert plan(64, q(fmt, 4096, sc=4104))["fwd_q_small_m"] == 0  # scales not 16-byte aligned
         cce.cce_set_forward_mode(1)
         try:
             assert plan(64, q(fmt, 4096))["fwd_q_small_m"] == 0
+            assert plan(200, q(fmt, 4096))["fwd_q_small_m"] == 0
+        finally:
+            cce.cce_set_forward_mode(0)
+        cce.cce_set_forward_mode(2)
+        try:
+            assert plan(1, q(fmt, 4096))["fwd_q_small_m"] == 2
+            assert plan(64, q(fmt, 4096))["fwd_q_small_m"] == 2
+            assert plan(256, q(fmt, 4096))["fwd_q_small_m"] == 2
+            assert plan(257, q(fmt, 4096))["fwd_q_small_m"] == 0
         finally:
             cce.cce_set_forward_mode(0)
         cce.cce_set_quant_staging(2)
