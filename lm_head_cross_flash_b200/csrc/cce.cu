@@ -1104,7 +1104,10 @@ cce_status qsmall_forward(const Operands& op, const cce_head* W, int64_t M, bool
                           float* tgt, uint32_t* status) {
   const int Mp = int(std::max<int64_t>(16, ceil_div(M, 16) * 16));
   CUtensorMap mp, mh;
-  if (!make_packed_map(&mp, W, op.qb, uint32_t(op.qb * 8), wide ? QW_UNIT : QS_BLK))
+  // one K step's packed rows: one group of 64 (wide), KG groups (narrow)
+  const int kg = wide ? 1 : (op.qb == 4 ? QsCfg<4>::KG : QsCfg<8>::KG);
+  if (!make_packed_map(&mp, W, op.qb, uint32_t(op.qb * 8 * kg),
+                       wide ? QW_UNIT : QS_BLK))
     return CCE_ERR_CUDA;
   if (!make_map(&mh, op.a, false, op.k, M, op.ld_a, 64, uint32_t(Mp))) return CCE_ERR_CUDA;
   QsArgs a;
@@ -1113,7 +1116,7 @@ cce_status qsmall_forward(const Operands& op, const cce_head* W, int64_t M, bool
   a.Mp = Mp;
   a.V = int(W->V);
   a.D = int(W->D);
-  a.nk = int(W->D / 64);
+  a.nk = int(W->D / 64 / kg);
   a.n_blk = int(ceil_div(W->V, QS_BLK));
   a.nacc = Mp <= 64 ? 2 : 1;
   a.wait_ns = g_wait_ns.load();

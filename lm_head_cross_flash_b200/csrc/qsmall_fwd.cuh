@@ -23,24 +23,26 @@
 // GEMM kernel).  H, the small operand, comes by TMA into shared memory.
 //
 // Per CTA: 256-row vocab blocks in turn (block b, then b + grid, ...), each
-// as two 128-row halves that share every K step's H slice; the K loop runs
-// over D in groups of 64, starting for block b at group b mod (D / 64) and
-// wrapping.  Every CTA reads the same small H, so with one K order for all
+// as two 128-row halves that share every K step's H slices; the K loop runs
+// over D in steps of KG groups of 64 (QsCfg), starting for block b at step
+// b mod (D / (64 KG)) and wrapping.  Every CTA reads the same small H, so with one K order for all
 // the SMs would fetch the same H slice from L2 at the same moment and a few
 // L2 slices would serve the whole GPU; rotated, they spread over all of H.
 // Roles (480 threads): warp 0 loads by TMA the packed rows of every K step
-// (256 rows of one group) and the matching 64 columns of H; warps 1 and 14
-// issue the MMAs, one 128-row half each (4 per K step: K = 16 each); warps
+// (256 rows of KG groups) and the matching 64-column slices of H; warps 1
+// and 14 issue the MMAs, one 128-row half each (4 per group: K = 16 each); warps
 // 2-9 dequantise, one vocab row per thread, into a ring of TMEM A slots;
 // warps 10-13 drain the accumulators (one vocab row per thread), reduce
 // each head row's maximum and sum of exponentials over the block's 256
 // vocab rows and write the block's partials.
 //
-// TMEM (512 columns): A ring, 4 slots x (2 halves x 32 columns); from column
-// 256 the accumulators, 2 halves x Mp columns, two buffers when Mp <= 64.
-// Shared-memory traffic per K step: packed 8 KB (4-bit) written by TMA and
-// read once by the dequantisers, the H slice (Mp x 128 bytes) written once
-// and read by the 8 MMAs; no operand stores by threads.
+// TMEM (512 columns): A ring of NA slots x (2 halves x KG groups x 32
+// columns); from column 256 the accumulators, 2 halves x Mp columns, two
+// buffers when Mp <= 64.  Shared-memory traffic per group: packed 8 KB
+// (4-bit) written by TMA and read once by the dequantisers, the H slice (Mp
+// x 128 bytes) written once and read by 8 MMAs; no operand stores by
+// threads.  Two groups per K step (4-bit heads) halve the hand-offs between the roles
+// (waits, commits, stores), which bound the one-group form.
 //
 // All waits are bounded; a timeout sets the status word.
 #pragma once
@@ -52,8 +54,7 @@ namespace cce {
 
 constexpr int QS_BLK = 256;          // vocab rows per block (two MMA halves)
 constexpr int QS_MAXM = 128;         // head rows at most
-constexpr int QS_NA = 4;             // TMEM A slots (one K step each)
-constexpr int QS_ACC0 = QS_NA * 64;  // first accumulator column
+constexpr int QS_ACC0 = 256;         // first accumulator column (the A ring below it)
 constexpr uint32_t QS_TMEM_COLS = 512;
 constexpr int QS_DQ0 = 2;            // first dequantisation warp (8 of them)
 constexpr int QS_EP0 = 10;           // first epilogue warp (4 of them)
@@ -61,14 +62,23 @@ constexpr int QS_ISS1 = 14;          // the second MMA issuer (half 1; warp 1 is
 constexpr int QS_THREADS = 15 * 32;
 constexpr int QS_MAXC = QS_MAXM / 32;  // 32-column chunks of the accumulator
 
-// Stage: packed [256 rows x QB*8 bytes], then H [Mp rows x 64 fp16] with the
-// 128-byte swizzle (1024-aligned).
+// KG groups of 64 weights per K step: 2 for 4-bit heads (half the
+// hand-offs between the roles per weight), 1 for 8-bit heads (whose
+// two-group stages would leave room for 3 stages instead of 6, too few to
+// cover HBM latency at twice the bytes: measured 10-15 % slower).
+// Stage: packed [256 rows x KG*QB*8 bytes], then per group H [Mp rows x
+// 64 fp16] with the 128-byte swizzle (1024-aligned, HG bytes apart).  TMEM
+// A ring below column 256: NA slots of 2 halves x KG groups x 32 columns.
 template <int QB>
 struct QsCfg {
-  static constexpr int PK = QS_BLK * QB * 8;
-  static constexpr int HB = QS_MAXM * 128;
+  static constexpr int KG = QB == 4 ? 2 : 1;
+  static constexpr int SLOT = 2 * KG * 32;
+  static constexpr int NA = QS_ACC0 / SLOT;
+  static constexpr int PK = QS_BLK * QB * 8 * KG;
+  static constexpr int HG = QS_MAXM * 128;
+  static constexpr int HB = KG * HG;
   static constexpr int STAGE = PK + HB;
-  static constexpr int NST = QB == 4 ? 8 : 6;
+  static constexpr int NST = QB == 4 ? 4 : 6;
   static constexpr int RED = 2 * 2 * 4 * QS_MAXM * 4;  // [parity][m|s][quarter][row]
   static constexpr int BC = 4 * 32 * 4;                // per epilogue warp broadcast row
   static constexpr int BARS = 512;
@@ -81,7 +91,8 @@ static_assert(QsCfg<4>::SMEM <= 232448 && QsCfg<8>::SMEM <= 232448,
 struct QsArgs {
   int M, Mp;       // head rows; rounded up to a multiple of 16 (the MMA's N)
   int V, D;
-  int nk;          // K steps (groups of 64) over D
+  int nk;          // K steps over D (QsCfg<QB>::KG groups of 64 each in qsmall_fwd.cuh,
+                   // one in qwide_fwd.cuh)
   int n_blk;       // 256-row vocab blocks
   int nacc;        // accumulator buffers (2 when Mp <= 64)
   uint64_t wait_ns;
@@ -166,13 +177,13 @@ struct QsStep {
   int s, a;
   uint32_t ph, aph;
 };
-template <int NST>
+template <int NST, int NA>
 __device__ __forceinline__ QsStep qs_step(uint32_t n) {
   QsStep r;
   r.s = static_cast<int>(n % NST);
   r.ph = (n / NST) & 1u;
-  r.a = static_cast<int>(n % QS_NA);
-  r.aph = (n / QS_NA) & 1u;
+  r.a = static_cast<int>(n % NA);
+  r.aph = (n / NA) & 1u;
   return r;
 }
 
@@ -190,9 +201,9 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(bc) + F::BC);
   uint64_t* full = bars;                   // [NST] stage landed (TMA bytes)
   uint64_t* empty = full + F::NST;         // [NST] 8 dequant warps read + MMAs done
-  uint64_t* afull = empty + F::NST;        // [QS_NA] 8 dequant warps stored
-  uint64_t* aempty = afull + QS_NA;        // [QS_NA] MMAs read
-  uint64_t* accfull = aempty + QS_NA;      // [2]
+  uint64_t* afull = empty + F::NST;        // [NA] 8 dequant warps stored
+  uint64_t* aempty = afull + F::NA;        // [NA] MMAs read
+  uint64_t* accfull = aempty + F::NA;      // [2]
   uint64_t* accempty = accfull + 2;        // [2] 4 epilogue warps drained
   uint64_t* drain = accempty + 2;          // [2] one per MMA issuer
   uint64_t* epibar = drain + 2;            // [2] 4 epilogue warps wrote their pairs
@@ -205,7 +216,7 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 10);
     }
-    for (int s = 0; s < QS_NA; ++s) {
+    for (int s = 0; s < F::NA; ++s) {
       mbar_init(&afull[s], 8);
       mbar_init(&aempty[s], 2);
     }
@@ -245,15 +256,17 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
         const int k0 = blk % nk;
         for (int i = 0; i < nk; ++i, ++n) {
           const int k = k0 + i < nk ? k0 + i : k0 + i - nk;
-          const QsStep q = qs_step<F::NST>(n);
+          const QsStep q = qs_step<F::NST, F::NA>(n);
           if (!wait_bounded(&empty[q.s], q.ph ^ 1u, a.wait_ns, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t* st = base + q.s * F::STAGE;
-          mbar_arrive_expect_tx(&full[q.s], static_cast<uint32_t>(F::PK) + hbytes);
-          tma_load_2d(st, &tmP, &full[q.s], k * QB * 8, blk * QS_BLK);
-          tma_load_2d(st + F::PK, &tmH, &full[q.s], k * 64, 0);
+          mbar_arrive_expect_tx(&full[q.s], static_cast<uint32_t>(F::PK) + F::KG * hbytes);
+          tma_load_2d(st, &tmP, &full[q.s], k * F::KG * QB * 8, blk * QS_BLK);
+#pragma unroll
+          for (int g = 0; g < F::KG; ++g)
+            tma_load_2d(st + F::PK + g * F::HG, &tmH, &full[q.s], (k * F::KG + g) * 64, 0);
         }
       }
       if (!ok) fail();
@@ -261,7 +274,7 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
       // steps' stages (earlier ones were consumed, hence landed).
       const uint32_t n0 = n > static_cast<uint32_t>(F::NST) ? n - F::NST : 0u;
       for (uint32_t i = n0; i < n; ++i) {
-        const QsStep q = qs_step<F::NST>(i);
+        const QsStep q = qs_step<F::NST, F::NA>(i);
         wait_bounded(&full[q.s], q.ph, DRAIN_LIMIT_NS, nullptr);
       }
     }
@@ -286,7 +299,7 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
         tc_fence_after();
         const uint32_t dcol = tmem_base + QS_ACC0 + static_cast<uint32_t>(buf * 2 * a.Mp);
         for (int i = 0; i < nk; ++i, ++n) {
-          const QsStep q = qs_step<F::NST>(n);
+          const QsStep q = qs_step<F::NST, F::NA>(n);
           if (!wait_bounded(&full[q.s], q.ph, a.wait_ns, abort_flag) ||
               !wait_bounded(&afull[q.a], q.aph, a.wait_ns, abort_flag)) {
             ok = false;
@@ -295,10 +308,14 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
           tc_fence_after();
           const uint32_t sH = smem_u32(base + q.s * F::STAGE + F::PK);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int g = 0; g < F::KG; ++g)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
               umma_f16_ts(dcol + static_cast<uint32_t>(h * a.Mp),
-                          tmem_base + static_cast<uint32_t>(q.a * 64 + h * 32 + j * 8),
-                          sdesc_sw128(sH + j * 32, 16, 1024), idesc, (i | j) != 0 ? 1u : 0u);
+                          tmem_base + static_cast<uint32_t>(q.a * F::SLOT + h * F::KG * 32 +
+                                                            g * 32 + j * 8),
+                          sdesc_sw128(sH + g * F::HG + j * 32, 16, 1024), idesc,
+                          (i | g | j) != 0 ? 1u : 0u);
           umma_commit(&empty[q.s]);
           umma_commit(&aempty[q.a]);
         }
@@ -313,9 +330,10 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
   } else if (warp < QS_EP0) {
     // ------------------------------------------------- dequantisation --
     // Thread = vocab row rin of the block (TMEM lane rin % 128 of half
-    // rin / 128).  Per K step: the row's packed words from the stage, its
-    // scale and bias (8 groups per 16-byte load, the next 8 fetched while
-    // these are used), 64 fp16 weights into the A slot.
+    // rin / 128).  Per K step: the row's packed words of KG groups from
+    // the stage, their scales and biases (8 groups per 16-byte load, the
+    // next 8 fetched while these are used), 64 fp16 weights per group into
+    // the A slot (one tcgen05.st each).
     const int q4 = warp & 3, h = (warp - QS_DQ0) >> 2;
     const int rin = h * 128 + q4 * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
@@ -328,9 +346,11 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
       const bool valid = v < a.V;
       const uint4* srow = reinterpret_cast<const uint4*>(a.q_scale + static_cast<size_t>(v) * gpr);
       const uint4* brow = reinterpret_cast<const uint4*>(a.q_bias + static_cast<size_t>(v) * gpr);
-      // the K loop starts at group k0 and wraps (as the producer's)
+      // the K loop starts at step k0 and wraps (as the producer's); group
+      // gi = k * KG + g of step k; scales and biases 8 groups per load,
+      // the next 8 fetched while these are used
       const int k0 = blk % nk, n8 = gpr / 8;
-      const int g8 = k0 >> 3, g8n = g8 + 1 < n8 ? g8 + 1 : 0;
+      const int g8 = (k0 * F::KG) >> 3, g8n = g8 + 1 < n8 ? g8 + 1 : 0;
       uint4 sc = make_uint4(0, 0, 0, 0), bi = sc, sc_n = sc, bi_n = sc;
       if (valid) {
         sc = __ldg(srow + g8);
@@ -340,56 +360,68 @@ __global__ void __launch_bounds__(QS_THREADS, 1)
       }
       for (int i = 0; i < nk; ++i, ++n) {
         const int k = k0 + i < nk ? k0 + i : k0 + i - nk;
-        if ((k & 7) == 0 && i > 0) {
-          sc = sc_n;
-          bi = bi_n;
-          const int nx = (k >> 3) + 1 < n8 ? (k >> 3) + 1 : 0;
-          if (valid) {
-            sc_n = __ldg(srow + nx);
-            bi_n = __ldg(brow + nx);
-          }
-        }
-        const QsStep q = qs_step<F::NST>(n);
+        const QsStep q = qs_step<F::NST, F::NA>(n);
         if (!__all_sync(0xffffffffu, wait_bounded(&full[q.s], q.ph, a.wait_ns, abort_flag))) {
           ok = false;
           break;
         }
-        uint4 w[NV];
-        const uint8_t* sP = base + q.s * F::STAGE + rin * (QB * 8);
+        uint4 w[F::KG][NV];
+        const uint8_t* sP = base + q.s * F::STAGE + rin * (F::KG * QB * 8);
 #pragma unroll
-        for (int i = 0; i < NV; ++i) w[i] = *reinterpret_cast<const uint4*>(sP + 16 * i);
+        for (int g = 0; g < F::KG; ++g)
+#pragma unroll
+          for (int t = 0; t < NV; ++t)
+            w[g][t] = *reinterpret_cast<const uint4*>(sP + g * (QB * 8) + 16 * t);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[q.s]);
-        const int g = k & 7;
-        const uint32_t ws = (g >> 1) == 0 ? sc.x : (g >> 1) == 1 ? sc.y : (g >> 1) == 2 ? sc.z : sc.w;
-        const uint32_t wb = (g >> 1) == 0 ? bi.x : (g >> 1) == 1 ? bi.y : (g >> 1) == 2 ? bi.z : bi.w;
-        const uint16_t sbits = static_cast<uint16_t>((g & 1) ? ws >> 16 : ws & 0xFFFFu);
-        const uint16_t bbits = static_cast<uint16_t>((g & 1) ? wb >> 16 : wb & 0xFFFFu);
-        uint4 out[8];
-        if (valid) {
-          if constexpr (QB == 8)
-            dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w), sbits, bbits, out);
-          else
-            dequant_group64(w[0], w[NV - 1], sbits, bbits, out);
-        } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
-        }
-        uint32_t r[32];
+        for (int g = 0; g < F::KG; ++g) {
+          const int gi = k * F::KG + g;
+          if ((gi & 7) == 0 && (i | g) != 0) {
+            sc = sc_n;
+            bi = bi_n;
+            const int nx = (gi >> 3) + 1 < n8 ? (gi >> 3) + 1 : 0;
+            if (valid) {
+              sc_n = __ldg(srow + nx);
+              bi_n = __ldg(brow + nx);
+            }
+          }
+          const int gg = gi & 7;
+          const uint32_t ws = (gg >> 1) == 0 ? sc.x : (gg >> 1) == 1 ? sc.y : (gg >> 1) == 2 ? sc.z : sc.w;
+          const uint32_t wb = (gg >> 1) == 0 ? bi.x : (gg >> 1) == 1 ? bi.y : (gg >> 1) == 2 ? bi.z : bi.w;
+          const uint16_t sbits = static_cast<uint16_t>((gg & 1) ? ws >> 16 : ws & 0xFFFFu);
+          const uint16_t bbits = static_cast<uint16_t>((gg & 1) ? wb >> 16 : wb & 0xFFFFu);
+          uint4 out[8];
+          if (valid) {
+            if constexpr (QB == 8)
+              dequant_group64_q8(*reinterpret_cast<const uint4(*)[4]>(w[g]), sbits, bbits, out);
+            else
+              dequant_group64(w[g][0], w[g][NV - 1], sbits, bbits, out);
+          } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          r[4 * c] = out[c].x;
-          r[4 * c + 1] = out[c].y;
-          r[4 * c + 2] = out[c].z;
-          r[4 * c + 3] = out[c].w;
+            for (int c = 0; c < 8; ++c) out[c] = make_uint4(0, 0, 0, 0);
+          }
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            r[4 * c] = out[c].x;
+            r[4 * c + 1] = out[c].y;
+            r[4 * c + 2] = out[c].z;
+            r[4 * c + 3] = out[c].w;
+          }
+          if (g == 0) {
+            if (!__all_sync(0xffffffffu,
+                            wait_bounded(&aempty[q.a], q.aph ^ 1u, a.wait_ns, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          tmem_st32(tmem_base + lane_addr +
+                        static_cast<uint32_t>(q.a * F::SLOT + h * F::KG * 32 + g * 32),
+                    r);
         }
-        if (!__all_sync(0xffffffffu,
-                        wait_bounded(&aempty[q.a], q.aph ^ 1u, a.wait_ns, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st32(tmem_base + lane_addr + static_cast<uint32_t>(q.a * 64 + h * 32), r);
+        if (!ok) break;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
