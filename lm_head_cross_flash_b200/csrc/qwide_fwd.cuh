@@ -1,7 +1,8 @@
-// qwide_fwd.cuh — the transposed forward of a 4/8-bit head for 129 to 256
-// head rows: S^T[v, m] = W_t[v, :] . H[m, :] with the dequantised head
-// tile as the A operand in TMEM, as in qsmall_fwd.cuh, but with N up to 256
-// (M rounded up to 16), so one accumulator is as wide as the head rows.
+// qwide_fwd.cuh — the transposed forward of a 4/8-bit head for up to 256
+// head rows (the library chooses it for 129 to 240): S^T[v, m] =
+// W_t[v, :] . H[m, :] with the dequantised head tile as the A operand in
+// TMEM, as in qsmall_fwd.cuh, but with N up to 256 (M rounded up to 16), so
+// one accumulator is as wide as the head rows.
 //
 // What it computes is the forward of the flash-CCE head (ORPO design 0.0.6,
 // fused-head implementation spec, "Forward"; Training design §5.6 for the
