@@ -63,9 +63,10 @@ constexpr int QS_THREADS = 15 * 32;
 constexpr int QS_MAXC = QS_MAXM / 32;  // 32-column chunks of the accumulator
 
 // KG groups of 64 weights per K step: 2 for 4-bit heads (half the
-// hand-offs between the roles per weight), 1 for 8-bit heads (whose
-// two-group stages would leave room for 3 stages instead of 6, too few to
-// cover HBM latency at twice the bytes: measured 10-15 % slower).
+// hand-offs between the roles per weight; 15 % faster at N = 64), 1 for
+// 8-bit heads, where two groups measured 10-15 % slower: with 3 stages of
+// 64 KB, and also with 4 of 48 KB when the H slots were sized for N <= 64
+// (which left 4-bit heads unchanged with 6 stages instead of 4).
 // Stage: packed [256 rows x KG*QB*8 bytes], then per group H [Mp rows x
 // 64 fp16] with the 128-byte swizzle (1024-aligned, HG bytes apart).  TMEM
 // A ring below column 256: NA slots of 2 halves x KG groups x 32 columns.
