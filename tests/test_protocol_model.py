@@ -20,6 +20,13 @@ shows that they can.
   else can), which opens the windows a lagging warp leaves.  The lead cap is
   a bounded hint, not a dependency, and is left out.  A CTA pair runs as one
   member.
+* The transposed small-M forwards (qsmall_fwd.cuh, qwide_fwd.cuh): the
+  producer, the MMA issuer(s), the eight dequantisation warps and the four
+  epilogue warps of one CTA, with the stage ring, the TMEM A ring, the
+  accumulators and the epilogue's merge barrier as phase objects; safety
+  (no stage, A slot, accumulator or merge buffer reused before its readers
+  are done) is tracked apart from the barriers, and every role is held back
+  in turn.
 * The sliced kernel (slice_bwd.cuh): per CTA of a cluster, the S and dH
   loaders and MMA issuers, the drain warps and the reducer warps, with the
   double-buffered partial (pfull, pempty), G'' (gfull, gempty) and S
@@ -469,3 +476,302 @@ def test_sliced_protocol_with_a_slow_role(n, ccl):
     for c in sorted({0, ccl - 1}):
         for r in range(SLICED_ROLES):
             assert _sliced_model(n, ccl, slow=[(c, r)]) == [], (c, r)
+
+
+# ------------------------------------------------ transposed small-M forward --
+def _qsmall_model(nblk, nk, nst, na, nacc, bug=None, slow=()):
+    """One CTA of qsmall_fwd_kernel: the producer, the two MMA issuers
+    (halves 0 and 1), eight dequantisation warps and four epilogue warps
+    over nblk blocks of nk K steps; stage ring (full, empty), TMEM A ring
+    (afull, aempty), accumulators (accfull, accempty; nacc buffers) and the
+    epilogue's merge barrier (epibar, two by block parity), each a phase
+    object tagged with its step or block.  Safety, tracked apart from the
+    barriers: a stage is reloaded only after its previous step's ten reads,
+    an A slot rewritten only after both issuers' MMAs of its previous step,
+    an accumulator overwritten only after the four warps drained its
+    previous block and drained only after both halves' MMAs, and a merge
+    buffer rewritten only after every warp read it.  bug: "aempty_one_back"
+    (a dequantisation warp waits for the slot's use two steps back instead
+    of one), "accempty_parity" (the issuers wait for the wrong buffer use)."""
+    steps = nblk * nk
+    st_tiles = lambda s: [n for n in range(steps) if n % nst == s]
+    a_tiles = lambda a: [n for n in range(steps) if n % na == a]
+    b_tiles = lambda b, m: [u for u in range(nblk) if u % m == b]
+    bars = {
+        "full": [_Phase(1, st_tiles(s)) for s in range(nst)],
+        "empty": [_Phase(10, st_tiles(s)) for s in range(nst)],
+        "afull": [_Phase(8, a_tiles(a)) for a in range(na)],
+        "aempty": [_Phase(2, a_tiles(a)) for a in range(na)],
+        "accfull": [_Phase(2, b_tiles(b, nacc)) for b in range(nacc)],
+        "accempty": [_Phase(4, b_tiles(b, nacc)) for b in range(nacc)],
+        "epibar": [_Phase(4, b_tiles(p, 2)) for p in range(2)],
+    }
+    seen = {"stage_reads": {}, "mma_done": {}, "drained": {}, "mma_block": {},
+            "red_written": {}, "red_read": {}, "violations": []}
+
+    def bump(key, k):
+        seen[key][k] = seen[key].get(k, 0) + 1
+
+    P = []
+    for n in range(steps):
+        s = n % nst
+        if n >= nst:
+            P.append(("wait", "empty", s, n - nst))
+        P += [("check_stage_free", n), ("arrive", "full", s, n)]
+    I = []
+    for h in range(2):
+        ops = []
+        for u in range(nblk):
+            b = u % nacc
+            prev = u - nacc if bug != "accempty_parity" else u - 2 * nacc
+            if prev >= 0:
+                ops.append(("wait", "accempty", b, prev))
+            ops.append(("check_acc_free", u))
+            for i in range(nk):
+                n = u * nk + i
+                ops += [("wait", "full", n % nst, n), ("wait", "afull", n % na, n),
+                        ("mma", n, u), ("arrive", "empty", n % nst, n),
+                        ("arrive", "aempty", n % na, n)]
+            ops.append(("arrive", "accfull", b, u))
+        I.append(ops)
+    Dq = []
+    for w in range(8):
+        ops = []
+        for n in range(steps):
+            back = na if bug != "aempty_one_back" else 2 * na
+            ops += [("wait", "full", n % nst, n), ("read_stage", n),
+                    ("arrive", "empty", n % nst, n)]
+            if n >= back:
+                ops.append(("wait", "aempty", n % na, n - back))
+            ops += [("check_slot_free", n), ("arrive", "afull", n % na, n)]
+        Dq.append(ops)
+    E = []
+    for w in range(4):
+        ops = []
+        for u in range(nblk):
+            b, par = u % nacc, u % 2
+            ops += [("wait", "accfull", b, u), ("check_acc_ready", u), ("drain", u),
+                    ("arrive", "accempty", b, u), ("check_red_free", w, u), ("write_red", w, u),
+                    ("arrive", "epibar", par, u), ("wait", "epibar", par, u), ("read_red", w, u)]
+        E.append(ops)
+    procs = [({}, [P] + I + Dq + E)]
+
+    def step(_, op, *a):
+        v = seen["violations"]
+        if op == "wait":
+            return bars[a[0]][a[1]].done(a[2])
+        if op == "arrive":
+            bars[a[0]][a[1]].arrive(a[2])
+            if a[0] == "full":  # the TMA bytes land with the arming
+                pass
+            return True
+        if op == "check_stage_free":
+            n = a[0]
+            if n >= nst and seen["stage_reads"].get(n - nst, 0) < 10:
+                v.append(("stage reloaded early", n))
+            return True
+        if op == "read_stage":
+            bump("stage_reads", a[0])
+            return True
+        if op == "mma":
+            bump("stage_reads", a[0])
+            bump("mma_done", a[0])
+            bump("mma_block", a[1])
+            return True
+        if op == "check_slot_free":
+            n = a[0]
+            if n >= na and seen["mma_done"].get(n - na, 0) < 2:
+                v.append(("A slot rewritten early", n))
+            return True
+        if op == "check_acc_free":
+            u = a[0]
+            if u >= nacc and seen["drained"].get(u - nacc, 0) < 4:
+                v.append(("accumulator overwritten early", u))
+            return True
+        if op == "check_acc_ready":
+            if seen["mma_block"].get(a[0], 0) < 2 * nk:
+                v.append(("accumulator drained early", a[0]))
+            return True
+        if op == "drain":
+            bump("drained", a[0])
+            return True
+        if op == "check_red_free":
+            w, u = a
+            if u >= 2 and seen["red_read"].get(u - 2, 0) < 4:
+                v.append(("merge buffer rewritten early", u))
+            return True
+        if op == "write_red":
+            bump("red_written", a[1])
+            return True
+        if op == "read_red":
+            if seen["red_written"].get(a[1], 0) < 4:
+                v.append(("merge buffer read early", a[1]))
+            bump("red_read", a[1])
+            return True
+        raise ValueError(op)
+
+    try:
+        stuck = _run(procs, step, slow=slow)
+    except AssertionError as e:
+        return [("phase", str(e))]
+    return stuck + seen["violations"]
+
+
+QSMALL_SHAPES = [(3, 5, 4, 2, 2), (3, 5, 6, 4, 2), (4, 7, 4, 2, 1), (5, 3, 6, 4, 1), (1, 1, 4, 2, 2)]
+QSMALL_ROLES = 1 + 2 + 8 + 4
+
+
+@pytest.mark.parametrize("nblk,nk,nst,na,nacc", QSMALL_SHAPES)
+def test_qsmall_protocol_runs_to_the_end(nblk, nk, nst, na, nacc):
+    """The transposed small-M forward's protocol (4-bit: 4 stages, 2 A
+    slots; 8-bit: 6 stages, 4 slots; one or two accumulators) runs to the
+    end, also with each role held back in turn, with no early reuse."""
+    assert _qsmall_model(nblk, nk, nst, na, nacc) == []
+    for r in range(QSMALL_ROLES):
+        assert _qsmall_model(nblk, nk, nst, na, nacc, slow=[(0, r)]) == [], r
+
+
+@pytest.mark.parametrize("bug", ["aempty_one_back", "accempty_parity"])
+def test_qsmall_protocol_model_catches_planted_mistakes(bug):
+    found = []
+    for r in range(QSMALL_ROLES):
+        found += _qsmall_model(4, 7, 4, 2, 2, bug=bug, slow=[(0, r)])
+    assert found, bug
+
+
+def _qwide_model(nblk, nk, nst=5, na=8, bug=None, slow=()):
+    """One CTA of qwide_fwd_kernel: the producer, one MMA issuer, eight
+    dequantisation warps and four epilogue warps; each block is two 128-row
+    units of nk K steps run one after the other into one accumulator.  The
+    same safety checks as _qsmall_model, per unit.  bug: "accempty_skip"
+    (the issuer does not wait for the drain of the previous unit)."""
+    units = 2 * nblk
+    steps = units * nk
+    st_tiles = lambda s: [n for n in range(steps) if n % nst == s]
+    a_tiles = lambda a: [n for n in range(steps) if n % na == a]
+    bars = {
+        "full": [_Phase(1, st_tiles(s)) for s in range(nst)],
+        "empty": [_Phase(9, st_tiles(s)) for s in range(nst)],
+        "afull": [_Phase(8, a_tiles(a)) for a in range(na)],
+        "aempty": [_Phase(1, a_tiles(a)) for a in range(na)],
+        "accfull": [_Phase(1, list(range(units)))],
+        "accempty": [_Phase(4, list(range(units)))],
+        "epibar": [_Phase(4, [u for u in range(nblk) if u % 2 == p]) for p in range(2)],
+    }
+    seen = {"stage_reads": {}, "mma_done": {}, "drained": {}, "mma_unit": {},
+            "red_written": {}, "red_read": {}, "violations": []}
+
+    def bump(key, k):
+        seen[key][k] = seen[key].get(k, 0) + 1
+
+    P = []
+    for n in range(steps):
+        if n >= nst:
+            P.append(("wait", "empty", n % nst, n - nst))
+        P += [("check_stage_free", n), ("arrive", "full", n % nst, n)]
+    X = []
+    for t in range(units):
+        if t >= 1 and bug != "accempty_skip":
+            X.append(("wait", "accempty", 0, t - 1))
+        X.append(("check_acc_free", t))
+        for i in range(nk):
+            n = t * nk + i
+            X += [("wait", "full", n % nst, n), ("wait", "afull", n % na, n), ("mma", n, t),
+                  ("arrive", "empty", n % nst, n), ("arrive", "aempty", n % na, n)]
+        X.append(("arrive", "accfull", 0, t))
+    Dq = []
+    for w in range(8):
+        ops = []
+        for n in range(steps):
+            ops += [("wait", "full", n % nst, n), ("read_stage", n),
+                    ("arrive", "empty", n % nst, n)]
+            if n >= na:
+                ops.append(("wait", "aempty", n % na, n - na))
+            ops += [("check_slot_free", n), ("arrive", "afull", n % na, n)]
+        Dq.append(ops)
+    E = []
+    for w in range(4):
+        ops = []
+        for u in range(nblk):
+            for h in range(2):
+                t = 2 * u + h
+                ops += [("wait", "accfull", 0, t), ("check_acc_ready", t), ("drain", t),
+                        ("arrive", "accempty", 0, t)]
+            ops += [("check_red_free", w, u), ("write_red", w, u), ("arrive", "epibar", u % 2, u),
+                    ("wait", "epibar", u % 2, u), ("read_red", w, u)]
+        E.append(ops)
+    procs = [({}, [P, X] + Dq + E)]
+
+    def step(_, op, *a):
+        v = seen["violations"]
+        if op == "wait":
+            return bars[a[0]][a[1]].done(a[2])
+        if op == "arrive":
+            bars[a[0]][a[1]].arrive(a[2])
+            return True
+        if op == "check_stage_free":
+            if a[0] >= nst and seen["stage_reads"].get(a[0] - nst, 0) < 9:
+                v.append(("stage reloaded early", a[0]))
+            return True
+        if op == "read_stage":
+            bump("stage_reads", a[0])
+            return True
+        if op == "mma":
+            bump("stage_reads", a[0])
+            bump("mma_done", a[0])
+            bump("mma_unit", a[1])
+            return True
+        if op == "check_slot_free":
+            if a[0] >= na and seen["mma_done"].get(a[0] - na, 0) < 1:
+                v.append(("A slot rewritten early", a[0]))
+            return True
+        if op == "check_acc_free":
+            if a[0] >= 1 and seen["drained"].get(a[0] - 1, 0) < 4:
+                v.append(("accumulator overwritten early", a[0]))
+            return True
+        if op == "check_acc_ready":
+            if seen["mma_unit"].get(a[0], 0) < nk:
+                v.append(("accumulator drained early", a[0]))
+            return True
+        if op == "drain":
+            bump("drained", a[0])
+            return True
+        if op == "check_red_free":
+            if a[1] >= 2 and seen["red_read"].get(a[1] - 2, 0) < 4:
+                v.append(("merge buffer rewritten early", a[1]))
+            return True
+        if op == "write_red":
+            bump("red_written", a[1])
+            return True
+        if op == "read_red":
+            if seen["red_written"].get(a[1], 0) < 4:
+                v.append(("merge buffer read early", a[1]))
+            bump("red_read", a[1])
+            return True
+        raise ValueError(op)
+
+    try:
+        stuck = _run(procs, step, slow=slow)
+    except AssertionError as e:
+        return [("phase", str(e))]
+    return stuck + seen["violations"]
+
+
+QWIDE_ROLES = 1 + 1 + 8 + 4
+
+
+@pytest.mark.parametrize("nblk,nk", [(3, 5), (4, 9), (1, 1), (2, 16)])
+def test_qwide_protocol_runs_to_the_end(nblk, nk):
+    """The wide transposed forward's protocol (5 stages, 8 A slots, one
+    accumulator for two units per block) runs to the end, also with each
+    role held back in turn, with no early reuse."""
+    assert _qwide_model(nblk, nk) == []
+    for r in range(QWIDE_ROLES):
+        assert _qwide_model(nblk, nk, slow=[(0, r)]) == [], r
+
+
+def test_qwide_protocol_model_catches_a_planted_mistake():
+    found = []
+    for r in range(QWIDE_ROLES):
+        found += _qwide_model(3, 5, bug="accempty_skip", slow=[(0, r)])
+    assert any(f[0] == "accumulator overwritten early" for f in found), found[:3]
